@@ -1,0 +1,52 @@
+"""The FLOP / parameter / byte model against the figures the pages print."""
+import json
+import os
+
+import pytest
+
+from token_mixing_feature_b200 import roofline, synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def test_appendix_b_flops():
+    """Three Mixer layers at B=256, T=8, d=256, h=1024 -> 6.442451 GFLOPs (Appendix B)."""
+    with open(os.path.join(GOLDEN, "appendix_b_flops.json")) as f:
+        g = json.load(f)
+    flops = g["L"] * roofline.dense_block_flops(g["B"], g["T"], g["D"], g["hidden"])
+    assert round(flops / 1e9, 6) == g["gflops"]
+    for row in g["rows"]:
+        # the TFLOP/s column is the GFLOPs over the ms column, which the table
+        # prints rounded to 1 us: the printed rate lies inside that interval
+        lo = flops / ((row["ms"] + 5e-4) * 1e-3) / 1e12
+        hi = flops / ((row["ms"] - 5e-4) * 1e-3) / 1e12
+        assert lo - 5e-4 <= row["tflops"] <= hi + 5e-4
+
+
+def test_pffn_param_formula():
+    """Per-token FFN parameters 2 T k D^2: T times a shared FFN's 2 k D^2."""
+    assert roofline.pffn_params(1, 768, 4 * 768) * 16 == roofline.pffn_params(16, 768, 4 * 768)
+    assert roofline.pffn_params(16, 768, 3072) == 2 * 16 * 4 * 768 ** 2
+
+
+@pytest.mark.parametrize("name,params", [("rm100m", 151e6), ("rm1b", 1.2e9)])
+def test_workload_param_counts(name, params):
+    wl = synth.WORKLOADS[name]
+    p = wl.L * roofline.pffn_params(wl.T, wl.D, wl.hidden)
+    assert abs(p - params) / params < 0.02
+
+
+def test_stack_flops_and_bytes_1b():
+    wl = synth.WORKLOADS["rm1b"]
+    assert roofline.stack_flops(wl) == 2 * 4 * 512 * 32 * 1536 * 6144
+    wbytes = 2 * 2 * 32 * 1536 * 6144 * 2
+    assert roofline.stack_bytes(wl) > wbytes
+    assert roofline.stack_bytes(wl) < wbytes * 1.1
+
+
+def test_moe_flops_need_active_counts():
+    wl = synth.WORKLOADS["moe"]
+    with pytest.raises(ValueError):
+        roofline.stack_flops(wl)
+    f = roofline.stack_flops(wl, [1000, 2000])
+    assert f == 3000 * 4 * 768 * 768 + 2 * (2 * 2048 * 16 * 768 * 8)
