@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""RankMixer stack forward benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload rm1b] [--impl ours|reference]
+
+One step = one rm_stack_forward over the whole batch of the workload (every
+block: token mixing + LN, the two per-token FFN projections, and the final
+LN + mean pooling; plus Pad-Split tokenisation and the head for the padsplit
+workload).  Inputs are synthetic (seeded), resident in HBM before timing.
+The 1B-scale stack reads 2.42 GB of weights per step, far above the 126 MB L2,
+so no L2 flush is needed between steps.
+
+Prints ONE JSON line on rank 0.  With N > 1 (torchrun, one process per GPU)
+every rank runs an independent replica of the workload (the forward pass has
+no cross-sample exchange); time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (rank 0
+only), each step a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from token_mixing_feature_b200 import roofline, synth  # noqa: E402
+
+METRIC = "RankMixer stack fwd samples/s and TFLOP/s as % of bf16 roofline on 1×B200"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+# ---------------------------------------------------------------- utilities
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons of one GPU while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            gid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={gid}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+        sm = [num(r[1]) for r in rows]
+        power = [num(r[3]) for r in rows]
+        pmax = max(p for p in power if p == p) if any(p == p for p in power) else 0.0
+        loaded = [s for s, p in zip(sm, power) if p == p and p >= 0.5 * pmax] or sm
+        reasons = sorted({self.REASONS[i] for r in rows for i in range(4) if "Active" == r[5 + i]
+                          or r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(num(r[2]) for r in rows),
+                "power_w_max": pmax, "samples": len(rows), "reasons": reasons}
+
+
+def traffic_from_profiles(kernel_key: str):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, if the
+    summary was taken on the current source of the GEMM kernel."""
+    path = os.path.join(ROOT, "profiles", "ncu_gemm_tc_rm1b.md")
+    src = os.path.join(ROOT, "token_mixing_feature_b200", "csrc", "rm_gemm_tc.cu")
+    try:
+        text = open(path).read()
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    m = re.search(r"source sha256\[:16\]:\s*([0-9a-f]{16})", text)
+    if not m or m.group(1) != digest:
+        return None
+    m = re.search(rf"dram_bytes_per_launch\s+{re.escape(kernel_key)}\s*[:=]\s*([0-9.eE+]+)", text)
+    return float(m.group(1)) if m else None
+
+
+# ----------------------------------------------------------- workload steps
+class Runner:
+    def __init__(self, wl: synth.Workload, device):
+        from token_mixing_feature_b200 import rankmixer as rm
+        from token_mixing_feature_b200.stack import RankMixerStack
+        self.rm = rm
+        self.wl = wl
+        self.device = device
+        d = synth.make_inputs(wl)
+        self.inputs = d
+        self.st = RankMixerStack(wl, d["blocks"], d.get("head"), device=device)
+        self.pooled = torch.empty(wl.B, wl.D, dtype=torch.float32, device=device)
+        if wl.group_widths:
+            self.groups = [g.to(device) for g in d["groups"]]
+            self.X0 = self.st.empty_act(wl.B)
+            self.prob = torch.empty(wl.B, dtype=torch.float32, device=device)
+        else:
+            self.X0 = d["X0"].to(device)
+
+    def launches_per_step(self) -> int:
+        wl = self.wl
+        per_block = 7 if wl.n_experts else 3   # MoE: mix, route, compact, gather, 2 GEMMs, combine
+        n = wl.L * per_block + 1
+        if wl.group_widths:
+            n += 2
+        return n
+
+    def step(self):
+        if self.wl.group_widths:
+            self.st.tokenize(self.groups, self.X0)
+        self.st.forward(self.X0, self.pooled)
+        if self.wl.head:
+            self.st.head_forward(self.pooled, self.prob)
+
+
+def moe_active_counts(runner: Runner):
+    """Per-block active expert counts, routing the real S of every block."""
+    rm, wl, st = runner.rm, runner.wl, runner.st
+    counts = []
+    x = runner.X0
+    G = torch.empty(wl.B, wl.T, wl.n_experts, dtype=torch.float32, device=runner.device)
+    V = torch.empty_like(x)
+    for l in range(wl.L):
+        blk = st.blocks[l]
+        # S = LN1(mix(X) + X) through the library (token mix, then LN of X + mix(X))
+        M = torch.empty_like(x)
+        rm.rm_token_mix(st.h, x, M, wl.B)
+        S = torch.empty_like(x)
+        rm.rm_layernorm(st.h, M, x, blk["ln1_g"], blk["ln1_b"], S, wl.B * wl.T)
+        rm.rm_moe_forward(st.h, blk, S, V, G, wl.B)
+        torch.cuda.synchronize()
+        counts.append(int((G > 0).sum().item()))
+        x = st.block(l, x)
+    return counts
+
+
+def time_steps(fn, K: int, stream) -> float:
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(K):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_blocks_f32(d):
+    import numpy as np
+    out = []
+    for blk in d["blocks"]:
+        out.append({k: np.ascontiguousarray(v.float().numpy()) for k, v in blk.items()})
+    return out
+
+
+def oracle_sample_run(wl, blocks_np, samples, seed=0):
+    """One bounded oracle step: the stack for the given samples.  Returns seconds."""
+    import numpy as np
+    from oracle import oracle as O
+    idx = torch.tensor(samples, dtype=torch.long)
+    if wl.group_widths:
+        X0 = O.padsplit(synth.make_groups(wl, seed, samples=idx), wl.padded_width)
+        X0 = X0.reshape(len(samples), wl.T, wl.D).astype(np.float32)
+    else:
+        X0 = synth.make_x0(wl, seed, samples=idx).float().numpy()
+    t0 = time.perf_counter()
+    r = O.stack(X0, blocks_np, want_last=False)
+    if wl.head:
+        d = synth.make_head(wl, seed)
+        O.head(r["pooled"], d["w"], float(d["b"][0]))
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, d, target_s: float = 15.0):
+    from oracle import oracle as O
+    threads = O.num_threads()
+    blocks_np = oracle_blocks_f32(d)
+    n = threads
+    secs = oracle_sample_run(wl, blocks_np, list(range(min(n, wl.B))))
+    done, total = min(n, wl.B), secs
+    while total < target_s and done < wl.B:
+        m = min(wl.B - done, max(threads, int(done * (target_s - total) / max(total, 1e-3))))
+        total += oracle_sample_run(wl, blocks_np, list(range(done, done + m)))
+        done += m
+    return {"value": done / total, "unit": "samples/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} of {wl.B} samples of the {wl.name} stack (fp64 C loops, OpenMP over "
+                      f"samples), {total:.1f} s"}
+
+
+# ------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="rm1b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = synth.WORKLOADS[a.workload]
+    cfg = {"workload": wl.name, "B": wl.B, "T": wl.T, "D": wl.D, "hidden": wl.hidden, "L": wl.L,
+           "n_experts": wl.n_experts, "global_batch": wl.B * max(world, 1),
+           "parallelism": f"replicas x{max(world, 1)}" if world > 1 else "single GPU",
+           "l2": "no flush: inputs larger than L2 "
+                 f"({roofline.stack_bytes(wl) / 1e9:.2f} GB read per step vs 126 MB L2)"}
+
+    if a.impl == "reference":
+        return run_reference(a, wl, cfg, rank, world)
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+        pg = dist
+
+    runner = Runner(wl, device)
+    stream = torch.cuda.current_stream(device)
+    rm = runner.rm
+    sampler = ClockSampler(local) if rank == 0 else None
+
+    for _ in range(a.warmup):
+        runner.step()
+    torch.cuda.synchronize(device)
+    if rm.rm_sync_status(runner.st.h) != rm.RM_OK:
+        raise SystemExit("device error during warm-up")
+
+    def barrier():
+        if pg:
+            pg.barrier(device_ids=[local])
+        torch.cuda.synchronize(device)
+
+    def max_over_ranks(x: float) -> float:
+        if not pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    # headline: K steps, device time, max over ranks
+    barrier()
+    ms = time_steps(runner.step, a.steps, stream)
+    barrier()
+    ms = max_over_ranks(ms)
+
+    # per-kernel times over a second timed region of K steps (events on the launch stream)
+    rm.rm_profile_begin(runner.st.h, a.steps * runner.launches_per_step() + 8)
+    barrier()
+    ms_prof = time_steps(runner.step, a.steps, stream)
+    barrier()
+    prof = rm.rm_profile_end(runner.st.h)
+    if rm.rm_sync_status(runner.st.h) != rm.RM_OK:
+        raise SystemExit("device error during timing")
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(runner, a, device)
+    e2e_ms = max_over_ranks(e2e.pop("_ms"))
+    e2e["value"] = wl.B * max(world, 1) * a.steps / (e2e_ms / 1e3)
+
+    clocks = sampler.stop() if sampler else None
+    active = moe_active_counts(runner) if wl.n_experts else None
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        flops = roofline.stack_flops(wl, active)
+        nbytes = roofline.stack_bytes(wl)
+        sec = ms / 1e3 / a.steps
+        t_roof = roofline.roofline_seconds(flops, nbytes, peaks["bf16_tflops"] * 1e12, peaks["hbm_gbs"] * 1e9)
+        kern = {k: {"ms_avg": v[0] / max(v[1], 1), "launches": v[1],
+                    "share": v[0] / max(sum(x[0] for x in prof.values()), 1e-9)} for k, v in prof.items()}
+        top = max(prof, key=lambda k: prof[k][0])
+        # algorithmic FLOPs per launch of the top kernel (both projections have 2 B T D kD)
+        if top in ("gemm1", "gemm2"):
+            if wl.n_experts:
+                per_launch = 2.0 * sum(active) * wl.D * wl.hidden / wl.L
+            else:
+                per_launch = 2.0 * wl.B * wl.T * wl.D * wl.hidden
+            achieved = per_launch / (kern[top]["ms_avg"] / 1e3) / 1e12
+            roof = {"kernel": f"gemm_tc ({top})", "bound": "tensor", "achieved": achieved,
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops"],
+                    "traffic": traffic_from_profiles(top),
+                    "peak_source": f"bf16 dense burst, of {peak_src}",
+                    "flops_per_launch": per_launch}
+        else:
+            roof = {"kernel": top, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": None, "traffic": None}
+        line = {
+            "metric": METRIC, "value": wl.B * max(world, 1) * a.steps / (ms / 1e3), "unit": "samples/s",
+            "n_gpus": max(world, 1), "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+            "data": "synthetic (seeded N(0,1) inputs, Xavier-normal weights)", "config": cfg,
+            "tflops": flops / sec / 1e12 / max(world, 1),
+            "stack_roofline": {"flops": flops, "bytes": nbytes, "t_roof_ms": t_roof * 1e3,
+                               "frac": t_roof / sec, "peaks": f"bf16 {peaks['bf16_tflops']} TFLOP/s, "
+                               f"HBM {peaks['hbm_gbs']} GB/s, of {peak_src}"},
+            "roofline": roof,
+            "kernels": kern,
+            "profiled_ms_per_step": ms_prof / a.steps,
+            "e2e": e2e,
+            "gpu_launches": a.steps * runner.launches_per_step(),
+            "clocks": clocks,
+        }
+        if active is not None:
+            line["moe_active_per_block"] = active
+            line["moe_active_fraction"] = [c / (wl.B * wl.T * wl.n_experts) for c in active]
+        if world == 1 and not a.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, runner.inputs)
+        print(json.dumps(line), flush=True)
+    runner.st.close()
+    if pg:
+        pg.barrier(device_ids=[local])
+        pg.destroy_process_group()
+
+
+def run_e2e(runner: Runner, a, device):
+    """K steps through the C ABI with host buffers: the step's inputs copied
+    from pinned host memory and its result read back, every step."""
+    wl, rm, st = runner.wl, runner.rm, runner.st
+    if wl.group_widths:
+        groups_h = [g.pin_memory() for g in runner.inputs["groups"]]
+        prob_h = torch.empty(wl.B, dtype=torch.float32).pin_memory()
+        gd = [torch.empty_like(g, device=device) for g in groups_h]
+
+        def step():
+            for src, dst in zip(groups_h, gd):
+                dst.copy_(src, non_blocking=True)
+            st.tokenize(gd, runner.X0)
+            st.forward(runner.X0, runner.pooled)
+            st.head_forward(runner.pooled, runner.prob)
+            prob_h.copy_(runner.prob, non_blocking=True)
+            torch.cuda.current_stream(device).synchronize()
+        h2d = sum(g.numel() * g.element_size() for g in groups_h)
+        d2h = prob_h.numel() * 4
+    else:
+        X0_h = runner.inputs["X0"].pin_memory()
+        pooled_h = torch.empty(wl.B, wl.D, dtype=torch.float32).pin_memory()
+
+        def step():
+            st.forward_host(X0_h, pooled_h)      # copies in, runs, copies out, synchronises
+        h2d = X0_h.numel() * X0_h.element_size()
+        d2h = pooled_h.numel() * 4
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(device)
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        step()
+    torch.cuda.synchronize(device)
+    elapsed = (time.perf_counter() - t0) * 1e3
+    return {"_ms": elapsed, "unit": "samples/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "api": "rm_stack_forward_host" if not wl.group_widths else
+                   "pinned copies + rm_padsplit_tokenize + rm_stack_forward + rm_head_forward"}
+
+
+def run_reference(a, wl, cfg, rank, world):
+    if rank != 0:
+        return
+    from oracle import oracle as O
+    d = synth.make_inputs(wl)
+    blocks_np = oracle_blocks_f32(d)
+    threads = O.num_threads()
+    per_step = min(wl.B, threads)
+    nxt = 0
+
+    def step():
+        nonlocal nxt
+        samples = [(nxt + i) % wl.B for i in range(per_step)]
+        nxt = (nxt + per_step) % wl.B
+        return oracle_sample_run(wl, blocks_np, samples)
+    for _ in range(a.warmup):
+        step()
+    total = sum(step() for _ in range(a.steps))
+    value = per_step * a.steps / total
+    sample = (f"{per_step} samples per step (one per host thread) of the {wl.name} stack, "
+              f"{a.steps} steps, fp64 C loops")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "samples/s", "n_gpus": max(world, 1),
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": total / a.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": cfg,
+            "cpu_baseline": {"value": value, "unit": "samples/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "samples/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

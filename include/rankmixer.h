@@ -1,0 +1,214 @@
+/*
+ * rankmixer.h -- C ABI of librankmixer.so, the B200 (sm_100a) forward pass of
+ * a stack of RankMixer blocks.
+ *
+ * Model (fun-rec chapter "Rankmixer: 硬件效率优化", section RankMixer整体架构):
+ *     S_{n-1} = LN(TokenMixing(X_{n-1}) + X_{n-1})
+ *     X_n     = LN(PFFN(S_{n-1}) + S_{n-1})
+ * for n = 1..L, then mean pooling over the T tokens.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, unless an entry
+ *     point says "host".  They must be 16-byte aligned.
+ *   - Activations are row-major [B, T, D]: token t of sample b starts at
+ *     element (b*T + t)*D.  Element type is the handle's dtype (RM_BF16 =
+ *     bfloat16, RM_F32 = float).  pooled outputs are always float.
+ *   - Weight matrices (handle dtype) are stored per token, output-major (the
+ *     orientation of the product W1 s_t in the Per-Token FFN equation):
+ *       dense  W1 [T][kD][D]      W2 [T][D][kD]      b1 [T][kD]  b2 [T][D]
+ *       MoE    W1 [T][Ne][kD][D]  W2 [T][Ne][D][kD]  b1 [T][Ne][kD]  b2 [T][Ne][D]
+ *              Wr [T][Ne][D]      br [T][Ne]
+ *     Biases, router and LayerNorm parameters are float.  LayerNorm
+ *     parameters are [D], one pair per LN instance, shared by all tokens.
+ *   - Calls are asynchronous on the given stream (NULL = legacy default
+ *     stream) and never synchronise the host, except rm_sync_status and
+ *     rm_stack_forward_host.  Argument errors are returned before anything is
+ *     launched.  Faults detected on the device (a bounded wait that ran out)
+ *     set the handle's device error word, read by rm_sync_status.
+ *   - A handle owns its device workspace (allocated by rm_create); the
+ *     forward calls allocate nothing.  One handle must not be used from two
+ *     streams or threads at the same time.
+ *   - Requirements: D % T == 0 (H = T heads of width D/T), D % 16 == 0 and
+ *     hidden % 16 == 0 for RM_BF16 (D % 4 == 0 for RM_F32), 1 <= B <= B_max,
+ *     1 <= T <= 64, n_experts <= 32.  Violations return RM_ERR_INVALID_ARG or
+ *     RM_ERR_UNSUPPORTED.
+ *   - RM_F32 handles compute on CUDA cores only (no tensor cores).  RM_BF16
+ *     handles run the FFN products on tcgen05 tensor cores with fp32
+ *     accumulation; S, the FFN hidden and the pre-LN rows are stored bf16.
+ */
+#ifndef RANKMIXER_H
+#define RANKMIXER_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *rm_stream_t;
+
+typedef enum {
+    RM_OK = 0,
+    RM_ERR_INVALID_ARG = 1,     /* null/misaligned pointer, bad size            */
+    RM_ERR_UNSUPPORTED = 2,     /* shape or mode this build does not implement  */
+    RM_ERR_CUDA = 3,            /* a CUDA runtime call failed                   */
+    RM_ERR_OOM = 4,             /* workspace allocation failed in rm_create     */
+    RM_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait ran out           */
+    RM_ERR_DEVICE_BOUNDS = 6    /* a device-side bounds check failed            */
+} rm_status;
+
+typedef enum { RM_F32 = 0, RM_BF16 = 1 } rm_dtype;
+
+typedef enum { RM_GELU_TANH = 0, RM_GELU_ERF = 1 } rm_gelu;
+
+typedef struct {
+    int B_max;       /* largest batch any call will pass                         */
+    int T;           /* tokens per sample (= heads H)                            */
+    int D;           /* token width                                              */
+    int hidden;      /* FFN hidden width kD (per expert for MoE)                 */
+    int L;           /* blocks in a stack                                        */
+    int n_experts;   /* 0 = dense per-token FFN; else experts per token (Ne)     */
+    rm_dtype dtype;
+    float ln_eps;    /* LayerNorm epsilon, inside the square root (e.g. 1e-5)    */
+    int gelu;        /* rm_gelu                                                  */
+} rm_config;
+
+typedef struct {
+    const void *W1, *b1, *W2, *b2;             /* see layout above; b1, b2 float */
+    const float *ln1_g, *ln1_b;                /* LN after token mixing [D]      */
+    const float *ln2_g, *ln2_b;                /* LN after the FFN [D]           */
+    const float *Wr, *br;                      /* MoE router (NULL when dense)   */
+} rm_block_weights;
+
+typedef struct rm_handle rm_handle;
+
+/* Create a handle on the current CUDA device and allocate its workspace for
+ * batches up to cfg->B_max.  *out receives the handle (NULL on error).
+ * Returns RM_ERR_OOM if the workspace does not fit. */
+rm_status rm_create(const rm_config *cfg, rm_handle **out);
+
+/* Release the workspace and the handle.  Waits for the handle's work. */
+rm_status rm_destroy(rm_handle *h);
+
+/* Bytes of device workspace the handle owns. */
+size_t rm_workspace_bytes(const rm_handle *h);
+
+/* Token mixing with H = T (section Token Mixing机制 of the fun-rec chapter:
+ * SplitHead, then Concat per head):
+ *     Y[b, h, t*dh + j] = X[b, t, h*dh + j],   dh = D / T.
+ * A pure permutation; X and Y [B, T, D] must not overlap. */
+rm_status rm_token_mix(rm_handle *h, const void *X, void *Y, int B, rm_stream_t stream);
+
+/* Row LayerNorm, out = LN(A + R) over D for rows = B*T rows (R may be NULL).
+ * gamma/beta [D] float.  A, R, out [rows, D] in the handle dtype; out may
+ * alias A. */
+rm_status rm_layernorm(rm_handle *h, const void *A, const void *R, const float *gamma,
+                       const float *beta, void *out, int rows, rm_stream_t stream);
+
+/* Per-token FFN (section Per-Token FFN of the fun-rec chapter):
+ *     V[b, t] = W2_t GELU(W1_t S[b, t] + b1_t) + b2_t
+ * S, V [B, T, D]; uses w->W1, b1, W2, b2.  No residual, no LayerNorm. */
+rm_status rm_pffn_forward(rm_handle *h, const rm_block_weights *w, const void *S, void *V,
+                          int B, rm_stream_t stream);
+
+/* Sparse-MoE per-token FFN with ReLU routing (section Sparse MoE扩展 of the
+ * fun-rec chapter; "特征交叉 —— RankMixer 精读笔记", PFFN paragraph):
+ *     G[b, t, j] = ReLU(Wr_t[j] . S[b, t] + br_t[j])
+ *     V[b, t]    = sum over j with G > 0 of G[b, t, j] * FFN_{t,j}(S[b, t])
+ * Experts whose gate is 0 are not evaluated.  gates (may be NULL) receives G
+ * [B, T, Ne] float.  Needs an MoE handle (n_experts > 0) of dtype RM_BF16. */
+rm_status rm_moe_forward(rm_handle *h, const rm_block_weights *w, const void *S, void *V,
+                         float *gates, int B, rm_stream_t stream);
+
+/* One RankMixer block: Xout = LN2(F(S) + S), S = LN1(TokenMixing(X) + X),
+ * F the dense or MoE per-token FFN.  X, Xout [B, T, D]; may alias. */
+rm_status rm_block_forward(rm_handle *h, const rm_block_weights *w, const void *X, void *Xout,
+                           int B, rm_stream_t stream);
+
+/* The stack: cfg.L blocks (blocks[0..L-1]) from X0, then the mean over the
+ * T tokens of the last block's output (section RankMixer整体架构):
+ *     pooled[b, :] = (1/T) sum_t X_L[b, t, :]          pooled [B, D] float
+ * Xlast (may be NULL) receives X_L [B, T, D].  X0 is not modified. */
+rm_status rm_stack_forward(rm_handle *h, const rm_block_weights *blocks, const void *X0,
+                           float *pooled, void *Xlast, int B, rm_stream_t stream);
+
+/* rm_stack_forward for callers whose X0 and pooled live in HOST memory
+ * (pinned memory gives full copy speed).  Copies X0 into the handle's
+ * workspace, runs the stack, copies pooled back, and synchronises the stream
+ * before returning.  Weights stay device pointers. */
+rm_status rm_stack_forward_host(rm_handle *h, const rm_block_weights *blocks,
+                                const void *X0_host, float *pooled_host, int B,
+                                rm_stream_t stream);
+
+/* Pad-Split tokenisation ("淘宝闪购-爆品团精排 Scaling Up 迭代实践", section
+ * 3.4: concatenate all feature-group embeddings, zero-pad, split into equal
+ * tokens, no projection):
+ *     X0[b, :] = [groups[0][b, :] ; ... ; groups[n-1][b, :] ; 0 ... 0]
+ * groups: HOST array of n_groups DEVICE pointers, groups[i] [B, widths[i]]
+ * in the handle dtype; widths: host array.  sum(widths) <= T*D, every width a
+ * multiple of 8; n_groups <= 32.  X0 [B, T*D]. */
+rm_status rm_padsplit_tokenize(rm_handle *h, const void *const *groups, const int *widths,
+                               int n_groups, void *X0, int B, rm_stream_t stream);
+
+/* Prediction head on the pooled vector: prob[b] = sigmoid(pooled[b] . w + bias).
+ * w [D] in the handle dtype, bias: device pointer to one float, pooled [B, D]
+ * float, prob [B] float. */
+rm_status rm_head_forward(rm_handle *h, const void *w, const float *bias, const float *pooled,
+                          float *prob, int B, rm_stream_t stream);
+
+/* Synchronise the stream, then return and clear the device error word
+ * (RM_OK, RM_ERR_DEVICE_TIMEOUT or RM_ERR_DEVICE_BOUNDS), or RM_ERR_CUDA. */
+rm_status rm_sync_status(rm_handle *h, rm_stream_t stream);
+
+/* Detail of the last device error: the site id of the wait that ran out. */
+int rm_last_error_site(const rm_handle *h);
+
+/* Budget, in nanoseconds, of every bounded device-side wait launched with
+ * this handle from now on (default 1e9, 1 second). */
+rm_status rm_set_wait_budget(rm_handle *h, unsigned long long ns);
+
+/* Diagnostic: launch a kernel whose single wait is on an mbarrier that no one
+ * ever arrives at, so the wait runs out after the handle's wait budget and the
+ * kernel records RM_ERR_DEVICE_TIMEOUT.  Exists to test the timeout path. */
+rm_status rm_selftest_wait_timeout(rm_handle *h, rm_stream_t stream);
+
+/* ---- launch profiling ----------------------------------------------------
+ * Kernel kinds launched by the forward entry points: */
+typedef enum {
+    RM_K_MIX_LN = 0,      /* token mixing + residual + LayerNorm (prev. LN2 on load) */
+    RM_K_GEMM1 = 1,       /* FFN first projection + bias + GELU (grouped GEMM)       */
+    RM_K_GEMM2 = 2,       /* FFN second projection + bias (+ residual / gate)        */
+    RM_K_LN_POOL = 3,     /* last LayerNorm + mean pooling                           */
+    RM_K_LAYERNORM = 4,
+    RM_K_TOKEN_MIX = 5,
+    RM_K_MOE_ROUTE = 6,   /* router + ReLU gates + compaction                        */
+    RM_K_MOE_GATHER = 7,
+    RM_K_MOE_COMBINE = 8,
+    RM_K_PADSPLIT = 9,
+    RM_K_HEAD = 10,
+    RM_K_COUNT = 11
+} rm_kernel_kind;
+
+/* Start recording a CUDA event pair around each kernel launch made through h
+ * (on the launch stream), for up to max_launches launches; later launches
+ * are not recorded.  Restarts any recording in progress. */
+rm_status rm_profile_begin(rm_handle *h, int max_launches);
+
+/* Stop recording, wait for the recorded events, and return per kind the
+ * summed elapsed milliseconds and the number of recorded launches (arrays of
+ * n_kinds entries, indexed by rm_kernel_kind; either may be NULL). */
+rm_status rm_profile_end(rm_handle *h, float *ms_by_kind, int *launches_by_kind, int n_kinds);
+
+/* Name of a kernel kind ("gemm1", ...), or "unknown". */
+const char *rm_kernel_name(int kind);
+
+/* Static description of a status code. */
+const char *rm_status_string(rm_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RANKMIXER_H */

@@ -1,0 +1,114 @@
+"""Whole-stack parity on the five synthetic workloads, through the C ABI.
+
+The small fp32 stack is compared in full.  The bf16 stacks run at their full
+batch in the launch configuration the benchmark times (rm_stack_forward over
+the whole batch); the oracle recomputes a sample of rows one by one (samples
+are independent), and every block output X_l, the last block output and the
+pooled output of those rows are compared.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_common import assert_close, dev, host64, sample_rows
+from token_mixing_feature_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rm():
+    from token_mixing_feature_b200 import rankmixer
+    return rankmixer
+
+
+def _stack(wl, d):
+    from token_mixing_feature_b200.stack import RankMixerStack
+    return RankMixerStack(wl, d["blocks"], d.get("head"))
+
+
+def test_tiny_f32_stack_full(rm, O):
+    wl = synth.WORKLOADS["tiny_f32"]
+    d = synth.make_inputs(wl)
+    st = _stack(wl, d)
+    X0 = dev(d["X0"])
+    Xlast = st.empty_act(wl.B)
+    pooled = st.forward(X0, Xlast=Xlast)
+    xs = [X0]
+    for l in range(wl.L):
+        xs.append(st.block(l, xs[-1]))
+    assert rm.rm_sync_status(st.h) == rm.RM_OK
+    ref = O.stack(d["X0"], d["blocks"], want_all=True)
+    for l in range(wl.L):
+        assert_close(host64(xs[l + 1]), ref["Xall"][l], "f32", f"X_{l + 1}")
+    assert_close(host64(Xlast), ref["Xlast"], "f32", "Xlast")
+    assert_close(host64(pooled), ref["pooled"], "f32", "pooled")
+    st.close()
+
+
+@pytest.mark.parametrize("name,nsamp", [("rm100m", 16), ("rm1b", 8), ("moe", 16)])
+def test_bf16_stack_sampled(rm, O, name, nsamp):
+    wl = synth.WORKLOADS[name]
+    d = synth.make_inputs(wl)
+    st = _stack(wl, d)
+    X0 = dev(d["X0"])
+    Xlast = st.empty_act(wl.B)
+    pooled = st.forward(X0, Xlast=Xlast)
+    xs = [X0]
+    for l in range(wl.L):
+        xs.append(st.block(l, xs[-1]))
+    assert rm.rm_sync_status(st.h) == rm.RM_OK
+    idx = sample_rows(wl.B, nsamp)
+    ref = O.stack(synth.make_x0(wl, samples=idx), d["blocks"], want_all=True)
+    for l in range(wl.L):
+        assert_close(host64(xs[l + 1][idx.to("cuda")]), ref["Xall"][l], "bf16", f"X_{l + 1}")
+    assert_close(host64(Xlast[idx.to("cuda")]), ref["Xlast"], "bf16", "Xlast")
+    assert_close(host64(pooled[idx.to("cuda")]), ref["pooled"], "bf16", "pooled")
+    st.close()
+
+
+def test_padsplit_stack_sampled(rm, O):
+    wl = synth.WORKLOADS["padsplit"]
+    d = synth.make_inputs(wl)
+    st = _stack(wl, d)
+    X0 = st.tokenize([dev(g) for g in d["groups"]])
+    pooled = st.forward(X0)
+    prob = st.head_forward(pooled)
+    assert rm.rm_sync_status(st.h) == rm.RM_OK
+    idx = sample_rows(wl.B, 24)
+    groups = synth.make_groups(wl, samples=idx)
+    X0ref = O.padsplit(groups, wl.padded_width).reshape(len(idx), wl.T, wl.D)
+    np.testing.assert_array_equal(host64(X0[idx.to("cuda")]), X0ref)
+    ref = O.stack(X0ref.astype(np.float32), d["blocks"], want_all=False)
+    assert_close(host64(pooled[idx.to("cuda")]), ref["pooled"], "bf16", "pooled")
+    pref = O.head(ref["pooled"], d["head"]["w"], float(d["head"]["b"][0]))
+    np.testing.assert_allclose(host64(prob[idx.to("cuda")]), pref, rtol=0, atol=2e-3)
+    st.close()
+
+
+def test_host_entry_matches_device_entry(rm):
+    wl = synth.WORKLOADS["rm100m"].with_batch(200)
+    d = synth.make_inputs(wl)
+    st = _stack(wl, d)
+    pooled_dev = st.forward(dev(d["X0"]))
+    X0h = d["X0"].pin_memory()
+    pooled_h = torch.empty(wl.B, wl.D, dtype=torch.float32).pin_memory()
+    st.forward_host(X0h, pooled_h)
+    assert rm.rm_sync_status(st.h) == rm.RM_OK
+    assert torch.equal(pooled_dev.cpu(), pooled_h)
+    st.close()
+
+
+def test_moe_active_rate_is_reported(rm):
+    """The MoE workload's routing statistics: fraction of active experts."""
+    wl = synth.WORKLOADS["moe"].with_batch(512)
+    d = synth.make_inputs(wl)
+    st = _stack(wl, d)
+    S = dev(d["X0"])
+    V = torch.empty_like(S)
+    G = torch.empty(wl.B, wl.T, wl.n_experts, dtype=torch.float32, device="cuda")
+    rm.rm_moe_forward(st.h, st.blocks[0], S, V, G, wl.B)
+    assert rm.rm_sync_status(st.h) == rm.RM_OK
+    rate = (G > 0).float().mean().item()
+    assert 0.0 < rate < 1.0
+    st.close()

@@ -1,0 +1,106 @@
+// Internal interface between the C ABI (rm_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/rankmixer.h"
+
+namespace rm {
+
+// Device error word and site id (both in device memory, owned by a handle).
+struct DeviceErr {
+    int* word;
+    int* site;
+};
+
+// Wait-site ids recorded with RM_ERR_DEVICE_TIMEOUT.
+enum WaitSite : int {
+    SITE_TC_PRODUCER = 1,
+    SITE_TC_MMA_FULL = 2,
+    SITE_TC_MMA_TMEM = 3,
+    SITE_TC_EPILOGUE = 4,
+    SITE_TC_DRAIN = 5,
+    SITE_SELFTEST = 9,
+};
+
+// ---- memory-bound kernels (rm_mem.cu); E = 0 float, 1 bf16 -------------
+cudaError_t launch_token_mix(int dtype, const void* X, void* Y, int B, int T, int D, cudaStream_t s);
+cudaError_t launch_layernorm(int dtype, const void* A, const void* R, const float* g, const float* b,
+                             void* out, long long rows, int D, float eps, cudaStream_t s);
+// S = LN1(TokenMixing(Xh) + Xh), Xh = pre_g ? LN_pre(X) : X (per token row).
+cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const float* pre_b,
+                          const float* g1, const float* b1, void* S, int B, int T, int D, float eps,
+                          cudaStream_t s);
+// Xh = LN(X) per token row; pooled[b] = mean_t Xh[b, t]; Xout optional.
+cudaError_t launch_ln_pool(int dtype, const void* X, const float* g, const float* b, float* pooled,
+                           void* Xout, int B, int T, int D, float eps, cudaStream_t s);
+struct PadSplitArgs {
+    const void* src[32];
+    int col0[33];   // first padded column of each group; col0[n] = sum of widths
+    int n;
+};
+cudaError_t launch_padsplit(int dtype, const PadSplitArgs& a, void* X0, int B, int width,
+                            cudaStream_t s);
+cudaError_t launch_head(int dtype, const float* pooled, const void* w, const float* bias, float* prob,
+                        int B, int D, cudaStream_t s);
+cudaError_t launch_selftest_wait(DeviceErr err, uint64_t budget_ns, cudaStream_t s);
+
+// ---- grouped GEMMs ------------------------------------------------------
+// out[g, m, n] = epi( sum_k A[g, m, k] * W[g, n, k] )  (W stored [G][N][K]).
+enum Epilogue : int {
+    EPI_GELU_TANH = 0,   // bf16( GELU_tanh(acc + bias) )
+    EPI_GELU_ERF = 1,    // bf16( GELU_erf(acc + bias) )
+    EPI_BIAS_RESID = 2,  // bf16( acc + bias [+ resid] )
+    EPI_BIAS_GATE = 3,   // bf16( gate[row] * (acc + bias) )
+};
+
+struct GroupedGemm {
+    int G, M, N, K;
+    // A operand: element (g, m, k) at A + g*a_gstride + m*a_ld + k (elements).
+    const void* A;
+    long long a_gstride, a_ld;
+    long long a_rows_total;   // variable-row mode: rows allocated in A (and out)
+    // W operand [G][N][K] contiguous.
+    const void* W;
+    // out element (g, m, n) at out + g*o_gstride + m*o_ld + n.
+    void* out;
+    long long o_gstride, o_ld;
+    const float* bias;        // [G][N]
+    const void* resid;        // EPI_BIAS_RESID (may be null): same indexing as out, strides below
+    long long r_gstride, r_ld;
+    const float* gate;        // EPI_BIAS_GATE: [rows] in variable-row mode
+    int epi;
+    // Variable-row mode (sparse MoE): group g owns rows [grp_off[g], grp_off[g] + grp_cnt[g])
+    // of A and out (g strides unused); mtile_prefix[g] = sum_{g' < g} ceil(cnt / 128).
+    const int* grp_cnt;
+    const int* grp_off;
+    const int* mtile_prefix;  // [G + 1]
+};
+
+cudaError_t launch_gemm_tc(const GroupedGemm& p, DeviceErr err, uint64_t budget_ns, int num_sms,
+                           cudaStream_t s);
+cudaError_t launch_gemm_simt(const GroupedGemm& p, cudaStream_t s);   // fp32, CUDA cores
+
+// ---- sparse MoE routing (rm_moe.cu) ----------------------------------------
+struct MoeWork {
+    float* gates;          // [B, T, Ne]
+    int* counts;           // [T*Ne]
+    int* offsets;          // [T*Ne]
+    int* mtile_prefix;     // [T*Ne + 1]
+    int* totals;           // [2]: active entries, m-tiles
+    int* slot_row;         // [B*T*Ne]: slot -> row b*T + t of S
+    float* slot_gate;      // [B*T*Ne]
+    int* slot_of;          // [B, T, Ne]: slot or -1
+    void* Sg;              // [B*T*Ne, D] bf16 gathered rows
+    void* Hg;              // [B*T*Ne, hidden] bf16
+    void* Eg;              // [B*T*Ne, D] bf16 gate-scaled expert outputs
+};
+cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, const MoeWork& w, int B,
+                             int T, int D, int Ne, cudaStream_t s);
+cudaError_t launch_moe_gather(const void* S, const MoeWork& w, int B, int T, int D, int Ne,
+                              cudaStream_t s);
+cudaError_t launch_moe_combine(const MoeWork& w, const void* resid, void* out, int B, int T, int D,
+                               int Ne, cudaStream_t s);
+
+}  // namespace rm

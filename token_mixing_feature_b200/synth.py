@@ -4,11 +4,12 @@ This module only draws random numbers and rounds them to the storage dtype.
 It holds none of the model's arithmetic, so both the CUDA path and the CPU
 oracle can take their inputs from it without sharing any computation.
 
-Every tensor is drawn from its own ``torch.Generator`` (CPU, Philox-free
-default mt19937) seeded with ``seed * 1_000_003 + index``, where ``index`` is
-fixed per tensor.  A tensor's values therefore do not depend on the batch size
-or on which other tensors were drawn, so a sub-batch of samples can be
-regenerated exactly for sampled parity checks.
+Every row along a tensor's first axis is drawn from its own CPU
+``torch.Generator`` (mt19937) seeded with a fixed function of (seed, tensor
+index, row).  A tensor's values therefore do not depend on the batch size, on
+which other tensors were drawn, or on how many threads drew them, and the
+rows of any subset of samples can be regenerated exactly for sampled parity
+checks.
 
 bf16 workloads draw in fp32 and round to bf16 (round-to-nearest-even) before
 anyone uses the values; the oracle consumes those rounded values widened to
@@ -24,11 +25,15 @@ Weight layout (per token t, "out-major", the orientation of the product
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
 import dataclasses
 import math
-from typing import Dict, List, Optional
+import os
+from typing import Dict, List, Optional, Sequence
 
 import torch
+
+_THREADS = os.cpu_count() or 1
 
 
 @dataclasses.dataclass(frozen=True)
@@ -81,19 +86,34 @@ WORKLOADS: Dict[str, Workload] = {
 }
 
 
-def _gen(seed: int, index: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
-    g.manual_seed(seed * 1_000_003 + index)
-    return g
+def _row_seed(seed: int, index: int, row: int) -> int:
+    return ((seed * 1_000_003 + index) * 1_000_000_007 + row) % (1 << 63)
 
 
-def _normal(shape, std: float, mean: float, seed: int, index: int) -> torch.Tensor:
-    t = torch.randn(*shape, generator=_gen(seed, index), dtype=torch.float32)
-    if std != 1.0:
-        t.mul_(std)
-    if mean != 0.0:
-        t.add_(mean)
-    return t
+def _normal(shape, std: float, mean: float, seed: int, index: int,
+            rows: Optional[Sequence[int]] = None) -> torch.Tensor:
+    """N(mean, std^2) fp32 tensor; row i of the first axis from its own stream.
+    With ``rows`` given, only those rows are drawn (in that order)."""
+    if len(shape) == 1:     # a vector is one row
+        return _normal((1,) + tuple(shape), std, mean, seed, index)[0]
+    rows = list(range(shape[0])) if rows is None else [int(r) for r in rows]
+    out = torch.empty((len(rows),) + tuple(shape[1:]), dtype=torch.float32)
+
+    def fill(lo: int, hi: int) -> None:
+        g = torch.Generator(device="cpu")
+        for k in range(lo, hi):
+            g.manual_seed(_row_seed(seed, index, rows[k]))
+            out[k].normal_(mean=mean, std=std, generator=g)
+
+    n = len(rows)
+    workers = max(1, min(_THREADS, n, (out.numel() >> 20) + 1))
+    if workers == 1:
+        fill(0, n)
+    else:
+        step = (n + workers - 1) // workers
+        with cf.ThreadPoolExecutor(workers) as ex:
+            list(ex.map(lambda lo: fill(lo, min(n, lo + step)), range(0, n, step)))
+    return out
 
 
 def _store(t: torch.Tensor, dtype: str) -> torch.Tensor:
@@ -112,9 +132,7 @@ _IDX_GROUP0 = 1
 
 def make_x0(wl: Workload, seed: int = 0, samples: Optional[torch.Tensor] = None) -> torch.Tensor:
     """X0 [B, T, D] in the workload's storage dtype (no Pad-Split)."""
-    x = _normal((wl.B, wl.T, wl.D), wl.x0_std, 0.0, seed, _IDX_X0)
-    if samples is not None:
-        x = x[samples].contiguous()
+    x = _normal((wl.B, wl.T, wl.D), wl.x0_std, 0.0, seed, _IDX_X0, rows=samples)
     return _store(x, wl.dtype)
 
 
@@ -122,9 +140,7 @@ def make_groups(wl: Workload, seed: int = 0, samples: Optional[torch.Tensor] = N
     """Pad-Split feature-group embeddings, one [B, w_i] tensor per group."""
     out = []
     for i, w in enumerate(wl.group_widths):
-        g = _normal((wl.B, w), wl.group_std, 0.0, seed, _IDX_GROUP0 + i)
-        if samples is not None:
-            g = g[samples].contiguous()
+        g = _normal((wl.B, w), wl.group_std, 0.0, seed, _IDX_GROUP0 + i, rows=samples)
         out.append(_store(g, wl.dtype))
     return out
 
