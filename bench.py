@@ -245,6 +245,8 @@ def main():
     ap.add_argument("--workload", default="rm1b", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernels-only", action="store_true",
+                    help="only the warm-up and the K timed steps (for profiler launch lists)")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -300,6 +302,15 @@ def main():
     ms = time_steps(runner.step, a.steps, stream)
     barrier()
     ms = max_over_ranks(ms)
+    if a.kernels_only:
+        if sampler:
+            sampler.stop()
+        if rank == 0:
+            print(json.dumps({"kernels_only": True, "workload": wl.name, "ms_per_step": ms / a.steps}))
+        runner.st.close()
+        if pg:
+            pg.destroy_process_group()
+        return
 
     # per-kernel times over a second timed region of K steps (events on the launch stream)
     rm.rm_profile_begin(runner.st.h, a.steps * runner.launches_per_step() + 8)

@@ -5,7 +5,9 @@ import torch
 # Tolerances.  bf16 storage with fp32 accumulation: every block output X_l and
 # the pooled output within 1e-2 relative L2 AND 5e-2 max-abs of the fp64
 # oracle; fp32 storage on CUDA cores: 1e-5 relative L2.  Token mixing,
-# Pad-Split and router masks: bit-exact.
+# Pad-Split and router masks: bit-exact.  Outputs that no LayerNorm scales
+# (the FFN / MoE output V alone) are not O(1): for those ("raw") the max-abs
+# bound applies to the error divided by max(1, max |reference|).
 BF16_REL_L2 = 1e-2
 BF16_MAX_ABS = 5e-2
 F32_REL_L2 = 1e-5
@@ -27,7 +29,7 @@ def max_abs(got: np.ndarray, ref: np.ndarray) -> float:
     return float(np.abs(got - ref).max()) if got.size else 0.0
 
 
-def assert_close(got, ref, dtype: str, what: str = "") -> None:
+def assert_close(got, ref, dtype: str, what: str = "", raw: bool = False) -> None:
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (got.shape, ref.shape)
@@ -37,6 +39,8 @@ def assert_close(got, ref, dtype: str, what: str = "") -> None:
         assert r <= F32_REL_L2, f"{what}: rel L2 {r:.3e} > {F32_REL_L2}"
     else:
         m = max_abs(got, ref)
+        if raw:
+            m /= max(1.0, float(np.abs(ref).max()))
         assert r <= BF16_REL_L2 and m <= BF16_MAX_ABS, f"{what}: rel L2 {r:.3e}, max abs {m:.3e}"
 
 

@@ -70,7 +70,7 @@ def test_pffn_bf16_tensor_cores(rm, O, T, D, hidden, B):
         rm.rm_pffn_forward(h, {k: dev(v) for k, v in blk.items()}, dev(S), V, B)
         assert rm.rm_sync_status(h) == rm.RM_OK
     ref = O.pffn(S, blk["W1"], blk["b1"], blk["W2"], blk["b2"])
-    assert_close(host64(V), ref, "bf16", "pffn")
+    assert_close(host64(V), ref, "bf16", "pffn", raw=True)
 
 
 @pytest.mark.parametrize("T,D,hidden,B", [(8, 64, 256, 64), (3, 24, 40, 5), (1, 128, 64, 70)])
@@ -94,7 +94,7 @@ def test_pffn_gelu_erf(rm, O):
         rm.rm_pffn_forward(h, {k: dev(v) for k, v in blk.items()}, dev(S), V, B)
         assert rm.rm_sync_status(h) == rm.RM_OK
     ref = O.pffn(S, blk["W1"], blk["b1"], blk["W2"], blk["b2"], gelu="erf")
-    assert_close(host64(V), ref, "bf16", "pffn erf")
+    assert_close(host64(V), ref, "bf16", "pffn erf", raw=True)
 
 
 # --------------------------------------------------------------------- block
@@ -156,7 +156,7 @@ def test_moe_router_masks_and_output(rm, O, B, T, D, hidden, Ne):
     decided = np.abs(logits) >= 1e-3      # the kernel decides in fp32, the oracle in fp64
     np.testing.assert_array_equal((g > 0)[decided], (logits > 0)[decided])
     np.testing.assert_allclose(g, np.maximum(logits, 0), rtol=0, atol=1e-4)
-    assert_close(host64(V), Vref, "bf16", "moe")
+    assert_close(host64(V), Vref, "bf16", "moe", raw=True)
 
 
 def test_moe_all_gates_closed(rm, O):
@@ -179,7 +179,7 @@ def test_moe_single_open_expert_is_pffn(rm, O):
         rm.rm_moe_forward(h, {k: dev(v) for k, v in blk.items()}, dev(S), V, None, B)
         assert rm.rm_sync_status(h) == rm.RM_OK
     ref = O.pffn(S, blk["W1"][:, 0], blk["b1"][:, 0], blk["W2"][:, 0], blk["b2"][:, 0])
-    assert_close(host64(V), ref, "bf16", "moe single expert")
+    assert_close(host64(V), ref, "bf16", "moe single expert", raw=True)
 
 
 def test_moe_block(rm, O):
