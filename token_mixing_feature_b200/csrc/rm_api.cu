@@ -23,7 +23,6 @@
 
 namespace rm {
 int gemm_tc_pick_bn(int G, int M, int N, bool var_rows, int num_sms);
-int mix_ln_max_d(int dtype);
 }  // namespace rm
 
 struct rm_handle {
@@ -234,7 +233,8 @@ rm_status run_stack(rm_handle* h, const rm_block_weights* blocks, const void* X0
         {
             ProfScope ps(h, RM_K_MIX_LN, s);
             e = rm::launch_mix_ln(c.dtype, l ? h->Y : X0, prev ? prev->ln2_g : nullptr,
-                                  prev ? prev->ln2_b : nullptr, w->ln1_g, w->ln1_b, h->S, B, c.T, c.D, c.ln_eps, s);
+                                  prev ? prev->ln2_b : nullptr, w->ln1_g, w->ln1_b, h->S, B, c.T, c.D, c.ln_eps,
+                                  h->num_sms, derr(h), h->budget_ns, s);
         }
         if (e != cudaSuccess) return RM_ERR_CUDA;
         rm_status st = run_ffn(h, w, h->S, h->Y, h->S, B, s);
@@ -243,7 +243,7 @@ rm_status run_stack(rm_handle* h, const rm_block_weights* blocks, const void* X0
     const rm_block_weights* last = &blocks[c.L - 1];
     ProfScope ps(h, RM_K_LN_POOL, s);
     return cuda_status(rm::launch_ln_pool(c.dtype, h->Y, last->ln2_g, last->ln2_b, pooled, Xlast, B, c.T, c.D,
-                                          c.ln_eps, s));
+                                          c.ln_eps, h->num_sms, derr(h), h->budget_ns, s));
 }
 
 template <typename T>
@@ -406,7 +406,8 @@ rm_status rm_block_forward(rm_handle* h, const rm_block_weights* w, const void* 
     cudaError_t e;
     {
         ProfScope ps(h, RM_K_MIX_LN, stream);
-        e = rm::launch_mix_ln(c.dtype, X, nullptr, nullptr, w->ln1_g, w->ln1_b, h->S, B, c.T, c.D, c.ln_eps, stream);
+        e = rm::launch_mix_ln(c.dtype, X, nullptr, nullptr, w->ln1_g, w->ln1_b, h->S, B, c.T, c.D, c.ln_eps,
+                              h->num_sms, derr(h), h->budget_ns, stream);
     }
     if (e != cudaSuccess) return RM_ERR_CUDA;
     if ((st = run_ffn(h, w, h->S, h->Y, h->S, B, stream)) != RM_OK) return st;

@@ -21,6 +21,8 @@ enum WaitSite : int {
     SITE_TC_MMA_TMEM = 3,
     SITE_TC_EPILOGUE = 4,
     SITE_TC_DRAIN = 5,
+    SITE_MIX_LN = 6,
+    SITE_LN_POOL = 7,
     SITE_SELFTEST = 9,
 };
 
@@ -28,13 +30,16 @@ enum WaitSite : int {
 cudaError_t launch_token_mix(int dtype, const void* X, void* Y, int B, int T, int D, cudaStream_t s);
 cudaError_t launch_layernorm(int dtype, const void* A, const void* R, const float* g, const float* b,
                              void* out, long long rows, int D, float eps, cudaStream_t s);
+// ---- rm_mix.cu ------------------------------------------------------------
 // S = LN1(TokenMixing(Xh) + Xh), Xh = pre_g ? LN_pre(X) : X (per token row).
 cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const float* pre_b,
                           const float* g1, const float* b1, void* S, int B, int T, int D, float eps,
-                          cudaStream_t s);
+                          int num_sms, DeviceErr err, uint64_t budget_ns, cudaStream_t s);
 // Xh = LN(X) per token row; pooled[b] = mean_t Xh[b, t]; Xout optional.
 cudaError_t launch_ln_pool(int dtype, const void* X, const float* g, const float* b, float* pooled,
-                           void* Xout, int B, int T, int D, float eps, cudaStream_t s);
+                           void* Xout, int B, int T, int D, float eps, int num_sms, DeviceErr err,
+                           uint64_t budget_ns, cudaStream_t s);
+int mix_ln_max_d(int dtype);
 struct PadSplitArgs {
     const void* src[32];
     int col0[33];   // first padded column of each group; col0[n] = sum of widths

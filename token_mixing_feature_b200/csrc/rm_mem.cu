@@ -1,14 +1,11 @@
-// Memory-bound kernels of the RankMixer stack: token mixing, LayerNorm, the
-// fused mix + residual + LayerNorm pass, the final LayerNorm + mean pooling,
-// Pad-Split tokenisation and the sigmoid head.
+// Memory-bound kernels of the RankMixer stack: standalone token mixing and
+// row LayerNorm (the unfused variants behind rm_token_mix / rm_layernorm),
+// Pad-Split tokenisation, the sigmoid head, and the wait self-test.
 //
 // Token mixing with H = T (fun-rec chapter "Rankmixer: 硬件效率优化", section
 // Token Mixing机制: SplitHead into H chunks of D/H, then Concat chunk h of
 // every token) maps output element (b, h, t*dh + j) to input element
-// (b, t, h*dh + j), dh = D/T.  It is a permutation within one sample, so the
-// kernels below stage one whole sample [T, D] in shared memory (read once,
-// coalesced) and apply the permutation through shared-memory addressing; no
-// transpose pass ever touches HBM.
+// (b, t, h*dh + j), dh = D/T.
 #include <cuda_bf16.h>
 
 #include "rm_device.cuh"
@@ -99,155 +96,6 @@ __global__ void __launch_bounds__(kThreads) layernorm_kernel(const E* A, const E
     }
 }
 
-// Load sample b ([T, D] contiguous) into shared memory with 16-byte vectors.
-template <typename E>
-__device__ __forceinline__ void load_sample(const E* X, E* xs, long long b, int TD) {
-    const uint4* src = reinterpret_cast<const uint4*>(X + b * TD);
-    uint4* dst = reinterpret_cast<uint4*>(xs);
-    const int n = TD * (int)sizeof(E) / 16;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = __ldg(src + i);
-}
-
-// Mean and reciprocal std of every token row of the staged sample.
-template <typename E>
-__device__ __forceinline__ void row_stats(const E* xs, int T, int D, float eps, float* mean_s, float* rstd_s) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    for (int t = warp; t < T; t += nw) {
-        const E* r = xs + t * D;
-        float s = 0.f;
-        for (int c = lane; c < D; c += 32) s += to_f(r[c]);
-        const float mu = warp_sum(s) / D;
-        float q = 0.f;
-        for (int c = lane; c < D; c += 32) {
-            const float d = to_f(r[c]) - mu;
-            q += d * d;
-        }
-        q = warp_sum(q);
-        if (lane == 0) {
-            mean_s[t] = mu;
-            rstd_s[t] = rsqrtf(q / D + eps);
-        }
-    }
-}
-
-// ---------------------------------------------------------- fused mix + LN
-// One CTA per sample.  Xh = PRE ? LN_pre(X) : X per token row (the previous
-// block's second LayerNorm, applied on load), then
-//   Z[h, c] = Xh[t, h*dh + j] + Xh[h, c],  c = t*dh + j
-//   S[h, :] = LN1(Z[h, :])
-// One warp per output row h; each lane keeps its NV vectors of Z in registers.
-template <typename E, bool PRE, bool CONTIG, int NV>
-__global__ void __launch_bounds__(kThreads) mix_ln_kernel(const E* __restrict__ X, const float* __restrict__ pre_g,
-                                                          const float* __restrict__ pre_b,
-                                                          const float* __restrict__ g1,
-                                                          const float* __restrict__ b1, E* __restrict__ S,
-                                                          int T, int D, float eps) {
-    constexpr int V = Vec16<E>::N;
-    extern __shared__ __align__(16) unsigned char smem[];
-    E* xs = reinterpret_cast<E*>(smem);
-    float* mean_s = reinterpret_cast<float*>(smem + (size_t)T * D * sizeof(E));
-    float* rstd_s = mean_s + T;
-    const long long b = blockIdx.x;
-    const int TD = T * D;
-    load_sample(X, xs, b, TD);
-    __syncthreads();
-    if (PRE) {
-        row_stats(xs, T, D, eps, mean_s, rstd_s);
-        __syncthreads();
-    }
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const int dh = D / T;
-    const int nv = D / V;
-    E* srow_base = S + b * TD;
-    for (int h = warp; h < T; h += nw) {
-        float z[NV][V];
-        float s = 0.f;
-        const float mh = PRE ? mean_s[h] : 0.f, rh = PRE ? rstd_s[h] : 1.f;
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            const int v = lane + 32 * i;
-            if (v < nv) {
-                const int c0 = v * V;
-                int t = c0 / dh, j = c0 - t * dh;
-#pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    if (!CONTIG && e > 0) {
-                        if (++j == dh) { j = 0; ++t; }
-                    }
-                    const int jj = CONTIG ? j + e : j;
-                    const int k = h * dh + jj;          // column of the source token
-                    const int c = c0 + e;
-                    float xm = to_f(xs[t * D + k]);
-                    float xr = to_f(xs[h * D + c]);
-                    if (PRE) {
-                        xm = (xm - mean_s[t]) * rstd_s[t] * __ldg(pre_g + k) + __ldg(pre_b + k);
-                        xr = (xr - mh) * rh * __ldg(pre_g + c) + __ldg(pre_b + c);
-                    }
-                    z[i][e] = xm + xr;
-                    s += z[i][e];
-                }
-            }
-        }
-        const float mu = warp_sum(s) / D;
-        float q = 0.f;
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            if (lane + 32 * i < nv) {
-#pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    const float d = z[i][e] - mu;
-                    q += d * d;
-                }
-            }
-        }
-        const float rstd = rsqrtf(warp_sum(q) / D + eps);
-        uint4* out4 = reinterpret_cast<uint4*>(srow_base + (long long)h * D);
-#pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            const int v = lane + 32 * i;
-            if (v < nv) {
-                Vec16<E> o;
-#pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    const int c = v * V + e;
-                    o.e[e] = from_f<E>(__ldg(g1 + c) * ((z[i][e] - mu) * rstd) + __ldg(b1 + c));
-                }
-                out4[v] = o.u;
-            }
-        }
-    }
-}
-
-// ------------------------------------------------------- final LN + pooling
-// One CTA per sample: Xh = LN(X) per token row; pooled[b, d] = (1/T) sum_t
-// Xh[t, d] summed in ascending t; Xout (optional) receives Xh.
-template <typename E>
-__global__ void __launch_bounds__(kThreads) ln_pool_kernel(const E* __restrict__ X, const float* __restrict__ g,
-                                                           const float* __restrict__ bta, float* __restrict__ pooled,
-                                                           E* __restrict__ Xout, int T, int D, float eps) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    E* xs = reinterpret_cast<E*>(smem);
-    float* mean_s = reinterpret_cast<float*>(smem + (size_t)T * D * sizeof(E));
-    float* rstd_s = mean_s + T;
-    const long long b = blockIdx.x;
-    const int TD = T * D;
-    load_sample(X, xs, b, TD);
-    __syncthreads();
-    row_stats(xs, T, D, eps, mean_s, rstd_s);
-    __syncthreads();
-    const float invT = 1.0f / T;
-    for (int d = threadIdx.x; d < D; d += blockDim.x) {
-        const float gd = __ldg(g + d), bd = __ldg(bta + d);
-        float acc = 0.f;
-        for (int t = 0; t < T; ++t) {
-            const float xh = gd * ((to_f(xs[t * D + d]) - mean_s[t]) * rstd_s[t]) + bd;
-            acc += xh;
-            if (Xout) Xout[b * TD + (long long)t * D + d] = from_f<E>(xh);
-        }
-        pooled[b * D + d] = acc * invT;
-    }
-}
-
 // ------------------------------------------------------------------ Pad-Split
 template <typename E>
 __global__ void __launch_bounds__(kThreads) padsplit_kernel(PadSplitArgs a, E* __restrict__ X0, long long B,
@@ -298,50 +146,7 @@ __global__ void selftest_wait_kernel(DeviceErr err, uint64_t budget_ns) {
     mbar_wait(smem_u32(&bar), 0, w, SITE_SELFTEST);
 }
 
-template <typename E, bool PRE, bool CONTIG>
-cudaError_t mix_ln_dispatch_nv(int nvl, const E* X, const float* pg, const float* pb, const float* g1,
-                               const float* b1, E* S, int B, int T, int D, float eps, size_t smem,
-                               cudaStream_t s) {
-#define RM_MIXLN_CASE(NVV)                                                                           \
-    if (nvl <= NVV) {                                                                                \
-        auto k = mix_ln_kernel<E, PRE, CONTIG, NVV>;                                                 \
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-        if (e != cudaSuccess) return e;                                                              \
-        k<<<B, kThreads, smem, s>>>(X, pg, pb, g1, b1, S, T, D, eps);                                \
-        return cudaGetLastError();                                                                   \
-    }
-    RM_MIXLN_CASE(1)
-    RM_MIXLN_CASE(2)
-    RM_MIXLN_CASE(4)
-    RM_MIXLN_CASE(8)
-    RM_MIXLN_CASE(16)
-#undef RM_MIXLN_CASE
-    return cudaErrorInvalidValue;
-}
-
-template <typename E>
-cudaError_t mix_ln_typed(const void* X, const float* pg, const float* pb, const float* g1, const float* b1,
-                         void* S, int B, int T, int D, float eps, cudaStream_t s) {
-    constexpr int V = Vec16<E>::N;
-    const int dh = D / T;
-    const int nv = D / V;
-    const int nvl = (nv + 31) / 32;
-    const size_t smem = (size_t)T * D * sizeof(E) + 2 * sizeof(float) * T;
-    const bool contig = (dh % V) == 0;
-    const E* x = static_cast<const E*>(X);
-    E* y = static_cast<E*>(S);
-    if (pg) {
-        return contig ? mix_ln_dispatch_nv<E, true, true>(nvl, x, pg, pb, g1, b1, y, B, T, D, eps, smem, s)
-                      : mix_ln_dispatch_nv<E, true, false>(nvl, x, pg, pb, g1, b1, y, B, T, D, eps, smem, s);
-    }
-    return contig ? mix_ln_dispatch_nv<E, false, true>(nvl, x, pg, pb, g1, b1, y, B, T, D, eps, smem, s)
-                  : mix_ln_dispatch_nv<E, false, false>(nvl, x, pg, pb, g1, b1, y, B, T, D, eps, smem, s);
-}
-
 }  // namespace
-
-// Largest D per dtype the register-cached mix kernel supports (16 vectors per lane).
-int mix_ln_max_d(int dtype) { return 32 * 16 * (dtype == RM_BF16 ? 8 : 4); }
 
 cudaError_t launch_token_mix(int dtype, const void* X, void* Y, int B, int T, int D, cudaStream_t s) {
     const int dh = D / T;
@@ -375,31 +180,6 @@ cudaError_t launch_layernorm(int dtype, const void* A, const void* R, const floa
     } else {
         layernorm_kernel<float><<<grid, kThreads, 0, s>>>((const float*)A, (const float*)R, g, b, (float*)out,
                                                            rows, D, eps);
-    }
-    return cudaGetLastError();
-}
-
-cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const float* pre_b, const float* g1,
-                          const float* b1, void* S, int B, int T, int D, float eps, cudaStream_t s) {
-    if (dtype == RM_BF16) return mix_ln_typed<__nv_bfloat16>(X, pre_g, pre_b, g1, b1, S, B, T, D, eps, s);
-    return mix_ln_typed<float>(X, pre_g, pre_b, g1, b1, S, B, T, D, eps, s);
-}
-
-cudaError_t launch_ln_pool(int dtype, const void* X, const float* g, const float* b, float* pooled, void* Xout,
-                           int B, int T, int D, float eps, cudaStream_t s) {
-    const size_t esz = dtype == RM_BF16 ? 2 : 4;
-    const size_t smem = (size_t)T * D * esz + 2 * sizeof(float) * T;
-    if (dtype == RM_BF16) {
-        using E = __nv_bfloat16;
-        auto k = ln_pool_kernel<E>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        k<<<B, kThreads, smem, s>>>((const E*)X, g, b, pooled, (E*)Xout, T, D, eps);
-    } else {
-        auto k = ln_pool_kernel<float>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        k<<<B, kThreads, smem, s>>>((const float*)X, g, b, pooled, (float*)Xout, T, D, eps);
     }
     return cudaGetLastError();
 }
