@@ -174,6 +174,32 @@ rm_status rm_set_wait_budget(rm_handle *h, unsigned long long ns);
  * kernel records RM_ERR_DEVICE_TIMEOUT.  Exists to test the timeout path. */
 rm_status rm_selftest_wait_timeout(rm_handle *h, rm_stream_t stream);
 
+/* ---- per-token FFN without device allocation ----------------------------
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory (code running where cudaMalloc is off
+ * limits, e.g. inside another runtime's memory pool or with all device memory
+ * reserved up front), so they cannot create a handle.
+ *
+ * Computes the same V = PFFN(S) as rm_pffn_forward (same kernels, same
+ * layouts; dtype and gelu as in rm_config), with no handle.  Its only scratch,
+ * the FFN hidden activations [T, B, hidden], lives in a fixed device array of
+ * RM_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits; the caller passes inputs and outputs
+ * only, and the call allocates nothing.
+ *   - Returns RM_ERR_INVALID_ARG, before launching anything, if
+ *     T * B * hidden * sizeof(element) > RM_STATIC_SCRATCH_BYTES - 256.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call uses the same array: calls that overlap on the GPU (other
+ *     streams, other host threads on the same device) race on it.
+ *   - device_status (device pointer to one int, may be NULL) receives, in
+ *     stream order, RM_OK or RM_ERR_DEVICE_TIMEOUT for this call. */
+#define RM_STATIC_SCRATCH_BYTES (16u << 20)
+rm_status rm_pffn_forward_static(const rm_block_weights *w, const void *S, void *V, int B, int T,
+                                 int D, int hidden, rm_dtype dtype, int gelu, int *device_status,
+                                 rm_stream_t stream);
+
 /* ---- launch profiling ----------------------------------------------------
  * Kernel kinds launched by the forward entry points: */
 typedef enum {

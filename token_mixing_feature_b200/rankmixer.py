@@ -25,8 +25,9 @@ EXPORTED = (
     "rm_pffn_forward", "rm_moe_forward", "rm_block_forward", "rm_stack_forward",
     "rm_stack_forward_host", "rm_padsplit_tokenize", "rm_head_forward", "rm_sync_status",
     "rm_last_error_site", "rm_set_wait_budget", "rm_selftest_wait_timeout", "rm_status_string",
-    "rm_profile_begin", "rm_profile_end", "rm_kernel_name",
+    "rm_profile_begin", "rm_profile_end", "rm_kernel_name", "rm_pffn_forward_static",
 )
+RM_STATIC_SCRATCH_BYTES = 16 << 20
 RM_K_COUNT = 11
 
 
@@ -73,6 +74,8 @@ def _load() -> ctypes.CDLL:
         "rm_profile_begin": (st, [vp, ci]),
         "rm_profile_end": (st, [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ci), ci]),
         "rm_kernel_name": (ctypes.c_char_p, [ci]),
+        "rm_pffn_forward_static": (st, [ctypes.POINTER(rm_block_weights), vp, vp, ci, ci, ci, ci, ci, ci,
+                                        vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -254,3 +257,14 @@ def rm_profile_end(h: Handle) -> Dict[str, tuple]:
 
 def rm_kernel_name(kind: int) -> str:
     return _lib.rm_kernel_name(kind).decode()
+
+
+def rm_pffn_forward_static(w: Dict, S, V, B: int, T: int, D: int, hidden: int, dtype: str = "bf16",
+                           gelu: str = "tanh", device_status=None, stream=None) -> None:
+    """V = PFFN(S) with no handle and no device allocation: the hidden
+    activations use a fixed array inside the library (RM_STATIC_SCRATCH_BYTES),
+    shared by all calls; overlapping calls race on it."""
+    bw = block_weights(w)
+    _check(_lib.rm_pffn_forward_static(ctypes.byref(bw), _ptr(S), _ptr(V), B, T, D, hidden, DTYPES[dtype],
+                                       GELUS[gelu], _ptr(device_status), _stream(stream)),
+           "rm_pffn_forward_static")
