@@ -22,7 +22,7 @@
 #include "rm_internal.h"
 
 namespace rm {
-int gemm_tc_pick_bn(int G, int M, int N, bool var_rows, int num_sms);
+int gemm_tc_pick_bn(int G, int M, int N, bool var_rows, int num_sms, int cg);
 }  // namespace rm
 
 struct rm_handle {

@@ -24,6 +24,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "rm_device.cuh"
@@ -41,6 +43,7 @@ struct KParams {
     int G, M, N, K;
     int var_rows;
     int a_g_inner;            // A map coordinate order (k, g, m) if 1, else (k, m, g)
+    int o_g_inner;            // out / resid map coordinate order (n, g, m) if 1, else (n, m, g)
     __nv_bfloat16* out;
     long long o_gstride, o_ld;
     const float* bias;
@@ -54,43 +57,57 @@ struct KParams {
     unsigned long long budget_ns;
 };
 
-template <int BN>
+// Tile shapes.  CG = 1: one CTA computes a 128 x BN tile.  CG = 2: a CTA pair
+// (cluster of 2) computes a 256 x BN tile with 2-SM MMAs; each CTA loads its
+// 128 rows of A and BN/2 rows of B and holds its 128 accumulator rows.
+template <int BN, int CG, bool VAR>
 struct Cfg {
+    static constexpr int BN_LOCAL = BN / CG;   // W rows this CTA loads per tile
+    static constexpr int TM = BM * CG;         // output rows per tile
     static constexpr int A_BYTES = BM * BK * 2;
-    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int B_BYTES = BN_LOCAL * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES_RAW = (216 * 1024) / STAGE_BYTES;
+    // Dense tiles leave the epilogue through a 32 x 64 bf16 staging buffer per
+    // epilogue warp (TMA stores); variable-row tiles store rows directly.
+    static constexpr int STAGING_BYTES = VAR ? 0 : kEpiWarps * 4096;
+    static constexpr int STAGES_RAW = (216 * 1024 - STAGING_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static constexpr int TMEM_COLS = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
-    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+    static constexpr int NBARS = 2 * STAGES + 5 + kEpiWarps;
+    static constexpr int BAR_BYTES = 8 * NBARS + 16;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES;
+    static_assert(BN % 128 == 0 || VAR, "dense tiles leave in 64-column chunks per half");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
     static_assert(B_BYTES % 1024 == 0, "stage alignment");
+    static_assert(CG == 1 || CG == 2, "CTA group");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
 struct Tile {
     int g;        // weight group
     int ag;       // A map group coordinate
-    int arow;     // A map row coordinate of the tile's first row
-    int rows;     // valid rows in this tile (<= BM)
-    int n0;
-    long long orow0;  // out / resid row index of the first row (group-local in dense mode)
+    int arow;     // A map row coordinate of this CTA's first row
+    int rows;     // valid rows of this CTA's 128 (may be <= 0)
+    int n0;       // first output column of the tile
+    long long orow0;  // out / resid row index of this CTA's first row (group-local in dense mode)
 };
 
-__device__ __forceinline__ Tile decode_tile(const KParams& p, long long idx, int nblk, int mblk) {
+template <int CG>
+__device__ __forceinline__ Tile decode_tile(const KParams& p, long long idx, int nblk, int mblk, int bn,
+                                            int rank) {
     Tile t;
     if (!p.var_rows) {
         const long long per_g = (long long)nblk * mblk;
         t.g = (int)(idx / per_g);
         const int r = (int)(idx - (long long)t.g * per_g);
         const int nb = r / mblk, mb = r - nb * mblk;
-        const int m0 = mb * BM;
+        const int m0 = mb * (BM * CG) + rank * BM;
         t.ag = t.g;
         t.arow = m0;
         t.rows = min(BM, p.M - m0);
-        t.n0 = nb;
+        t.n0 = nb * bn;
         t.orow0 = m0;
-    } else {
+    } else {   // CG == 1 only
         int lo = 0, hi = p.G;
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
@@ -106,7 +123,7 @@ __device__ __forceinline__ Tile decode_tile(const KParams& p, long long idx, int
         t.ag = 0;
         t.arow = off + m0;
         t.rows = min(BM, __ldg(p.grp_cnt + lo) - m0);
-        t.n0 = nb;
+        t.n0 = nb * bn;
         t.orow0 = off + m0;
     }
     return t;
@@ -120,25 +137,30 @@ __device__ __forceinline__ float gelu_tanh_approx(float x) {
     return 0.5f * x * (1.0f + th);
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int CG, bool VAR>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
                    const KParams p) {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, CG, VAR>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     unsigned char* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(smem);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    const uint32_t staging0 = sbase + C::STAGES * C::STAGE_BYTES;   // 1024-aligned
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::STAGING_BYTES);
     const uint32_t full0 = smem_u32(bars);
     const uint32_t empty0 = full0 + 8 * C::STAGES;
     const uint32_t tfull0 = empty0 + 8 * C::STAGES;
     const uint32_t tempty0 = tfull0 + 16;
     const uint32_t drain_bar = tempty0 + 16;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+    const uint32_t rbar0 = drain_bar + 8;      // one per epilogue warp: residual tile loads
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(full0 + 8 * s, 1);
@@ -146,29 +168,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull0 + 8 * a, 1);
-            mbar_init(tempty0 + 8 * a, kEpiWarps * 32);
+            mbar_init(tempty0 + 8 * a, CG * kEpiWarps * 32);
         }
         mbar_init(drain_bar, 1);
+        for (int w = 0; w < kEpiWarps; ++w) mbar_init(rbar0 + 8 * w, 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        if (!VAR) prefetch_tmap(&tmO);
     }
     if (warp == 0) {
-        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
-        tmem_relinquish();
+        if (CG == 2) {
+            tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync_all();   // the peer's barriers exist before anyone signals them
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
     const WaitCtx wc{abort_flag, p.budget_ns, p.err};
     const int nblk = (p.N + BN - 1) / BN;
-    const int mblk = (p.M + BM - 1) / BM;
+    const int mblk = (p.M + C::TM - 1) / C::TM;
     const int num_kb = (p.K + BK - 1) / BK;
     const long long total = p.var_rows ? (long long)__ldg(p.mtile_prefix + p.G) * nblk
                                        : (long long)p.G * nblk * mblk;
+    const long long unit = blockIdx.x / CG, nunits = gridDim.x / CG;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -176,40 +207,50 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0, issued = 0, issued_phase = 0;
             bool ok = true;
-            for (long long idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-                const Tile t = decode_tile(p, idx, nblk, mblk);
-                const int n0 = t.n0 * BN;
+            for (long long idx = unit; idx < total && ok; idx += nunits) {
+                const Tile t = decode_tile<CG>(p, idx, nblk, mblk, BN, (int)rank);
+                const int nb0 = t.n0 + (int)rank * C::BN_LOCAL;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, wc, SITE_TC_PRODUCER)) {
                         ok = false;
                         break;
                     }
                     const uint32_t fb = full0 + 8 * stage;
-                    mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+                    if (leader) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
                     const uint32_t sa = sbase + stage * C::STAGE_BYTES;
                     const int kc = kb * BK;
-                    if (p.a_g_inner) tma_load_3d(sa, &tmA, fb, kc, t.ag, t.arow);
-                    else tma_load_3d(sa, &tmA, fb, kc, t.arow, t.ag);
-                    tma_load_3d(sa + C::A_BYTES, &tmB, fb, kc, n0, t.g);
+                    if (CG == 2) {
+                        const uint32_t fbl = mapa_shared(fb, 0);   // the pair counts bytes on the even CTA
+                        if (p.a_g_inner) tma_load_3d_pair(sa, &tmA, fbl, kc, t.ag, t.arow);
+                        else tma_load_3d_pair(sa, &tmA, fbl, kc, t.arow, t.ag);
+                        tma_load_3d_pair(sa + C::A_BYTES, &tmB, fbl, kc, nb0, t.g);
+                    } else {
+                        if (p.a_g_inner) tma_load_3d(sa, &tmA, fb, kc, t.ag, t.arow);
+                        else tma_load_3d(sa, &tmA, fb, kc, t.arow, t.ag);
+                        tma_load_3d(sa + C::A_BYTES, &tmB, fb, kc, nb0, t.g);
+                    }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            // Every issued copy must land before the CTA's shared memory goes away.
-            for (int s = 0; s < C::STAGES; ++s)
-                if (issued & (1u << s)) mbar_wait(full0 + 8 * s, (issued_phase >> s) & 1u, wc, SITE_TC_DRAIN, false);
+            // Every issued copy must land before the CTA's shared memory goes
+            // away (for a pair, the even CTA's barrier counts both CTAs' bytes).
+            if (leader)
+                for (int s = 0; s < C::STAGES; ++s)
+                    if (issued & (1u << s))
+                        mbar_wait(full0 + 8 * s, (issued_phase >> s) & 1u, wc, SITE_TC_DRAIN, false);
         }
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+            constexpr uint32_t idesc = idesc_bf16_f32(C::TM, BN);
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true, any = false;
             int it = 0;
-            for (long long idx = blockIdx.x; idx < total && ok; idx += gridDim.x, ++it) {
+            for (long long idx = unit; idx < total && ok; idx += nunits, ++it) {
                 const int acc = it & 1;
                 const uint32_t aph = (uint32_t)(it >> 1) & 1u;
                 if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, wc, SITE_TC_MMA_TMEM)) break;
@@ -227,33 +268,160 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         // advance the start address by k * 32 bytes (16-byte units)
-                        tc_mma_f16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
-                                   (kb | k) != 0 ? 1u : 0u);
+                        if (CG == 2)
+                            tc_mma_f16_pair(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
+                                            (kb | k) != 0 ? 1u : 0u);
+                        else
+                            tc_mma_f16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
+                                       (kb | k) != 0 ? 1u : 0u);
                     }
-                    tc_commit(empty0 + 8 * stage);
+                    if (CG == 2) tc_commit_pair_mc(empty0 + 8 * stage, 0x3);
+                    else tc_commit(empty0 + 8 * stage);
                     any = true;
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                tc_commit(tfull0 + 8 * acc);
+                if (CG == 2) tc_commit_pair_mc(tfull0 + 8 * acc, 0x3);
+                else tc_commit(tfull0 + 8 * acc);
             }
             // Every issued MMA must complete before tensor memory is released.
             if (any) {
-                tc_commit(drain_bar);
+                if (CG == 2) tc_commit_pair(drain_bar);
+                else tc_commit(drain_bar);
                 mbar_wait(drain_bar, 0, wc, SITE_TC_DRAIN, false);
             }
         }
         __syncwarp();
+    } else if constexpr (!VAR) {
+        // ------------------------------------- epilogue, dense: TMA stores
+        // Each warp owns 32 accumulator rows (its TMEM lane quarter) and half
+        // of the BN columns, in 64-column chunks: tcgen05.ld -> registers ->
+        // bias / GELU / residual -> bf16 into a 128-byte-swizzled 32 x 64
+        // staging buffer -> one TMA bulk store.  The residual tile arrives in
+        // the same buffer by TMA first.  The accumulator is released right
+        // after the tile's last tcgen05.ld.
+        const int ew = warp - 2;
+        const int quarter = warp & 3;
+        const int half = ew >> 2;
+        constexpr int HALF = BN / 2;
+        const uint32_t tempty_leader = CG == 2 ? mapa_shared(tempty0, 0) : tempty0;
+        const uint32_t stg = staging0 + (uint32_t)ew * 4096u;
+        const uint32_t rbar = rbar0 + 8u * (uint32_t)ew;
+        uint32_t rphase = 0;
+        const bool has_resid = EPI == EPI_BIAS_RESID && p.resid != nullptr;
+        const uint32_t my_row = stg + (uint32_t)lane * 128u;
+        const uint32_t swz = (uint32_t)(lane & 7);
+        int it = 0;
+        for (long long idx = unit; idx < total; idx += nunits, ++it) {
+            const Tile t = decode_tile<CG>(p, idx, nblk, mblk, BN, (int)rank);
+            const int acc = it & 1;
+            const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+            if (!mbar_wait(tfull0 + 8 * acc, aph, wc, SITE_TC_EPILOGUE)) break;
+            tc_fence_after();
+            const int wrow0 = (int)t.orow0 + quarter * 32;
+            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+            const float* bias_g = p.bias + (long long)t.g * p.N;
+            bool ok = true;
+#pragma unroll 1
+            for (int c = half * HALF; c < (half + 1) * HALF; c += 64) {
+                const int n = t.n0 + c;
+                const bool live = n < p.N;   // warp-uniform
+                if (lane == 0) bulk_wait_read_all();   // the previous store has read the buffer
+                __syncwarp();
+                if (has_resid && live && lane == 0) {
+                    mbar_arrive_expect_tx(rbar, 4096);
+                    if (p.o_g_inner) tma_load_3d(stg, &tmR, rbar, n, t.g, wrow0);
+                    else tma_load_3d(stg, &tmR, rbar, n, wrow0, t.g);
+                }
+                float v[64];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float w16[16];
+                    tmem_ld16(tbase + (uint32_t)(c + 16 * q), w16);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[16 * q + e] = w16[e];
+                }
+                tmem_ld_wait();
+                if (c + 64 >= (half + 1) * HALF) {   // last chunk: the accumulator may be reused
+                    tc_fence_before();
+                    if (CG == 2 && !leader) mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
+                    else mbar_arrive(tempty0 + 8 * acc);
+                }
+                if (!live) continue;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (n + 16 * q < p.N) {
+                        const float4* b4 = reinterpret_cast<const float4*>(bias_g + n + 16 * q);
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const float4 bb = __ldg(b4 + r);
+                            v[16 * q + 4 * r + 0] += bb.x;
+                            v[16 * q + 4 * r + 1] += bb.y;
+                            v[16 * q + 4 * r + 2] += bb.z;
+                            v[16 * q + 4 * r + 3] += bb.w;
+                        }
+                    }
+                }
+                if (EPI == EPI_GELU_TANH) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) v[e] = gelu_tanh_approx(v[e]);
+                } else if (EPI == EPI_GELU_ERF) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) v[e] = 0.5f * v[e] * (1.0f + erff(v[e] * 0.7071067811865476f));
+                } else if (EPI == EPI_BIAS_RESID) {
+                    if (has_resid) {
+                        if (!mbar_wait(rbar, rphase, wc, SITE_TC_EPILOGUE)) {
+                            ok = false;
+                            break;
+                        }
+                        rphase ^= 1u;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            uint4 u;
+                            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
+                                         : "r"(my_row + ((((uint32_t)j) ^ swz) << 4)));
+                            Vec16<__nv_bfloat16> r;
+                            r.u = u;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) v[8 * j + e] += __bfloat162float(r.e[e]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t a0 = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+                    const uint32_t a1 = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+                    const uint32_t a2 = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+                    const uint32_t a3 = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(my_row + ((((uint32_t)j) ^ swz) << 4)),
+                                 "r"(a0), "r"(a1), "r"(a2), "r"(a3)
+                                 : "memory");
+                }
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    if (p.o_g_inner) tma_store_3d(&tmO, stg, n, t.g, wrow0);
+                    else tma_store_3d(&tmO, stg, n, wrow0, t.g);
+                    bulk_commit_group();
+                }
+            }
+            if (!ok) break;
+        }
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
     } else {
-        // ---------------------------------------------------- epilogue
+        // ------------------------------ epilogue, variable rows: row stores
         const int ew = warp - 2;
         const int quarter = warp & 3;          // TMEM lanes this warp may access
         const int half = ew >> 2;              // which half of the BN columns
         const int row = quarter * 32 + lane;
         constexpr int HALF = BN / 2;
+        // the pair's accumulator-free barrier lives on the even CTA
+        const uint32_t tempty_leader = CG == 2 ? mapa_shared(tempty0, 0) : tempty0;
         int it = 0;
-        for (long long idx = blockIdx.x; idx < total; idx += gridDim.x, ++it) {
-            const Tile t = decode_tile(p, idx, nblk, mblk);
+        for (long long idx = unit; idx < total; idx += nunits, ++it) {
+            const Tile t = decode_tile<CG>(p, idx, nblk, mblk, BN, (int)rank);
             const int acc = it & 1;
             const uint32_t aph = (uint32_t)(it >> 1) & 1u;
             if (!mbar_wait(tfull0 + 8 * acc, aph, wc, SITE_TC_EPILOGUE)) break;
@@ -270,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float v[16];
                 tmem_ld16(tbase + (uint32_t)c, v);
                 tmem_ld_wait();
-                const int n = t.n0 * BN + c;
+                const int n = t.n0 + c;
                 if (row_ok && n < p.N) {
                     const float4* b4 = reinterpret_cast<const float4*>(bias_g + n);
 #pragma unroll
@@ -318,15 +486,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(tempty0 + 8 * acc);
+            if (CG == 2 && !leader) mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
+            else mbar_arrive(tempty0 + 8 * acc);
         }
     }
 
     tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync_all();   // the pair's MMAs and copies are done before either CTA leaves
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
+        if (CG == 2) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+        else tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 }
 
@@ -364,49 +535,71 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, int EPI>
-cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap& mb, const KParams& kp, int grid,
-                         cudaStream_t s) {
-    auto k = gemm_tc_kernel<BN, EPI>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::SMEM_BYTES);
+struct Maps {
+    CUtensorMap a, b, o, r;
+};
+
+template <int BN, int EPI, int CG, bool VAR>
+cudaError_t launch_typed(const Maps& m, const KParams& kp, int grid, cudaStream_t s) {
+    using C = Cfg<BN, CG, VAR>;
+    auto k = gemm_tc_kernel<BN, EPI, CG, VAR>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    k<<<grid, kThreads, Cfg<BN>::SMEM_BYTES, s>>>(ma, mb, kp);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, m.a, m.b, m.o, m.r, kp);
 }
 
-template <int BN>
-cudaError_t launch_bn(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const KParams& kp, int grid,
-                      cudaStream_t s) {
+template <int BN, int CG, bool VAR>
+cudaError_t launch_bn(int epi, const Maps& m, const KParams& kp, int grid, cudaStream_t s) {
     switch (epi) {
-        case EPI_GELU_TANH: return launch_typed<BN, EPI_GELU_TANH>(ma, mb, kp, grid, s);
-        case EPI_GELU_ERF: return launch_typed<BN, EPI_GELU_ERF>(ma, mb, kp, grid, s);
-        case EPI_BIAS_RESID: return launch_typed<BN, EPI_BIAS_RESID>(ma, mb, kp, grid, s);
-        case EPI_BIAS_GATE: return launch_typed<BN, EPI_BIAS_GATE>(ma, mb, kp, grid, s);
+        case EPI_GELU_TANH: return launch_typed<BN, EPI_GELU_TANH, CG, VAR>(m, kp, grid, s);
+        case EPI_GELU_ERF: return launch_typed<BN, EPI_GELU_ERF, CG, VAR>(m, kp, grid, s);
+        case EPI_BIAS_RESID:
+            if constexpr (!VAR) return launch_typed<BN, EPI_BIAS_RESID, CG, VAR>(m, kp, grid, s);
+            break;
+        case EPI_BIAS_GATE:
+            if constexpr (VAR) return launch_typed<BN, EPI_BIAS_GATE, CG, VAR>(m, kp, grid, s);
+            break;
     }
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-// Tile width for N: the candidate with the best product of column fill, wave
-// fill over the SMs, and a per-width tensor-core efficiency (wider tiles read
-// less shared memory per MMA).
-int gemm_tc_pick_bn(int G, int M, int N, bool var_rows, int num_sms) {
+// Tile width for N: the candidate with the best product of column fill, a
+// per-width tensor-core efficiency measured on B200 with 2-SM tiles at
+// K = 1536..6144 (BN 256 : 192 : 128 = 1 : 0.88 : 0.74), and a damped wave
+// fill over the SMs (a partial last wave costs less than its share, since the
+// tiles of that wave see less L2 contention).
+int gemm_tc_pick_bn(int G, int M, int N, bool var_rows, int num_sms, int cg) {
     const int cands[4] = {256, 192, 160, 128};
-    const double mma_eff[4] = {1.0, 0.95, 0.92, 0.86};
+    const double mma_eff[4] = {1.0, 0.88, 0.8, 0.74};
     int best = 256;
     double best_s = -1.0;
     for (int i = 0; i < 4; ++i) {
         const int bn = cands[i];
+        if (!var_rows && bn % 128) continue;   // dense tiles leave in 64-column chunks per half
         const long long nblk = (N + bn - 1) / bn;
         const double col_fill = (double)N / (double)(nblk * bn);
         double wave_fill = 1.0;
         if (!var_rows) {
-            const long long tiles = (long long)G * ((M + BM - 1) / BM) * nblk;
-            const long long waves = (tiles + num_sms - 1) / num_sms;
-            wave_fill = (double)tiles / (double)(waves * num_sms);
+            const long long units = num_sms / cg;
+            const long long tiles = (long long)G * ((M + BM * cg - 1) / (BM * cg)) * nblk;
+            const long long waves = (tiles + units - 1) / units;
+            wave_fill = (double)tiles / (double)(waves * units);
         }
-        const double sc = col_fill * wave_fill * mma_eff[i];
+        const double sc = col_fill * mma_eff[i] * (0.5 + 0.5 * wave_fill);
         if (sc > best_s + 1e-9) {
             best_s = sc;
             best = bn;
@@ -438,37 +631,71 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     kp.err = err;
     kp.budget_ns = budget_ns;
 
-    const int bn = gemm_tc_pick_bn(g.G, g.M, g.N, var, num_sms);
-    CUtensorMap ma, mb;
+    // 2-SM (256-row) tiles for dense problems with more than one 128-row block;
+    // the variable-row (MoE) groups keep 128-row tiles.
+    int cg = (!var && g.M > BM) ? 2 : 1;
+    int bn = gemm_tc_pick_bn(g.G, g.M, g.N, var, num_sms, cg);
+    // Tuning overrides (same kernel, other tile shape): RM_GEMM_CG=1|2, RM_GEMM_BN=256|192|160|128.
+    if (const char* e = getenv("RM_GEMM_CG")) {
+        const int v = atoi(e);
+        if ((v == 1 || (v == 2 && !var)) ) cg = v;
+    }
+    if (const char* e = getenv("RM_GEMM_BN")) {
+        const int v = atoi(e);
+        if (v == 256 || v == 128 || (var && (v == 192 || v == 160))) bn = v;
+    }
+    Maps m;
+    memset(&m, 0, sizeof(m));
     bool ok;
     if (var) {
         // compacted rows [rows_total, K]
-        ok = make_map(&ma, g.A, g.K, g.a_rows_total, 1, g.a_ld * 2, g.a_rows_total * g.a_ld * 2, BM, 1);
+        ok = make_map(&m.a, g.A, g.K, g.a_rows_total, 1, g.a_ld * 2, g.a_rows_total * g.a_ld * 2, BM, 1);
         kp.a_g_inner = 0;
     } else if (g.a_gstride <= g.a_ld) {
         // group stride inside the row stride, e.g. S [B, T, D]: dims (K, G, M)
-        ok = make_map(&ma, g.A, g.K, g.G, g.M, g.a_gstride * 2, g.a_ld * 2, 1, BM);
+        ok = make_map(&m.a, g.A, g.K, g.G, g.M, g.a_gstride * 2, g.a_ld * 2, 1, BM);
         kp.a_g_inner = 1;
     } else {
         // groups outermost, e.g. H [T, B, kD]: dims (K, M, G)
-        ok = make_map(&ma, g.A, g.K, g.M, g.G, g.a_ld * 2, g.a_gstride * 2, BM, 1);
+        ok = make_map(&m.a, g.A, g.K, g.M, g.G, g.a_ld * 2, g.a_gstride * 2, BM, 1);
         kp.a_g_inner = 0;
     }
-    ok = ok && make_map(&mb, g.W, g.K, g.N, g.G, (uint64_t)g.K * 2, (uint64_t)g.N * g.K * 2, (uint32_t)bn, 1);
+    ok = ok && make_map(&m.b, g.W, g.K, g.N, g.G, (uint64_t)g.K * 2, (uint64_t)g.N * g.K * 2, (uint32_t)(bn / cg), 1);
+    if (!var) {
+        // output (and residual) tiles of 32 rows x 64 columns, same orientation as A
+        if (g.o_gstride <= g.o_ld) {
+            ok = ok && make_map(&m.o, g.out, g.N, g.G, g.M, g.o_gstride * 2, g.o_ld * 2, 1, 32);
+            kp.o_g_inner = 1;
+        } else {
+            ok = ok && make_map(&m.o, g.out, g.N, g.M, g.G, g.o_ld * 2, g.o_gstride * 2, 32, 1);
+            kp.o_g_inner = 0;
+        }
+        if (g.resid) {
+            if ((g.r_gstride <= g.r_ld) != (kp.o_g_inner == 1)) return cudaErrorInvalidValue;
+            ok = ok && (kp.o_g_inner ? make_map(&m.r, g.resid, g.N, g.G, g.M, g.r_gstride * 2, g.r_ld * 2, 1, 32)
+                                     : make_map(&m.r, g.resid, g.N, g.M, g.G, g.r_ld * 2, g.r_gstride * 2, 32, 1));
+        }
+    }
     if (!ok) return cudaErrorInvalidValue;
 
-    int grid = num_sms;
+    int units = num_sms / cg;
     if (!var) {
-        const long long tiles = (long long)g.G * ((g.M + BM - 1) / BM) * ((g.N + bn - 1) / bn);
+        const long long tiles = (long long)g.G * ((g.M + BM * cg - 1) / (BM * cg)) * ((g.N + bn - 1) / bn);
         if (tiles == 0) return cudaSuccess;
-        if (tiles < grid) grid = (int)tiles;
+        if (tiles < units) units = (int)tiles;
     }
-    switch (bn) {
-        case 256: return launch_bn<256>(g.epi, ma, mb, kp, grid, s);
-        case 192: return launch_bn<192>(g.epi, ma, mb, kp, grid, s);
-        case 160: return launch_bn<160>(g.epi, ma, mb, kp, grid, s);
-        default: return launch_bn<128>(g.epi, ma, mb, kp, grid, s);
+    const int grid = units * cg;
+    if (var) {
+        switch (bn) {
+            case 256: return launch_bn<256, 1, true>(g.epi, m, kp, grid, s);
+            case 192: return launch_bn<192, 1, true>(g.epi, m, kp, grid, s);
+            case 160: return launch_bn<160, 1, true>(g.epi, m, kp, grid, s);
+            default: return launch_bn<128, 1, true>(g.epi, m, kp, grid, s);
+        }
     }
+    if (cg == 2) return bn == 256 ? launch_bn<256, 2, false>(g.epi, m, kp, grid, s)
+                                  : launch_bn<128, 2, false>(g.epi, m, kp, grid, s);
+    return bn == 256 ? launch_bn<256, 1, false>(g.epi, m, kp, grid, s) : launch_bn<128, 1, false>(g.epi, m, kp, grid, s);
 }
 
 }  // namespace rm
