@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from token_mixing_feature_b200 import roofline, synth  # noqa: E402
+from token_mixing_feature_b200 import replicas, roofline, synth  # noqa: E402
 
 METRIC = "RankMixer stack fwd samples/s and TFLOP/s as % of bf16 roofline on 1×B200"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
@@ -291,11 +291,7 @@ def main():
         torch.cuda.synchronize(device)
 
     def max_over_ranks(x: float) -> float:
-        if not pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(x, device)
 
     # headline: K steps, device time, max over ranks
     barrier()

@@ -24,7 +24,7 @@ _SRC = _HERE / "rankmixer_oracle.c"
 _LIB_PATH = _HERE / "_build" / "liboracle.so"
 _lib = None
 
-GELU_MODES = {"tanh": 0, "erf": 1}
+GELU_MODES = {"tanh": 0, "erf": 1, "relu": 2}   # FFN activation: GELU forms or ReLU
 MAX_EXPERTS = 64
 
 
@@ -153,8 +153,10 @@ def _dims(blk: Dict, T: int, D: int):
     return int(W1.shape[2]), int(W1.shape[1])
 
 
-def block(X, blk: Dict, eps: float = 1e-5, gelu: str = "tanh", want_logits: bool = False):
-    """X' = LN2(PFFN(S) + S), S = LN1(TokenMixing(X) + X)."""
+def block(X, blk: Dict, eps: float = 1e-5, gelu: str = "tanh", want_logits: bool = False,
+          mix_addnorm: bool = True):
+    """X' = LN2(PFFN(S) + S), S = LN1(TokenMixing(X) + X) (or S = TokenMixing(X)
+    without the Add & Norm when mix_addnorm is False)."""
     X = _np(X, np.float64)
     B, T, D = X.shape
     Hd, Ne = _dims(blk, T, D)
@@ -163,13 +165,13 @@ def block(X, blk: Dict, eps: float = 1e-5, gelu: str = "tanh", want_logits: bool
     logits = np.empty((B, T, max(Ne, 1)), dtype=np.float64) if (Ne and want_logits) else None
     _load().orc_block(ctypes.c_long(B), ctypes.c_int(T), ctypes.c_int(D), ctypes.c_int(Hd),
                       ctypes.c_int(Ne), _p(X), ctypes.byref(prm), ctypes.c_double(eps),
-                      ctypes.c_int(GELU_MODES[gelu]), _p(Y), _p(logits))
+                      ctypes.c_int(GELU_MODES[gelu]), ctypes.c_int(1 if mix_addnorm else 0), _p(Y), _p(logits))
     del keep
     return (Y, logits) if want_logits else Y
 
 
 def stack(X0, blocks: Sequence[Dict], eps: float = 1e-5, gelu: str = "tanh",
-          want_all: bool = False, want_last: bool = True) -> Dict[str, np.ndarray]:
+          want_all: bool = False, want_last: bool = True, mix_addnorm: bool = True) -> Dict[str, np.ndarray]:
     """L blocks then mean pooling over tokens.  Returns pooled [B, D], and
     optionally Xlast [B, T, D] and Xall [L, B, T, D]."""
     X0 = _np(X0, np.float32)
@@ -186,7 +188,8 @@ def stack(X0, blocks: Sequence[Dict], eps: float = 1e-5, gelu: str = "tanh",
     Xall = np.empty((L, B, T, D), dtype=np.float64) if want_all else None
     _load().orc_stack(ctypes.c_long(B), ctypes.c_int(T), ctypes.c_int(D), ctypes.c_int(Hd),
                       ctypes.c_int(Ne), ctypes.c_int(L), _p(X0), arr, ctypes.c_double(eps),
-                      ctypes.c_int(GELU_MODES[gelu]), _p(pooled), _p(Xlast), _p(Xall))
+                      ctypes.c_int(GELU_MODES[gelu]), ctypes.c_int(1 if mix_addnorm else 0), _p(pooled), _p(Xlast),
+                      _p(Xall))
     del keep
     out = {"pooled": pooled}
     if want_last:

@@ -27,7 +27,12 @@
  *     eps inside the square root, one (gamma, beta) pair of length D per LN
  *     instance shared by all tokens.
  *   - GELU is the tanh form 0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3)))
- *     of Hendrycks & Gimpel (mode 0); mode 1 is the exact erf form.
+ *     of Hendrycks & Gimpel (mode 0); mode 1 is the exact erf form; mode 2
+ *     is ReLU, the activation of the Mixer backbone timed in Appendix B of
+ *     "重新理解 RankMixer：扩参为什么有效，又为什么划算？".
+ *   - Variant without the Add & Norm after token mixing (mix_addnorm = 0):
+ *     S = TokenMixing(X), the configuration "淘宝闪购-爆品团精排 Scaling Up
+ *     迭代实践" reports in section 3.5 (RankMixer 层数).
  *   - Weights are stored out-major, W1_t [kD][D], W2_t [D][kD], router
  *     Wr_t [Ne][D], so u = W1_t s_t is a row-by-vector product as written in
  *     the PFFN equation.
@@ -95,6 +100,7 @@ static void ln_row(int D, const double *z, const float *g, const float *b, doubl
 }
 
 double orc_gelu(double u, int mode) {
+    if (mode == 2) return u > 0.0 ? u : 0.0;
     if (mode == 1) return 0.5 * u * (1.0 + erf(u / sqrt(2.0)));
     const double c = sqrt(2.0 / M_PI);
     return 0.5 * u * (1.0 + tanh(c * (u + 0.044715 * u * u * u)));
@@ -146,17 +152,21 @@ static void moe_vec(int t, int D, int Hd, int Ne, const double *s, const orc_blo
 
 /* One RankMixer block on one sample: x, y are [T][D]. */
 static void block_sample(int T, int D, int Hd, int Ne, const double *x, const orc_block_params *p,
-                         double eps, int gelu, double *y, double *logits_out, double *work) {
+                         double eps, int gelu, int mix_addnorm, double *y, double *logits_out, double *work) {
     double *z = work;                       /* [T][D] */
     double *s = z + (size_t)T * D;          /* [T][D] */
     double *v = s + (size_t)T * D;          /* [D]    */
     double *e = v + D;                      /* [D]    */
     double *hb = e + D;                     /* [Hd]   */
     double lg[64];
-    /* S = LN(TokenMixing(X) + X) */
+    /* S = LN(TokenMixing(X) + X), or S = TokenMixing(X) without the Add & Norm */
     mix_sample(T, D, x, z);
-    for (size_t i = 0; i < (size_t)T * D; ++i) z[i] += x[i];
-    for (int t = 0; t < T; ++t) ln_row(D, z + (size_t)t * D, p->ln1_g, p->ln1_b, eps, s + (size_t)t * D);
+    if (mix_addnorm) {
+        for (size_t i = 0; i < (size_t)T * D; ++i) z[i] += x[i];
+        for (int t = 0; t < T; ++t) ln_row(D, z + (size_t)t * D, p->ln1_g, p->ln1_b, eps, s + (size_t)t * D);
+    } else {
+        for (size_t i = 0; i < (size_t)T * D; ++i) s[i] = z[i];
+    }
     /* X' = LN(PFFN(S) + S) */
     for (int t = 0; t < T; ++t) {
         const double *st = s + (size_t)t * D;
@@ -235,13 +245,13 @@ void orc_moe(long B, int T, int D, int Hd, int Ne, const double *S, const orc_bl
 
 /* One block over B samples. logits [B][T][Ne] (MoE only, may be NULL). */
 void orc_block(long B, int T, int D, int Hd, int Ne, const double *X, const orc_block_params *p,
-               double eps, int gelu, double *Y, double *logits) {
+               double eps, int gelu, int mix_addnorm, double *Y, double *logits) {
     #pragma omp parallel
     {
         double *work = (double *)malloc(sizeof(double) * block_work_doubles(T, D, Hd));
         #pragma omp for schedule(dynamic)
         for (long b = 0; b < B; ++b)
-            block_sample(T, D, Hd, Ne, X + (size_t)b * T * D, p, eps, gelu, Y + (size_t)b * T * D,
+            block_sample(T, D, Hd, Ne, X + (size_t)b * T * D, p, eps, gelu, mix_addnorm, Y + (size_t)b * T * D,
                          logits ? logits + (size_t)b * T * Ne : NULL, work);
         free(work);
     }
@@ -251,7 +261,7 @@ void orc_block(long B, int T, int D, int Hd, int Ne, const double *X, const orc_
  * Xall (may be NULL): [L][B][T][D], every block's output.
  * Xlast (may be NULL): [B][T][D], the last block's output. */
 void orc_stack(long B, int T, int D, int Hd, int Ne, int L, const float *X0,
-               const orc_block_params *blocks, double eps, int gelu,
+               const orc_block_params *blocks, double eps, int gelu, int mix_addnorm,
                double *pooled, double *Xlast, double *Xall) {
     #pragma omp parallel
     {
@@ -263,7 +273,7 @@ void orc_stack(long B, int T, int D, int Hd, int Ne, int L, const float *X0,
         for (long b = 0; b < B; ++b) {
             for (size_t i = 0; i < td; ++i) xa[i] = (double)X0[(size_t)b * td + i];
             for (int l = 0; l < L; ++l) {
-                block_sample(T, D, Hd, Ne, xa, &blocks[l], eps, gelu, xb, NULL, work);
+                block_sample(T, D, Hd, Ne, xa, &blocks[l], eps, gelu, mix_addnorm, xb, NULL, work);
                 if (Xall) memcpy(Xall + ((size_t)l * B + b) * td, xb, sizeof(double) * td);
                 double *tmp = xa; xa = xb; xb = tmp;
             }

@@ -267,3 +267,32 @@ def test_head_sigmoid(O):
     w = synth.random_activations((32,), seed=62)
     ref = torch.sigmoid(P @ w.double() + 0.25)
     np.testing.assert_allclose(O.head(P, w, 0.25), ref.numpy(), rtol=0, atol=1e-15)
+
+
+# ------------------------------------------------ variants on the pages
+def test_relu_activation_matches_library(O):
+    """ReLU per-token FFN (the Appendix B Mixer's activation)."""
+    B, T, D, Hd = 4, 4, 16, 32
+    blk = synth.random_like_block(T, D, Hd, seed=71)
+    S = synth.random_activations((B, T, D), seed=72).double()
+    W1, b1, W2, b2 = (blk[k].double() for k in ("W1", "b1", "W2", "b2"))
+    ref = torch.einsum("bth,tdh->btd", torch.relu(torch.einsum("btd,thd->bth", S, W1) + b1), W2) + b2
+    np.testing.assert_allclose(O.pffn(S, blk["W1"], blk["b1"], blk["W2"], blk["b2"], gelu="relu"),
+                               ref.numpy(), rtol=0, atol=1e-12)
+    u = np.linspace(-3, 3, 13)
+    np.testing.assert_array_equal(O.gelu(u, "relu"), np.maximum(u, 0))
+
+
+def test_block_without_mix_addnorm(O):
+    """S = TokenMixing(X) (no residual, no LayerNorm after the mix)."""
+    B, T, dh, Hd = 5, 4, 6, 40
+    D = T * dh
+    blk = synth.random_like_block(T, D, Hd, seed=73)
+    X = synth.random_activations((B, T, D), seed=74).double()
+    S = X.view(B, T, T, dh).transpose(1, 2).reshape(B, T, D)
+    W1, b1, W2, b2 = (blk[k].double() for k in ("W1", "b1", "W2", "b2"))
+    V = torch.einsum("bth,tdh->btd", F.gelu(torch.einsum("btd,thd->bth", S, W1) + b1, approximate="tanh"), W2) + b2
+    ref = F.layer_norm(V + S, (D,), blk["ln2_g"].double(), blk["ln2_b"].double(), eps=EPS)
+    np.testing.assert_allclose(O.block(X, blk, EPS, mix_addnorm=False), ref.numpy(), rtol=0, atol=1e-12)
+    # the variant differs from the equation on the pages
+    assert np.abs(O.block(X, blk, EPS) - ref.numpy()).max() > 1e-3
