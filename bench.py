@@ -213,7 +213,7 @@ def oracle_sample_run(wl, blocks_np, samples, seed=0):
     else:
         X0 = synth.make_x0(wl, seed, samples=idx).float().numpy()
     t0 = time.perf_counter()
-    r = O.stack(X0, blocks_np, want_last=False)
+    r = O.stack(X0, blocks_np, want_last=False, gelu=wl.act, mix_addnorm=wl.mix_addnorm)
     if wl.head:
         d = synth.make_head(wl, seed)
         O.head(r["pooled"], d["w"], float(d["b"][0]))

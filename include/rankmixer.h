@@ -61,7 +61,9 @@ typedef enum {
 
 typedef enum { RM_F32 = 0, RM_BF16 = 1 } rm_dtype;
 
-typedef enum { RM_GELU_TANH = 0, RM_GELU_ERF = 1 } rm_gelu;
+/* FFN activation: GELU (tanh form or exact erf form), or ReLU (the activation
+ * of the Mixer backbone timed in Appendix B of "重新理解 RankMixer"). */
+typedef enum { RM_ACT_GELU_TANH = 0, RM_ACT_GELU_ERF = 1, RM_ACT_RELU = 2 } rm_act;
 
 typedef struct {
     int B_max;       /* largest batch any call will pass                         */
@@ -72,7 +74,10 @@ typedef struct {
     int n_experts;   /* 0 = dense per-token FFN; else experts per token (Ne)     */
     rm_dtype dtype;
     float ln_eps;    /* LayerNorm epsilon, inside the square root (e.g. 1e-5)    */
-    int gelu;        /* rm_gelu                                                  */
+    int act;         /* rm_act                                                   */
+    int mix_addnorm; /* 1: S = LN(TokenMixing(X) + X), the block equation;        */
+                     /* 0: S = TokenMixing(X), the variant without Add & Norm     */
+                     /*    after mixing ("淘宝闪购-爆品团精排 Scaling Up 迭代实践", 3.5) */
 } rm_config;
 
 typedef struct {
@@ -122,8 +127,9 @@ rm_status rm_pffn_forward(rm_handle *h, const rm_block_weights *w, const void *S
 rm_status rm_moe_forward(rm_handle *h, const rm_block_weights *w, const void *S, void *V,
                          float *gates, int B, rm_stream_t stream);
 
-/* One RankMixer block: Xout = LN2(F(S) + S), S = LN1(TokenMixing(X) + X),
- * F the dense or MoE per-token FFN.  X, Xout [B, T, D]; may alias. */
+/* One RankMixer block: Xout = LN2(F(S) + S), S = LN1(TokenMixing(X) + X)
+ * (S = TokenMixing(X) when cfg.mix_addnorm is 0), F the dense or MoE
+ * per-token FFN.  X, Xout [B, T, D]; may alias. */
 rm_status rm_block_forward(rm_handle *h, const rm_block_weights *w, const void *X, void *Xout,
                            int B, rm_stream_t stream);
 
@@ -181,7 +187,7 @@ rm_status rm_selftest_wait_timeout(rm_handle *h, rm_stream_t stream);
  * reserved up front), so they cannot create a handle.
  *
  * Computes the same V = PFFN(S) as rm_pffn_forward (same kernels, same
- * layouts; dtype and gelu as in rm_config), with no handle.  Its only scratch,
+ * layouts; dtype and act as in rm_config), with no handle.  Its only scratch,
  * the FFN hidden activations [T, B, hidden], lives in a fixed device array of
  * RM_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads the
  * library holds until the process exits; the caller passes inputs and outputs
@@ -197,7 +203,7 @@ rm_status rm_selftest_wait_timeout(rm_handle *h, rm_stream_t stream);
  *     stream order, RM_OK or RM_ERR_DEVICE_TIMEOUT for this call. */
 #define RM_STATIC_SCRATCH_BYTES (16u << 20)
 rm_status rm_pffn_forward_static(const rm_block_weights *w, const void *S, void *V, int B, int T,
-                                 int D, int hidden, rm_dtype dtype, int gelu, int *device_status,
+                                 int D, int hidden, rm_dtype dtype, int act, int *device_status,
                                  rm_stream_t stream);
 
 /* ---- launch profiling ----------------------------------------------------

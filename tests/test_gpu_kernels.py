@@ -234,3 +234,33 @@ def test_argument_errors(rm):
             rm.rm_moe_forward(h, {}, X, Y, None, 4)          # dense handle
         assert e.value.status == rm.RM_ERR_UNSUPPORTED
         assert rm.rm_sync_status(h) == rm.RM_OK
+
+
+# ------------------------------------------------ variants on the pages
+@pytest.mark.parametrize("dtype,act,addnorm,T,D,hidden,B", [
+    ("bf16", "relu", True, 8, 256, 1024, 130),      # the Appendix B Mixer's ReLU
+    ("bf16", "tanh", False, 16, 320, 1280, 70),     # no Add & Norm after mixing (dh = 20)
+    ("bf16", "relu", False, 8, 128, 512, 3),
+    ("f32", "relu", False, 8, 64, 256, 64),
+    ("f32", "erf", True, 4, 32, 64, 9)])
+def test_block_variants(rm, O, dtype, act, addnorm, T, D, hidden, B):
+    blk = synth.random_like_block(T, D, hidden, dtype, seed=D + 3 * T)
+    X = synth.random_activations((B, T, D), dtype, seed=19)
+    with rm.rm_create(B, T, D, hidden, 1, 0, dtype, 1e-5, act, addnorm) as h:
+        Xout = torch.empty(B, T, D, dtype=TD[dtype], device="cuda")
+        rm.rm_block_forward(h, {k: dev(v) for k, v in blk.items()}, dev(X), Xout, B)
+        assert rm.rm_sync_status(h) == rm.RM_OK
+    assert_close(host64(Xout), O.block(X, blk, gelu=act, mix_addnorm=addnorm), dtype, f"block {act} {addnorm}")
+
+
+def test_stack_without_mix_addnorm(rm, O):
+    import dataclasses
+    wl = dataclasses.replace(synth.WORKLOADS["rm100m"], B=96, mix_addnorm=False)
+    d = synth.make_inputs(wl)
+    from token_mixing_feature_b200.stack import RankMixerStack
+    st = RankMixerStack(wl, d["blocks"])
+    pooled = st.forward(dev(d["X0"]))
+    assert rm.rm_sync_status(st.h) == rm.RM_OK
+    ref = O.stack(d["X0"], d["blocks"], mix_addnorm=False)
+    assert_close(host64(pooled), ref["pooled"], "bf16", "pooled, no Add & Norm")
+    st.close()

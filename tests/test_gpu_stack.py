@@ -27,8 +27,10 @@ def _stack(wl, d):
     return RankMixerStack(wl, d["blocks"], d.get("head"))
 
 
-def test_tiny_f32_stack_full(rm, O):
-    wl = synth.WORKLOADS["tiny_f32"]
+@pytest.mark.parametrize("name", ["tiny_f32", "appendix_b"])
+def test_small_stack_full(rm, O, name):
+    """Every sample: the fp32 stack, and the Appendix B three-layer ReLU Mixer (bf16)."""
+    wl = synth.WORKLOADS[name]
     d = synth.make_inputs(wl)
     st = _stack(wl, d)
     X0 = dev(d["X0"])
@@ -38,11 +40,11 @@ def test_tiny_f32_stack_full(rm, O):
     for l in range(wl.L):
         xs.append(st.block(l, xs[-1]))
     assert rm.rm_sync_status(st.h) == rm.RM_OK
-    ref = O.stack(d["X0"], d["blocks"], want_all=True)
+    ref = O.stack(d["X0"], d["blocks"], want_all=True, gelu=wl.act)
     for l in range(wl.L):
-        assert_close(host64(xs[l + 1]), ref["Xall"][l], "f32", f"X_{l + 1}")
-    assert_close(host64(Xlast), ref["Xlast"], "f32", "Xlast")
-    assert_close(host64(pooled), ref["pooled"], "f32", "pooled")
+        assert_close(host64(xs[l + 1]), ref["Xall"][l], wl.dtype, f"X_{l + 1}")
+    assert_close(host64(Xlast), ref["Xlast"], wl.dtype, "Xlast")
+    assert_close(host64(pooled), ref["pooled"], wl.dtype, "pooled")
     st.close()
 
 

@@ -100,8 +100,8 @@ rm_status check_batch(const rm_handle* h, int B) {
 rm_status check_block_weights(const rm_handle* h, const rm_block_weights* w, bool need_ln) {
     if (!w) return RM_ERR_INVALID_ARG;
     if (!aligned16(w->W1) || !aligned16(w->W2) || !aligned16(w->b1) || !aligned16(w->b2)) return RM_ERR_INVALID_ARG;
-    if (need_ln && (!aligned16(w->ln1_g) || !aligned16(w->ln1_b) || !aligned16(w->ln2_g) || !aligned16(w->ln2_b)))
-        return RM_ERR_INVALID_ARG;
+    if (need_ln && h->cfg.mix_addnorm && (!aligned16(w->ln1_g) || !aligned16(w->ln1_b))) return RM_ERR_INVALID_ARG;
+    if (need_ln && (!aligned16(w->ln2_g) || !aligned16(w->ln2_b))) return RM_ERR_INVALID_ARG;
     if (h->cfg.n_experts > 0 && (!aligned16(w->Wr) || !aligned16(w->br))) return RM_ERR_INVALID_ARG;
     return RM_OK;
 }
@@ -123,7 +123,7 @@ rm_status run_pffn(rm_handle* h, const rm_block_weights* w, const void* S, void*
     g1.o_gstride = (long long)B * c.hidden;
     g1.o_ld = c.hidden;
     g1.bias = static_cast<const float*>(w->b1);
-    g1.epi = c.gelu == RM_GELU_ERF ? rm::EPI_GELU_ERF : rm::EPI_GELU_TANH;
+    g1.epi = rm::epi_for_act(c.act);
 
     rm::GroupedGemm g2{};
     g2.G = c.T;
@@ -185,7 +185,7 @@ rm_status run_moe(rm_handle* h, const rm_block_weights* w, const void* S, void* 
     g1.out = h->moe.Hg;
     g1.o_ld = c.hidden;
     g1.bias = static_cast<const float*>(w->b1);
-    g1.epi = c.gelu == RM_GELU_ERF ? rm::EPI_GELU_ERF : rm::EPI_GELU_TANH;
+    g1.epi = rm::epi_for_act(c.act);
     g1.grp_cnt = h->moe.counts;
     g1.grp_off = h->moe.offsets;
     g1.mtile_prefix = h->moe.mtile_prefix;
@@ -234,7 +234,7 @@ rm_status run_stack(rm_handle* h, const rm_block_weights* blocks, const void* X0
             ProfScope ps(h, RM_K_MIX_LN, s);
             e = rm::launch_mix_ln(c.dtype, l ? h->Y : X0, prev ? prev->ln2_g : nullptr,
                                   prev ? prev->ln2_b : nullptr, w->ln1_g, w->ln1_b, h->S, B, c.T, c.D, c.ln_eps,
-                                  h->num_sms, derr(h), h->budget_ns, s);
+                                  c.mix_addnorm, h->num_sms, derr(h), h->budget_ns, s);
         }
         if (e != cudaSuccess) return RM_ERR_CUDA;
         rm_status st = run_ffn(h, w, h->S, h->Y, h->S, B, s);
@@ -277,7 +277,8 @@ rm_status rm_create(const rm_config* cfg, rm_handle** out) {
     const rm_config c = *cfg;
     if (c.B_max < 1 || c.T < 1 || c.D < 1 || c.hidden < 1 || c.L < 1 || c.n_experts < 0) return RM_ERR_INVALID_ARG;
     if (c.dtype != RM_F32 && c.dtype != RM_BF16) return RM_ERR_INVALID_ARG;
-    if (c.gelu != RM_GELU_TANH && c.gelu != RM_GELU_ERF) return RM_ERR_INVALID_ARG;
+    if (c.act != RM_ACT_GELU_TANH && c.act != RM_ACT_GELU_ERF && c.act != RM_ACT_RELU) return RM_ERR_INVALID_ARG;
+    if (c.mix_addnorm != 0 && c.mix_addnorm != 1) return RM_ERR_INVALID_ARG;
     if (!(c.ln_eps > 0.f)) return RM_ERR_INVALID_ARG;
     if (c.T > 64 || c.n_experts > 32 || c.D % c.T) return RM_ERR_UNSUPPORTED;
     const size_t esz = c.dtype == RM_BF16 ? 2 : 4;
@@ -407,7 +408,7 @@ rm_status rm_block_forward(rm_handle* h, const rm_block_weights* w, const void* 
     {
         ProfScope ps(h, RM_K_MIX_LN, stream);
         e = rm::launch_mix_ln(c.dtype, X, nullptr, nullptr, w->ln1_g, w->ln1_b, h->S, B, c.T, c.D, c.ln_eps,
-                              h->num_sms, derr(h), h->budget_ns, stream);
+                              c.mix_addnorm, h->num_sms, derr(h), h->budget_ns, stream);
     }
     if (e != cudaSuccess) return RM_ERR_CUDA;
     if ((st = run_ffn(h, w, h->S, h->Y, h->S, B, stream)) != RM_OK) return st;

@@ -57,6 +57,8 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GroupedGemm p) {
                 v = 0.5f * v * (1.0f + tanhf(0.7978845608028654f * (v + 0.044715f * v * v * v)));
             } else if (EPI == EPI_GELU_ERF) {
                 v = 0.5f * v * (1.0f + erff(v * 0.7071067811865476f));
+            } else if (EPI == EPI_RELU) {
+                v = fmaxf(v, 0.0f);
             } else if (EPI == EPI_BIAS_RESID) {
                 if (resid) v += resid[(long long)g * p.r_gstride + (long long)m * p.r_ld + n];
             }
@@ -74,6 +76,7 @@ cudaError_t launch_gemm_simt(const GroupedGemm& p, cudaStream_t s) {
     switch (p.epi) {
         case EPI_GELU_TANH: gemm_simt_kernel<EPI_GELU_TANH><<<grid, 256, 0, s>>>(p); break;
         case EPI_GELU_ERF: gemm_simt_kernel<EPI_GELU_ERF><<<grid, 256, 0, s>>>(p); break;
+        case EPI_RELU: gemm_simt_kernel<EPI_RELU><<<grid, 256, 0, s>>>(p); break;
         default: gemm_simt_kernel<EPI_BIAS_RESID><<<grid, 256, 0, s>>>(p); break;
     }
     return cudaGetLastError();

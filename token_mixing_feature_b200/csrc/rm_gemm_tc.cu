@@ -362,7 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                if (EPI == EPI_GELU_TANH) {
+                if (EPI == EPI_RELU) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) v[e] = fmaxf(v[e], 0.0f);
+                } else if (EPI == EPI_GELU_TANH) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e) v[e] = gelu_tanh_approx(v[e]);
                 } else if (EPI == EPI_GELU_ERF) {
@@ -449,7 +452,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         v[4 * q + 2] += bb.z;
                         v[4 * q + 3] += bb.w;
                     }
-                    if (EPI == EPI_GELU_TANH) {
+                    if (EPI == EPI_RELU) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = fmaxf(v[e], 0.0f);
+                    } else if (EPI == EPI_GELU_TANH) {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = gelu_tanh_approx(v[e]);
                     } else if (EPI == EPI_GELU_ERF) {
@@ -565,6 +571,7 @@ cudaError_t launch_bn(int epi, const Maps& m, const KParams& kp, int grid, cudaS
     switch (epi) {
         case EPI_GELU_TANH: return launch_typed<BN, EPI_GELU_TANH, CG, VAR>(m, kp, grid, s);
         case EPI_GELU_ERF: return launch_typed<BN, EPI_GELU_ERF, CG, VAR>(m, kp, grid, s);
+        case EPI_RELU: return launch_typed<BN, EPI_RELU, CG, VAR>(m, kp, grid, s);
         case EPI_BIAS_RESID:
             if constexpr (!VAR) return launch_typed<BN, EPI_BIAS_RESID, CG, VAR>(m, kp, grid, s);
             break;

@@ -31,10 +31,11 @@ cudaError_t launch_token_mix(int dtype, const void* X, void* Y, int B, int T, in
 cudaError_t launch_layernorm(int dtype, const void* A, const void* R, const float* g, const float* b,
                              void* out, long long rows, int D, float eps, cudaStream_t s);
 // ---- rm_mix.cu ------------------------------------------------------------
-// S = LN1(TokenMixing(Xh) + Xh), Xh = pre_g ? LN_pre(X) : X (per token row).
+// S = LN1(TokenMixing(Xh) + Xh), Xh = pre_g ? LN_pre(X) : X (per token row);
+// with addnorm == 0, S = TokenMixing(Xh) (g1, b1 unused).
 cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const float* pre_b,
                           const float* g1, const float* b1, void* S, int B, int T, int D, float eps,
-                          int num_sms, DeviceErr err, uint64_t budget_ns, cudaStream_t s);
+                          int addnorm, int num_sms, DeviceErr err, uint64_t budget_ns, cudaStream_t s);
 // Xh = LN(X) per token row; pooled[b] = mean_t Xh[b, t]; Xout optional.
 cudaError_t launch_ln_pool(int dtype, const void* X, const float* g, const float* b, float* pooled,
                            void* Xout, int B, int T, int D, float eps, int num_sms, DeviceErr err,
@@ -58,7 +59,9 @@ enum Epilogue : int {
     EPI_GELU_ERF = 1,    // bf16( GELU_erf(acc + bias) )
     EPI_BIAS_RESID = 2,  // bf16( acc + bias [+ resid] )
     EPI_BIAS_GATE = 3,   // bf16( gate[row] * (acc + bias) )
+    EPI_RELU = 4,        // bf16( max(acc + bias, 0) )
 };
+inline int epi_for_act(int act) { return act == RM_ACT_GELU_ERF ? EPI_GELU_ERF : act == RM_ACT_RELU ? EPI_RELU : EPI_GELU_TANH; }
 
 struct GroupedGemm {
     int G, M, N, K;

@@ -18,6 +18,7 @@
 // mix_ln:  Xh = PRE ? LN_pre(X) : X          (previous block's LN, row-wise)
 //          Z[h, t*dh + j] = Xh[t, h*dh + j] + Xh[h, t*dh + j]
 //          S[h, :] = LN1(Z[h, :])             (one warp per output row h)
+//          or, without the Add & Norm after mixing, S[h, t*dh + j] = Xh[t, h*dh + j]
 // ln_pool: Xh = LN(X);  pooled[b, :] = (1/T) sum_t Xh[t, :]  (ascending t)
 #include <cuda_bf16.h>
 
@@ -163,7 +164,7 @@ __device__ __forceinline__ void normalize_in_place(E* xs, int T, int D, const fl
     }
 }
 
-template <typename E, bool PRE, bool CONTIG, int NV>
+template <typename E, bool PRE, bool CONTIG, int NV, bool ADDNORM>
 __global__ void __launch_bounds__(NV >= 16 ? 256 : 512) mix_ln_kernel(const E* __restrict__ X, const float* __restrict__ pre_g,
                                                     const float* __restrict__ pre_b, const float* __restrict__ g1,
                                                     const float* __restrict__ b1, E* __restrict__ S, int B, int T,
@@ -205,7 +206,31 @@ __global__ void __launch_bounds__(NV >= 16 ? 256 : 512) mix_ln_kernel(const E* _
             __syncthreads();
         }
         E* srow = S + (size_t)b * TD;
-        for (int h = warp; h < T; h += nw) {
+        if (!ADDNORM) {
+            // S = TokenMixing(Xh): a permutation of the (normalised) staged sample
+            for (int h = warp; h < T; h += nw) {
+                for (int v = lane; v < nv; v += 32) {
+                    const int c0 = v * V;
+                    Vec16<E> o;
+                    if (CONTIG) {
+                        const int t = c0 / dh, k0 = h * dh + (c0 - t * dh);
+                        o.u = *reinterpret_cast<const uint4*>(xs + (size_t)t * D + k0);
+                    } else {
+                        int t = c0 / dh, j = c0 - t * dh;
+#pragma unroll
+                        for (int e = 0; e < V; ++e) {
+                            o.e[e] = xs[(size_t)t * D + h * dh + j];
+                            if (++j == dh) {
+                                j = 0;
+                                ++t;
+                            }
+                        }
+                    }
+                    *reinterpret_cast<uint4*>(srow + (size_t)h * D + c0) = o.u;
+                }
+            }
+        }
+        for (int h = warp; ADDNORM && h < T; h += nw) {
             float z[NV][V];
             float s = 0.f;
 #pragma unroll
@@ -379,7 +404,7 @@ cudaError_t persistent_launch(K kernel, int threads, size_t smem, int B, int num
     return cudaSuccess;
 }
 
-template <typename E, bool PRE, bool CONTIG, int NVV>
+template <typename E, bool PRE, bool CONTIG, int NVV, bool ADDNORM = true>
 cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, const float* g1, const float* b1, E* S, int B,
                       int T, int D, float eps, int num_sms, DeviceErr err, uint64_t budget, cudaStream_t s) {
     int nbuf;
@@ -387,7 +412,7 @@ cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, const float*
     ring_shape(T, D, sizeof(E), 0, &nbuf, &smem);
     // one slot: 256 threads so that two CTAs fit an SM's registers as well
     const int threads = (NVV >= 16 || nbuf == 1 || T < 16) ? 256 : 512;
-    auto k = mix_ln_kernel<E, PRE, CONTIG, NVV>;
+    auto k = mix_ln_kernel<E, PRE, CONTIG, NVV, ADDNORM>;
     int grid = 0;
     cudaError_t e = persistent_launch(k, threads, smem, B, num_sms, s, &grid);
     if (e != cudaSuccess) return e;
@@ -408,12 +433,20 @@ cudaError_t mix_ln_nv(int nvl, const E* X, const float* pg, const float* pb, con
 
 template <typename E>
 cudaError_t mix_ln_typed(const void* X, const float* pg, const float* pb, const float* g1, const float* b1, void* S,
-                         int B, int T, int D, float eps, int num_sms, DeviceErr err, uint64_t budget, cudaStream_t s) {
+                         int B, int T, int D, float eps, int addnorm, int num_sms, DeviceErr err, uint64_t budget,
+                         cudaStream_t s) {
     constexpr int V = Vec16<E>::N;
     const int nvl = (D / V + 31) / 32;
     const bool contig = ((D / T) % V) == 0;
     const E* x = static_cast<const E*>(X);
     E* y = static_cast<E*>(S);
+    if (!addnorm) {
+        if (pg)
+            return contig ? mix_ln_go<E, true, true, 1, false>(x, pg, pb, g1, b1, y, B, T, D, eps, num_sms, err, budget, s)
+                          : mix_ln_go<E, true, false, 1, false>(x, pg, pb, g1, b1, y, B, T, D, eps, num_sms, err, budget, s);
+        return contig ? mix_ln_go<E, false, true, 1, false>(x, pg, pb, g1, b1, y, B, T, D, eps, num_sms, err, budget, s)
+                      : mix_ln_go<E, false, false, 1, false>(x, pg, pb, g1, b1, y, B, T, D, eps, num_sms, err, budget, s);
+    }
     if (pg)
         return contig ? mix_ln_nv<E, true, true>(nvl, x, pg, pb, g1, b1, y, B, T, D, eps, num_sms, err, budget, s)
                       : mix_ln_nv<E, true, false>(nvl, x, pg, pb, g1, b1, y, B, T, D, eps, num_sms, err, budget, s);
@@ -442,11 +475,12 @@ cudaError_t ln_pool_typed(const void* X, const float* g, const float* b, float* 
 int mix_ln_max_d(int dtype) { return 32 * 16 * (dtype == RM_BF16 ? 8 : 4); }
 
 cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const float* pre_b, const float* g1,
-                          const float* b1, void* S, int B, int T, int D, float eps, int num_sms, DeviceErr err,
-                          uint64_t budget_ns, cudaStream_t s) {
+                          const float* b1, void* S, int B, int T, int D, float eps, int addnorm, int num_sms,
+                          DeviceErr err, uint64_t budget_ns, cudaStream_t s) {
     if (dtype == RM_BF16)
-        return mix_ln_typed<__nv_bfloat16>(X, pre_g, pre_b, g1, b1, S, B, T, D, eps, num_sms, err, budget_ns, s);
-    return mix_ln_typed<float>(X, pre_g, pre_b, g1, b1, S, B, T, D, eps, num_sms, err, budget_ns, s);
+        return mix_ln_typed<__nv_bfloat16>(X, pre_g, pre_b, g1, b1, S, B, T, D, eps, addnorm, num_sms, err, budget_ns,
+                                           s);
+    return mix_ln_typed<float>(X, pre_g, pre_b, g1, b1, S, B, T, D, eps, addnorm, num_sms, err, budget_ns, s);
 }
 
 cudaError_t launch_ln_pool(int dtype, const void* X, const float* g, const float* b, float* pooled, void* Xout, int B,

@@ -51,14 +51,14 @@ inline bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(
 }  // namespace
 
 extern "C" rm_status rm_pffn_forward_static(const rm_block_weights* w, const void* S, void* V, int B, int T, int D,
-                                            int hidden, rm_dtype dtype, int gelu, int* device_status,
+                                            int hidden, rm_dtype dtype, int act, int* device_status,
                                             rm_stream_t stream) {
     if (!w || !aligned16(S) || !aligned16(V) || !aligned16(w->W1) || !aligned16(w->b1) || !aligned16(w->W2) ||
         !aligned16(w->b2))
         return RM_ERR_INVALID_ARG;
     if (B < 1 || T < 1 || D < 1 || hidden < 1) return RM_ERR_INVALID_ARG;
     if (dtype != RM_BF16 && dtype != RM_F32) return RM_ERR_INVALID_ARG;
-    if (gelu != RM_GELU_TANH && gelu != RM_GELU_ERF) return RM_ERR_INVALID_ARG;
+    if (act != RM_ACT_GELU_TANH && act != RM_ACT_GELU_ERF && act != RM_ACT_RELU) return RM_ERR_INVALID_ARG;
     if (dtype == RM_BF16 && (D % 16 || hidden % 16)) return RM_ERR_UNSUPPORTED;
     if (dtype == RM_F32 && (D % 4 || hidden % 4)) return RM_ERR_UNSUPPORTED;
     const size_t esz = dtype == RM_BF16 ? 2 : 4;
@@ -92,7 +92,7 @@ extern "C" rm_status rm_pffn_forward_static(const rm_block_weights* w, const voi
     g1.o_gstride = (long long)B * hidden;
     g1.o_ld = hidden;
     g1.bias = static_cast<const float*>(w->b1);
-    g1.epi = gelu == RM_GELU_ERF ? rm::EPI_GELU_ERF : rm::EPI_GELU_TANH;
+    g1.epi = rm::epi_for_act(act);
 
     rm::GroupedGemm g2{};
     g2.G = T;

@@ -16,9 +16,9 @@ _LIB_PATH = pathlib.Path(__file__).resolve().with_name("librankmixer.so")
 RM_OK, RM_ERR_INVALID_ARG, RM_ERR_UNSUPPORTED, RM_ERR_CUDA, RM_ERR_OOM, \
     RM_ERR_DEVICE_TIMEOUT, RM_ERR_DEVICE_BOUNDS = range(7)
 RM_F32, RM_BF16 = 0, 1
-RM_GELU_TANH, RM_GELU_ERF = 0, 1
+RM_ACT_GELU_TANH, RM_ACT_GELU_ERF, RM_ACT_RELU = 0, 1, 2
 DTYPES = {"f32": RM_F32, "bf16": RM_BF16}
-GELUS = {"tanh": RM_GELU_TANH, "erf": RM_GELU_ERF}
+ACTS = {"tanh": RM_ACT_GELU_TANH, "erf": RM_ACT_GELU_ERF, "relu": RM_ACT_RELU}
 
 EXPORTED = (
     "rm_create", "rm_destroy", "rm_workspace_bytes", "rm_token_mix", "rm_layernorm",
@@ -34,7 +34,8 @@ RM_K_COUNT = 11
 class rm_config(ctypes.Structure):
     _fields_ = [("B_max", ctypes.c_int), ("T", ctypes.c_int), ("D", ctypes.c_int),
                 ("hidden", ctypes.c_int), ("L", ctypes.c_int), ("n_experts", ctypes.c_int),
-                ("dtype", ctypes.c_int), ("ln_eps", ctypes.c_float), ("gelu", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("ln_eps", ctypes.c_float), ("act", ctypes.c_int),
+                ("mix_addnorm", ctypes.c_int)]
 
 
 class rm_block_weights(ctypes.Structure):
@@ -147,8 +148,9 @@ class Handle:
 
 
 def rm_create(B_max: int, T: int, D: int, hidden: int, L: int = 1, n_experts: int = 0,
-              dtype: str = "bf16", ln_eps: float = 1e-5, gelu: str = "tanh") -> Handle:
-    cfg = rm_config(B_max, T, D, hidden, L, n_experts, DTYPES[dtype], ln_eps, GELUS[gelu])
+              dtype: str = "bf16", ln_eps: float = 1e-5, act: str = "tanh", mix_addnorm: bool = True) -> Handle:
+    """act: "tanh" / "erf" (GELU forms) or "relu"."""
+    cfg = rm_config(B_max, T, D, hidden, L, n_experts, DTYPES[dtype], ln_eps, ACTS[act], 1 if mix_addnorm else 0)
     out = ctypes.c_void_p()
     _check(_lib.rm_create(ctypes.byref(cfg), ctypes.byref(out)), "rm_create")
     return Handle(out.value, cfg)
@@ -260,11 +262,11 @@ def rm_kernel_name(kind: int) -> str:
 
 
 def rm_pffn_forward_static(w: Dict, S, V, B: int, T: int, D: int, hidden: int, dtype: str = "bf16",
-                           gelu: str = "tanh", device_status=None, stream=None) -> None:
+                           act: str = "tanh", device_status=None, stream=None) -> None:
     """V = PFFN(S) with no handle and no device allocation: the hidden
     activations use a fixed array inside the library (RM_STATIC_SCRATCH_BYTES),
     shared by all calls; overlapping calls race on it."""
     bw = block_weights(w)
     _check(_lib.rm_pffn_forward_static(ctypes.byref(bw), _ptr(S), _ptr(V), B, T, D, hidden, DTYPES[dtype],
-                                       GELUS[gelu], _ptr(device_status), _stream(stream)),
+                                       ACTS[act], _ptr(device_status), _stream(stream)),
            "rm_pffn_forward_static")

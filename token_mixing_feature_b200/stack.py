@@ -21,14 +21,14 @@ def to_device(blk: Dict[str, torch.Tensor], device) -> Dict[str, torch.Tensor]:
 
 class RankMixerStack:
     def __init__(self, wl: Workload, blocks: Sequence[Dict[str, torch.Tensor]], head: Optional[Dict] = None,
-                 device="cuda", B_max: Optional[int] = None, gelu: str = "tanh", ln_eps: float = 1e-5):
+                 device="cuda", B_max: Optional[int] = None, ln_eps: float = 1e-5):
         self.wl = wl
         self.device = torch.device(device)
         self.dtype = TORCH_DTYPE[wl.dtype]
         self.B_max = B_max or wl.B
         with torch.cuda.device(self.device):
             self.h = rm.rm_create(self.B_max, wl.T, wl.D, wl.hidden, wl.L, wl.n_experts, wl.dtype,
-                                  ln_eps, gelu)
+                                  ln_eps, wl.act, wl.mix_addnorm)
         self.blocks: List[Dict[str, torch.Tensor]] = [to_device(b, self.device) for b in blocks]
         self.head = to_device(head, self.device) if head else None
 

@@ -56,6 +56,8 @@ class Workload:
     head: bool = False          # D -> 1 linear head + sigmoid after pooling
     router_std: float = 0.02
     router_bias: float = -0.5
+    act: str = "tanh"           # FFN activation: "tanh" / "erf" (GELU) or "relu"
+    mix_addnorm: bool = True    # False: S = TokenMixing(X), no Add & Norm after mixing
 
     @property
     def dh(self) -> int:
@@ -83,6 +85,9 @@ WORKLOADS: Dict[str, Workload] = {
                                        352, 352, 320, 288),
                          head=True),
     "moe": Workload("moe", B=2048, T=16, D=768, hidden=768, L=2, n_experts=8),
+    # the three-layer Mixer backbone timed in Appendix B of the MFU re-reading
+    # article: batch 256, 8 tokens of width 256, FFN hidden 1024, ReLU, no MoE
+    "appendix_b": Workload("appendix_b", B=256, T=8, D=256, hidden=1024, L=3, act="relu"),
 }
 
 
