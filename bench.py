@@ -309,7 +309,7 @@ def main():
         return
 
     # per-kernel times over a second timed region of K steps (events on the launch stream)
-    rm.rm_profile_begin(runner.st.h, a.steps * runner.launches_per_step() + 8)
+    rm.rm_profile_begin(runner.st.h, a.steps * (runner.launches_per_step() + runner.wl.L) + 8)
     barrier()
     ms_prof = time_steps(runner.step, a.steps, stream)
     barrier()
@@ -363,7 +363,9 @@ def main():
             "kernels": kern,
             "profiled_ms_per_step": ms_prof / a.steps,
             "e2e": e2e,
-            "gpu_launches": a.steps * runner.launches_per_step(),
+            # launches counted by the library's per-launch events in the profiled
+            # region (the router scope covers two kernels: route + compaction)
+            "gpu_launches": sum(v[1] for v in prof.values()) + prof.get("moe_route", (0.0, 0))[1],
             "clocks": clocks,
         }
         if active is not None:

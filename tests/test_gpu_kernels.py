@@ -100,7 +100,10 @@ def test_pffn_gelu_erf(rm, O):
 # --------------------------------------------------------------------- block
 @pytest.mark.parametrize("dtype,T,D,hidden,B", [
     ("bf16", 16, 768, 3072, 96), ("bf16", 16, 320, 1280, 130), ("bf16", 8, 128, 512, 3),
-    ("f32", 8, 64, 256, 64), ("f32", 4, 32, 64, 7)])
+    ("bf16", 8, 96, 256, 33),     # dh = 12: mixed term in 8-byte pieces
+    ("bf16", 8, 80, 256, 17),     # dh = 10: mixed term element by element
+    ("f32", 8, 64, 256, 64), ("f32", 4, 32, 64, 7),
+    ("f32", 4, 24, 64, 5)])       # dh = 6: 8-byte pieces of fp32
 def test_block_forward(rm, O, dtype, T, D, hidden, B):
     blk = synth.random_like_block(T, D, hidden, dtype, seed=D + T)
     X = synth.random_activations((B, T, D), dtype, seed=9)

@@ -37,6 +37,8 @@ struct rm_handle {
     void* Y;
     void* X0buf;
     float* pooledbuf;
+    float2* ystats;   // LayerNorm partials of the pre-LN block outputs Y [B_max*T][stat_P]
+    int stat_P;
     rm::MoeWork moe;
     int* err;       // [0] error word, [1] site
     unsigned long long budget_ns;
@@ -106,9 +108,11 @@ rm_status check_block_weights(const rm_handle* h, const rm_block_weights* w, boo
     return RM_OK;
 }
 
-// V = F(S) (+ resid when resid != nullptr); F the dense per-token FFN.
+// V = F(S) (+ resid when resid != nullptr); F the dense per-token FFN.  With
+// stats != nullptr the second projection's epilogue also writes the LayerNorm
+// partials of V (h->stat_P slices per row); *stats_done tells whether it did.
 rm_status run_pffn(rm_handle* h, const rm_block_weights* w, const void* S, void* V, const void* resid, int B,
-                   cudaStream_t s) {
+                   cudaStream_t s, float2* stats = nullptr, bool* stats_done = nullptr) {
     const rm_config& c = h->cfg;
     rm::GroupedGemm g1{};
     g1.G = c.T;
@@ -142,6 +146,13 @@ rm_status run_pffn(rm_handle* h, const rm_block_weights* w, const void* S, void*
     g2.r_gstride = c.D;
     g2.r_ld = (long long)c.T * c.D;
     g2.epi = rm::EPI_BIAS_RESID;
+    const bool gemm_stats = stats && c.dtype == RM_BF16 && c.D % 64 == 0;
+    if (gemm_stats) {
+        g2.stats = stats;
+        g2.s_gstride = h->stat_P;
+        g2.s_ld = (long long)c.T * h->stat_P;
+    }
+    if (stats_done) *stats_done = gemm_stats;
 
     cudaError_t e;
     {
@@ -157,9 +168,10 @@ rm_status run_pffn(rm_handle* h, const rm_block_weights* w, const void* S, void*
     return cuda_status(e);
 }
 
-// V = sum_j ReLU-gate * expert(S) (+ resid); gates_out optional copy of G.
+// V = sum_j ReLU-gate * expert(S) (+ resid); gates_out optional copy of G;
+// stats (optional) receives the LayerNorm statistics of V (one slice per row).
 rm_status run_moe(rm_handle* h, const rm_block_weights* w, const void* S, void* V, const void* resid,
-                  float* gates_out, int B, cudaStream_t s) {
+                  float* gates_out, int B, cudaStream_t s, float2* stats = nullptr) {
     const rm_config& c = h->cfg;
     const int Ne = c.n_experts;
     const int G = c.T * Ne;
@@ -210,17 +222,24 @@ rm_status run_moe(rm_handle* h, const rm_block_weights* w, const void* S, void* 
     }
     if (e == cudaSuccess) {
         ProfScope ps(h, RM_K_MOE_COMBINE, s);
-        e = rm::launch_moe_combine(h->moe, resid, V, B, c.T, c.D, Ne, s);
+        e = rm::launch_moe_combine(h->moe, resid, V, stats, B, c.T, c.D, Ne, s);
     }
     if (e == cudaSuccess && gates_out)
         e = cudaMemcpyAsync(gates_out, h->moe.gates, sizeof(float) * (size_t)B * c.T * Ne, cudaMemcpyDeviceToDevice, s);
     return cuda_status(e);
 }
 
+// V = F(S) + resid; with stats, also the LayerNorm statistics of V in
+// h->stat_P slices per row (from the producing epilogue when it can, else by
+// a row-statistics pass).
 rm_status run_ffn(rm_handle* h, const rm_block_weights* w, const void* S, void* V, const void* resid, int B,
-                  cudaStream_t s) {
-    if (h->cfg.n_experts > 0) return run_moe(h, w, S, V, resid, nullptr, B, s);
-    return run_pffn(h, w, S, V, resid, B, s);
+                  cudaStream_t s, float2* stats = nullptr) {
+    if (h->cfg.n_experts > 0) return run_moe(h, w, S, V, resid, nullptr, B, s, stats);
+    bool done = false;
+    rm_status st = run_pffn(h, w, S, V, resid, B, s, stats, &done);
+    if (st != RM_OK || !stats || done) return st;
+    ProfScope ps(h, RM_K_LAYERNORM, s);
+    return cuda_status(rm::launch_row_stats(h->cfg.dtype, V, stats, (long long)B * h->cfg.T, h->cfg.D, s));
 }
 
 rm_status run_stack(rm_handle* h, const rm_block_weights* blocks, const void* X0, float* pooled, void* Xlast,
@@ -229,21 +248,23 @@ rm_status run_stack(rm_handle* h, const rm_block_weights* blocks, const void* X0
     for (int l = 0; l < c.L; ++l) {
         const rm_block_weights* w = &blocks[l];
         const rm_block_weights* prev = l ? &blocks[l - 1] : nullptr;
+        const rm::RowStats ys{h->ystats, h->stat_P};
         cudaError_t e;
         {
             ProfScope ps(h, RM_K_MIX_LN, s);
             e = rm::launch_mix_ln(c.dtype, l ? h->Y : X0, prev ? prev->ln2_g : nullptr,
-                                  prev ? prev->ln2_b : nullptr, w->ln1_g, w->ln1_b, h->S, B, c.T, c.D, c.ln_eps,
+                                  prev ? prev->ln2_b : nullptr, ys, w->ln1_g, w->ln1_b, h->S, B, c.T, c.D, c.ln_eps,
                                   c.mix_addnorm, h->num_sms, derr(h), h->budget_ns, s);
         }
         if (e != cudaSuccess) return RM_ERR_CUDA;
-        rm_status st = run_ffn(h, w, h->S, h->Y, h->S, B, s);
+        rm_status st = run_ffn(h, w, h->S, h->Y, h->S, B, s, h->ystats);
         if (st != RM_OK) return st;
     }
     const rm_block_weights* last = &blocks[c.L - 1];
     ProfScope ps(h, RM_K_LN_POOL, s);
-    return cuda_status(rm::launch_ln_pool(c.dtype, h->Y, last->ln2_g, last->ln2_b, pooled, Xlast, B, c.T, c.D,
-                                          c.ln_eps, h->num_sms, derr(h), h->budget_ns, s));
+    return cuda_status(rm::launch_ln_pool(c.dtype, h->Y, rm::RowStats{h->ystats, h->stat_P}, last->ln2_g,
+                                          last->ln2_b, pooled, Xlast, B, c.T, c.D, c.ln_eps, h->num_sms, derr(h),
+                                          h->budget_ns, s));
 }
 
 template <typename T>
@@ -285,6 +306,7 @@ rm_status rm_create(const rm_config* cfg, rm_handle** out) {
     if (c.dtype == RM_BF16 && (c.D % 16 || c.hidden % 16)) return RM_ERR_UNSUPPORTED;
     if (c.dtype == RM_F32 && (c.D % 4 || c.hidden % 4)) return RM_ERR_UNSUPPORTED;
     if (c.n_experts > 0 && c.dtype != RM_BF16) return RM_ERR_UNSUPPORTED;
+    if ((size_t)c.n_experts * c.D * sizeof(float) > 160 * 1024) return RM_ERR_UNSUPPORTED;   // router staged in smem
     if (c.D > rm::mix_ln_max_d(c.dtype)) return RM_ERR_UNSUPPORTED;
     if ((size_t)c.T * c.D * esz + 8 * (size_t)c.T > 220 * 1024) return RM_ERR_UNSUPPORTED;
 
@@ -311,6 +333,8 @@ rm_status rm_create(const rm_config* cfg, rm_handle** out) {
         h->Y = carve<unsigned char>(base, off, BTD * esz);
         h->X0buf = carve<unsigned char>(base, off, BTD * esz);
         h->pooledbuf = carve<float>(base, off, (size_t)c.B_max * c.D * sizeof(float));
+        h->stat_P = (c.dtype == RM_BF16 && c.n_experts == 0 && c.D % 64 == 0) ? c.D / 64 : 1;
+        h->ystats = carve<float2>(base, off, (size_t)c.B_max * c.T * h->stat_P * sizeof(float2));
         h->H = c.n_experts == 0 ? carve<unsigned char>(base, off, (size_t)c.T * c.B_max * c.hidden * esz) : nullptr;
         if (c.n_experts > 0) {
             rm::MoeWork& m = h->moe;
@@ -407,8 +431,8 @@ rm_status rm_block_forward(rm_handle* h, const rm_block_weights* w, const void* 
     cudaError_t e;
     {
         ProfScope ps(h, RM_K_MIX_LN, stream);
-        e = rm::launch_mix_ln(c.dtype, X, nullptr, nullptr, w->ln1_g, w->ln1_b, h->S, B, c.T, c.D, c.ln_eps,
-                              c.mix_addnorm, h->num_sms, derr(h), h->budget_ns, stream);
+        e = rm::launch_mix_ln(c.dtype, X, nullptr, nullptr, rm::RowStats{nullptr, 0}, w->ln1_g, w->ln1_b, h->S, B,
+                              c.T, c.D, c.ln_eps, c.mix_addnorm, h->num_sms, derr(h), h->budget_ns, stream);
     }
     if (e != cudaSuccess) return RM_ERR_CUDA;
     if ((st = run_ffn(h, w, h->S, h->Y, h->S, B, stream)) != RM_OK) return st;

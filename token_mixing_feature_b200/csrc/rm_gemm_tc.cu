@@ -53,6 +53,8 @@ struct KParams {
     const int* grp_cnt;
     const int* grp_off;
     const int* mtile_prefix;
+    float2* stats;            // LayerNorm partials of stored rows (dense EPI_BIAS_RESID), or null
+    long long s_gstride, s_ld;
     DeviceErr err;
     unsigned long long budget_ns;
 };
@@ -391,14 +393,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
+                uint32_t w[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                if (EPI == EPI_BIAS_RESID && p.stats != nullptr && wrow0 + lane < p.M) {
+                    // LayerNorm partials of the stored (rounded) 64 values: (mean, M2)
+                    float s1 = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) s1 += __uint_as_float(w[j] << 16) + __uint_as_float(w[j] & 0xffff0000u);
+                    const float mean = s1 * (1.0f / 64.0f);
+                    float q = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float d0 = __uint_as_float(w[j] << 16) - mean;
+                        const float d1 = __uint_as_float(w[j] & 0xffff0000u) - mean;
+                        q = fmaf(d0, d0, fmaf(d1, d1, q));
+                    }
+                    p.stats[(long long)t.g * p.s_gstride + (long long)(wrow0 + lane) * p.s_ld + (n >> 6)] =
+                        make_float2(mean, q);
+                }
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const uint32_t a0 = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-                    const uint32_t a1 = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-                    const uint32_t a2 = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-                    const uint32_t a3 = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(my_row + ((((uint32_t)j) ^ swz) << 4)),
-                                 "r"(a0), "r"(a1), "r"(a2), "r"(a3)
+                                 "r"(w[4 * j]), "r"(w[4 * j + 1]), "r"(w[4 * j + 2]), "r"(w[4 * j + 3])
                                  : "memory");
                 }
                 fence_proxy_async_shared();
@@ -635,6 +652,10 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     kp.grp_cnt = g.grp_cnt;
     kp.grp_off = g.grp_off;
     kp.mtile_prefix = g.mtile_prefix;
+    kp.stats = g.stats;
+    kp.s_gstride = g.s_gstride;
+    kp.s_ld = g.s_ld;
+    if (g.stats && (var || g.epi != EPI_BIAS_RESID || g.N % 64)) return cudaErrorInvalidValue;
     kp.err = err;
     kp.budget_ns = budget_ns;
 

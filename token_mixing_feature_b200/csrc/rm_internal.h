@@ -31,15 +31,23 @@ cudaError_t launch_token_mix(int dtype, const void* X, void* Y, int B, int T, in
 cudaError_t launch_layernorm(int dtype, const void* A, const void* R, const float* g, const float* b,
                              void* out, long long rows, int D, float eps, cudaStream_t s);
 // ---- rm_mix.cu ------------------------------------------------------------
-// S = LN1(TokenMixing(Xh) + Xh), Xh = pre_g ? LN_pre(X) : X (per token row);
-// with addnorm == 0, S = TokenMixing(Xh) (g1, b1 unused).
-cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const float* pre_b,
-                          const float* g1, const float* b1, void* S, int B, int T, int D, float eps,
-                          int addnorm, int num_sms, DeviceErr err, uint64_t budget_ns, cudaStream_t s);
-// Xh = LN(X) per token row; pooled[b] = mean_t Xh[b, t]; Xout optional.
-cudaError_t launch_ln_pool(int dtype, const void* X, const float* g, const float* b, float* pooled,
+// LayerNorm statistics of rows (row = b*T + t) in partial form: part[row*P + p]
+// = (mean, M2) over the D/P columns of slice p, as written by the producer.
+struct RowStats {
+    float2* part;
+    int P;
+};
+// S = LN1(TokenMixing(Xh) + Xh), Xh = pre_g ? LN_pre(X) : X (per token row,
+// statistics from pre_stats); with addnorm == 0, S = TokenMixing(Xh).
+cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const float* pre_b, RowStats pre_stats,
+                          const float* g1, const float* b1, void* S, int B, int T, int D, float eps, int addnorm,
+                          int num_sms, DeviceErr err, uint64_t budget_ns, cudaStream_t s);
+// pooled[b] = mean_t LN(X[b, t]) (statistics given); Xout (optional) = LN(X).
+cudaError_t launch_ln_pool(int dtype, const void* X, RowStats stats, const float* g, const float* b, float* pooled,
                            void* Xout, int B, int T, int D, float eps, int num_sms, DeviceErr err,
                            uint64_t budget_ns, cudaStream_t s);
+// out[row] = (mean, M2) of each row over all D columns (P = 1).
+cudaError_t launch_row_stats(int dtype, const void* X, float2* out, long long rows, int D, cudaStream_t s);
 int mix_ln_max_d(int dtype);
 struct PadSplitArgs {
     const void* src[32];
@@ -79,6 +87,11 @@ struct GroupedGemm {
     long long r_gstride, r_ld;
     const float* gate;        // EPI_BIAS_GATE: [rows] in variable-row mode
     int epi;
+    // Optional LayerNorm partial statistics of the stored (rounded) output rows,
+    // EPI_BIAS_RESID dense only, N % 64 == 0: (mean, M2) of columns
+    // [64c, 64c + 64) of row (g, m) at stats + g*s_gstride + m*s_ld + c.
+    float2* stats;
+    long long s_gstride, s_ld;
     // Variable-row mode (sparse MoE): group g owns rows [grp_off[g], grp_off[g] + grp_cnt[g])
     // of A and out (g strides unused); mtile_prefix[g] = sum_{g' < g} ceil(cnt / 128).
     const int* grp_cnt;
@@ -108,7 +121,9 @@ cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, co
                              int T, int D, int Ne, cudaStream_t s);
 cudaError_t launch_moe_gather(const void* S, const MoeWork& w, int B, int T, int D, int Ne,
                               cudaStream_t s);
-cudaError_t launch_moe_combine(const MoeWork& w, const void* resid, void* out, int B, int T, int D,
+// out[r] = resid[r] + sum_j Eg[slot_of[r, j]]; stats (may be null) = (mean, M2)
+// of each stored row (P = 1).
+cudaError_t launch_moe_combine(const MoeWork& w, const void* resid, void* out, float2* stats, int B, int T, int D,
                                int Ne, cudaStream_t s);
 
 }  // namespace rm

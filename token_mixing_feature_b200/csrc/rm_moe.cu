@@ -21,49 +21,104 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// One warp per (b, t) row of S.  NE is the compile-time capacity (>= Ne).
+// Router logits, ReLU gates and per-expert active counts.  CTA (t, chunk)
+// stages router t's weights Wr_t [Ne][D] in shared memory once and serves
+// kRouteRows samples b.  A warp takes RW = 32 / NE rows (b, t) of S at a time:
+// lane l multiplies columns 4l, 4l+128, ... of all RW rows with all NE
+// experts, so each shared-memory weight vector feeds RW rows and each S
+// vector NE experts, with conflict-free 16-byte shared loads.  The RW x NE =
+// 32 partial dot products per lane are reduced across the warp by a
+// transposing butterfly (31 shuffles in all), after which lane l holds the
+// logit of row l / NE, expert l % NE.  Active counts are summed in shared
+// memory and added to the global counts once per CTA.
+constexpr int kRouteRows = 64;
+
+// acc[i] summed over the warp; afterwards acc[0] of lane l is the sum of
+// everyone's acc[l].
+__device__ __forceinline__ void warp_reduce_transpose32(float (&acc)[32]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+            const float send = upper ? acc[i] : acc[i + o];
+            const float keep = upper ? acc[i + o] : acc[i];
+            acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+}
+
 template <int NE>
 __global__ void __launch_bounds__(kThreads) route_kernel(const __nv_bfloat16* __restrict__ S,
                                                          const float* __restrict__ Wr,
                                                          const float* __restrict__ br, float* __restrict__ gates,
-                                                         int* __restrict__ counts, long long rows, int T, int D,
-                                                         int Ne) {
-    const int lane = threadIdx.x & 31;
-    const long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (r >= rows) return;
-    const int t = (int)(r % T);
-    const __nv_bfloat16* srow = S + r * D;
-    const float* w = Wr + (long long)t * Ne * D;
-    float acc[NE];
+                                                         int* __restrict__ counts, int B, int T, int D, int Ne) {
+    constexpr int RW = 32 / NE;
+    extern __shared__ __align__(16) float wsm[];   // [Ne][D]
+    __shared__ int cnt[NE];
+    const int t = blockIdx.x;
+    const int b0 = blockIdx.y * kRouteRows;
+    const int bend = min(B, b0 + kRouteRows);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    {
+        const float4* src = reinterpret_cast<const float4*>(Wr + (size_t)t * Ne * D);
+        float4* dst = reinterpret_cast<float4*>(wsm);
+        for (int i = threadIdx.x; i < Ne * D / 4; i += blockDim.x) dst[i] = __ldg(src + i);
+        if (threadIdx.x < NE) cnt[threadIdx.x] = 0;
+    }
+    __syncthreads();
+    const int nv = D / 4;
+    const int jl = lane % NE, rl = lane / NE;   // this lane's (row, expert) after the reduction
+    const float bias = jl < Ne ? __ldg(br + (long long)t * Ne + jl) : 0.f;
+    for (int bw = b0 + warp * RW; bw < bend; bw += nw * RW) {
+        float acc[32];
 #pragma unroll
-    for (int j = 0; j < NE; ++j) acc[j] = 0.f;
-    for (int v = lane; v < D / 8; v += 32) {
-        Vec16<__nv_bfloat16> x;
-        x.u = __ldg(reinterpret_cast<const uint4*>(srow) + v);
-        float xf[8];
+        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+        for (int v = lane; v < nv; v += 32) {
+            float xf[RW][4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) xf[e] = __bfloat162float(x.e[e]);
+            for (int q = 0; q < RW; ++q) {
+                const int b = bw + q;
+                if (b < bend) {
+                    const uint2 u = __ldg(reinterpret_cast<const uint2*>(S + ((long long)b * T + t) * D) + v);
+                    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+                    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+                    xf[q][0] = lo.x;
+                    xf[q][1] = lo.y;
+                    xf[q][2] = hi.x;
+                    xf[q][3] = hi.y;
+                } else {
+                    xf[q][0] = xf[q][1] = xf[q][2] = xf[q][3] = 0.f;
+                }
+            }
 #pragma unroll
-        for (int j = 0; j < NE; ++j) {
-            if (j < Ne) {
-                const float4* w4 = reinterpret_cast<const float4*>(w + (long long)j * D + v * 8);
-                const float4 a = __ldg(w4), b = __ldg(w4 + 1);
-                acc[j] += xf[0] * a.x + xf[1] * a.y + xf[2] * a.z + xf[3] * a.w + xf[4] * b.x + xf[5] * b.y +
-                          xf[6] * b.z + xf[7] * b.w;
+            for (int j = 0; j < NE; ++j) {
+                if (j < Ne) {
+                    const float4 w = *reinterpret_cast<const float4*>(wsm + (size_t)j * D + 4 * v);
+#pragma unroll
+                    for (int q = 0; q < RW; ++q) {
+                        float a = acc[q * NE + j];
+                        a = fmaf(xf[q][0], w.x, a);
+                        a = fmaf(xf[q][1], w.y, a);
+                        a = fmaf(xf[q][2], w.z, a);
+                        a = fmaf(xf[q][3], w.w, a);
+                        acc[q * NE + j] = a;
+                    }
+                }
             }
         }
-    }
-#pragma unroll
-    for (int j = 0; j < NE; ++j) {
-        if (j < Ne) {
-            const float logit = warp_sum(acc[j]) + __ldg(br + (long long)t * Ne + j);
+        warp_reduce_transpose32(acc);
+        const int b = bw + rl;
+        if (jl < Ne && b < bend) {
+            const float logit = acc[0] + bias;
             const float gate = logit > 0.f ? logit : 0.f;
-            if (lane == 0) {
-                gates[r * Ne + j] = gate;
-                if (gate > 0.f) atomicAdd(counts + (long long)t * Ne + j, 1);
-            }
+            gates[((long long)b * T + t) * Ne + jl] = gate;
+            if (gate > 0.f) atomicAdd(&cnt[jl], 1);
         }
     }
+    __syncthreads();
+    if (threadIdx.x < Ne && cnt[threadIdx.x]) atomicAdd(counts + (long long)t * Ne + threadIdx.x, cnt[threadIdx.x]);
 }
 
 __device__ __forceinline__ int warp_isum(int v) {
@@ -157,16 +212,18 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const __nv_bfloat16* _
 }
 
 // out[r] = resid[r] + sum over j ascending of Eg[slot_of[r, j]] (active only),
-// summed in fp32.  One warp per (b, t) row.
+// summed in fp32.  One warp per (b, t) row.  stats (optional) = (mean, M2) of
+// the stored row, from sums shifted by the row's first stored value.
 __global__ void __launch_bounds__(kThreads) combine_kernel(const __nv_bfloat16* __restrict__ Eg,
                                                            const int* __restrict__ slot_of,
                                                            const __nv_bfloat16* __restrict__ resid,
-                                                           __nv_bfloat16* __restrict__ out, long long rows, int D,
-                                                           int Ne) {
+                                                           __nv_bfloat16* __restrict__ out, float2* __restrict__ stats,
+                                                           long long rows, int D, int Ne) {
     const int lane = threadIdx.x & 31;
     const long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5);
     if (r >= rows) return;
     const int nv = D / 8;
+    float K = 0.f, s1 = 0.f, s2 = 0.f;
     for (int v = lane; v < nv; v += 32) {
         float acc[8];
         if (resid) {
@@ -192,6 +249,21 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const __nv_bfloat16* 
         o.z = pack_bf16x2(acc[4], acc[5]);
         o.w = pack_bf16x2(acc[6], acc[7]);
         reinterpret_cast<uint4*>(out + r * D)[v] = o;
+        if (stats) {
+            const uint32_t w[4] = {o.x, o.y, o.z, o.w};
+            if (v == lane) K = __shfl_sync(__activemask(), __uint_as_float(o.x << 16), 0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float d0 = __uint_as_float(w[q] << 16) - K, d1 = __uint_as_float(w[q] & 0xffff0000u) - K;
+                s1 += d0 + d1;
+                s2 = fmaf(d0, d0, fmaf(d1, d1, s2));
+            }
+        }
+    }
+    if (stats) {
+        s1 = warp_sum(s1);
+        s2 = warp_sum(s2);
+        if (lane == 0) stats[r] = make_float2(K + s1 / D, fmaxf(s2 - s1 * s1 / D, 0.f));
     }
 }
 
@@ -201,15 +273,22 @@ cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, co
                              int D, int Ne, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(w.counts, 0, sizeof(int) * T * Ne, s);
     if (e != cudaSuccess) return e;
-    const long long rows = (long long)B * T;
-    const int grid = (int)((rows + kThreads / 32 - 1) / (kThreads / 32));
+    const dim3 grid(T, (B + kRouteRows - 1) / kRouteRows);
+    const size_t smem = sizeof(float) * (size_t)Ne * D;
     const auto* Sb = static_cast<const __nv_bfloat16*>(S);
-    if (Ne <= 1) route_kernel<1><<<grid, kThreads, 0, s>>>(Sb, Wr, br, w.gates, w.counts, rows, T, D, Ne);
-    else if (Ne <= 2) route_kernel<2><<<grid, kThreads, 0, s>>>(Sb, Wr, br, w.gates, w.counts, rows, T, D, Ne);
-    else if (Ne <= 4) route_kernel<4><<<grid, kThreads, 0, s>>>(Sb, Wr, br, w.gates, w.counts, rows, T, D, Ne);
-    else if (Ne <= 8) route_kernel<8><<<grid, kThreads, 0, s>>>(Sb, Wr, br, w.gates, w.counts, rows, T, D, Ne);
-    else if (Ne <= 16) route_kernel<16><<<grid, kThreads, 0, s>>>(Sb, Wr, br, w.gates, w.counts, rows, T, D, Ne);
-    else route_kernel<32><<<grid, kThreads, 0, s>>>(Sb, Wr, br, w.gates, w.counts, rows, T, D, Ne);
+#define RM_ROUTE(NEV)                                                                                    \
+    {                                                                                                    \
+        e = cudaFuncSetAttribute(route_kernel<NEV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+        if (e != cudaSuccess) return e;                                                                  \
+        route_kernel<NEV><<<grid, kThreads, smem, s>>>(Sb, Wr, br, w.gates, w.counts, B, T, D, Ne);      \
+    }
+    if (Ne <= 1) RM_ROUTE(1)
+    else if (Ne <= 2) RM_ROUTE(2)
+    else if (Ne <= 4) RM_ROUTE(4)
+    else if (Ne <= 8) RM_ROUTE(8)
+    else if (Ne <= 16) RM_ROUTE(16)
+    else RM_ROUTE(32)
+#undef RM_ROUTE
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     compact_kernel<<<T * Ne, 1024, 0, s>>>(w.gates, w.counts, w.offsets, w.mtile_prefix, w.totals, w.slot_row,
@@ -226,13 +305,13 @@ cudaError_t launch_moe_gather(const void* S, const MoeWork& w, int B, int T, int
     return cudaGetLastError();
 }
 
-cudaError_t launch_moe_combine(const MoeWork& w, const void* resid, void* out, int B, int T, int D, int Ne,
-                               cudaStream_t s) {
+cudaError_t launch_moe_combine(const MoeWork& w, const void* resid, void* out, float2* stats, int B, int T, int D,
+                               int Ne, cudaStream_t s) {
     const long long rows = (long long)B * T;
     const int grid = (int)((rows + kThreads / 32 - 1) / (kThreads / 32));
     combine_kernel<<<grid, kThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(w.Eg), w.slot_of,
                                              static_cast<const __nv_bfloat16*>(resid),
-                                             static_cast<__nv_bfloat16*>(out), rows, D, Ne);
+                                             static_cast<__nv_bfloat16*>(out), stats, rows, D, Ne);
     return cudaGetLastError();
 }
 
