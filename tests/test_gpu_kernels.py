@@ -97,6 +97,33 @@ def test_pffn_gelu_erf(rm, O):
     assert_close(host64(V), ref, "bf16", "pffn erf", raw=True)
 
 
+@pytest.mark.parametrize("T,D,hidden,B", [(4, 256, 2048, 256), (4, 320, 1536, 300)])
+def test_pffn_split_k_tail(rm, O, monkeypatch, T, D, hidden, B):
+    """Few output tiles over a long K: the second projection's last wave is
+    split into K slices on otherwise idle SMs, summed in slice order by the
+    slice that finishes last.  Parity with the oracle, bitwise repeatability
+    (whichever slice finishes last), agreement with the unsplit kernel."""
+    blk = synth.random_like_block(T, D, hidden, "bf16", seed=D + hidden)
+    S = synth.random_activations((B, T, D), "bf16", seed=21)
+    with _handle(rm, B, T, D, hidden, "bf16") as h:
+        w = {k: dev(v) for k, v in blk.items()}
+        Sd = dev(S)
+        runs = []
+        for _ in range(3):
+            V = torch.empty(B, T, D, dtype=torch.bfloat16, device="cuda")
+            rm.rm_pffn_forward(h, w, Sd, V, B)
+            runs.append(V)
+        monkeypatch.setenv("RM_GEMM_SPLIT", "0")
+        V0 = torch.empty(B, T, D, dtype=torch.bfloat16, device="cuda")
+        rm.rm_pffn_forward(h, w, Sd, V0, B)
+        assert rm.rm_sync_status(h) == rm.RM_OK
+    for V in runs[1:]:
+        assert torch.equal(V, runs[0])
+    ref = O.pffn(S, blk["W1"], blk["b1"], blk["W2"], blk["b2"])
+    assert_close(host64(runs[0]), ref, "bf16", "pffn split-K", raw=True)
+    assert_close(host64(V0), ref, "bf16", "pffn unsplit", raw=True)
+
+
 # --------------------------------------------------------------------- block
 @pytest.mark.parametrize("dtype,T,D,hidden,B", [
     ("bf16", 16, 768, 3072, 96), ("bf16", 16, 320, 1280, 130), ("bf16", 8, 128, 512, 3),

@@ -21,10 +21,6 @@
 
 #include "rm_internal.h"
 
-namespace rm {
-int gemm_tc_pick_bn(int G, int M, int N, bool var_rows, int num_sms, int cg);
-}  // namespace rm
-
 struct rm_handle {
     rm_config cfg;
     int device;
@@ -39,6 +35,8 @@ struct rm_handle {
     float* pooledbuf;
     float2* ystats;   // LayerNorm partials of the pre-LN block outputs Y [B_max*T][stat_P]
     int stat_P;
+    float* sk_ws;     // split-K partial tiles of the dense tcgen05 GEMMs (null for fp32 / MoE)
+    int* sk_cnt;      // their arrival counters (zero between launches)
     rm::MoeWork moe;
     int* err;       // [0] error word, [1] site
     unsigned long long budget_ns;
@@ -146,6 +144,8 @@ rm_status run_pffn(rm_handle* h, const rm_block_weights* w, const void* S, void*
     g2.r_gstride = c.D;
     g2.r_ld = (long long)c.T * c.D;
     g2.epi = rm::EPI_BIAS_RESID;
+    g1.sk_ws = g2.sk_ws = h->sk_ws;
+    g1.sk_cnt = g2.sk_cnt = h->sk_cnt;
     const bool gemm_stats = stats && c.dtype == RM_BF16 && c.D % 64 == 0;
     if (gemm_stats) {
         g2.stats = stats;
@@ -336,6 +336,9 @@ rm_status rm_create(const rm_config* cfg, rm_handle** out) {
         h->stat_P = (c.dtype == RM_BF16 && c.n_experts == 0 && c.D % 64 == 0) ? c.D / 64 : 1;
         h->ystats = carve<float2>(base, off, (size_t)c.B_max * c.T * h->stat_P * sizeof(float2));
         h->H = c.n_experts == 0 ? carve<unsigned char>(base, off, (size_t)c.T * c.B_max * c.hidden * esz) : nullptr;
+        const bool split = c.dtype == RM_BF16 && c.n_experts == 0;
+        h->sk_cnt = split ? carve<int>(base, off, rm::gemm_tc_split_cnt_ints(h->num_sms) * sizeof(int)) : nullptr;
+        h->sk_ws = split ? carve<float>(base, off, rm::gemm_tc_split_ws_bytes(h->num_sms)) : nullptr;
         if (c.n_experts > 0) {
             rm::MoeWork& m = h->moe;
             m.gates = carve<float>(base, off, slots * sizeof(float));
@@ -359,7 +362,8 @@ rm_status rm_create(const rm_config* cfg, rm_handle** out) {
             }
         }
     }
-    if (cudaMemset(h->err, 0, 2 * sizeof(int)) != cudaSuccess) {
+    if (cudaMemset(h->err, 0, 2 * sizeof(int)) != cudaSuccess ||
+        (h->sk_cnt && cudaMemset(h->sk_cnt, 0, rm::gemm_tc_split_cnt_ints(h->num_sms) * sizeof(int)) != cudaSuccess)) {
         cudaFree(h->ws);
         delete h;
         return RM_ERR_CUDA;
@@ -504,6 +508,9 @@ rm_status rm_sync_status(rm_handle* h, rm_stream_t stream) {
     if (v[0] != 0) {
         h->last_site = v[1];
         if (cudaMemset(h->err, 0, sizeof(v)) != cudaSuccess) return RM_ERR_CUDA;
+        // a GEMM that stopped early may have left split-K arrival counts behind
+        if (h->sk_cnt && cudaMemset(h->sk_cnt, 0, rm::gemm_tc_split_cnt_ints(h->num_sms) * sizeof(int)) != cudaSuccess)
+            return RM_ERR_CUDA;
     }
     return static_cast<rm_status>(v[0]);
 }

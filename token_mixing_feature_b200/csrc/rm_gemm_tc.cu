@@ -24,6 +24,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -55,6 +56,14 @@ struct KParams {
     const int* mtile_prefix;
     float2* stats;            // LayerNorm partials of stored rows (dense EPI_BIAS_RESID), or null
     long long s_gstride, s_ld;
+    // Split-K tail (dense only): tiles [full_tiles, tiles) are each computed
+    // as nsplit K-slices by different CTAs; fp32 partials go to sk_ws and the
+    // last slice to finish (per-warp arrival counters sk_cnt) sums them in
+    // slice order and runs the epilogue.  nsplit = 1: no split items.
+    long long full_tiles;
+    int nsplit;
+    float* sk_ws;
+    int* sk_cnt;
     DeviceErr err;
     unsigned long long budget_ns;
 };
@@ -131,6 +140,34 @@ __device__ __forceinline__ Tile decode_tile(const KParams& p, long long idx, int
     return t;
 }
 
+// Work item idx -> tile index, K-block range and (for split items) the tail
+// tile's ordinal and this item's slice.  Items below full_tiles are whole tiles.
+struct Item {
+    long long tile;
+    int kb_lo, kb_hi;
+    int tj;      // tail tile ordinal (split items), else -1
+    int slice;
+};
+
+__device__ __forceinline__ Item decode_item(const KParams& p, long long idx, int num_kb) {
+    Item it;
+    if (idx < p.full_tiles || p.nsplit == 1) {
+        it.tile = idx;
+        it.kb_lo = 0;
+        it.kb_hi = num_kb;
+        it.tj = -1;
+        it.slice = 0;
+    } else {
+        const long long j = idx - p.full_tiles;
+        it.tj = (int)(j / p.nsplit);
+        it.slice = (int)(j - (long long)it.tj * p.nsplit);
+        it.tile = p.full_tiles + it.tj;
+        it.kb_lo = (int)((long long)it.slice * num_kb / p.nsplit);
+        it.kb_hi = (int)((long long)(it.slice + 1) * num_kb / p.nsplit);
+    }
+    return it;
+}
+
 __device__ __forceinline__ float gelu_tanh_approx(float x) {
     // 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), tanh from the SFU.
     const float u = 0.7978845608028654f * fmaf(0.044715f * x * x, x, x);
@@ -200,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int mblk = (p.M + C::TM - 1) / C::TM;
     const int num_kb = (p.K + BK - 1) / BK;
     const long long total = p.var_rows ? (long long)__ldg(p.mtile_prefix + p.G) * nblk
-                                       : (long long)p.G * nblk * mblk;
+                                       : p.full_tiles + ((long long)p.G * nblk * mblk - p.full_tiles) * p.nsplit;
     const long long unit = blockIdx.x / CG, nunits = gridDim.x / CG;
 
     if (warp == 0) {
@@ -210,9 +247,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0, issued = 0, issued_phase = 0;
             bool ok = true;
             for (long long idx = unit; idx < total && ok; idx += nunits) {
-                const Tile t = decode_tile<CG>(p, idx, nblk, mblk, BN, (int)rank);
+                const Item item = decode_item(p, idx, num_kb);
+                const Tile t = decode_tile<CG>(p, item.tile, nblk, mblk, BN, (int)rank);
                 const int nb0 = t.n0 + (int)rank * C::BN_LOCAL;
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int kb = item.kb_lo; kb < item.kb_hi; ++kb) {
                     if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, wc, SITE_TC_PRODUCER)) {
                         ok = false;
                         break;
@@ -258,7 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, wc, SITE_TC_MMA_TMEM)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < num_kb; ++kb) {
+                const Item item = decode_item(p, idx, num_kb);
+                for (int kb = item.kb_lo; kb < item.kb_hi; ++kb) {
                     if (!mbar_wait(full0 + 8 * stage, phase, wc, SITE_TC_MMA_FULL)) {
                         ok = false;
                         break;
@@ -270,12 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         // advance the start address by k * 32 bytes (16-byte units)
+                        const uint32_t accum = (kb != item.kb_lo || k != 0) ? 1u : 0u;
                         if (CG == 2)
                             tc_mma_f16_pair(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
-                                            (kb | k) != 0 ? 1u : 0u);
+                                            accum);
                         else
-                            tc_mma_f16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
-                                       (kb | k) != 0 ? 1u : 0u);
+                            tc_mma_f16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc, accum);
                     }
                     if (CG == 2) tc_commit_pair_mc(empty0 + 8 * stage, 0x3);
                     else tc_commit(empty0 + 8 * stage);
@@ -315,7 +354,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t swz = (uint32_t)(lane & 7);
         int it = 0;
         for (long long idx = unit; idx < total; idx += nunits, ++it) {
-            const Tile t = decode_tile<CG>(p, idx, nblk, mblk, BN, (int)rank);
+            const Item item = decode_item(p, idx, num_kb);
+            const Tile t = decode_tile<CG>(p, item.tile, nblk, mblk, BN, (int)rank);
             const int acc = it & 1;
             const uint32_t aph = (uint32_t)(it >> 1) & 1u;
             if (!mbar_wait(tfull0 + 8 * acc, aph, wc, SITE_TC_EPILOGUE)) break;
@@ -323,6 +363,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int wrow0 = (int)t.orow0 + quarter * 32;
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
             const float* bias_g = p.bias + (long long)t.g * p.N;
+            const bool split = item.tj >= 0;
+            // this warp's 32 x HALF block of slice s of tail tile tj: [chunk][16 float4][lane]
+            const long long wsblk = split ? (((long long)item.tj * p.nsplit) * CG + rank) * kEpiWarps + ew : 0;
+            const long long wstride = (long long)CG * kEpiWarps * (32 * HALF / 4);   // float4s between slices
+            float4* wsw = split ? reinterpret_cast<float4*>(p.sk_ws) + wsblk * (32 * HALF / 4) : nullptr;
+            if (split) {
+                // dump this slice's partial sums, release the accumulator, count the arrival
+#pragma unroll 1
+                for (int c = half * HALF; c < (half + 1) * HALF; c += 64) {
+                    float v[64];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float w16[16];
+                        tmem_ld16(tbase + (uint32_t)(c + 16 * q), w16);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[16 * q + e] = w16[e];
+                    }
+                    tmem_ld_wait();
+                    float4* dst = wsw + (long long)item.slice * wstride + ((c - half * HALF) / 64) * 16 * 32 + lane;
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) __stcg(dst + q * 32, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
+                }
+                tc_fence_before();
+                if (CG == 2 && !leader) mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
+                else mbar_arrive(tempty0 + 8 * acc);
+                __threadfence();
+                __syncwarp();
+                int* cnt = p.sk_cnt + ((long long)item.tj * CG + rank) * kEpiWarps + ew;
+                int last = 0;
+                if (lane == 0) {
+                    int old;
+                    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(cnt) : "memory");
+                    last = old == p.nsplit - 1;
+                    if (last) *cnt = 0;   // ready for the next launch
+                }
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (!last) continue;
+                __threadfence();
+            }
             bool ok = true;
 #pragma unroll 1
             for (int c = half * HALF; c < (half + 1) * HALF; c += 64) {
@@ -336,15 +415,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                     else tma_load_3d(stg, &tmR, rbar, n, wrow0, t.g);
                 }
                 float v[64];
+                if (split) {
+                    // the tile's sum over its K slices, always in slice order
+                    const float4* src = wsw + ((c - half * HALF) / 64) * 16 * 32 + lane;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float w16[16];
-                    tmem_ld16(tbase + (uint32_t)(c + 16 * q), w16);
+                    for (int q = 0; q < 16; ++q) {
+                        const float4 a = __ldcg(src + q * 32);
+                        v[4 * q] = a.x;
+                        v[4 * q + 1] = a.y;
+                        v[4 * q + 2] = a.z;
+                        v[4 * q + 3] = a.w;
+                    }
+#pragma unroll 1
+                    for (int sl = 1; sl < p.nsplit; ++sl) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[16 * q + e] = w16[e];
+                        for (int q = 0; q < 16; ++q) {
+                            const float4 a = __ldcg(src + sl * wstride + q * 32);
+                            v[4 * q] += a.x;
+                            v[4 * q + 1] += a.y;
+                            v[4 * q + 2] += a.z;
+                            v[4 * q + 3] += a.w;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float w16[16];
+                        tmem_ld16(tbase + (uint32_t)(c + 16 * q), w16);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[16 * q + e] = w16[e];
+                    }
+                    tmem_ld_wait();
                 }
-                tmem_ld_wait();
-                if (c + 64 >= (half + 1) * HALF) {   // last chunk: the accumulator may be reused
+                if (!split && c + 64 >= (half + 1) * HALF) {   // last chunk: the accumulator may be reused
                     tc_fence_before();
                     if (CG == 2 && !leader) mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
                     else mbar_arrive(tempty0 + 8 * acc);
@@ -606,7 +709,26 @@ cudaError_t launch_bn(int epi, const Maps& m, const KParams& kp, int grid, cudaS
 // K = 1536..6144 (BN 256 : 192 : 128 = 1 : 0.88 : 0.74), and a damped wave
 // fill over the SMs (a partial last wave costs less than its share, since the
 // tiles of that wave see less L2 contention).
-int gemm_tc_pick_bn(int G, int M, int N, bool var_rows, int num_sms, int cg) {
+// K slices per tail tile: the last partial wave's `tail` tiles are spread
+// over the otherwise idle units, each slice keeping >= 8 K blocks.
+static int split_slices(long long tiles, int units, int num_kb) {
+    const long long tail = tiles % units;
+    if (tail == 0) return 1;
+    long long S = units / tail;
+    if (S > 8) S = 8;
+    while (S > 1 && num_kb / S < 8) --S;
+    return (int)S;
+}
+
+static cudaError_t launch_gemm_tc_nosplit(const GroupedGemm& g, DeviceErr err, uint64_t budget_ns, int num_sms,
+                                   cudaStream_t s) {
+    GroupedGemm h = g;
+    h.sk_ws = nullptr;
+    h.sk_cnt = nullptr;
+    return launch_gemm_tc(h, err, budget_ns, num_sms, s);
+}
+
+static int gemm_tc_pick_bn(int G, int M, int N, int K, bool var_rows, int num_sms, int cg, bool split) {
     const int cands[4] = {256, 192, 160, 128};
     const double mma_eff[4] = {1.0, 0.88, 0.8, 0.74};
     int best = 256;
@@ -622,6 +744,10 @@ int gemm_tc_pick_bn(int G, int M, int N, bool var_rows, int num_sms, int cg) {
             const long long tiles = (long long)G * ((M + BM * cg - 1) / (BM * cg)) * nblk;
             const long long waves = (tiles + units - 1) / units;
             wave_fill = (double)tiles / (double)(waves * units);
+            if (split) {   // the tail wave costs about 1/S of a wave
+                const int S = split_slices(tiles, (int)units, (K + BK - 1) / BK);
+                if (S > 1) wave_fill = (double)tiles / ((double)(tiles / units) * units + (double)units / S);
+            }
         }
         const double sc = col_fill * mma_eff[i] * (0.5 + 0.5 * wave_fill);
         if (sc > best_s + 1e-9) {
@@ -656,13 +782,17 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     kp.s_gstride = g.s_gstride;
     kp.s_ld = g.s_ld;
     if (g.stats && (var || g.epi != EPI_BIAS_RESID || g.N % 64)) return cudaErrorInvalidValue;
+    kp.full_tiles = 0;
+    kp.nsplit = 1;
+    kp.sk_ws = g.sk_ws;
+    kp.sk_cnt = g.sk_cnt;
     kp.err = err;
     kp.budget_ns = budget_ns;
 
     // 2-SM (256-row) tiles for dense problems with more than one 128-row block;
     // the variable-row (MoE) groups keep 128-row tiles.
     int cg = (!var && g.M > BM) ? 2 : 1;
-    int bn = gemm_tc_pick_bn(g.G, g.M, g.N, var, num_sms, cg);
+    int bn = gemm_tc_pick_bn(g.G, g.M, g.N, g.K, var, num_sms, cg, g.sk_ws && g.sk_cnt);
     // Tuning overrides (same kernel, other tile shape): RM_GEMM_CG=1|2, RM_GEMM_BN=256|192|160|128.
     if (const char* e = getenv("RM_GEMM_CG")) {
         const int v = atoi(e);
@@ -710,7 +840,18 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     if (!var) {
         const long long tiles = (long long)g.G * ((g.M + BM * cg - 1) / (BM * cg)) * ((g.N + bn - 1) / bn);
         if (tiles == 0) return cudaSuccess;
-        if (tiles < units) units = (int)tiles;
+        const int num_kb = (g.K + BK - 1) / BK;
+        const int S = (g.sk_ws && g.sk_cnt) ? split_slices(tiles, units, num_kb) : 1;
+        if (const char* e = getenv("RM_GEMM_SPLIT"))   // tuning override: 0 disables the split tail
+            if (atoi(e) == 0 && S > 1) return launch_gemm_tc_nosplit(g, err, budget_ns, num_sms, s);
+        const long long tail = S > 1 ? tiles % units : 0;
+        kp.full_tiles = tiles - tail;
+        kp.nsplit = S;
+        const long long items = kp.full_tiles + tail * S;
+        if (items < units) units = (int)items;
+        if (getenv("RM_GEMM_LOG"))
+            fprintf(stderr, "gemm_tc G=%d M=%d N=%d K=%d epi=%d cg=%d bn=%d tiles=%lld tail=%lld slices=%d grid=%d\n",
+                    g.G, g.M, g.N, g.K, g.epi, cg, bn, tiles, tail, S, units * cg);
     }
     const int grid = units * cg;
     if (var) {
@@ -725,5 +866,8 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
                                   : launch_bn<128, 2, false>(g.epi, m, kp, grid, s);
     return bn == 256 ? launch_bn<256, 1, false>(g.epi, m, kp, grid, s) : launch_bn<128, 1, false>(g.epi, m, kp, grid, s);
 }
+
+size_t gemm_tc_split_ws_bytes(int num_sms) { return (size_t)num_sms * BM * 256 * sizeof(float); }
+size_t gemm_tc_split_cnt_ints(int num_sms) { return (size_t)num_sms * kEpiWarps; }
 
 }  // namespace rm

@@ -97,7 +97,16 @@ struct GroupedGemm {
     const int* grp_cnt;
     const int* grp_off;
     const int* mtile_prefix;  // [G + 1]
+    // Optional split-K workspace for the dense tcgen05 path (both null: no
+    // split).  sk_ws holds gemm_tc_split_ws_bytes(num_sms) bytes; sk_cnt holds
+    // gemm_tc_split_cnt_ints(num_sms) ints, zero before the first use (the
+    // kernel leaves them zero when it completes).
+    float* sk_ws;
+    int* sk_cnt;
 };
+
+size_t gemm_tc_split_ws_bytes(int num_sms);
+size_t gemm_tc_split_cnt_ints(int num_sms);
 
 cudaError_t launch_gemm_tc(const GroupedGemm& p, DeviceErr err, uint64_t budget_ns, int num_sms,
                            cudaStream_t s);
