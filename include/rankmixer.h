@@ -30,8 +30,9 @@
  *     streams or threads at the same time.
  *   - Requirements: D % T == 0 (H = T heads of width D/T), D % 16 == 0 and
  *     hidden % 16 == 0 for RM_BF16 (D % 4 == 0 for RM_F32), 1 <= B <= B_max,
- *     1 <= T <= 64, n_experts <= 32, n_experts * D <= 40960.  Violations return RM_ERR_INVALID_ARG or
- *     RM_ERR_UNSUPPORTED.
+ *     1 <= T <= 64, n_experts <= 32, n_experts * D <= 40960, D <= 2048 (bf16) or 1024 (fp32), and
+ *     one sample (T * D elements, rows padded by < 128 bytes) plus T * 8 + D * 4 bytes within
+ *     226 KB of shared memory.  Violations return RM_ERR_INVALID_ARG or RM_ERR_UNSUPPORTED.
  *   - RM_F32 handles compute on CUDA cores only (no tensor cores).  RM_BF16
  *     handles run the FFN products on tcgen05 tensor cores with fp32
  *     accumulation; S, the FFN hidden and the pre-LN rows are stored bf16.

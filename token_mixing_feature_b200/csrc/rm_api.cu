@@ -308,7 +308,7 @@ rm_status rm_create(const rm_config* cfg, rm_handle** out) {
     if (c.n_experts > 0 && c.dtype != RM_BF16) return RM_ERR_UNSUPPORTED;
     if ((size_t)c.n_experts * c.D * sizeof(float) > 160 * 1024) return RM_ERR_UNSUPPORTED;   // router staged in smem
     if (c.D > rm::mix_ln_max_d(c.dtype)) return RM_ERR_UNSUPPORTED;
-    if ((size_t)c.T * c.D * esz + 8 * (size_t)c.T > 220 * 1024) return RM_ERR_UNSUPPORTED;
+    if (!rm::mix_ln_sample_fits(c.dtype, c.T, c.D)) return RM_ERR_UNSUPPORTED;   // a sample is staged in smem
 
     rm_handle* h = new (std::nothrow) rm_handle();
     if (!h) return RM_ERR_OOM;

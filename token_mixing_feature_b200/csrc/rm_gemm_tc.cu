@@ -81,7 +81,9 @@ struct Cfg {
     // Dense tiles leave the epilogue through a 32 x 64 bf16 staging buffer per
     // epilogue warp (TMA stores); variable-row tiles store rows directly.
     static constexpr int STAGING_BYTES = VAR ? 0 : kEpiWarps * 4096;
-    static constexpr int STAGES_RAW = (216 * 1024 - STAGING_BYTES) / STAGE_BYTES;
+    // as many ring stages as fit next to the staging buffers, the 1 KB
+    // alignment slack and the barriers (227 KB per CTA)
+    static constexpr int STAGES_RAW = (227 * 1024 - 1024 - 512 - STAGING_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static constexpr int TMEM_COLS = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
     static constexpr int NBARS = 2 * STAGES + 5 + kEpiWarps;

@@ -49,6 +49,7 @@ cudaError_t launch_ln_pool(int dtype, const void* X, RowStats stats, const float
 // out[row] = (mean, M2) of each row over all D columns (P = 1).
 cudaError_t launch_row_stats(int dtype, const void* X, float2* out, long long rows, int D, cudaStream_t s);
 int mix_ln_max_d(int dtype);
+bool mix_ln_sample_fits(int dtype, int T, int D);
 struct PadSplitArgs {
     const void* src[32];
     int col0[33];   // first padded column of each group; col0[n] = sum of widths

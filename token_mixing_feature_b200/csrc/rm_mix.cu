@@ -39,6 +39,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+template <int NP>
+__device__ __forceinline__ void load_pairs(const float* __restrict__ p, float2 (&o)[NP]) {
+#pragma unroll
+    for (int q = 0; q < NP / 2; ++q) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(p) + q);
+        o[2 * q] = make_float2(v.x, v.y);
+        o[2 * q + 1] = make_float2(v.z, v.w);
+    }
+}
+
 template <int N>
 __device__ __forceinline__ void load_params(const float* __restrict__ p, float (&o)[N]) {
 #pragma unroll
@@ -51,27 +61,43 @@ __device__ __forceinline__ void load_params(const float* __restrict__ p, float (
     }
 }
 
-// Two-slot ring of whole samples in shared memory (slot state kept in bit
-// masks so nothing is indexed dynamically).
+// Ring of whole samples in shared memory.  Slot s holds one sample's T rows
+// at a row stride of rs >= D elements; it fills from one cp.async.bulk copy
+// (rs == D) or T row copies issued by the lanes of warp 0, on the slot's
+// mbarrier.  Slot bookkeeping lives in bit masks in lane 0 of warp 0.
+constexpr int kMaxSlots = 4;
+
 template <typename E>
 struct SampleRing {
-    unsigned char* base;   // slot s at base + s * bytes
+    unsigned char* base;   // slot s at base + s * slot_bytes
     uint32_t bar0;         // mbarrier of slot s at bar0 + 8 * s
-    int nbuf;
-    uint32_t bytes;
+    int nslots, T, D, rs;
+    uint32_t slot_bytes;
     uint32_t outstanding;  // bit s: a copy into slot s was issued and not yet waited for
     uint32_t parity;       // bit s: parity of slot s's next completion
 
-    __device__ __forceinline__ E* buf(int slot) const { return reinterpret_cast<E*>(base + (size_t)slot * bytes); }
+    __device__ __forceinline__ E* buf(int slot) const { return reinterpret_cast<E*>(base + (size_t)slot * slot_bytes); }
     __device__ __forceinline__ uint32_t bar(int slot) const { return bar0 + 8u * (uint32_t)slot; }
 
-    __device__ void issue(int slot, const E* src) {   // thread 0 only
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(bar(slot), bytes);
-        bulk_load(smem_u32(buf(slot)), src, bytes, bar(slot));
-        outstanding |= 1u << slot;
+    // all lanes of warp 0: sample src [T, D] (contiguous) into `slot`
+    __device__ void issue(int slot, const E* src) {
+        const int lane = threadIdx.x & 31;
+        const uint32_t row_bytes = (uint32_t)(D * sizeof(E));
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar(slot), row_bytes * (uint32_t)T);
+            outstanding |= 1u << slot;
+        }
+        __syncwarp();
+        fence_proxy_async_smem();   // earlier generic accesses to the slot come first
+        const uint32_t dst = smem_u32(buf(slot));
+        if (rs == D) {   // unpadded rows: the sample is one contiguous copy
+            if (lane == 0) bulk_load(dst, src, row_bytes * (uint32_t)T, bar(slot));
+            return;
+        }
+        for (int r = lane; r < T; r += 32)
+            bulk_load(dst + (uint32_t)(r * rs) * (uint32_t)sizeof(E), src + (size_t)r * D, row_bytes, bar(slot));
     }
-    // thread 0 only: wait for the copy in `slot`; false if it ran out.
+    // thread 0 only: wait for the copies into `slot`; false if the wait ran out.
     __device__ bool wait(int slot, const WaitCtx& wc, int site) {
         const bool ok = mbar_wait(bar(slot), (parity >> slot) & 1u, wc, site, false);
         if (ok) {
@@ -82,26 +108,47 @@ struct SampleRing {
     }
     // thread 0 only: let every copy still in flight land before the CTA exits.
     __device__ void drain(const WaitCtx& wc, int site) {
-        for (int s = 0; s < nbuf; ++s)
+        for (int s = 0; s < nslots; ++s)
             if ((outstanding >> s) & 1u) mbar_wait(bar(s), (parity >> s) & 1u, wc, site, false);
     }
 };
 
-// Carves the ring and the per-row statistics out of dynamic shared memory.
+// Bytes of one ring slot (128-byte multiple).
+inline __host__ __device__ size_t slot_bytes_of(int T, int rs, size_t esz) {
+    return ((size_t)T * rs * esz + 127) / 128 * 128;
+}
+
+// Carves the ring (nslots slots), its barriers and the per-row statistics
+// (mean_s[T], rstd_s[T]) out of dynamic shared memory; returns the first
+// float after them.
 template <typename E>
-__device__ __forceinline__ SampleRing<E> make_ring(unsigned char* smem, int TD, int nbuf, float*& mean_s,
-                                                   float*& rstd_s, int T) {
-    SampleRing<E> r;
-    r.bytes = (uint32_t)((size_t)TD * sizeof(E));
-    r.nbuf = nbuf;
+__device__ __forceinline__ float* make_ring(SampleRing<E>& r, unsigned char* smem, int T, int D, int rs, int nslots,
+                                            float*& mean_s, float*& rstd_s) {
+    r.slot_bytes = (uint32_t)slot_bytes_of(T, rs, sizeof(E));
+    r.nslots = nslots;
+    r.T = T;
+    r.D = D;
+    r.rs = rs;
     r.base = smem;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)nbuf * r.bytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)nslots * r.slot_bytes);
     r.bar0 = smem_u32(bars);
     r.outstanding = 0;
     r.parity = 0;
-    mean_s = reinterpret_cast<float*>(bars + 2);
+    mean_s = reinterpret_cast<float*>(bars + kMaxSlots);
     rstd_s = mean_s + T;
-    return r;
+    return rstd_s + T;
+}
+
+// Row stride of the staged sample for the mixing kernel: D plus a pad that
+// makes consecutive token rows start (dh - D) * esz bytes apart modulo 128,
+// so the 16-byte pieces that consecutive lanes gather from consecutive token
+// rows fall in consecutive banks.  Only for whole-vector pieces.
+inline int mix_row_stride(int D, int dh, size_t esz) {
+    const long long bytes = (long long)dh * (long long)esz;
+    if (bytes % 16) return D;
+    long long pad = ((long long)(dh - D) * (long long)esz) % 128;
+    if (pad < 0) pad += 128;
+    return D + (int)(pad / (long long)esz);
 }
 
 // Merge partial statistics (count, mean, M2) b into a (Chan et al.).
@@ -179,70 +226,94 @@ __device__ __forceinline__ void load_mixed(const E* mixed, int rs, int hoff, int
     }
 }
 
-// In-place LayerNorm of the staged sample (row statistics already in shared
-// memory).  Thread i owns column vector i % nv and walks the rows of its row
-// group, so each thread loads its columns' gamma/beta once per sample.
+// Threads of the mixing kernel form `groups` row groups of nv = D/V
+// column-vector threads: thread (grp, v) owns columns [v*V, v*V + V) of rows
+// grp, grp + groups, ... in the element-wise passes, so the source offset of
+// its mixed vector and its gamma/beta stay in registers.
+constexpr int kMixMaxThreads = 384;
+
+// In-place LayerNorm of the staged sample (row statistics in shared memory),
+// in fp32 pairs: y = ((x r) - m r) gamma + beta.
 template <typename E>
-__device__ __forceinline__ void normalize_in_place(E* xs, int T, int D, const float* __restrict__ g,
-                                                   const float* __restrict__ bta, const float* mean_s,
-                                                   const float* rstd_s) {
-    constexpr int V = Vec16<E>::N;
-    const int nv = D / V;
-    const int groups = max(1, (int)blockDim.x / nv);
-    const int grp = threadIdx.x / nv;
-    if (grp >= groups) return;
-    for (int v = threadIdx.x - grp * nv; v < nv; v += (groups == 1 ? blockDim.x : nv)) {
-        const int c0 = v * V;
-        float gg[V], bb[V];
-        load_params(g + c0, gg);
-        load_params(bta + c0, bb);
-        for (int t = grp; t < T; t += groups) {
-            uint4* p = reinterpret_cast<uint4*>(xs + (size_t)t * D + c0);
-            Vec16<E> x;
-            x.u = *p;
-            const float m = mean_s[t], r = rstd_s[t];
+__device__ __forceinline__ void normalize_in_place(E* xs, int T, int rs, int c0, int grp, int groups,
+                                                   const float* __restrict__ g, const float* __restrict__ bta,
+                                                   const float* mean_s, const float* rstd_s) {
+    constexpr int NP = Vec16<E>::N / 2;
+    float2 gp[NP], bp[NP];
+    load_pairs(g + c0, gp);
+    load_pairs(bta + c0, bp);
+#pragma unroll 2
+    for (int t = grp; t < T; t += groups) {
+        uint4* p = reinterpret_cast<uint4*>(xs + (size_t)t * rs + c0);
+        float2 x[NP];
+        unpack_pairs(*p, x);
+        const float r = rstd_s[t];
+        const float2 r2 = f2(r), mr2 = f2(-mean_s[t] * r);
 #pragma unroll
-            for (int e = 0; e < V; ++e) x.e[e] = from_f<E>(fmaf((to_f(x.e[e]) - m) * r, gg[e], bb[e]));
-            *p = x.u;
-        }
+        for (int j = 0; j < NP; ++j) x[j] = f2_fma(f2_fma(x[j], r2, mr2), gp[j], bp[j]);
+        *p = pack_pairs(x);
     }
 }
 
+// Mixed vector of output row h at column c0 of a sample staged at row stride
+// rs: whole-vector pieces come from a precomputed h-independent offset
+// moff = t (rs - dh) + c0 (source token t = c0/dh), others piecewise.
+template <typename E, int MV>
+__device__ __forceinline__ void mixed_vec(const E* xs, int rs, int dh, int h, int c0, int moff, Vec16<E>& o) {
+    constexpr int V = Vec16<E>::N;
+    if constexpr (MV == V)
+        o.u = *reinterpret_cast<const uint4*>(xs + moff + h * dh);
+    else
+        load_mixed<E, MV>(xs, rs, h * dh, dh, c0, o);
+}
+
 template <typename E, bool PRE, int MV, int NV, bool ADDNORM>
-__global__ void __launch_bounds__(NV >= 16 ? 256 : 512) mix_ln_kernel(
+__global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
     const E* __restrict__ X, const float* __restrict__ pre_g, const float* __restrict__ pre_b,
     const float2* __restrict__ pstats, int P, const float* __restrict__ g1, const float* __restrict__ b1,
-    E* __restrict__ S, int B, int T, int D, float eps, int nbuf, DeviceErr err, uint64_t budget_ns) {
+    E* __restrict__ S, int B, int T, int D, float eps, int rs, int nslots, int groups, DeviceErr err,
+    uint64_t budget_ns) {
     constexpr int V = Vec16<E>::N;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int abort_flag, s_ok;
     const int TD = T * D;
     float *mean_s, *rstd_s;
-    SampleRing<E> ring = make_ring<E>(smem, TD, nbuf, mean_s, rstd_s, T);
+    SampleRing<E> ring;
+    make_ring<E>(ring, smem, T, D, rs, nslots, mean_s, rstd_s);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const WaitCtx wc{&abort_flag, budget_ns, err};
     if (tid == 0) {
-        mbar_init(ring.bar(0), 1);
-        mbar_init(ring.bar(1), 1);
+        for (int k = 0; k < nslots; ++k) mbar_init(ring.bar(k), 1);
         abort_flag = 0;
         fence_mbar_init();
-        if (blockIdx.x < B) ring.issue(0, X + (size_t)blockIdx.x * TD);
     }
     __syncthreads();
+    if (warp == 0)
+        for (int k = 0; k < nslots; ++k) {
+            const long long bk = blockIdx.x + (long long)k * gridDim.x;
+            if (bk < B) ring.issue(k, X + (size_t)bk * TD);
+        }
     const int dh = D / T;
     const int nv = D / V;
-    // Whole-vector pieces: the mixed vector i of output row h sits at
-    // moff[i] + h*dh (its source token t = c0/dh does not depend on h).
-    int moff[NV];
+    const int grp = tid / nv, c0 = (tid - grp * nv) * V;
+    const bool active = grp < groups;
+    const int moff = (c0 / dh) * (rs - dh) + c0;   // used when MV == V
+    constexpr int NP = V / 2;
+    float2 g1p[NP], b1p[NP];
+    if (ADDNORM && active) {
+        load_pairs(g1 + c0, g1p);
+        load_pairs(b1 + c0, b1p);
+    }
+    // statistics pass: lane l of a warp takes vectors l, l + 32, ... of a row
+    int moffA[NV];
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-        const int c0 = (lane + 32 * i) * V, t = c0 / dh;
-        moff[i] = t * (D - dh) + c0;
+        const int c = (lane + 32 * i) * V;
+        moffA[i] = (c / dh) * (rs - dh) + c;
     }
     int it = 0;
     for (int b = blockIdx.x; b < B; b += gridDim.x, ++it) {
-        const int cur = nbuf == 2 ? (it & 1) : 0;
-        const int nb = b + gridDim.x;
+        const int cur = it % nslots;
         if (PRE) {   // statistics of this sample's rows, from the producer's partials
             for (int t = warp; t < T; t += nw) {
                 float m, r;
@@ -253,79 +324,73 @@ __global__ void __launch_bounds__(NV >= 16 ? 256 : 512) mix_ln_kernel(
                 }
             }
         }
-        if (tid == 0) {
-            if (nbuf == 2 && nb < B) ring.issue(cur ^ 1, X + (size_t)nb * TD);
-            s_ok = ring.wait(cur, wc, SITE_MIX_LN);
-        }
+        if (tid == 0) s_ok = ring.wait(cur, wc, SITE_MIX_LN);
         __syncthreads();
         if (!s_ok) break;
         E* xs = ring.buf(cur);
         if (PRE) {
             // the previous block's LayerNorm, applied once per element, in place
-            normalize_in_place(xs, T, D, pre_g, pre_b, mean_s, rstd_s);
+            if (active) normalize_in_place(xs, T, rs, c0, grp, groups, pre_g, pre_b, mean_s, rstd_s);
             __syncthreads();
         }
         E* srow = S + (size_t)b * TD;
-        for (int h = warp; h < T; h += nw) {
-            const int hoff = h * dh;
-            if (!ADDNORM) {   // S = TokenMixing(Xh): a permutation of the staged sample
-                for (int v = lane; v < nv; v += 32) {
-                    Vec16<E> o;
-                    load_mixed<E, MV>(xs, D, hoff, dh, v * V, o);
-                    *reinterpret_cast<uint4*>(srow + (size_t)h * D + v * V) = o.u;
-                }
-                continue;
-            }
-            float z[NV][V];
-            float s = 0.f;
+        if (ADDNORM) {
+            // pass A: mean and rstd of Z[h, :] = mix[h, :] + Xh[h, :], one warp
+            // per row, sums shifted by the row's first element
+            for (int h = warp; h < T; h += nw) {
+                const float K = to_f(xs[h * dh]) + to_f(xs[(size_t)h * rs]);
+                const float2 nK = f2(-K);
+                float2 a1 = f2(0.f), a2 = f2(0.f);
 #pragma unroll
-            for (int i = 0; i < NV; ++i) {
-                const int v = lane + 32 * i;
-                if (v < nv) {
-                    const int c0 = v * V;
-                    Vec16<E> xr, xm;
-                    xr.u = *reinterpret_cast<const uint4*>(xs + (size_t)h * D + c0);
-                    if constexpr (MV == V)
-                        xm.u = *reinterpret_cast<const uint4*>(xs + moff[i] + hoff);
-                    else
-                        load_mixed<E, MV>(xs, D, hoff, dh, c0, xm);
+                for (int i = 0; i < NV; ++i) {
+                    const int v = lane + 32 * i;
+                    if (v < nv) {
+                        Vec16<E> xm;
+                        mixed_vec<E, MV>(xs, rs, dh, h, v * V, moffA[i], xm);
+                        float2 pm[NP], pr[NP];
+                        unpack_pairs(xm.u, pm);
+                        unpack_pairs(*reinterpret_cast<const uint4*>(xs + (size_t)h * rs + v * V), pr);
 #pragma unroll
-                    for (int e = 0; e < V; ++e) {
-                        z[i][e] = to_f(xm.e[e]) + to_f(xr.e[e]);
-                        s += z[i][e];
+                        for (int j = 0; j < NP; ++j) {
+                            const float2 d = f2_add(f2_add(pm[j], pr[j]), nK);
+                            a1 = f2_add(a1, d);
+                            a2 = f2_fma(d, d, a2);
+                        }
                     }
                 }
-            }
-            const float mu = warp_sum(s) / D;
-            float q = 0.f;
-#pragma unroll
-            for (int i = 0; i < NV; ++i) {
-                if (lane + 32 * i < nv) {
-#pragma unroll
-                    for (int e = 0; e < V; ++e) {
-                        const float d = z[i][e] - mu;
-                        q = fmaf(d, d, q);
-                    }
+                const float s1 = warp_sum(a1.x + a1.y);
+                const float s2 = warp_sum(a2.x + a2.y);
+                if (lane == 0) {
+                    const float m1 = s1 / D;
+                    mean_s[h] = K + m1;
+                    rstd_s[h] = rsqrtf(fmaxf(s2 / D - m1 * m1, 0.f) + eps);
                 }
             }
-            const float rstd = rsqrtf(warp_sum(q) / D + eps);
+            __syncthreads();
+        }
+        // pass B: element-wise, thread (grp, v) over rows grp, grp + groups, ...
+        if (active) {
+#pragma unroll 2
+            for (int h = grp; h < T; h += groups) {
+                Vec16<E> xm;
+                mixed_vec<E, MV>(xs, rs, dh, h, c0, moff, xm);
+                uint4 o = xm.u;   // without Add & Norm: S = TokenMixing(Xh), a permutation
+                if (ADDNORM) {
+                    float2 pm[NP], pr[NP];
+                    unpack_pairs(xm.u, pm);
+                    unpack_pairs(*reinterpret_cast<const uint4*>(xs + (size_t)h * rs + c0), pr);
+                    const float r = rstd_s[h];
+                    const float2 r2 = f2(r), mr2 = f2(-mean_s[h] * r);
 #pragma unroll
-            for (int i = 0; i < NV; ++i) {
-                const int v = lane + 32 * i;
-                if (v < nv) {
-                    const int c0 = v * V;
-                    float gg[V], bb[V];
-                    load_params(g1 + c0, gg);
-                    load_params(b1 + c0, bb);
-                    Vec16<E> o;
-#pragma unroll
-                    for (int e = 0; e < V; ++e) o.e[e] = from_f<E>(fmaf((z[i][e] - mu) * rstd, gg[e], bb[e]));
-                    *reinterpret_cast<uint4*>(srow + (size_t)h * D + c0) = o.u;
+                    for (int j = 0; j < NP; ++j) pm[j] = f2_fma(f2_fma(f2_add(pm[j], pr[j]), r2, mr2), g1p[j], b1p[j]);
+                    o = pack_pairs(pm);
                 }
+                *reinterpret_cast<uint4*>(srow + (size_t)h * D + c0) = o;
             }
         }
         __syncthreads();   // the slot and the statistics are free again
-        if (nbuf == 1 && tid == 0 && nb < B) ring.issue(0, X + (size_t)nb * TD);
+        const long long nb = b + (long long)nslots * gridDim.x;
+        if (warp == 0 && nb < B) ring.issue(cur, X + (size_t)nb * TD);
     }
     if (tid == 0) ring.drain(wc, SITE_MIX_LN);
 }
@@ -340,42 +405,45 @@ constexpr int kPoolThreads = 512;
 constexpr size_t kMaxSmemPerCta = 227 * 1024;
 
 template <typename E>
-__global__ void __launch_bounds__(kPoolThreads) ln_pool_kernel(const E* __restrict__ X,
+__global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __restrict__ X,
                                                               const float2* __restrict__ pstats, int P,
                                                               const float* __restrict__ g,
                                                               const float* __restrict__ bta,
                                                               float* __restrict__ pooled, E* __restrict__ Xout,
-                                                              int B, int T, int D, float eps, int nbuf, int groups,
-                                                              DeviceErr err, uint64_t budget_ns) {
+                                                              int B, int T, int D, float eps, int nslots,
+                                                              int groups, DeviceErr err, uint64_t budget_ns) {
     constexpr int V = Vec16<E>::N;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int abort_flag, s_ok;
     const int TD = T * D;
     float *mean_s, *rstd_s;
-    SampleRing<E> ring = make_ring<E>(smem, TD, nbuf, mean_s, rstd_s, T);
-    float* part = rstd_s + T;   // [groups][D] partial sums of (x - m_t) r_t
+    SampleRing<E> ring;
+    float* part = make_ring<E>(ring, smem, T, D, D, nslots, mean_s, rstd_s);   // [groups][D] partial sums
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const WaitCtx wc{&abort_flag, budget_ns, err};
     if (tid == 0) {
-        mbar_init(ring.bar(0), 1);
-        mbar_init(ring.bar(1), 1);
+        for (int k = 0; k < nslots; ++k) mbar_init(ring.bar(k), 1);
         abort_flag = 0;
         fence_mbar_init();
-        if (blockIdx.x < B) ring.issue(0, X + (size_t)blockIdx.x * TD);
     }
     __syncthreads();
+    if (warp == 0)
+        for (int k = 0; k < nslots; ++k) {
+            const long long bk = blockIdx.x + (long long)k * gridDim.x;
+            if (bk < B) ring.issue(k, X + (size_t)bk * TD);
+        }
     const int nv = D / V;
     const int grp = tid / nv, v = tid - grp * nv, c0 = v * V;
     const float invT = 1.0f / T;
-    float gg[V], bb[V];
+    constexpr int NP = V / 2;
+    float2 gp[NP], bp[NP];
     if (Xout && grp < groups) {
-        load_params(g + c0, gg);
-        load_params(bta + c0, bb);
+        load_pairs(g + c0, gp);
+        load_pairs(bta + c0, bp);
     }
     int it = 0;
     for (int b = blockIdx.x; b < B; b += gridDim.x, ++it) {
-        const int cur = nbuf == 2 ? (it & 1) : 0;
-        const int nb = b + gridDim.x;
+        const int cur = it % nslots;
         for (int t = warp; t < T; t += nw) {
             float m, r;
             row_mean_rstd(pstats, P, D, (long long)b * T + t, eps, m, r);
@@ -384,34 +452,35 @@ __global__ void __launch_bounds__(kPoolThreads) ln_pool_kernel(const E* __restri
                 rstd_s[t] = r;
             }
         }
-        if (tid == 0) {
-            if (nbuf == 2 && nb < B) ring.issue(cur ^ 1, X + (size_t)nb * TD);
-            s_ok = ring.wait(cur, wc, SITE_LN_POOL);
-        }
+        if (tid == 0) s_ok = ring.wait(cur, wc, SITE_LN_POOL);
         __syncthreads();
         if (!s_ok) break;
         const E* xs = ring.buf(cur);
         if (grp < groups) {
-            float acc[V];
+            float2 acc[NP];
 #pragma unroll
-            for (int e = 0; e < V; ++e) acc[e] = 0.f;
+            for (int j = 0; j < NP; ++j) acc[j] = f2(0.f);
+#pragma unroll 2
             for (int t = grp; t < T; t += groups) {
-                Vec16<E> x;
-                x.u = *reinterpret_cast<const uint4*>(xs + (size_t)t * D + c0);
-                const float mt = mean_s[t], rt = rstd_s[t];
-                Vec16<E> o;
+                float2 x[NP];
+                unpack_pairs(*reinterpret_cast<const uint4*>(xs + (size_t)t * D + c0), x);
+                const float rt = rstd_s[t];
+                const float2 r2 = f2(rt), mr2 = f2(-mean_s[t] * rt);
 #pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    const float u = (to_f(x.e[e]) - mt) * rt;
-                    acc[e] += u;
-                    if (Xout) o.e[e] = from_f<E>(fmaf(u, gg[e], bb[e]));
+                for (int j = 0; j < NP; ++j) {
+                    x[j] = f2_fma(x[j], r2, mr2);   // (x - m_t) r_t
+                    acc[j] = f2_add(acc[j], x[j]);
                 }
-                if (Xout) *reinterpret_cast<uint4*>(Xout + (size_t)b * TD + (size_t)t * D + c0) = o.u;
+                if (Xout) {
+#pragma unroll
+                    for (int j = 0; j < NP; ++j) x[j] = f2_fma(x[j], gp[j], bp[j]);
+                    *reinterpret_cast<uint4*>(Xout + (size_t)b * TD + (size_t)t * D + c0) = pack_pairs(x);
+                }
             }
             float4* dst = reinterpret_cast<float4*>(part + (size_t)grp * D + c0);
 #pragma unroll
-            for (int q = 0; q < V / 4; ++q)
-                dst[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+            for (int q = 0; q < NP / 2; ++q)
+                dst[q] = make_float4(acc[2 * q].x, acc[2 * q].y, acc[2 * q + 1].x, acc[2 * q + 1].y);
         }
         __syncthreads();
         for (int c = tid; c < D; c += blockDim.x) {
@@ -420,7 +489,8 @@ __global__ void __launch_bounds__(kPoolThreads) ln_pool_kernel(const E* __restri
             pooled[(size_t)b * D + c] = fmaf(__ldg(g + c), a * invT, __ldg(bta + c));
         }
         __syncthreads();   // slot, statistics and partials are free again
-        if (nbuf == 1 && tid == 0 && nb < B) ring.issue(0, X + (size_t)nb * TD);
+        const long long nb = b + (long long)nslots * gridDim.x;
+        if (warp == 0 && nb < B) ring.issue(cur, X + (size_t)nb * TD);
     }
     if (tid == 0) ring.drain(wc, SITE_LN_POOL);
 }
@@ -452,24 +522,47 @@ __global__ void __launch_bounds__(256) row_stats_kernel(const E* __restrict__ X,
     if (lane == 0) out[r] = make_float2(K + s1 / D, fmaxf(s2 - s1 * s1 / D, 0.f));
 }
 
-// One slot per CTA once a sample is large enough that two CTAs (each with its
-// own slot) fit an SM only that way: the co-resident CTA overlaps the loads.
-inline void ring_shape(int T, int D, size_t esz, size_t extra_floats, int* nbuf, size_t* smem) {
-    const size_t one = (size_t)T * D * esz;
-    const size_t extra = 2 * sizeof(uint64_t) + sizeof(float) * (2 * (size_t)T + extra_floats);
-    *nbuf = one <= 56 * 1024 ? 2 : 1;
-    *smem = (size_t)(*nbuf) * one + extra;
+// Ring slots (up to kMaxSlots, at least 1) and dynamic shared memory for
+// samples of T rows at row stride rs, plus extra_floats floats after the
+// per-row statistics.  Two CTAs share an SM whenever one slot each fits:
+// measured in the stack, two independent CTAs (one computes while the other
+// waits for its copy) beat one CTA with a deeper ring.
+inline void ring_shape(int T, int rs, size_t esz, size_t extra_floats, int* nslots, size_t* smem) {
+    const size_t one = slot_bytes_of(T, rs, esz);
+    const size_t fixed = 8 * kMaxSlots + sizeof(float) * (2 * (size_t)T + extra_floats);
+    const size_t full = 227 * 1024 - 1024;    // static shared memory and slack
+    const size_t half = full / 2 - 1024;
+    const size_t avail = one + fixed <= half ? half : full;
+    long long n = avail > fixed ? (long long)((avail - fixed) / one) : 0;
+    if (n > kMaxSlots) n = kMaxSlots;
+    if (n < 1) n = 1;
+    *nslots = (int)n;
+    *smem = (size_t)n * one + fixed;
+}
+
+// Row groups: the largest divisor of T (so every group gets the same rows)
+// with groups * nv <= kMixMaxThreads.
+inline int mix_groups(int T, int nv) {
+    int g = kMixMaxThreads / nv;
+    if (g > T) g = T;
+    while (g > 1 && T % g) --g;
+    return g < 1 ? 1 : g;
 }
 
 template <typename E, bool PRE, int MV, int NVV, bool ADDNORM>
 cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps, const float* g1, const float* b1,
                       E* S, int B, int T, int D, float eps, int num_sms, DeviceErr err, uint64_t budget,
                       cudaStream_t s) {
-    int nbuf;
+    constexpr int V = Vec16<E>::N;
+    const int nv = D / V;
+    if (nv < 1 || nv > kMixMaxThreads) return cudaErrorInvalidValue;
+    const int groups = mix_groups(T, nv);
+    int threads = (groups * nv + 31) / 32 * 32;
+    if (threads < 64) threads = 64;
+    const int rs = MV == V ? mix_row_stride(D, D / T, sizeof(E)) : D;
+    int nslots;
     size_t smem;
-    ring_shape(T, D, sizeof(E), 0, &nbuf, &smem);
-    // one slot: 256 threads so that two CTAs fit an SM's registers as well
-    const int threads = (NVV >= 16 || nbuf == 1 || T < 16) ? 256 : 512;
+    ring_shape(T, rs, sizeof(E), 0, &nslots, &smem);
     auto k = mix_ln_kernel<E, PRE, MV, NVV, ADDNORM>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
@@ -481,7 +574,8 @@ cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps,
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const long long g = (long long)num_sms * per_sm;
     const int grid = (int)(g < B ? g : B);
-    k<<<grid, threads, smem, s>>>(X, pg, pb, ps.part, ps.P, g1, b1, S, B, T, D, eps, nbuf, err, budget);
+    k<<<grid, threads, smem, s>>>(X, pg, pb, ps.part, ps.P, g1, b1, S, B, T, D, eps, rs, nslots, groups, err,
+                                  budget);
     return cudaGetLastError();
 }
 
@@ -525,12 +619,12 @@ cudaError_t ln_pool_go(const void* X, RowStats stats, const float* g, const floa
     if (nv < 1 || nv > kPoolThreads) return cudaErrorInvalidValue;
     int groups = kPoolThreads / nv;
     if (groups > T) groups = T;
-    int nbuf;
+    int nslots;
     size_t smem;
-    ring_shape(T, D, sizeof(E), (size_t)groups * D, &nbuf, &smem);
+    ring_shape(T, D, sizeof(E), (size_t)groups * D, &nslots, &smem);
     while (groups > 1 && smem > kMaxSmemPerCta) {   // large samples: fewer row groups
         --groups;
-        ring_shape(T, D, sizeof(E), (size_t)groups * D, &nbuf, &smem);
+        ring_shape(T, D, sizeof(E), (size_t)groups * D, &nslots, &smem);
     }
     auto k = ln_pool_kernel<E>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -544,14 +638,26 @@ cudaError_t ln_pool_go(const void* X, RowStats stats, const float* g, const floa
     const long long gr = (long long)num_sms * per_sm;
     const int grid = (int)(gr < B ? gr : B);
     k<<<grid, kPoolThreads, smem, s>>>(static_cast<const E*>(X), stats.part, stats.P, g, b, pooled, static_cast<E*>(Xout),
-                                       B, T, D, eps, nbuf, groups, err, budget);
+                                       B, T, D, eps, nslots, groups, err, budget);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-// Largest D per dtype the register-cached mix kernel supports (8 vectors per lane).
+// Largest D per dtype the mixing kernel supports (8 vectors per lane in its
+// statistics pass).
 int mix_ln_max_d(int dtype) { return 32 * 8 * (dtype == RM_BF16 ? 8 : 4); }
+
+// Whether one staged sample (padded for the mixing gather) plus the kernels'
+// per-row and pooling scratch fits a CTA's shared memory.
+bool mix_ln_sample_fits(int dtype, int T, int D) {
+    const size_t esz = dtype == RM_BF16 ? 2 : 4;
+    const int V = (int)(16 / esz);
+    const int dh = D / T;
+    const int rs = dh % V == 0 ? mix_row_stride(D, dh, esz) : D;
+    const size_t fixed = 8 * kMaxSlots + sizeof(float) * (2 * (size_t)T + (size_t)D);   // one pooling group
+    return slot_bytes_of(T, rs, esz) + fixed <= 227 * 1024 - 1024;
+}
 
 cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const float* pre_b, RowStats pre_stats,
                           const float* g1, const float* b1, void* S, int B, int T, int D, float eps, int addnorm,
