@@ -149,6 +149,25 @@ rm_status rm_stack_forward_host(rm_handle *h, const rm_block_weights *blocks,
                                 const void *X0_host, float *pooled_host, int B,
                                 rm_stream_t stream);
 
+/* Asynchronous form of rm_stack_forward_host for back-to-back batches (a
+ * serving runtime facility; the pages define no such call).  Returns after
+ * enqueueing: X0_host is copied into one of two device input buffers on the
+ * handle's own copy stream, the stack runs on `stream` once that copy and the
+ * previous read-back of the same buffer pair are done, and pooled is copied
+ * into pooled_host on a second copy stream.  So the input copy of call i+1
+ * overlaps the stack of call i.  X0_host must stay unchanged and pooled_host
+ * unread until rm_host_wait returns.  All asynchronous calls of a handle use
+ * the same `stream`, with the handle's device current.  Host buffers should
+ * be pinned (pageable memory makes the copies synchronous). */
+rm_status rm_stack_forward_host_async(rm_handle *h, const rm_block_weights *blocks,
+                                      const void *X0_host, float *pooled_host, int B,
+                                      rm_stream_t stream);
+
+/* Blocks until every rm_stack_forward_host_async call of the handle has
+ * written its pooled_host.  RM_ERR_CUDA if a copy or launch failed; device
+ * errors are read by rm_sync_status. */
+rm_status rm_host_wait(rm_handle *h);
+
 /* Pad-Split tokenisation ("淘宝闪购-爆品团精排 Scaling Up 迭代实践", section
  * 3.4: concatenate all feature-group embeddings, zero-pad, split into equal
  * tokens, no projection):

@@ -48,6 +48,30 @@ def test_small_stack_full(rm, O, name):
     st.close()
 
 
+@pytest.mark.parametrize("dtype,T,D,hidden,B,mix_addnorm", [
+    ("bf16", 5, 80, 64, 37, True),      # odd T; several samples per staged chunk, ragged last chunk
+    ("f32", 3, 24, 16, 11, True),       # odd T, fp32, dh = 8 bytes pieces
+    ("bf16", 16, 320, 256, 70, True),   # Pad-Split width: dh = 20 (8-byte pieces)
+    ("bf16", 8, 128, 64, 3, True),      # fewer samples than one chunk holds
+    ("bf16", 5, 80, 64, 37, False),     # no Add & Norm after mixing
+])
+def test_stack_small_shapes_full(rm, O, dtype, T, D, hidden, B, mix_addnorm):
+    """Two-block stacks compared in full on shapes that exercise the staged
+    chunks of several samples, odd T and the narrow-piece mixing paths."""
+    wl = synth.Workload("small", B=B, T=T, D=D, hidden=hidden, L=2, dtype=dtype, ln_params="perturbed",
+                        mix_addnorm=mix_addnorm)
+    d = synth.make_inputs(wl)
+    st = _stack(wl, d)
+    X0 = dev(d["X0"])
+    Xlast = st.empty_act(wl.B)
+    pooled = st.forward(X0, Xlast=Xlast)
+    assert rm.rm_sync_status(st.h) == rm.RM_OK
+    ref = O.stack(d["X0"], d["blocks"], want_all=False, mix_addnorm=mix_addnorm)
+    assert_close(host64(Xlast), ref["Xlast"], dtype, "Xlast")
+    assert_close(host64(pooled), ref["pooled"], dtype, "pooled")
+    st.close()
+
+
 @pytest.mark.parametrize("name,nsamp", [("rm100m", 16), ("rm1b", 8), ("moe", 16)])
 def test_bf16_stack_sampled(rm, O, name, nsamp):
     wl = synth.WORKLOADS[name]
@@ -98,6 +122,26 @@ def test_host_entry_matches_device_entry(rm):
     st.forward_host(X0h, pooled_h)
     assert rm.rm_sync_status(st.h) == rm.RM_OK
     assert torch.equal(pooled_dev.cpu(), pooled_h)
+    st.close()
+
+
+def test_host_async_pipeline_matches_device_entry(rm):
+    """Back-to-back asynchronous host calls (two device buffer sets used in
+    turn, so the third call reuses the first set): each call's pooled output
+    equals the device entry point's on the same input."""
+    wl = synth.WORKLOADS["rm100m"].with_batch(160)
+    d = synth.make_inputs(wl)
+    st = _stack(wl, d)
+    inputs = [synth.random_activations((wl.B, wl.T, wl.D), "bf16", seed=40 + i) for i in range(3)]
+    expect = [st.forward(dev(x)).cpu() for x in inputs]
+    hosts = [x.pin_memory() for x in inputs]
+    outs = [torch.full((wl.B, wl.D), float("nan"), dtype=torch.float32).pin_memory() for _ in range(3)]
+    for xh, oh in zip(hosts, outs):
+        st.forward_host_async(xh, oh)
+    st.host_wait()
+    assert rm.rm_sync_status(st.h) == rm.RM_OK
+    for i in range(3):
+        assert torch.equal(outs[i], expect[i]), f"call {i}"
     st.close()
 
 

@@ -33,6 +33,14 @@ struct rm_handle {
     void* Y;
     void* X0buf;
     float* pooledbuf;
+    // asynchronous host entry: second buffer set, copy streams and events
+    // (created on first use), slot of the next call
+    void* X0buf2;
+    float* pooledbuf2;
+    cudaStream_t h2d, d2h;
+    cudaEvent_t ev_copied[2], ev_computed[2], ev_read[2];
+    bool pipe_ready;
+    int host_slot;
     float2* ystats;   // LayerNorm partials of the pre-LN block outputs Y [B_max*T][stat_P]
     int stat_P;
     float* sk_ws;     // split-K partial tiles of the dense tcgen05 GEMMs (null for fp32 / MoE)
@@ -333,6 +341,8 @@ rm_status rm_create(const rm_config* cfg, rm_handle** out) {
         h->Y = carve<unsigned char>(base, off, BTD * esz);
         h->X0buf = carve<unsigned char>(base, off, BTD * esz);
         h->pooledbuf = carve<float>(base, off, (size_t)c.B_max * c.D * sizeof(float));
+        h->X0buf2 = carve<unsigned char>(base, off, BTD * esz);
+        h->pooledbuf2 = carve<float>(base, off, (size_t)c.B_max * c.D * sizeof(float));
         h->stat_P = (c.dtype == RM_BF16 && c.n_experts == 0 && c.D % 64 == 0) ? c.D / 64 : 1;
         h->ystats = carve<float2>(base, off, (size_t)c.B_max * c.T * h->stat_P * sizeof(float2));
         h->H = c.n_experts == 0 ? carve<unsigned char>(base, off, (size_t)c.T * c.B_max * c.hidden * esz) : nullptr;
@@ -379,6 +389,15 @@ rm_status rm_destroy(rm_handle* h) {
     cudaSetDevice(h->device);
     cudaDeviceSynchronize();
     free_events(h);
+    if (h->pipe_ready) {
+        cudaStreamDestroy(h->h2d);
+        cudaStreamDestroy(h->d2h);
+        for (int i = 0; i < 2; ++i) {
+            cudaEventDestroy(h->ev_copied[i]);
+            cudaEventDestroy(h->ev_computed[i]);
+            cudaEventDestroy(h->ev_read[i]);
+        }
+    }
     cudaError_t e = cudaFree(h->ws);
     cudaSetDevice(cur);
     delete h;
@@ -470,6 +489,56 @@ rm_status rm_stack_forward_host(rm_handle* h, const rm_block_weights* blocks, co
                         stream) != cudaSuccess)
         return RM_ERR_CUDA;
     return cuda_status(cudaStreamSynchronize(stream));
+}
+
+rm_status rm_stack_forward_host_async(rm_handle* h, const rm_block_weights* blocks, const void* X0_host,
+                                      float* pooled_host, int B, rm_stream_t stream) {
+    rm_status st = check_batch(h, B);
+    if (st != RM_OK) return st;
+    if (!blocks || !X0_host || !pooled_host) return RM_ERR_INVALID_ARG;
+    for (int l = 0; l < h->cfg.L; ++l)
+        if ((st = check_block_weights(h, &blocks[l], true)) != RM_OK) return st;
+    if (!h->pipe_ready) {
+        int cur = 0;
+        if (cudaGetDevice(&cur) != cudaSuccess || cur != h->device) return RM_ERR_INVALID_ARG;
+        bool ok = cudaStreamCreateWithFlags(&h->h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&h->d2h, cudaStreamNonBlocking) == cudaSuccess;
+        for (int i = 0; i < 2 && ok; ++i)
+            ok = cudaEventCreateWithFlags(&h->ev_copied[i], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&h->ev_computed[i], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&h->ev_read[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) return RM_ERR_CUDA;
+        h->pipe_ready = true;
+    }
+    const int s = h->host_slot;
+    h->host_slot ^= 1;
+    void* xb = s ? h->X0buf2 : h->X0buf;
+    float* pb = s ? h->pooledbuf2 : h->pooledbuf;
+    const size_t in_bytes = (size_t)B * h->cfg.T * h->cfg.D * h->esz;
+    const size_t out_bytes = (size_t)B * h->cfg.D * sizeof(float);
+    // input slot s is free once the stack that last read it has run
+    if (cudaStreamWaitEvent(h->h2d, h->ev_computed[s], 0) != cudaSuccess ||
+        cudaMemcpyAsync(xb, X0_host, in_bytes, cudaMemcpyHostToDevice, h->h2d) != cudaSuccess ||
+        cudaEventRecord(h->ev_copied[s], h->h2d) != cudaSuccess)
+        return RM_ERR_CUDA;
+    // the stack waits for its input and for the previous read-back of output slot s
+    if (cudaStreamWaitEvent(stream, h->ev_copied[s], 0) != cudaSuccess ||
+        cudaStreamWaitEvent(stream, h->ev_read[s], 0) != cudaSuccess)
+        return RM_ERR_CUDA;
+    if ((st = run_stack(h, blocks, xb, pb, nullptr, B, stream)) != RM_OK) return st;
+    if (cudaEventRecord(h->ev_computed[s], stream) != cudaSuccess ||
+        cudaStreamWaitEvent(h->d2h, h->ev_computed[s], 0) != cudaSuccess ||
+        cudaMemcpyAsync(pooled_host, pb, out_bytes, cudaMemcpyDeviceToHost, h->d2h) != cudaSuccess ||
+        cudaEventRecord(h->ev_read[s], h->d2h) != cudaSuccess)
+        return RM_ERR_CUDA;
+    return RM_OK;
+}
+
+rm_status rm_host_wait(rm_handle* h) {
+    if (!h) return RM_ERR_INVALID_ARG;
+    if (!h->pipe_ready) return RM_OK;
+    // every call's read-back is ordered after its stack, which follows its copy in
+    return cuda_status(cudaStreamSynchronize(h->d2h));
 }
 
 rm_status rm_padsplit_tokenize(rm_handle* h, const void* const* groups, const int* widths, int n_groups, void* X0,

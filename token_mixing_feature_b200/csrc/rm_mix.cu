@@ -71,7 +71,7 @@ template <typename E>
 struct SampleRing {
     unsigned char* base;   // slot s at base + s * slot_bytes
     uint32_t bar0;         // mbarrier of slot s at bar0 + 8 * s
-    int nslots, T, D, rs;
+    int nslots, D, rs;
     uint32_t slot_bytes;
     uint32_t outstanding;  // bit s: a copy into slot s was issued and not yet waited for
     uint32_t parity;       // bit s: parity of slot s's next completion
@@ -79,22 +79,22 @@ struct SampleRing {
     __device__ __forceinline__ E* buf(int slot) const { return reinterpret_cast<E*>(base + (size_t)slot * slot_bytes); }
     __device__ __forceinline__ uint32_t bar(int slot) const { return bar0 + 8u * (uint32_t)slot; }
 
-    // all lanes of warp 0: sample src [T, D] (contiguous) into `slot`
-    __device__ void issue(int slot, const E* src) {
+    // all lanes of warp 0: `rows` contiguous rows [rows, D] from src into `slot`
+    __device__ void issue(int slot, const E* src, int rows) {
         const int lane = threadIdx.x & 31;
         const uint32_t row_bytes = (uint32_t)(D * sizeof(E));
         if (lane == 0) {
-            mbar_arrive_expect_tx(bar(slot), row_bytes * (uint32_t)T);
+            mbar_arrive_expect_tx(bar(slot), row_bytes * (uint32_t)rows);
             outstanding |= 1u << slot;
         }
         __syncwarp();
         fence_proxy_async_smem();   // earlier generic accesses to the slot come first
         const uint32_t dst = smem_u32(buf(slot));
-        if (rs == D) {   // unpadded rows: the sample is one contiguous copy
-            if (lane == 0) bulk_load(dst, src, row_bytes * (uint32_t)T, bar(slot));
+        if (rs == D) {   // unpadded rows: one contiguous copy
+            if (lane == 0) bulk_load(dst, src, row_bytes * (uint32_t)rows, bar(slot));
             return;
         }
-        for (int r = lane; r < T; r += 32)
+        for (int r = lane; r < rows; r += 32)
             bulk_load(dst + (uint32_t)(r * rs) * (uint32_t)sizeof(E), src + (size_t)r * D, row_bytes, bar(slot));
     }
     // thread 0 only: wait for the copies into `slot`; false if the wait ran out.
@@ -118,15 +118,14 @@ inline __host__ __device__ size_t slot_bytes_of(int T, int rs, size_t esz) {
     return ((size_t)T * rs * esz + 127) / 128 * 128;
 }
 
-// Carves the ring (nslots slots), its barriers and the per-row statistics
-// (mean_s[T], rstd_s[T]) out of dynamic shared memory; returns the first
-// float after them.
+// Carves the ring (nslots slots of `rows` rows), its barriers and the
+// per-row statistics (mean_s[rows], rstd_s[rows]) out of dynamic shared
+// memory; returns the first float after them.
 template <typename E>
-__device__ __forceinline__ float* make_ring(SampleRing<E>& r, unsigned char* smem, int T, int D, int rs, int nslots,
-                                            float*& mean_s, float*& rstd_s) {
-    r.slot_bytes = (uint32_t)slot_bytes_of(T, rs, sizeof(E));
+__device__ __forceinline__ float* make_ring(SampleRing<E>& r, unsigned char* smem, int rows, int D, int rs,
+                                            int nslots, float*& mean_s, float*& rstd_s) {
+    r.slot_bytes = (uint32_t)slot_bytes_of(rows, rs, sizeof(E));
     r.nslots = nslots;
-    r.T = T;
     r.D = D;
     r.rs = rs;
     r.base = smem;
@@ -135,8 +134,8 @@ __device__ __forceinline__ float* make_ring(SampleRing<E>& r, unsigned char* sme
     r.outstanding = 0;
     r.parity = 0;
     mean_s = reinterpret_cast<float*>(bars + kMaxSlots);
-    rstd_s = mean_s + T;
-    return rstd_s + T;
+    rstd_s = mean_s + rows;
+    return reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(rstd_s + rows) + 15) & ~static_cast<uintptr_t>(15));
 }
 
 // Row stride of the staged sample for the mixing kernel: D plus a pad that
@@ -151,42 +150,39 @@ inline int mix_row_stride(int D, int dh, size_t esz) {
     return D + (int)(pad / (long long)esz);
 }
 
-// Merge partial statistics (count, mean, M2) b into a (Chan et al.).
-__device__ __forceinline__ void stats_merge(float& na, float& ma, float& qa, float nb, float mb, float qb) {
-    if (nb == 0.f) return;
-    if (na == 0.f) {
-        na = nb;
-        ma = mb;
-        qa = qb;
-        return;
-    }
-    const float n = na + nb, d = mb - ma, f = nb / n;
-    ma += d * f;
-    qa += qb + d * d * na * f;
-    na = n;
-}
-
-// Mean and 1/sqrt(var + eps) of row `row` from its P partials (each over
-// D/P columns); the warp merges lane-strided partials, then a fixed
-// shfl_down tree (deterministic).  Result valid in every lane.
-__device__ __forceinline__ void row_mean_rstd(const float2* __restrict__ part, int P, int D, long long row, float eps,
-                                              float& mean, float& rstd) {
-    const int lane = threadIdx.x & 31;
-    const float per = (float)D / (float)P;
-    float n = 0.f, m = 0.f, q = 0.f;
-    for (int p = lane; p < P; p += 32) {
-        const float2 v = __ldg(part + row * P + p);
-        stats_merge(n, m, q, per, v.x, v.y);
-    }
+// Mean and 1/sqrt(var + eps) of a row from its P partials (mean_p, M2_p),
+// each over the same n = D/P columns.  With equal counts the pairwise
+// (Chan et al.) combination reduces to mean = (1/P) sum_p mean_p and
+// M2 = sum_p M2_p + n sum_p (mean_p - mean)^2: two warp sums in a fixed
+// butterfly order (deterministic), no divisions; P <= 32.
+// Row statistics of rows row0 .. row0+R-1 into mean_s/rstd_s, all warps of
+// the CTA: each warp loads the partials of up to four rows before reducing
+// them, so the loads' latency is paid once per four rows.
+__device__ __forceinline__ void chunk_stats(const float2* __restrict__ part, int P, int D, long long row0, int R,
+                                            float eps, float* mean_s, float* rstd_s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const float n = (float)D / (float)P;
+    for (int r = warp; r < R; r += 4 * nw) {
+        float2 v[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float nb = __shfl_down_sync(0xffffffffu, n, o);
-        const float mb = __shfl_down_sync(0xffffffffu, m, o);
-        const float qb = __shfl_down_sync(0xffffffffu, q, o);
-        if (lane < o) stats_merge(n, m, q, nb, mb, qb);
+        for (int k = 0; k < 4; ++k) {
+            const int rr = r + k * nw;
+            v[k] = (rr < R && lane < P) ? __ldg(part + (row0 + rr) * P + lane) : make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int rr = r + k * nw;
+            if (rr < R) {   // warp-uniform
+                const float mean = warp_sum(v[k].x) / (float)P;
+                const float d = v[k].x - mean;
+                const float q = warp_sum(lane < P ? fmaf(n * d, d, v[k].y) : 0.f);
+                if (lane == 0) {
+                    mean_s[rr] = mean;
+                    rstd_s[rr] = rsqrtf(q / D + eps);
+                }
+            }
+        }
     }
-    mean = __shfl_sync(0xffffffffu, m, 0);
-    rstd = rsqrtf(__shfl_sync(0xffffffffu, q, 0) / D + eps);
 }
 
 // Columns c0 .. c0+V-1 of output row h, mixed term: source token t = c / dh,
@@ -235,7 +231,7 @@ constexpr int kMixMaxThreads = 384;
 // In-place LayerNorm of the staged sample (row statistics in shared memory),
 // in fp32 pairs: y = ((x r) - m r) gamma + beta.
 template <typename E>
-__device__ __forceinline__ void normalize_in_place(E* xs, int T, int rs, int c0, int grp, int groups,
+__device__ __forceinline__ void normalize_in_place(E* xs, int rows, int rs, int c0, int grp, int groups,
                                                    const float* __restrict__ g, const float* __restrict__ bta,
                                                    const float* mean_s, const float* rstd_s) {
     constexpr int NP = Vec16<E>::N / 2;
@@ -243,7 +239,7 @@ __device__ __forceinline__ void normalize_in_place(E* xs, int T, int rs, int c0,
     load_pairs(g + c0, gp);
     load_pairs(bta + c0, bp);
 #pragma unroll 2
-    for (int t = grp; t < T; t += groups) {
+    for (int t = grp; t < rows; t += groups) {
         uint4* p = reinterpret_cast<uint4*>(xs + (size_t)t * rs + c0);
         float2 x[NP];
         unpack_pairs(*p, x);
@@ -255,31 +251,52 @@ __device__ __forceinline__ void normalize_in_place(E* xs, int T, int rs, int c0,
     }
 }
 
-// Mixed vector of output row h at column c0 of a sample staged at row stride
-// rs: whole-vector pieces come from a precomputed h-independent offset
-// moff = t (rs - dh) + c0 (source token t = c0/dh), others piecewise.
+// Source offsets of the mixed vector at column c0 (h-independent): piece k
+// (16 bytes if MV == V, else 8 bytes at c = c0 + k*V/2) comes from token
+// t = c/dh at element t (rs - dh) + c + h*dh of the staged sample.
+struct MixOff {
+    int a, b;
+};
 template <typename E, int MV>
-__device__ __forceinline__ void mixed_vec(const E* xs, int rs, int dh, int h, int c0, int moff, Vec16<E>& o) {
+__device__ __forceinline__ MixOff mix_off(int c0, int dh, int rs) {
     constexpr int V = Vec16<E>::N;
-    if constexpr (MV == V)
-        o.u = *reinterpret_cast<const uint4*>(xs + moff + h * dh);
-    else
+    MixOff m;
+    m.a = (c0 / dh) * (rs - dh) + c0;
+    const int c1 = c0 + V / 2;
+    m.b = MV * 2 == V ? (c1 / dh) * (rs - dh) + c1 : 0;
+    return m;
+}
+
+// Mixed vector of output row h at column c0 of a sample staged at row stride
+// rs, from precomputed offsets (16- or 8-byte pieces) or element by element.
+template <typename E, int MV>
+__device__ __forceinline__ void mixed_vec(const E* xs, int rs, int dh, int h, int c0, MixOff mo, Vec16<E>& o) {
+    constexpr int V = Vec16<E>::N;
+    if constexpr (MV == V) {
+        o.u = *reinterpret_cast<const uint4*>(xs + mo.a + h * dh);
+    } else if constexpr (MV * 2 == V) {
+        const uint2 q0 = *reinterpret_cast<const uint2*>(xs + mo.a + h * dh);
+        const uint2 q1 = *reinterpret_cast<const uint2*>(xs + mo.b + h * dh);
+        o.u = make_uint4(q0.x, q0.y, q1.x, q1.y);
+    } else {
         load_mixed<E, MV>(xs, rs, h * dh, dh, c0, o);
+    }
 }
 
 template <typename E, bool PRE, int MV, int NV, bool ADDNORM>
 __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
     const E* __restrict__ X, const float* __restrict__ pre_g, const float* __restrict__ pre_b,
     const float2* __restrict__ pstats, int P, const float* __restrict__ g1, const float* __restrict__ b1,
-    E* __restrict__ S, int B, int T, int D, float eps, int rs, int nslots, int groups, DeviceErr err,
+    E* __restrict__ S, int B, int T, int D, float eps, int rs, int spb, int nslots, int groups, DeviceErr err,
     uint64_t budget_ns) {
     constexpr int V = Vec16<E>::N;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int abort_flag, s_ok;
     const int TD = T * D;
+    const int nchunks = (B + spb - 1) / spb;   // chunk c: samples [c*spb, c*spb + spb) in one slot
     float *mean_s, *rstd_s;
     SampleRing<E> ring;
-    make_ring<E>(ring, smem, T, D, rs, nslots, mean_s, rstd_s);
+    make_ring<E>(ring, smem, spb * T, D, rs, nslots, mean_s, rstd_s);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const WaitCtx wc{&abort_flag, budget_ns, err};
     if (tid == 0) {
@@ -288,16 +305,17 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
         fence_mbar_init();
     }
     __syncthreads();
+    auto chunk_rows = [&](long long c) { return (int)(min((long long)spb, B - c * spb) * T); };
     if (warp == 0)
         for (int k = 0; k < nslots; ++k) {
-            const long long bk = blockIdx.x + (long long)k * gridDim.x;
-            if (bk < B) ring.issue(k, X + (size_t)bk * TD);
+            const long long ck = blockIdx.x + (long long)k * gridDim.x;
+            if (ck < nchunks) ring.issue(k, X + (size_t)ck * spb * TD, chunk_rows(ck));
         }
     const int dh = D / T;
     const int nv = D / V;
     const int grp = tid / nv, c0 = (tid - grp * nv) * V;
     const bool active = grp < groups;
-    const int moff = (c0 / dh) * (rs - dh) + c0;   // used when MV == V
+    const MixOff moff = mix_off<E, MV>(c0, dh, rs);
     constexpr int NP = V / 2;
     float2 g1p[NP], b1p[NP];
     if (ADDNORM && active) {
@@ -305,40 +323,33 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
         load_pairs(b1 + c0, b1p);
     }
     // statistics pass: lane l of a warp takes vectors l, l + 32, ... of a row
-    int moffA[NV];
+    MixOff moffA[NV];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const int c = (lane + 32 * i) * V;
-        moffA[i] = (c / dh) * (rs - dh) + c;
-    }
+    for (int i = 0; i < NV; ++i) moffA[i] = mix_off<E, MV>((lane + 32 * i) * V, dh, rs);
+    const int sstride = T * rs;   // elements between the staged samples of a chunk
     int it = 0;
-    for (int b = blockIdx.x; b < B; b += gridDim.x, ++it) {
+    for (long long c = blockIdx.x; c < nchunks; c += gridDim.x, ++it) {
         const int cur = it % nslots;
-        if (PRE) {   // statistics of this sample's rows, from the producer's partials
-            for (int t = warp; t < T; t += nw) {
-                float m, r;
-                row_mean_rstd(pstats, P, D, (long long)b * T + t, eps, m, r);
-                if (lane == 0) {
-                    mean_s[t] = m;
-                    rstd_s[t] = r;
-                }
-            }
-        }
+        const int R = chunk_rows(c);
+        const long long row0 = c * spb * T;   // global row of the chunk's first row
+        if (PRE) chunk_stats(pstats, P, D, row0, R, eps, mean_s, rstd_s);   // from the producer's partials
         if (tid == 0) s_ok = ring.wait(cur, wc, SITE_MIX_LN);
         __syncthreads();
         if (!s_ok) break;
         E* xs = ring.buf(cur);
         if (PRE) {
             // the previous block's LayerNorm, applied once per element, in place
-            if (active) normalize_in_place(xs, T, rs, c0, grp, groups, pre_g, pre_b, mean_s, rstd_s);
+            if (active) normalize_in_place(xs, R, rs, c0, grp, groups, pre_g, pre_b, mean_s, rstd_s);
             __syncthreads();
         }
-        E* srow = S + (size_t)b * TD;
+        E* srow = S + (size_t)row0 * D;
         if (ADDNORM) {
             // pass A: mean and rstd of Z[h, :] = mix[h, :] + Xh[h, :], one warp
             // per row, sums shifted by the row's first element
-            for (int h = warp; h < T; h += nw) {
-                const float K = to_f(xs[h * dh]) + to_f(xs[(size_t)h * rs]);
+            for (int r = warp; r < R; r += nw) {
+                const int s = r / T, h = r - s * T;
+                const E* xsm = xs + (size_t)s * sstride;   // this row's sample
+                const float K = to_f(xsm[h * dh]) + to_f(xs[(size_t)r * rs]);
                 const float2 nK = f2(-K);
                 float2 a1 = f2(0.f), a2 = f2(0.f);
 #pragma unroll
@@ -346,10 +357,10 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
                     const int v = lane + 32 * i;
                     if (v < nv) {
                         Vec16<E> xm;
-                        mixed_vec<E, MV>(xs, rs, dh, h, v * V, moffA[i], xm);
+                        mixed_vec<E, MV>(xsm, rs, dh, h, v * V, moffA[i], xm);
                         float2 pm[NP], pr[NP];
                         unpack_pairs(xm.u, pm);
-                        unpack_pairs(*reinterpret_cast<const uint4*>(xs + (size_t)h * rs + v * V), pr);
+                        unpack_pairs(*reinterpret_cast<const uint4*>(xs + (size_t)r * rs + v * V), pr);
 #pragma unroll
                         for (int j = 0; j < NP; ++j) {
                             const float2 d = f2_add(f2_add(pm[j], pr[j]), nK);
@@ -362,63 +373,73 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
                 const float s2 = warp_sum(a2.x + a2.y);
                 if (lane == 0) {
                     const float m1 = s1 / D;
-                    mean_s[h] = K + m1;
-                    rstd_s[h] = rsqrtf(fmaxf(s2 / D - m1 * m1, 0.f) + eps);
+                    mean_s[r] = K + m1;
+                    rstd_s[r] = rsqrtf(fmaxf(s2 / D - m1 * m1, 0.f) + eps);
                 }
             }
             __syncthreads();
         }
         // pass B: element-wise, thread (grp, v) over rows grp, grp + groups, ...
+        // (groups divides T, so h wraps to the next sample exactly)
         if (active) {
+            int h = grp;
+            const E* xsm = xs;
 #pragma unroll 2
-            for (int h = grp; h < T; h += groups) {
+            for (int r = grp; r < R; r += groups) {
                 Vec16<E> xm;
-                mixed_vec<E, MV>(xs, rs, dh, h, c0, moff, xm);
+                mixed_vec<E, MV>(xsm, rs, dh, h, c0, moff, xm);
                 uint4 o = xm.u;   // without Add & Norm: S = TokenMixing(Xh), a permutation
                 if (ADDNORM) {
                     float2 pm[NP], pr[NP];
                     unpack_pairs(xm.u, pm);
-                    unpack_pairs(*reinterpret_cast<const uint4*>(xs + (size_t)h * rs + c0), pr);
-                    const float r = rstd_s[h];
-                    const float2 r2 = f2(r), mr2 = f2(-mean_s[h] * r);
+                    unpack_pairs(*reinterpret_cast<const uint4*>(xs + (size_t)r * rs + c0), pr);
+                    const float rr = rstd_s[r];
+                    const float2 r2 = f2(rr), mr2 = f2(-mean_s[r] * rr);
 #pragma unroll
                     for (int j = 0; j < NP; ++j) pm[j] = f2_fma(f2_fma(f2_add(pm[j], pr[j]), r2, mr2), g1p[j], b1p[j]);
                     o = pack_pairs(pm);
                 }
-                *reinterpret_cast<uint4*>(srow + (size_t)h * D + c0) = o;
+                *reinterpret_cast<uint4*>(srow + (size_t)r * D + c0) = o;
+                h += groups;
+                if (h >= T) {
+                    h -= T;
+                    xsm += sstride;
+                }
             }
         }
         __syncthreads();   // the slot and the statistics are free again
-        const long long nb = b + (long long)nslots * gridDim.x;
-        if (warp == 0 && nb < B) ring.issue(cur, X + (size_t)nb * TD);
+        const long long nc = c + (long long)nslots * gridDim.x;
+        if (warp == 0 && nc < nchunks) ring.issue(cur, X + (size_t)nc * spb * TD, chunk_rows(nc));
     }
     if (tid == 0) ring.drain(wc, SITE_MIX_LN);
 }
 
 // pooled[b, c] = gamma[c] * (1/T) sum_t (x[t, c] - m_t) r_t + beta[c]; Xout
-// (optional) receives LN(x).  Persistent CTAs stage whole samples in the same
-// shared-memory ring as mix_ln (one bulk copy per sample: far more bytes in
-// flight than per-thread loads).  The threads form `groups` row groups of
-// nv = D/V column-vector threads; group q sums rows q, q+groups, ... and the
-// groups' partial sums are added in ascending q (deterministic).
+// (optional) receives LN(x).  Persistent CTAs stream chunks of spb whole
+// samples through the shared-memory ring.  The threads form `groups` row
+// groups (groups divides T) of nv = D/V column-vector threads; group q sums
+// rows q, q + groups, ... of each sample, and the groups' partial sums are
+// added in ascending q (deterministic).
 constexpr int kPoolThreads = 512;
 constexpr size_t kMaxSmemPerCta = 227 * 1024;
 
 template <typename E>
 __global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __restrict__ X,
-                                                              const float2* __restrict__ pstats, int P,
-                                                              const float* __restrict__ g,
-                                                              const float* __restrict__ bta,
-                                                              float* __restrict__ pooled, E* __restrict__ Xout,
-                                                              int B, int T, int D, float eps, int nslots,
-                                                              int groups, DeviceErr err, uint64_t budget_ns) {
+                                                                 const float2* __restrict__ pstats, int P,
+                                                                 const float* __restrict__ g,
+                                                                 const float* __restrict__ bta,
+                                                                 float* __restrict__ pooled, E* __restrict__ Xout,
+                                                                 int B, int T, int D, float eps, int spb, int nslots,
+                                                                 int groups, DeviceErr err, uint64_t budget_ns) {
     constexpr int V = Vec16<E>::N;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int abort_flag, s_ok;
     const int TD = T * D;
+    const int nchunks = (B + spb - 1) / spb;
     float *mean_s, *rstd_s;
     SampleRing<E> ring;
-    float* part = make_ring<E>(ring, smem, T, D, D, nslots, mean_s, rstd_s);   // [groups][D] partial sums
+    // partial sums [spb][groups][D] after the ring and the statistics
+    float* part = make_ring<E>(ring, smem, spb * T, D, D, nslots, mean_s, rstd_s);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const WaitCtx wc{&abort_flag, budget_ns, err};
     if (tid == 0) {
@@ -427,13 +448,14 @@ __global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __res
         fence_mbar_init();
     }
     __syncthreads();
+    auto chunk_samples = [&](long long c) { return (int)min((long long)spb, B - c * spb); };
     if (warp == 0)
         for (int k = 0; k < nslots; ++k) {
-            const long long bk = blockIdx.x + (long long)k * gridDim.x;
-            if (bk < B) ring.issue(k, X + (size_t)bk * TD);
+            const long long ck = blockIdx.x + (long long)k * gridDim.x;
+            if (ck < nchunks) ring.issue(k, X + (size_t)ck * spb * TD, chunk_samples(ck) * T);
         }
     const int nv = D / V;
-    const int grp = tid / nv, v = tid - grp * nv, c0 = v * V;
+    const int grp = tid / nv, c0 = (tid - grp * nv) * V;
     const float invT = 1.0f / T;
     constexpr int NP = V / 2;
     float2 gp[NP], bp[NP];
@@ -442,55 +464,56 @@ __global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __res
         load_pairs(bta + c0, bp);
     }
     int it = 0;
-    for (int b = blockIdx.x; b < B; b += gridDim.x, ++it) {
+    for (long long c = blockIdx.x; c < nchunks; c += gridDim.x, ++it) {
         const int cur = it % nslots;
-        for (int t = warp; t < T; t += nw) {
-            float m, r;
-            row_mean_rstd(pstats, P, D, (long long)b * T + t, eps, m, r);
-            if (lane == 0) {
-                mean_s[t] = m;
-                rstd_s[t] = r;
-            }
-        }
+        const int ns = chunk_samples(c);
+        const int R = ns * T;
+        const long long row0 = c * spb * T;
+        chunk_stats(pstats, P, D, row0, R, eps, mean_s, rstd_s);
         if (tid == 0) s_ok = ring.wait(cur, wc, SITE_LN_POOL);
         __syncthreads();
         if (!s_ok) break;
         const E* xs = ring.buf(cur);
         if (grp < groups) {
-            float2 acc[NP];
+            for (int sm = 0; sm < ns; ++sm) {
+                float2 acc[NP];
 #pragma unroll
-            for (int j = 0; j < NP; ++j) acc[j] = f2(0.f);
+                for (int j = 0; j < NP; ++j) acc[j] = f2(0.f);
 #pragma unroll 2
-            for (int t = grp; t < T; t += groups) {
-                float2 x[NP];
-                unpack_pairs(*reinterpret_cast<const uint4*>(xs + (size_t)t * D + c0), x);
-                const float rt = rstd_s[t];
-                const float2 r2 = f2(rt), mr2 = f2(-mean_s[t] * rt);
+                for (int h = grp; h < T; h += groups) {
+                    const int r = sm * T + h;
+                    float2 x[NP];
+                    unpack_pairs(*reinterpret_cast<const uint4*>(xs + (size_t)r * D + c0), x);
+                    const float rt = rstd_s[r];
+                    const float2 r2 = f2(rt), mr2 = f2(-mean_s[r] * rt);
 #pragma unroll
-                for (int j = 0; j < NP; ++j) {
-                    x[j] = f2_fma(x[j], r2, mr2);   // (x - m_t) r_t
-                    acc[j] = f2_add(acc[j], x[j]);
-                }
-                if (Xout) {
+                    for (int j = 0; j < NP; ++j) {
+                        x[j] = f2_fma(x[j], r2, mr2);   // (x - m_t) r_t
+                        acc[j] = f2_add(acc[j], x[j]);
+                    }
+                    if (Xout) {
 #pragma unroll
-                    for (int j = 0; j < NP; ++j) x[j] = f2_fma(x[j], gp[j], bp[j]);
-                    *reinterpret_cast<uint4*>(Xout + (size_t)b * TD + (size_t)t * D + c0) = pack_pairs(x);
+                        for (int j = 0; j < NP; ++j) x[j] = f2_fma(x[j], gp[j], bp[j]);
+                        *reinterpret_cast<uint4*>(Xout + (size_t)(row0 + r) * D + c0) = pack_pairs(x);
+                    }
                 }
+                float4* dst = reinterpret_cast<float4*>(part + ((size_t)sm * groups + grp) * D + c0);
+#pragma unroll
+                for (int q = 0; q < NP / 2; ++q)
+                    dst[q] = make_float4(acc[2 * q].x, acc[2 * q].y, acc[2 * q + 1].x, acc[2 * q + 1].y);
             }
-            float4* dst = reinterpret_cast<float4*>(part + (size_t)grp * D + c0);
-#pragma unroll
-            for (int q = 0; q < NP / 2; ++q)
-                dst[q] = make_float4(acc[2 * q].x, acc[2 * q].y, acc[2 * q + 1].x, acc[2 * q + 1].y);
         }
         __syncthreads();
-        for (int c = tid; c < D; c += blockDim.x) {
-            float a = part[c];
-            for (int q = 1; q < groups; ++q) a += part[(size_t)q * D + c];
-            pooled[(size_t)b * D + c] = fmaf(__ldg(g + c), a * invT, __ldg(bta + c));
+        for (int i = tid; i < ns * D; i += blockDim.x) {
+            const int sm = i / D, cc = i - sm * D;
+            const float* ps = part + (size_t)sm * groups * D + cc;
+            float a = ps[0];
+            for (int q = 1; q < groups; ++q) a += ps[(size_t)q * D];
+            pooled[(size_t)(c * spb + sm) * D + cc] = fmaf(__ldg(g + cc), a * invT, __ldg(bta + cc));
         }
         __syncthreads();   // slot, statistics and partials are free again
-        const long long nb = b + (long long)nslots * gridDim.x;
-        if (warp == 0 && nb < B) ring.issue(cur, X + (size_t)nb * TD);
+        const long long nc = c + (long long)nslots * gridDim.x;
+        if (warp == 0 && nc < nchunks) ring.issue(cur, X + (size_t)nc * spb * TD, chunk_samples(nc) * T);
     }
     if (tid == 0) ring.drain(wc, SITE_LN_POOL);
 }
@@ -522,14 +545,24 @@ __global__ void __launch_bounds__(256) row_stats_kernel(const E* __restrict__ X,
     if (lane == 0) out[r] = make_float2(K + s1 / D, fmaxf(s2 - s1 * s1 / D, 0.f));
 }
 
+// Samples per ring slot: small samples travel in chunks of about 32 KB, so
+// the per-chunk synchronisation and statistics are amortised.
+constexpr size_t kChunkTargetBytes = 32 * 1024;
+inline int samples_per_chunk(int T, int rs, size_t esz, int B) {
+    const size_t one = (size_t)T * rs * esz;
+    long long spb = one >= kChunkTargetBytes ? 1 : (long long)(kChunkTargetBytes / one);
+    if (spb > B) spb = B;
+    return spb < 1 ? 1 : (int)spb;
+}
+
 // Ring slots (up to kMaxSlots, at least 1) and dynamic shared memory for
-// samples of T rows at row stride rs, plus extra_floats floats after the
+// chunks of `rows` rows at row stride rs, plus extra_floats floats after the
 // per-row statistics.  Two CTAs share an SM whenever one slot each fits:
 // measured in the stack, two independent CTAs (one computes while the other
 // waits for its copy) beat one CTA with a deeper ring.
-inline void ring_shape(int T, int rs, size_t esz, size_t extra_floats, int* nslots, size_t* smem) {
-    const size_t one = slot_bytes_of(T, rs, esz);
-    const size_t fixed = 8 * kMaxSlots + sizeof(float) * (2 * (size_t)T + extra_floats);
+inline void ring_shape(int rows, int rs, size_t esz, size_t extra_floats, int* nslots, size_t* smem) {
+    const size_t one = slot_bytes_of(rows, rs, esz);
+    const size_t fixed = 8 * kMaxSlots + sizeof(float) * (2 * (size_t)rows + extra_floats) + 16;
     const size_t full = 227 * 1024 - 1024;    // static shared memory and slack
     const size_t half = full / 2 - 1024;
     const size_t avail = one + fixed <= half ? half : full;
@@ -541,13 +574,14 @@ inline void ring_shape(int T, int rs, size_t esz, size_t extra_floats, int* nslo
 }
 
 // Row groups: the largest divisor of T (so every group gets the same rows)
-// with groups * nv <= kMixMaxThreads.
-inline int mix_groups(int T, int nv) {
-    int g = kMixMaxThreads / nv;
+// with groups * nv <= cap threads.
+inline int mix_groups_cap(int T, int nv, int cap) {
+    int g = cap / nv;
     if (g > T) g = T;
     while (g > 1 && T % g) --g;
     return g < 1 ? 1 : g;
 }
+inline int mix_groups(int T, int nv) { return mix_groups_cap(T, nv, kMixMaxThreads); }
 
 template <typename E, bool PRE, int MV, int NVV, bool ADDNORM>
 cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps, const float* g1, const float* b1,
@@ -560,9 +594,10 @@ cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps,
     int threads = (groups * nv + 31) / 32 * 32;
     if (threads < 64) threads = 64;
     const int rs = MV == V ? mix_row_stride(D, D / T, sizeof(E)) : D;
+    const int spb = samples_per_chunk(T, rs, sizeof(E), B);
     int nslots;
     size_t smem;
-    ring_shape(T, rs, sizeof(E), 0, &nslots, &smem);
+    ring_shape(spb * T, rs, sizeof(E), 0, &nslots, &smem);
     auto k = mix_ln_kernel<E, PRE, MV, NVV, ADDNORM>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
@@ -572,9 +607,10 @@ cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps,
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const long long nchunks = (B + spb - 1) / spb;
     const long long g = (long long)num_sms * per_sm;
-    const int grid = (int)(g < B ? g : B);
-    k<<<grid, threads, smem, s>>>(X, pg, pb, ps.part, ps.P, g1, b1, S, B, T, D, eps, rs, nslots, groups, err,
+    const int grid = (int)(g < nchunks ? g : nchunks);
+    k<<<grid, threads, smem, s>>>(X, pg, pb, ps.part, ps.P, g1, b1, S, B, T, D, eps, rs, spb, nslots, groups, err,
                                   budget);
     return cudaGetLastError();
 }
@@ -617,14 +653,16 @@ cudaError_t ln_pool_go(const void* X, RowStats stats, const float* g, const floa
     constexpr int V = Vec16<E>::N;
     const int nv = D / V;
     if (nv < 1 || nv > kPoolThreads) return cudaErrorInvalidValue;
-    int groups = kPoolThreads / nv;
-    if (groups > T) groups = T;
+    int groups = mix_groups_cap(T, nv, kPoolThreads);   // divides T
+    // chunk partials [spb][groups][D] stay within 32 KB
+    int spb = samples_per_chunk(T, D, sizeof(E), B);
+    while (spb > 1 && (size_t)spb * groups * D * sizeof(float) > kChunkTargetBytes) --spb;
     int nslots;
     size_t smem;
-    ring_shape(T, D, sizeof(E), (size_t)groups * D, &nslots, &smem);
-    while (groups > 1 && smem > kMaxSmemPerCta) {   // large samples: fewer row groups
-        --groups;
-        ring_shape(T, D, sizeof(E), (size_t)groups * D, &nslots, &smem);
+    ring_shape(spb * T, D, sizeof(E), (size_t)spb * groups * D, &nslots, &smem);
+    while (groups > 1 && smem > kMaxSmemPerCta - 1024) {   // large samples: fewer row groups
+        groups = mix_groups_cap(T, nv, groups * nv - 1);
+        ring_shape(spb * T, D, sizeof(E), (size_t)spb * groups * D, &nslots, &smem);
     }
     auto k = ln_pool_kernel<E>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -635,10 +673,11 @@ cudaError_t ln_pool_go(const void* X, RowStats stats, const float* g, const floa
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kPoolThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const long long nchunks = (B + spb - 1) / spb;
     const long long gr = (long long)num_sms * per_sm;
-    const int grid = (int)(gr < B ? gr : B);
+    const int grid = (int)(gr < nchunks ? gr : nchunks);
     k<<<grid, kPoolThreads, smem, s>>>(static_cast<const E*>(X), stats.part, stats.P, g, b, pooled, static_cast<E*>(Xout),
-                                       B, T, D, eps, nslots, groups, err, budget);
+                                       B, T, D, eps, spb, nslots, groups, err, budget);
     return cudaGetLastError();
 }
 
@@ -662,7 +701,7 @@ bool mix_ln_sample_fits(int dtype, int T, int D) {
 cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const float* pre_b, RowStats pre_stats,
                           const float* g1, const float* b1, void* S, int B, int T, int D, float eps, int addnorm,
                           int num_sms, DeviceErr err, uint64_t budget_ns, cudaStream_t s) {
-    if (pre_g && !pre_stats.part) return cudaErrorInvalidValue;
+    if (pre_g && (!pre_stats.part || pre_stats.P < 1 || pre_stats.P > 32)) return cudaErrorInvalidValue;
     if (dtype == RM_BF16)
         return mix_ln_typed<__nv_bfloat16>(X, pre_g, pre_b, pre_stats, g1, b1, S, B, T, D, eps, addnorm, num_sms,
                                            err, budget_ns, s);
@@ -673,6 +712,7 @@ cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const fl
 cudaError_t launch_ln_pool(int dtype, const void* X, RowStats stats, const float* g, const float* b, float* pooled,
                            void* Xout, int B, int T, int D, float eps, int num_sms, DeviceErr err, uint64_t budget_ns,
                            cudaStream_t s) {
+    if (!stats.part || stats.P < 1 || stats.P > 32) return cudaErrorInvalidValue;
     if (dtype == RM_BF16)
         return ln_pool_go<__nv_bfloat16>(X, stats, g, b, pooled, Xout, B, T, D, eps, num_sms, err, budget_ns, s);
     return ln_pool_go<float>(X, stats, g, b, pooled, Xout, B, T, D, eps, num_sms, err, budget_ns, s);

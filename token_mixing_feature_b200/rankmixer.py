@@ -26,6 +26,7 @@ EXPORTED = (
     "rm_stack_forward_host", "rm_padsplit_tokenize", "rm_head_forward", "rm_sync_status",
     "rm_last_error_site", "rm_set_wait_budget", "rm_selftest_wait_timeout", "rm_status_string",
     "rm_profile_begin", "rm_profile_end", "rm_kernel_name", "rm_pffn_forward_static",
+    "rm_stack_forward_host_async", "rm_host_wait",
 )
 RM_STATIC_SCRATCH_BYTES = 16 << 20
 RM_K_COUNT = 11
@@ -65,6 +66,8 @@ def _load() -> ctypes.CDLL:
         "rm_block_forward": (st, [vp, ctypes.POINTER(rm_block_weights), vp, vp, ci, vp]),
         "rm_stack_forward": (st, [vp, ctypes.POINTER(rm_block_weights), vp, vp, vp, ci, vp]),
         "rm_stack_forward_host": (st, [vp, ctypes.POINTER(rm_block_weights), vp, vp, ci, vp]),
+        "rm_stack_forward_host_async": (st, [vp, ctypes.POINTER(rm_block_weights), vp, vp, ci, vp]),
+        "rm_host_wait": (st, [vp]),
         "rm_padsplit_tokenize": (st, [vp, ctypes.POINTER(vp), ctypes.POINTER(ci), ci, vp, ci, vp]),
         "rm_head_forward": (st, [vp, vp, vp, vp, vp, ci, vp]),
         "rm_sync_status": (st, [vp, vp]),
@@ -210,6 +213,18 @@ def rm_stack_forward_host(h: Handle, blocks: Sequence[Dict], X0_host, pooled_hos
     arr = _block_array(blocks)
     _check(_lib.rm_stack_forward_host(h.ptr, arr, _ptr(X0_host), _ptr(pooled_host), B,
                                       _stream(stream)), "rm_stack_forward_host")
+
+
+def rm_stack_forward_host_async(h: Handle, blocks: Sequence[Dict], X0_host, pooled_host, B: int,
+                                stream=None) -> None:
+    """Enqueue one host-buffer stack call; results valid after rm_host_wait."""
+    arr = _block_array(blocks)
+    _check(_lib.rm_stack_forward_host_async(h.ptr, arr, _ptr(X0_host), _ptr(pooled_host), B,
+                                            _stream(stream)), "rm_stack_forward_host_async")
+
+
+def rm_host_wait(h: Handle) -> None:
+    _check(_lib.rm_host_wait(h.ptr), "rm_host_wait")
 
 
 def rm_padsplit_tokenize(h: Handle, groups: Sequence, X0, B: int, stream=None) -> None:

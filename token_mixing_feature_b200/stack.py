@@ -50,6 +50,13 @@ class RankMixerStack:
         rm.rm_stack_forward_host(self.h, self.blocks, X0_host, pooled_host, X0_host.shape[0], stream)
         return pooled_host
 
+    def forward_host_async(self, X0_host: torch.Tensor, pooled_host: torch.Tensor, stream=None) -> None:
+        """Enqueue one host-buffer call (input copy overlaps the previous call's stack)."""
+        rm.rm_stack_forward_host_async(self.h, self.blocks, X0_host, pooled_host, X0_host.shape[0], stream)
+
+    def host_wait(self) -> None:
+        rm.rm_host_wait(self.h)
+
     def block(self, l: int, X: torch.Tensor, Xout: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         Xout = self.empty_act(X.shape[0]) if Xout is None else Xout
         rm.rm_block_forward(self.h, self.blocks[l], X, Xout, X.shape[0], stream)
