@@ -170,12 +170,16 @@ __device__ __forceinline__ Item decode_item(const KParams& p, long long idx, int
     return it;
 }
 
-__device__ __forceinline__ float gelu_tanh_approx(float x) {
-    // 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), tanh from the SFU.
-    const float u = 0.7978845608028654f * fmaf(0.044715f * x * x, x, x);
-    float th;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(u));
-    return 0.5f * x * (1.0f + th);
+// GELU (tanh form) of a pair: 0.5 x (1 + tanh(u)), u = sqrt(2/pi) x (1 + 0.044715 x^2),
+// written as h + h tanh(u) with h = x/2; paired fp32 arithmetic, tanh from the SFU.
+__device__ __forceinline__ float2 gelu_tanh_pair(float2 x) {
+    const float2 p = f2_fma(f2_mul(x, x), f2(0.7978845608028654f * 0.044715f), f2(0.7978845608028654f));
+    const float2 u = f2_mul(x, p);
+    float2 th;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(u.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(u.y));
+    const float2 hx = f2_mul(x, f2(0.5f));
+    return f2_fma(hx, th, hx);
 }
 
 template <int BN, int EPI, int CG, bool VAR>
@@ -462,10 +466,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int r = 0; r < 4; ++r) {
                             const float4 bb = __ldg(b4 + r);
-                            v[16 * q + 4 * r + 0] += bb.x;
-                            v[16 * q + 4 * r + 1] += bb.y;
-                            v[16 * q + 4 * r + 2] += bb.z;
-                            v[16 * q + 4 * r + 3] += bb.w;
+                            const int e = 16 * q + 4 * r;
+                            const float2 lo = f2_add(make_float2(v[e], v[e + 1]), make_float2(bb.x, bb.y));
+                            const float2 hi = f2_add(make_float2(v[e + 2], v[e + 3]), make_float2(bb.z, bb.w));
+                            v[e] = lo.x;
+                            v[e + 1] = lo.y;
+                            v[e + 2] = hi.x;
+                            v[e + 3] = hi.y;
                         }
                     }
                 }
@@ -474,7 +481,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < 64; ++e) v[e] = fmaxf(v[e], 0.0f);
                 } else if (EPI == EPI_GELU_TANH) {
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) v[e] = gelu_tanh_approx(v[e]);
+                    for (int e = 0; e < 64; e += 2) {
+                        const float2 y = gelu_tanh_pair(make_float2(v[e], v[e + 1]));
+                        v[e] = y.x;
+                        v[e + 1] = y.y;
+                    }
                 } else if (EPI == EPI_GELU_ERF) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e) v[e] = 0.5f * v[e] * (1.0f + erff(v[e] * 0.7071067811865476f));
@@ -491,10 +502,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                                          : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
                                          : "r"(my_row + ((((uint32_t)j) ^ swz) << 4)));
-                            Vec16<__nv_bfloat16> r;
-                            r.u = u;
+                            float2 rp[4];
+                            unpack_pairs(u, rp);
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) v[8 * j + e] += __bfloat162float(r.e[e]);
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 y = f2_add(make_float2(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]), rp[e]);
+                                v[8 * j + 2 * e] = y.x;
+                                v[8 * j + 2 * e + 1] = y.y;
+                            }
                         }
                     }
                 }
@@ -503,17 +518,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < 32; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
                 if (EPI == EPI_BIAS_RESID && p.stats != nullptr && wrow0 + lane < p.M) {
                     // LayerNorm partials of the stored (rounded) 64 values: (mean, M2)
-                    float s1 = 0.f;
+                    float2 a1 = f2(0.f);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) s1 += __uint_as_float(w[j] << 16) + __uint_as_float(w[j] & 0xffff0000u);
-                    const float mean = s1 * (1.0f / 64.0f);
-                    float q = 0.f;
+                    for (int j = 0; j < 32; ++j)
+                        a1 = f2_add(a1, make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u)));
+                    const float mean = (a1.x + a1.y) * (1.0f / 64.0f);
+                    const float2 nm = f2(-mean);
+                    float2 a2 = f2(0.f);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const float d0 = __uint_as_float(w[j] << 16) - mean;
-                        const float d1 = __uint_as_float(w[j] & 0xffff0000u) - mean;
-                        q = fmaf(d0, d0, fmaf(d1, d1, q));
+                        const float2 d = f2_add(make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u)), nm);
+                        a2 = f2_fma(d, d, a2);
                     }
+                    const float q = a2.x + a2.y;
                     p.stats[(long long)t.g * p.s_gstride + (long long)(wrow0 + lane) * p.s_ld + (n >> 6)] =
                         make_float2(mean, q);
                 }
@@ -569,17 +586,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const float4 bb = __ldg(b4 + q);
-                        v[4 * q + 0] += bb.x;
-                        v[4 * q + 1] += bb.y;
-                        v[4 * q + 2] += bb.z;
-                        v[4 * q + 3] += bb.w;
+                        const float2 lo = f2_add(make_float2(v[4 * q], v[4 * q + 1]), make_float2(bb.x, bb.y));
+                        const float2 hi = f2_add(make_float2(v[4 * q + 2], v[4 * q + 3]), make_float2(bb.z, bb.w));
+                        v[4 * q] = lo.x;
+                        v[4 * q + 1] = lo.y;
+                        v[4 * q + 2] = hi.x;
+                        v[4 * q + 3] = hi.y;
                     }
                     if (EPI == EPI_RELU) {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = fmaxf(v[e], 0.0f);
                     } else if (EPI == EPI_GELU_TANH) {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] = gelu_tanh_approx(v[e]);
+                        for (int e = 0; e < 16; e += 2) {
+                            const float2 y = gelu_tanh_pair(make_float2(v[e], v[e + 1]));
+                            v[e] = y.x;
+                            v[e + 1] = y.y;
+                        }
                     } else if (EPI == EPI_GELU_ERF) {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = 0.5f * v[e] * (1.0f + erff(v[e] * 0.7071067811865476f));
@@ -597,7 +620,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     } else {  // EPI_BIAS_GATE
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] *= gate;
+                        for (int e = 0; e < 16; e += 2) {
+                            const float2 y = f2_mul(make_float2(v[e], v[e + 1]), f2(gate));
+                            v[e] = y.x;
+                            v[e + 1] = y.y;
+                        }
                     }
                     uint4 o0, o1;
                     o0.x = pack_bf16x2(v[0], v[1]);

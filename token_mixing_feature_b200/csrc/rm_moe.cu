@@ -72,9 +72,9 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __nv_bfloat16* __
     const int jl = lane % NE, rl = lane / NE;   // this lane's (row, expert) after the reduction
     const float bias = jl < Ne ? __ldg(br + (long long)t * Ne + jl) : 0.f;
     for (int bw = b0 + warp * RW; bw < bend; bw += nw * RW) {
-        float acc[32];
+        float2 acc2[32];   // paired partial dot products (even / odd columns)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+        for (int i = 0; i < 32; ++i) acc2[i] = f2(0.f);
         for (int v = lane; v < nv; v += 32) {
             float xf[RW][4];
 #pragma unroll
@@ -96,18 +96,20 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __nv_bfloat16* __
             for (int j = 0; j < NE; ++j) {
                 if (j < Ne) {
                     const float4 w = *reinterpret_cast<const float4*>(wsm + (size_t)j * D + 4 * v);
+                    const float2 wl = make_float2(w.x, w.y), wh = make_float2(w.z, w.w);
 #pragma unroll
                     for (int q = 0; q < RW; ++q) {
-                        float a = acc[q * NE + j];
-                        a = fmaf(xf[q][0], w.x, a);
-                        a = fmaf(xf[q][1], w.y, a);
-                        a = fmaf(xf[q][2], w.z, a);
-                        a = fmaf(xf[q][3], w.w, a);
-                        acc[q * NE + j] = a;
+                        float2 a = acc2[q * NE + j];
+                        a = f2_fma(make_float2(xf[q][0], xf[q][1]), wl, a);
+                        a = f2_fma(make_float2(xf[q][2], xf[q][3]), wh, a);
+                        acc2[q * NE + j] = a;
                     }
                 }
             }
         }
+        float acc[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] = acc2[i].x + acc2[i].y;
         warp_reduce_transpose32(acc);
         const int b = bw + rl;
         if (jl < Ne && b < bend) {
@@ -207,13 +209,25 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const __nv_bfloat16* _
          s += (long long)gridDim.x * (blockDim.x >> 5)) {
         const uint4* src = reinterpret_cast<const uint4*>(S + (long long)slot_row[s] * D);
         uint4* dst = reinterpret_cast<uint4*>(Sg + s * D);
-        for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+        for (int v0 = lane; v0 < nv; v0 += 128) {   // up to four loads in flight per lane
+            uint4 t[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (v0 + 32 * k < nv) t[k] = __ldg(src + v0 + 32 * k);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (v0 + 32 * k < nv) dst[v0 + 32 * k] = t[k];
+        }
     }
 }
 
 // out[r] = resid[r] + sum over j ascending of Eg[slot_of[r, j]] (active only),
-// summed in fp32.  One warp per (b, t) row.  stats (optional) = (mean, M2) of
-// the stored row, from sums shifted by the row's first stored value.
+// summed in fp32 pairs.  One warp per (b, t) row: the row's expert slots are
+// read once (lane j holds slot j), lane l keeps vectors l, l + 32, ... of the
+// row (NVL of them) in registers, and each active expert's vectors are loaded
+// together.  stats (optional) = (mean, M2) of the stored row, from sums
+// shifted by the row's first stored value.
+template <int NVL>
 __global__ void __launch_bounds__(kThreads) combine_kernel(const __nv_bfloat16* __restrict__ Eg,
                                                            const int* __restrict__ slot_of,
                                                            const __nv_bfloat16* __restrict__ resid,
@@ -221,48 +235,63 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const __nv_bfloat16* 
                                                            long long rows, int D, int Ne) {
     const int lane = threadIdx.x & 31;
     const long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (r >= rows) return;
+    if (r >= rows) return;   // warp-uniform
     const int nv = D / 8;
-    float K = 0.f, s1 = 0.f, s2 = 0.f;
-    for (int v = lane; v < nv; v += 32) {
-        float acc[8];
-        if (resid) {
-            Vec16<__nv_bfloat16> x;
-            x.u = __ldg(reinterpret_cast<const uint4*>(resid + r * D) + v);
+    const int myslot = lane < Ne ? __ldg(slot_of + r * Ne + lane) : -1;
+    const unsigned act = __ballot_sync(0xffffffffu, myslot >= 0);
+    float2 acc[NVL][4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = __bfloat162float(x.e[e]);
+    for (int i = 0; i < NVL; ++i) {
+        const int v = lane + 32 * i;
+        if (resid && v < nv) {
+            unpack_pairs(__ldg(reinterpret_cast<const uint4*>(resid + r * D) + v), acc[i]);
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+            for (int e = 0; e < 4; ++e) acc[i][e] = f2(0.f);
         }
-        for (int j = 0; j < Ne; ++j) {
-            const int slot = __ldg(slot_of + r * Ne + j);
-            if (slot < 0) continue;
-            Vec16<__nv_bfloat16> x;
-            x.u = __ldg(reinterpret_cast<const uint4*>(Eg + (long long)slot * D) + v);
+    }
+    for (unsigned m = act; m; m &= m - 1) {   // active experts, ascending j
+        const int slot = __shfl_sync(0xffffffffu, myslot, __ffs(m) - 1);
+        const uint4* src = reinterpret_cast<const uint4*>(Eg + (long long)slot * D);
+        uint4 x[NVL];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] += __bfloat162float(x.e[e]);
-        }
-        uint4 o;
-        o.x = pack_bf16x2(acc[0], acc[1]);
-        o.y = pack_bf16x2(acc[2], acc[3]);
-        o.z = pack_bf16x2(acc[4], acc[5]);
-        o.w = pack_bf16x2(acc[6], acc[7]);
-        reinterpret_cast<uint4*>(out + r * D)[v] = o;
-        if (stats) {
-            const uint32_t w[4] = {o.x, o.y, o.z, o.w};
-            if (v == lane) K = __shfl_sync(__activemask(), __uint_as_float(o.x << 16), 0);
+        for (int i = 0; i < NVL; ++i)
+            if (lane + 32 * i < nv) x[i] = __ldg(src + lane + 32 * i);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float d0 = __uint_as_float(w[q] << 16) - K, d1 = __uint_as_float(w[q] & 0xffff0000u) - K;
-                s1 += d0 + d1;
-                s2 = fmaf(d0, d0, fmaf(d1, d1, s2));
+        for (int i = 0; i < NVL; ++i) {
+            if (lane + 32 * i < nv) {
+                float2 p[4];
+                unpack_pairs(x[i], p);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[i][e] = f2_add(acc[i][e], p[e]);
             }
         }
     }
+    uint4 o[NVL];
+#pragma unroll
+    for (int i = 0; i < NVL; ++i) {
+        o[i] = pack_pairs(acc[i]);
+        if (lane + 32 * i < nv) reinterpret_cast<uint4*>(out + r * D)[lane + 32 * i] = o[i];
+    }
     if (stats) {
-        s1 = warp_sum(s1);
-        s2 = warp_sum(s2);
+        const float K = __shfl_sync(0xffffffffu, __uint_as_float(o[0].x << 16), 0);   // stored element 0
+        const float2 nK = f2(-K);
+        float2 a1 = f2(0.f), a2 = f2(0.f);
+#pragma unroll
+        for (int i = 0; i < NVL; ++i) {
+            if (lane + 32 * i < nv) {
+                float2 p[4];
+                unpack_pairs(o[i], p);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 d = f2_add(p[e], nK);
+                    a1 = f2_add(a1, d);
+                    a2 = f2_fma(d, d, a2);
+                }
+            }
+        }
+        const float s1 = warp_sum(a1.x + a1.y);
+        const float s2 = warp_sum(a2.x + a2.y);
         if (lane == 0) stats[r] = make_float2(K + s1 / D, fmaxf(s2 - s1 * s1 / D, 0.f));
     }
 }
@@ -309,9 +338,15 @@ cudaError_t launch_moe_combine(const MoeWork& w, const void* resid, void* out, f
                                int Ne, cudaStream_t s) {
     const long long rows = (long long)B * T;
     const int grid = (int)((rows + kThreads / 32 - 1) / (kThreads / 32));
-    combine_kernel<<<grid, kThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(w.Eg), w.slot_of,
-                                             static_cast<const __nv_bfloat16*>(resid),
-                                             static_cast<__nv_bfloat16*>(out), stats, rows, D, Ne);
+    const int nvl = (D / 8 + 31) / 32;
+    const auto* eg = static_cast<const __nv_bfloat16*>(w.Eg);
+    const auto* rs = static_cast<const __nv_bfloat16*>(resid);
+    auto* o = static_cast<__nv_bfloat16*>(out);
+    if (nvl <= 1) combine_kernel<1><<<grid, kThreads, 0, s>>>(eg, w.slot_of, rs, o, stats, rows, D, Ne);
+    else if (nvl <= 2) combine_kernel<2><<<grid, kThreads, 0, s>>>(eg, w.slot_of, rs, o, stats, rows, D, Ne);
+    else if (nvl <= 4) combine_kernel<4><<<grid, kThreads, 0, s>>>(eg, w.slot_of, rs, o, stats, rows, D, Ne);
+    else if (nvl <= 8) combine_kernel<8><<<grid, kThreads, 0, s>>>(eg, w.slot_of, rs, o, stats, rows, D, Ne);
+    else return cudaErrorInvalidValue;
     return cudaGetLastError();
 }
 
