@@ -545,12 +545,13 @@ __global__ void __launch_bounds__(256) row_stats_kernel(const E* __restrict__ X,
     if (lane == 0) out[r] = make_float2(K + s1 / D, fmaxf(s2 - s1 * s1 / D, 0.f));
 }
 
-// Samples per ring slot: small samples travel in chunks of about 32 KB, so
-// the per-chunk synchronisation and statistics are amortised.
-constexpr size_t kChunkTargetBytes = 32 * 1024;
+// Samples per ring slot: small samples travel in chunks of about 48 KB (the
+// nearest whole number of samples), so the per-chunk synchronisation and
+// statistics are amortised while two CTAs with two slots each fit an SM.
+constexpr size_t kChunkTargetBytes = 48 * 1024;
 inline int samples_per_chunk(int T, int rs, size_t esz, int B) {
     const size_t one = (size_t)T * rs * esz;
-    long long spb = one >= kChunkTargetBytes ? 1 : (long long)(kChunkTargetBytes / one);
+    long long spb = (long long)((kChunkTargetBytes + one / 2) / one);
     if (spb > B) spb = B;
     return spb < 1 ? 1 : (int)spb;
 }
@@ -622,6 +623,7 @@ cudaError_t mix_ln_nv(int nvl, int addnorm, const E* X, const float* pg, const f
     if (!addnorm) return mix_ln_go<E, PRE, MV, 1, false>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
     if (nvl <= 1) return mix_ln_go<E, PRE, MV, 1, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
     if (nvl <= 2) return mix_ln_go<E, PRE, MV, 2, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
+    if (nvl <= 3) return mix_ln_go<E, PRE, MV, 3, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
     if (nvl <= 4) return mix_ln_go<E, PRE, MV, 4, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
     if (nvl <= 6) return mix_ln_go<E, PRE, MV, 6, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
     if (nvl <= 8) return mix_ln_go<E, PRE, MV, 8, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);

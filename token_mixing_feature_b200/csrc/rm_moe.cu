@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __nv_bfloat16* __
         float2 acc2[32];   // paired partial dot products (even / odd columns)
 #pragma unroll
         for (int i = 0; i < 32; ++i) acc2[i] = f2(0.f);
+#pragma unroll 2
         for (int v = lane; v < nv; v += 32) {
             float xf[RW][4];
 #pragma unroll
