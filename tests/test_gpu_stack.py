@@ -145,6 +145,41 @@ def test_host_async_pipeline_matches_device_entry(rm):
     st.close()
 
 
+def test_programmatic_launch_changes_no_bits(rm, tmp_path):
+    """Kernels overlap their launch with the previous kernel's tail
+    (programmatic dependent launch); a process with it switched off
+    (RM_NO_PDL) computes bit-identical stacks (dense, MoE, Pad-Split + head)."""
+    import os
+    import subprocess
+    import sys
+    script = tmp_path / "run.py"
+    script.write_text(
+        "import sys, torch\n"
+        "sys.path.insert(0, %r)\n"
+        "from token_mixing_feature_b200 import synth\n"
+        "from token_mixing_feature_b200.stack import RankMixerStack\n"
+        "out = {}\n"
+        "for name, B in (('rm100m', 96), ('moe', 128), ('padsplit', 200)):\n"
+        "    wl = synth.WORKLOADS[name].with_batch(B)\n"
+        "    d = synth.make_inputs(wl)\n"
+        "    st = RankMixerStack(wl, d['blocks'], d.get('head'))\n"
+        "    X0 = st.tokenize([g.cuda() for g in d['groups']]) if wl.group_widths else d['X0'].cuda()\n"
+        "    pooled = st.forward(X0)\n"
+        "    out[name] = (st.head_forward(pooled) if wl.head else pooled).cpu()\n"
+        "    st.close()\n"
+        "torch.save(out, sys.argv[1])\n" % os.getcwd())
+    results = []
+    for env_extra in ({}, {"RM_NO_PDL": "1"}):
+        env = dict(os.environ)
+        env.pop("RM_NO_PDL", None)
+        env.update(env_extra)
+        path = tmp_path / f"out{len(results)}.pt"
+        subprocess.run([sys.executable, str(script), str(path)], check=True, env=env, timeout=600)
+        results.append(torch.load(path))
+    for name in results[0]:
+        assert torch.equal(results[0][name], results[1][name]), name
+
+
 def test_moe_active_rate_is_reported(rm):
     """The MoE workload's routing statistics: fraction of active experts."""
     wl = synth.WORKLOADS["moe"].with_batch(512)

@@ -4,6 +4,9 @@
 #pragma once
 
 #include <cuda_bf16.h>
+
+#include <cstdlib>
+#include <utility>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -88,6 +91,45 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
+}
+
+// ------------------------------------------------------ programmatic launch
+// Every kernel of the library is launched with programmatic stream
+// serialisation (launch_pdl), so it may begin while the previous kernel of
+// the stream drains, and calls pdl_enter() before its first global-memory
+// access: that lets the next kernel launch once this grid is resident, then
+// waits until the previous grid has completed and its writes are visible.
+// Since every kernel waits, the ordering is transitive along the stream.
+// Consequence for loads: a kernel's lifetime now overlaps its predecessors'
+// writes, so the read-only path (__ldg, ld.global.nc) is used only for data
+// no kernel writes (weights, biases, LayerNorm and router parameters); data
+// produced by earlier kernels is read with __ldcg (L2, coherent), plain loads
+// through non-restrict pointers, or TMA / bulk copies.
+__device__ __forceinline__ void pdl_enter() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Process-wide switch (RM_NO_PDL set in the environment: plain serialisation).
+inline bool pdl_enabled() {
+    static const bool on = getenv("RM_NO_PDL") == nullptr;
+    return on;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ---------------------------------------------------------------- error word

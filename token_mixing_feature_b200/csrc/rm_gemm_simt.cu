@@ -12,6 +12,7 @@ constexpr int TM = 64, TN = 64, TK = 16;
 
 template <int EPI>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(GroupedGemm p) {
+    pdl_enter();
     __shared__ float As[TK][TM + 4];
     __shared__ float Ws[TK][TN + 4];
     const int g = blockIdx.z;
@@ -74,12 +75,11 @@ cudaError_t launch_gemm_simt(const GroupedGemm& p, cudaStream_t s) {
     if (p.M == 0) return cudaSuccess;
     dim3 grid((p.N + TN - 1) / TN, (p.M + TM - 1) / TM, p.G);
     switch (p.epi) {
-        case EPI_GELU_TANH: gemm_simt_kernel<EPI_GELU_TANH><<<grid, 256, 0, s>>>(p); break;
-        case EPI_GELU_ERF: gemm_simt_kernel<EPI_GELU_ERF><<<grid, 256, 0, s>>>(p); break;
-        case EPI_RELU: gemm_simt_kernel<EPI_RELU><<<grid, 256, 0, s>>>(p); break;
-        default: gemm_simt_kernel<EPI_BIAS_RESID><<<grid, 256, 0, s>>>(p); break;
+        case EPI_GELU_TANH: return launch_pdl(gemm_simt_kernel<EPI_GELU_TANH>, grid, 256, 0, s, p);
+        case EPI_GELU_ERF: return launch_pdl(gemm_simt_kernel<EPI_GELU_ERF>, grid, 256, 0, s, p);
+        case EPI_RELU: return launch_pdl(gemm_simt_kernel<EPI_RELU>, grid, 256, 0, s, p);
+        default: return launch_pdl(gemm_simt_kernel<EPI_BIAS_RESID>, grid, 256, 0, s, p);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace rm

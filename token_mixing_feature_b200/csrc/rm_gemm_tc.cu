@@ -124,18 +124,18 @@ __device__ __forceinline__ Tile decode_tile(const KParams& p, long long idx, int
         int lo = 0, hi = p.G;
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if ((long long)__ldg(p.mtile_prefix + mid) * nblk <= idx) lo = mid; else hi = mid;
+            if ((long long)__ldcg(p.mtile_prefix + mid) * nblk <= idx) lo = mid; else hi = mid;
         }
-        const int p0 = __ldg(p.mtile_prefix + lo);
-        const int mt = __ldg(p.mtile_prefix + lo + 1) - p0;
+        const int p0 = __ldcg(p.mtile_prefix + lo);
+        const int mt = __ldcg(p.mtile_prefix + lo + 1) - p0;
         const int local = (int)(idx - (long long)p0 * nblk);
         const int nb = local / mt, mb = local - nb * mt;
         const int m0 = mb * BM;
-        const int off = __ldg(p.grp_off + lo);
+        const int off = __ldcg(p.grp_off + lo);
         t.g = lo;
         t.ag = 0;
         t.arow = off + m0;
-        t.rows = min(BM, __ldg(p.grp_cnt + lo) - m0);
+        t.rows = min(BM, __ldcg(p.grp_cnt + lo) - m0);
         t.n0 = nb * bn;
         t.orow0 = off + m0;
     }
@@ -237,12 +237,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (CG == 2) cluster_sync_all();   // the peer's barriers exist before anyone signals them
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_enter();   // set-up above overlaps the previous kernel's tail; global memory only from here
 
     const WaitCtx wc{abort_flag, p.budget_ns, p.err};
     const int nblk = (p.N + BN - 1) / BN;
     const int mblk = (p.M + C::TM - 1) / C::TM;
     const int num_kb = (p.K + BK - 1) / BK;
-    const long long total = p.var_rows ? (long long)__ldg(p.mtile_prefix + p.G) * nblk
+    const long long total = p.var_rows ? (long long)__ldcg(p.mtile_prefix + p.G) * nblk
                                        : p.full_tiles + ((long long)p.G * nblk * mblk - p.full_tiles) * p.nsplit;
     const long long unit = blockIdx.x / CG, nunits = gridDim.x / CG;
 
@@ -574,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float* bias_g = p.bias + (long long)t.g * p.N;
             __nv_bfloat16* out_row = p.out + (long long)t.g * p.o_gstride + orow * p.o_ld;
             float gate = 0.f;
-            if (EPI == EPI_BIAS_GATE && row_ok) gate = __ldg(p.gate + orow);
+            if (EPI == EPI_BIAS_GATE && row_ok) gate = __ldcg(p.gate + orow);
 #pragma unroll 1
             for (int c = half * HALF; c < (half + 1) * HALF; c += 16) {
                 float v[16];
@@ -613,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int q = 0; q < 2; ++q) {
                                 Vec16<__nv_bfloat16> r;
-                                r.u = __ldg(r4 + q);
+                                r.u = __ldcg(r4 + q);
 #pragma unroll
                                 for (int e = 0; e < 8; ++e) v[8 * q + e] += __bfloat162float(r.e[e]);
                             }
@@ -705,13 +706,15 @@ cudaError_t launch_typed(const Maps& m, const KParams& kp, int grid, cudaStream_
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CG;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, k, m.a, m.b, m.o, m.r, kp);
 }
 

@@ -28,6 +28,7 @@ inline int grid_for(long long work, int per_block) {
 template <typename E, int V>
 __global__ void __launch_bounds__(kThreads) token_mix_kernel(const E* __restrict__ X, E* __restrict__ Y,
                                                              long long nvec, int T, int D, int dh) {
+    pdl_enter();
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nvec;
          i += (long long)gridDim.x * blockDim.x) {
         const long long o = i * V;
@@ -38,9 +39,9 @@ __global__ void __launch_bounds__(kThreads) token_mix_kernel(const E* __restrict
         const int t = c / dh, j = c - t * dh;
         const E* src = X + (b * T + t) * D + (long long)h * dh + j;
         if constexpr (V == 1) {
-            Y[o] = *src;
+            Y[o] = __ldcg(src);
         } else {
-            *reinterpret_cast<uint4*>(Y + o) = __ldg(reinterpret_cast<const uint4*>(src));
+            *reinterpret_cast<uint4*>(Y + o) = __ldcg(reinterpret_cast<const uint4*>(src));
         }
     }
 }
@@ -52,6 +53,7 @@ template <typename E>
 __global__ void __launch_bounds__(kThreads) layernorm_kernel(const E* A, const E* R, const float* __restrict__ g,
                                                              const float* __restrict__ bta, E* out, long long rows,
                                                              int D, float eps) {
+    pdl_enter();
     constexpr int V = Vec16<E>::N;
     const int lane = threadIdx.x & 31;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -100,6 +102,7 @@ __global__ void __launch_bounds__(kThreads) layernorm_kernel(const E* A, const E
 template <typename E>
 __global__ void __launch_bounds__(kThreads) padsplit_kernel(PadSplitArgs a, E* __restrict__ X0, long long B,
                                                             int width) {
+    pdl_enter();
     constexpr int V = Vec16<E>::N;
     const int wv = width / V;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < B * wv;
@@ -112,7 +115,7 @@ __global__ void __launch_bounds__(kThreads) padsplit_kernel(PadSplitArgs a, E* _
         if (gi < a.n) {
             const int w = a.col0[gi + 1] - a.col0[gi];
             const E* src = reinterpret_cast<const E*>(a.src[gi]) + b * w + (c - a.col0[gi]);
-            v = __ldg(reinterpret_cast<const uint4*>(src));
+            v = __ldcg(reinterpret_cast<const uint4*>(src));
         }
         *reinterpret_cast<uint4*>(X0 + b * width + c) = v;
     }
@@ -123,11 +126,12 @@ template <typename E>
 __global__ void __launch_bounds__(kThreads) head_kernel(const float* __restrict__ pooled, const E* __restrict__ w,
                                                         const float* __restrict__ bias, float* __restrict__ prob,
                                                         int B, int D) {
+    pdl_enter();
     const int lane = threadIdx.x & 31;
     const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (b >= B) return;
     float s = 0.f;
-    for (int d = lane; d < D; d += 32) s += pooled[(long long)b * D + d] * to_f(w[d]);
+    for (int d = lane; d < D; d += 32) s += __ldcg(pooled + (long long)b * D + d) * to_f(w[d]);
     s = warp_sum(s);
     if (lane == 0) prob[b] = 1.0f / (1.0f + expf(-(s + bias[0])));
 }
@@ -153,22 +157,17 @@ cudaError_t launch_token_mix(int dtype, const void* X, void* Y, int B, int T, in
     const long long n = (long long)B * T * D;
     if (dtype == RM_BF16) {
         using E = __nv_bfloat16;
-        if (dh % 8 == 0) {
-            token_mix_kernel<E, 8><<<grid_for(n / 8, kThreads), kThreads, 0, s>>>(
-                (const E*)X, (E*)Y, n / 8, T, D, dh);
-        } else {
-            token_mix_kernel<E, 1><<<grid_for(n, kThreads), kThreads, 0, s>>>((const E*)X, (E*)Y, n, T, D, dh);
-        }
-    } else {
-        if (dh % 4 == 0) {
-            token_mix_kernel<float, 4><<<grid_for(n / 4, kThreads), kThreads, 0, s>>>(
-                (const float*)X, (float*)Y, n / 4, T, D, dh);
-        } else {
-            token_mix_kernel<float, 1><<<grid_for(n, kThreads), kThreads, 0, s>>>((const float*)X, (float*)Y,
-                                                                                n, T, D, dh);
-        }
+        if (dh % 8 == 0)
+            return launch_pdl(token_mix_kernel<E, 8>, grid_for(n / 8, kThreads), kThreads, 0, s, (const E*)X, (E*)Y,
+                              n / 8, T, D, dh);
+        return launch_pdl(token_mix_kernel<E, 1>, grid_for(n, kThreads), kThreads, 0, s, (const E*)X, (E*)Y, n, T, D,
+                          dh);
     }
-    return cudaGetLastError();
+    if (dh % 4 == 0)
+        return launch_pdl(token_mix_kernel<float, 4>, grid_for(n / 4, kThreads), kThreads, 0, s, (const float*)X,
+                          (float*)Y, n / 4, T, D, dh);
+    return launch_pdl(token_mix_kernel<float, 1>, grid_for(n, kThreads), kThreads, 0, s, (const float*)X, (float*)Y, n,
+                      T, D, dh);
 }
 
 cudaError_t launch_layernorm(int dtype, const void* A, const void* R, const float* g, const float* b, void* out,
@@ -176,31 +175,29 @@ cudaError_t launch_layernorm(int dtype, const void* A, const void* R, const floa
     const int grid = grid_for(rows, kThreads / 32);
     if (dtype == RM_BF16) {
         using E = __nv_bfloat16;
-        layernorm_kernel<E><<<grid, kThreads, 0, s>>>((const E*)A, (const E*)R, g, b, (E*)out, rows, D, eps);
-    } else {
-        layernorm_kernel<float><<<grid, kThreads, 0, s>>>((const float*)A, (const float*)R, g, b, (float*)out,
-                                                           rows, D, eps);
+        return launch_pdl(layernorm_kernel<E>, grid, kThreads, 0, s, (const E*)A, (const E*)R, g, b, (E*)out, rows, D,
+                          eps);
     }
-    return cudaGetLastError();
+    return launch_pdl(layernorm_kernel<float>, grid, kThreads, 0, s, (const float*)A, (const float*)R, g, b,
+                      (float*)out, rows, D, eps);
 }
 
 cudaError_t launch_padsplit(int dtype, const PadSplitArgs& a, void* X0, int B, int width, cudaStream_t s) {
     const long long n = (long long)B * width / (dtype == RM_BF16 ? 8 : 4);
     if (dtype == RM_BF16)
-        padsplit_kernel<__nv_bfloat16><<<grid_for(n, kThreads), kThreads, 0, s>>>(a, (__nv_bfloat16*)X0, B, width);
-    else
-        padsplit_kernel<float><<<grid_for(n, kThreads), kThreads, 0, s>>>(a, (float*)X0, B, width);
-    return cudaGetLastError();
+        return launch_pdl(padsplit_kernel<__nv_bfloat16>, grid_for(n, kThreads), kThreads, 0, s, a,
+                          (__nv_bfloat16*)X0, (long long)B, width);
+    return launch_pdl(padsplit_kernel<float>, grid_for(n, kThreads), kThreads, 0, s, a, (float*)X0, (long long)B,
+                      width);
 }
 
 cudaError_t launch_head(int dtype, const float* pooled, const void* w, const float* bias, float* prob, int B,
                         int D, cudaStream_t s) {
     const int grid = (B + kThreads / 32 - 1) / (kThreads / 32);
     if (dtype == RM_BF16)
-        head_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(pooled, (const __nv_bfloat16*)w, bias, prob, B, D);
-    else
-        head_kernel<float><<<grid, kThreads, 0, s>>>(pooled, (const float*)w, bias, prob, B, D);
-    return cudaGetLastError();
+        return launch_pdl(head_kernel<__nv_bfloat16>, grid, kThreads, 0, s, pooled, (const __nv_bfloat16*)w, bias,
+                          prob, B, D);
+    return launch_pdl(head_kernel<float>, grid, kThreads, 0, s, pooled, (const float*)w, bias, prob, B, D);
 }
 
 cudaError_t launch_selftest_wait(DeviceErr err, uint64_t budget_ns, cudaStream_t s) {

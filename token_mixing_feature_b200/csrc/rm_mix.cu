@@ -167,7 +167,7 @@ __device__ __forceinline__ void chunk_stats(const float2* __restrict__ part, int
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int rr = r + k * nw;
-            v[k] = (rr < R && lane < P) ? __ldg(part + (row0 + rr) * P + lane) : make_float2(0.f, 0.f);
+            v[k] = (rr < R && lane < P) ? __ldcg(part + (row0 + rr) * P + lane) : make_float2(0.f, 0.f);
         }
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -289,6 +289,7 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
     const float2* __restrict__ pstats, int P, const float* __restrict__ g1, const float* __restrict__ b1,
     E* __restrict__ S, int B, int T, int D, float eps, int rs, int spb, int nslots, int groups, DeviceErr err,
     uint64_t budget_ns) {
+    pdl_enter();
     constexpr int V = Vec16<E>::N;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int abort_flag, s_ok;
@@ -431,6 +432,7 @@ __global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __res
                                                                  float* __restrict__ pooled, E* __restrict__ Xout,
                                                                  int B, int T, int D, float eps, int spb, int nslots,
                                                                  int groups, DeviceErr err, uint64_t budget_ns) {
+    pdl_enter();
     constexpr int V = Vec16<E>::N;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ int abort_flag, s_ok;
@@ -523,6 +525,7 @@ __global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __res
 template <typename E>
 __global__ void __launch_bounds__(256) row_stats_kernel(const E* __restrict__ X, float2* __restrict__ out,
                                                        long long rows, int D) {
+    pdl_enter();
     constexpr int V = Vec16<E>::N;
     const int lane = threadIdx.x & 31;
     const long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -532,7 +535,7 @@ __global__ void __launch_bounds__(256) row_stats_kernel(const E* __restrict__ X,
     float s1 = 0.f, s2 = 0.f;
     for (int v = lane; v < D / V; v += 32) {
         Vec16<E> u;
-        u.u = __ldg(reinterpret_cast<const uint4*>(x) + v);
+        u.u = __ldcg(reinterpret_cast<const uint4*>(x) + v);
 #pragma unroll
         for (int e = 0; e < V; ++e) {
             const float d = to_f(u.e[e]) - K;
@@ -611,9 +614,8 @@ cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps,
     const long long nchunks = (B + spb - 1) / spb;
     const long long g = (long long)num_sms * per_sm;
     const int grid = (int)(g < nchunks ? g : nchunks);
-    k<<<grid, threads, smem, s>>>(X, pg, pb, ps.part, ps.P, g1, b1, S, B, T, D, eps, rs, spb, nslots, groups, err,
-                                  budget);
-    return cudaGetLastError();
+    return launch_pdl(k, grid, threads, smem, s, X, pg, pb, ps.part, ps.P, g1, b1, S, B, T, D, eps, rs, spb, nslots,
+                      groups, err, budget);
 }
 
 template <typename E, bool PRE, int MV>
@@ -678,9 +680,8 @@ cudaError_t ln_pool_go(const void* X, RowStats stats, const float* g, const floa
     const long long nchunks = (B + spb - 1) / spb;
     const long long gr = (long long)num_sms * per_sm;
     const int grid = (int)(gr < nchunks ? gr : nchunks);
-    k<<<grid, kPoolThreads, smem, s>>>(static_cast<const E*>(X), stats.part, stats.P, g, b, pooled, static_cast<E*>(Xout),
-                                       B, T, D, eps, spb, nslots, groups, err, budget);
-    return cudaGetLastError();
+    return launch_pdl(k, grid, kPoolThreads, smem, s, static_cast<const E*>(X), stats.part, stats.P, g, b, pooled,
+                      static_cast<E*>(Xout), B, T, D, eps, spb, nslots, groups, err, budget);
 }
 
 }  // namespace
@@ -723,10 +724,9 @@ cudaError_t launch_ln_pool(int dtype, const void* X, RowStats stats, const float
 cudaError_t launch_row_stats(int dtype, const void* X, float2* out, long long rows, int D, cudaStream_t s) {
     const int grid = (int)((rows + 7) / 8);
     if (dtype == RM_BF16)
-        row_stats_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(X), out, rows, D);
-    else
-        row_stats_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(X), out, rows, D);
-    return cudaGetLastError();
+        return launch_pdl(row_stats_kernel<__nv_bfloat16>, grid, 256, 0, s, static_cast<const __nv_bfloat16*>(X), out,
+                          rows, D);
+    return launch_pdl(row_stats_kernel<float>, grid, 256, 0, s, static_cast<const float*>(X), out, rows, D);
 }
 
 }  // namespace rm

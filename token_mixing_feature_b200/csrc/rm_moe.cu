@@ -54,6 +54,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __nv_bfloat16* __
                                                          const float* __restrict__ Wr,
                                                          const float* __restrict__ br, float* __restrict__ gates,
                                                          int* __restrict__ counts, int B, int T, int D, int Ne) {
+    pdl_enter();
     constexpr int RW = 32 / NE;
     extern __shared__ __align__(16) float wsm[];   // [Ne][D]
     __shared__ int cnt[NE];
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __nv_bfloat16* __
             for (int q = 0; q < RW; ++q) {
                 const int b = bw + q;
                 if (b < bend) {
-                    const uint2 u = __ldg(reinterpret_cast<const uint2*>(S + ((long long)b * T + t) * D) + v);
+                    const uint2 u = __ldcg(reinterpret_cast<const uint2*>(S + ((long long)b * T + t) * D) + v);
                     const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
                     const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
                     xf[q][0] = lo.x;
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__
                                                        int* __restrict__ mtile_prefix, int* __restrict__ totals,
                                                        int* __restrict__ slot_row, float* __restrict__ slot_gate,
                                                        int* __restrict__ slot_of, int B, int T, int Ne) {
+    pdl_enter();
     __shared__ int s_off;
     __shared__ int s_warp[32];
     const int G = T * Ne;
@@ -147,7 +149,7 @@ __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__
     if (warp == 0) {
         int off = 0, mt = 0;
         for (int q = lane; q < g; q += 32) {
-            const int c = counts[q];
+            const int c = __ldcg(counts + q);
             off += c;
             mt += (c + 127) / 128;
         }
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__
             offsets[g] = off;
             mtile_prefix[g] = mt;
             if (g == G - 1) {
-                const int c = counts[g];
+                const int c = __ldcg(counts + g);
                 mtile_prefix[G] = mt + (c + 127) / 128;
                 totals[0] = off + c;
                 totals[1] = mt + (c + 127) / 128;
@@ -171,7 +173,7 @@ __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__
     for (int b0 = 0; b0 < B; b0 += 1024) {
         const int b = b0 + threadIdx.x;
         const long long e = ((long long)b * T + t) * Ne + j;
-        const float gate = b < B ? gates[e] : 0.f;
+        const float gate = b < B ? __ldcg(gates + e) : 0.f;
         const bool act = gate > 0.f;
         const unsigned m = __ballot_sync(0xffffffffu, act);
         const int before = __popc(m & ((1u << lane) - 1u));
@@ -203,18 +205,19 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const __nv_bfloat16* _
                                                           const int* __restrict__ slot_row,
                                                           const int* __restrict__ totals,
                                                           __nv_bfloat16* __restrict__ Sg, int D) {
+    pdl_enter();
     const int lane = threadIdx.x & 31;
-    const int n = totals[0];
+    const int n = __ldcg(totals);
     const int nv = D / 8;
     for (long long s = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); s < n;
          s += (long long)gridDim.x * (blockDim.x >> 5)) {
-        const uint4* src = reinterpret_cast<const uint4*>(S + (long long)slot_row[s] * D);
+        const uint4* src = reinterpret_cast<const uint4*>(S + (long long)__ldcg(slot_row + s) * D);
         uint4* dst = reinterpret_cast<uint4*>(Sg + s * D);
         for (int v0 = lane; v0 < nv; v0 += 128) {   // up to four loads in flight per lane
             uint4 t[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-                if (v0 + 32 * k < nv) t[k] = __ldg(src + v0 + 32 * k);
+                if (v0 + 32 * k < nv) t[k] = __ldcg(src + v0 + 32 * k);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 if (v0 + 32 * k < nv) dst[v0 + 32 * k] = t[k];
@@ -234,18 +237,19 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const __nv_bfloat16* 
                                                            const __nv_bfloat16* __restrict__ resid,
                                                            __nv_bfloat16* __restrict__ out, float2* __restrict__ stats,
                                                            long long rows, int D, int Ne) {
+    pdl_enter();
     const int lane = threadIdx.x & 31;
     const long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5);
     if (r >= rows) return;   // warp-uniform
     const int nv = D / 8;
-    const int myslot = lane < Ne ? __ldg(slot_of + r * Ne + lane) : -1;
+    const int myslot = lane < Ne ? __ldcg(slot_of + r * Ne + lane) : -1;
     const unsigned act = __ballot_sync(0xffffffffu, myslot >= 0);
     float2 acc[NVL][4];
 #pragma unroll
     for (int i = 0; i < NVL; ++i) {
         const int v = lane + 32 * i;
         if (resid && v < nv) {
-            unpack_pairs(__ldg(reinterpret_cast<const uint4*>(resid + r * D) + v), acc[i]);
+            unpack_pairs(__ldcg(reinterpret_cast<const uint4*>(resid + r * D) + v), acc[i]);
         } else {
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[i][e] = f2(0.f);
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const __nv_bfloat16* 
         uint4 x[NVL];
 #pragma unroll
         for (int i = 0; i < NVL; ++i)
-            if (lane + 32 * i < nv) x[i] = __ldg(src + lane + 32 * i);
+            if (lane + 32 * i < nv) x[i] = __ldcg(src + lane + 32 * i);
 #pragma unroll
         for (int i = 0; i < NVL; ++i) {
             if (lane + 32 * i < nv) {
@@ -310,7 +314,8 @@ cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, co
     {                                                                                                    \
         e = cudaFuncSetAttribute(route_kernel<NEV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
         if (e != cudaSuccess) return e;                                                                  \
-        route_kernel<NEV><<<grid, kThreads, smem, s>>>(Sb, Wr, br, w.gates, w.counts, B, T, D, Ne);      \
+        e = launch_pdl(route_kernel<NEV>, grid, kThreads, smem, s, Sb, Wr, br, w.gates, w.counts, B, T, D, Ne); \
+        if (e != cudaSuccess) return e;                                                                  \
     }
     if (Ne <= 1) RM_ROUTE(1)
     else if (Ne <= 2) RM_ROUTE(2)
@@ -319,20 +324,16 @@ cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, co
     else if (Ne <= 16) RM_ROUTE(16)
     else RM_ROUTE(32)
 #undef RM_ROUTE
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    compact_kernel<<<T * Ne, 1024, 0, s>>>(w.gates, w.counts, w.offsets, w.mtile_prefix, w.totals, w.slot_row,
-                                           w.slot_gate, w.slot_of, B, T, Ne);
-    return cudaGetLastError();
+    return launch_pdl(compact_kernel, T * Ne, 1024, 0, s, w.gates, w.counts, w.offsets, w.mtile_prefix, w.totals,
+                      w.slot_row, w.slot_gate, w.slot_of, B, T, Ne);
 }
 
 cudaError_t launch_moe_gather(const void* S, const MoeWork& w, int B, int T, int D, int Ne, cudaStream_t s) {
     (void)B;
     (void)T;
     (void)Ne;
-    gather_kernel<<<148 * 8, kThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(S), w.slot_row, w.totals,
-                                               static_cast<__nv_bfloat16*>(w.Sg), D);
-    return cudaGetLastError();
+    return launch_pdl(gather_kernel, 148 * 8, kThreads, 0, s, static_cast<const __nv_bfloat16*>(S), w.slot_row,
+                      w.totals, static_cast<__nv_bfloat16*>(w.Sg), D);
 }
 
 cudaError_t launch_moe_combine(const MoeWork& w, const void* resid, void* out, float2* stats, int B, int T, int D,
@@ -343,12 +344,11 @@ cudaError_t launch_moe_combine(const MoeWork& w, const void* resid, void* out, f
     const auto* eg = static_cast<const __nv_bfloat16*>(w.Eg);
     const auto* rs = static_cast<const __nv_bfloat16*>(resid);
     auto* o = static_cast<__nv_bfloat16*>(out);
-    if (nvl <= 1) combine_kernel<1><<<grid, kThreads, 0, s>>>(eg, w.slot_of, rs, o, stats, rows, D, Ne);
-    else if (nvl <= 2) combine_kernel<2><<<grid, kThreads, 0, s>>>(eg, w.slot_of, rs, o, stats, rows, D, Ne);
-    else if (nvl <= 4) combine_kernel<4><<<grid, kThreads, 0, s>>>(eg, w.slot_of, rs, o, stats, rows, D, Ne);
-    else if (nvl <= 8) combine_kernel<8><<<grid, kThreads, 0, s>>>(eg, w.slot_of, rs, o, stats, rows, D, Ne);
-    else return cudaErrorInvalidValue;
-    return cudaGetLastError();
+    if (nvl <= 1) return launch_pdl(combine_kernel<1>, grid, kThreads, 0, s, eg, w.slot_of, rs, o, stats, rows, D, Ne);
+    if (nvl <= 2) return launch_pdl(combine_kernel<2>, grid, kThreads, 0, s, eg, w.slot_of, rs, o, stats, rows, D, Ne);
+    if (nvl <= 4) return launch_pdl(combine_kernel<4>, grid, kThreads, 0, s, eg, w.slot_of, rs, o, stats, rows, D, Ne);
+    if (nvl <= 8) return launch_pdl(combine_kernel<8>, grid, kThreads, 0, s, eg, w.slot_of, rs, o, stats, rows, D, Ne);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace rm
