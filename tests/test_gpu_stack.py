@@ -180,6 +180,40 @@ def test_programmatic_launch_changes_no_bits(rm, tmp_path):
         assert torch.equal(results[0][name], results[1][name]), name
 
 
+@pytest.mark.parametrize("name,B", [("rm100m", 96), ("moe", 128)])
+def test_cuda_graph_replay_equals_direct_launch(rm, name, B):
+    """The stack captured once in a CUDA graph (kernel launches, programmatic
+    dependencies and the router's memset become graph nodes) and replayed on
+    new inputs copied into the captured buffer gives the direct launches'
+    bits."""
+    wl = synth.WORKLOADS[name].with_batch(B)
+    d = synth.make_inputs(wl)
+    st = _stack(wl, d)
+    X0 = dev(d["X0"])
+    pooled = torch.empty(wl.B, wl.D, dtype=torch.float32, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        st.forward(X0, pooled, stream=side.cuda_stream)
+        side.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            st.forward(X0, pooled, stream=side.cuda_stream)
+    torch.cuda.synchronize()
+    for i in range(2):
+        x = synth.random_activations((wl.B, wl.T, wl.D), "bf16", seed=60 + i)
+        X0.copy_(dev(x))
+        g.replay()
+        torch.cuda.synchronize()
+        got = pooled.clone()
+        expect = st.forward(dev(x))
+        torch.cuda.synchronize()
+        assert rm.rm_sync_status(st.h) == rm.RM_OK
+        assert torch.equal(got, expect), f"replay {i}"
+    del g
+    st.close()
+
+
 def test_moe_active_rate_is_reported(rm):
     """The MoE workload's routing statistics: fraction of active experts."""
     wl = synth.WORKLOADS["moe"].with_batch(512)

@@ -105,9 +105,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 // no kernel writes (weights, biases, LayerNorm and router parameters); data
 // produced by earlier kernels is read with __ldcg (L2, coherent), plain loads
 // through non-restrict pointers, or TMA / bulk copies.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_enter() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_trigger();
+    pdl_wait();
 }
 
 // Process-wide switch (RM_NO_PDL set in the environment: plain serialisation).

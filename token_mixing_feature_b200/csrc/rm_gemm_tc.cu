@@ -237,7 +237,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (CG == 2) cluster_sync_all();   // the peer's barriers exist before anyone signals them
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    pdl_enter();   // set-up above overlaps the previous kernel's tail; global memory only from here
+    // The set-up above overlaps the previous kernel's tail (programmatic
+    // launch).  Every thread waits for that kernel before it touches data an
+    // earlier kernel wrote; only the producer's first weight tiles come before
+    // the wait (no kernel writes weights).
+    pdl_trigger();
+    if (VAR) pdl_wait();   // the tile count comes from the routing kernels
 
     const WaitCtx wc{abort_flag, p.budget_ns, p.err};
     const int nblk = (p.N + BN - 1) / BN;
@@ -253,33 +258,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0, issued = 0, issued_phase = 0;
             bool ok = true;
+            // Weight (B) tiles of the first tile's first stages, before the wait.
+            int npre = 0;
+            if (!VAR && unit < total) {
+                const Item it0 = decode_item(p, unit, num_kb);
+                const Tile t0 = decode_tile<CG>(p, it0.tile, nblk, mblk, BN, (int)rank);
+                const int nb0 = t0.n0 + (int)rank * C::BN_LOCAL;
+                npre = min(C::STAGES, it0.kb_hi - it0.kb_lo);
+                for (int k = 0; k < npre; ++k) {   // fresh ring: every slot is free
+                    const uint32_t fb = full0 + 8 * k;
+                    if (leader) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
+                    const uint32_t sb = sbase + k * C::STAGE_BYTES + C::A_BYTES;
+                    const int kc = (it0.kb_lo + k) * BK;
+                    if (CG == 2) tma_load_3d_pair(sb, &tmB, mapa_shared(fb, 0), kc, nb0, t0.g);
+                    else tma_load_3d(sb, &tmB, fb, kc, nb0, t0.g);
+                }
+            }
+            pdl_wait();
+            bool first = true;
             for (long long idx = unit; idx < total && ok; idx += nunits) {
                 const Item item = decode_item(p, idx, num_kb);
                 const Tile t = decode_tile<CG>(p, item.tile, nblk, mblk, BN, (int)rank);
                 const int nb0 = t.n0 + (int)rank * C::BN_LOCAL;
                 for (int kb = item.kb_lo; kb < item.kb_hi; ++kb) {
-                    if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, wc, SITE_TC_PRODUCER)) {
+                    const bool pre = first && kb - item.kb_lo < npre;   // B already issued
+                    if (!pre && !mbar_wait(empty0 + 8 * stage, phase ^ 1u, wc, SITE_TC_PRODUCER)) {
                         ok = false;
                         break;
                     }
                     const uint32_t fb = full0 + 8 * stage;
-                    if (leader) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
+                    if (leader && !pre) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
                     const uint32_t sa = sbase + stage * C::STAGE_BYTES;
                     const int kc = kb * BK;
                     if (CG == 2) {
                         const uint32_t fbl = mapa_shared(fb, 0);   // the pair counts bytes on the even CTA
                         if (p.a_g_inner) tma_load_3d_pair(sa, &tmA, fbl, kc, t.ag, t.arow);
                         else tma_load_3d_pair(sa, &tmA, fbl, kc, t.arow, t.ag);
-                        tma_load_3d_pair(sa + C::A_BYTES, &tmB, fbl, kc, nb0, t.g);
+                        if (!pre) tma_load_3d_pair(sa + C::A_BYTES, &tmB, fbl, kc, nb0, t.g);
                     } else {
                         if (p.a_g_inner) tma_load_3d(sa, &tmA, fb, kc, t.ag, t.arow);
                         else tma_load_3d(sa, &tmA, fb, kc, t.arow, t.ag);
-                        tma_load_3d(sa + C::A_BYTES, &tmB, fb, kc, nb0, t.g);
+                        if (!pre) tma_load_3d(sa + C::A_BYTES, &tmB, fb, kc, nb0, t.g);
                     }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
                 }
+                first = false;
             }
             // Every issued copy must land before the CTA's shared memory goes
             // away (for a pair, the even CTA's barrier counts both CTAs' bytes).
@@ -290,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
+        pdl_wait();   // (reads no global memory; keeps every thread ordered after the previous kernel)
         if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issuer
             constexpr uint32_t idesc = idesc_bf16_f32(C::TM, BN);
@@ -341,6 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if constexpr (!VAR) {
+        pdl_wait();
         // ------------------------------------- epilogue, dense: TMA stores
         // Each warp owns 32 accumulator rows (its TMEM lane quarter) and half
         // of the BN columns, in 64-column chunks: tcgen05.ld -> registers ->
@@ -554,6 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) bulk_wait_all();
         __syncwarp();
     } else {
+        // (the wait for the routing kernels came before the tile count)
         // ------------------------------ epilogue, variable rows: row stores
         const int ew = warp - 2;
         const int quarter = warp & 3;          // TMEM lanes this warp may access
