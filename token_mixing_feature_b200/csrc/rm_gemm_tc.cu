@@ -39,6 +39,7 @@ constexpr int BK = 64;       // bf16 elements per 128-byte swizzle row
 constexpr int UMMA_K = 16;   // K per tcgen05.mma of kind::f16
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr int kMaxVarGroups = 2048 + 1;   // entries of the variable-row tile prefix (G <= 2048)
 
 struct KParams {
     int G, M, N, K;
@@ -83,12 +84,14 @@ struct Cfg {
     static constexpr int STAGING_BYTES = VAR ? 0 : kEpiWarps * 4096;
     // as many ring stages as fit next to the staging buffers, the 1 KB
     // alignment slack and the barriers (227 KB per CTA)
-    static constexpr int STAGES_RAW = (227 * 1024 - 1024 - 512 - STAGING_BYTES) / STAGE_BYTES;
+    // variable-row tiles keep the tile prefix table (G + 1 ints) in shared memory
+    static constexpr int TABLE_BYTES = VAR ? kMaxVarGroups * 4 + 16 : 0;
+    static constexpr int STAGES_RAW = (227 * 1024 - 1024 - 512 - STAGING_BYTES - TABLE_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static constexpr int TMEM_COLS = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
     static constexpr int NBARS = 2 * STAGES + 5 + kEpiWarps;
     static constexpr int BAR_BYTES = 8 * NBARS + 16;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + TABLE_BYTES;
     static_assert(BN % 128 == 0 || VAR, "dense tiles leave in 64-column chunks per half");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
     static_assert(B_BYTES % 1024 == 0, "stage alignment");
@@ -105,9 +108,10 @@ struct Tile {
     long long orow0;  // out / resid row index of this CTA's first row (group-local in dense mode)
 };
 
+// mt: the variable-row tile prefix (mtile_prefix, staged in shared memory).
 template <int CG>
 __device__ __forceinline__ Tile decode_tile(const KParams& p, long long idx, int nblk, int mblk, int bn,
-                                            int rank) {
+                                            int rank, const int* mt = nullptr) {
     Tile t;
     if (!p.var_rows) {
         const long long per_g = (long long)nblk * mblk;
@@ -124,12 +128,12 @@ __device__ __forceinline__ Tile decode_tile(const KParams& p, long long idx, int
         int lo = 0, hi = p.G;
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if ((long long)__ldcg(p.mtile_prefix + mid) * nblk <= idx) lo = mid; else hi = mid;
+            if ((long long)mt[mid] * nblk <= idx) lo = mid; else hi = mid;
         }
-        const int p0 = __ldcg(p.mtile_prefix + lo);
-        const int mt = __ldcg(p.mtile_prefix + lo + 1) - p0;
+        const int p0 = mt[lo];
+        const int nt = mt[lo + 1] - p0;
         const int local = (int)(idx - (long long)p0 * nblk);
-        const int nb = local / mt, mb = local - nb * mt;
+        const int nb = local / nt, mb = local - nb * nt;
         const int m0 = mb * BM;
         const int off = __ldcg(p.grp_off + lo);
         t.g = lo;
@@ -201,6 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t drain_bar = tempty0 + 16;
     const uint32_t rbar0 = drain_bar + 8;      // one per epilogue warp: residual tile loads
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+    int* mt_table = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES + C::STAGING_BYTES + C::BAR_BYTES);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -242,13 +247,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // earlier kernel wrote; only the producer's first weight tiles come before
     // the wait (no kernel writes weights).
     pdl_trigger();
-    if (VAR) pdl_wait();   // the tile count comes from the routing kernels
+    if (VAR) {   // the tile count and prefix come from the routing kernels
+        pdl_wait();
+        for (int i = threadIdx.x; i <= p.G; i += blockDim.x) mt_table[i] = __ldcg(p.mtile_prefix + i);
+        __syncthreads();
+    }
 
     const WaitCtx wc{abort_flag, p.budget_ns, p.err};
     const int nblk = (p.N + BN - 1) / BN;
     const int mblk = (p.M + C::TM - 1) / C::TM;
     const int num_kb = (p.K + BK - 1) / BK;
-    const long long total = p.var_rows ? (long long)__ldcg(p.mtile_prefix + p.G) * nblk
+    const long long total = p.var_rows ? (long long)mt_table[p.G] * nblk
                                        : p.full_tiles + ((long long)p.G * nblk * mblk - p.full_tiles) * p.nsplit;
     const long long unit = blockIdx.x / CG, nunits = gridDim.x / CG;
 
@@ -262,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int npre = 0;
             if (!VAR && unit < total) {
                 const Item it0 = decode_item(p, unit, num_kb);
-                const Tile t0 = decode_tile<CG>(p, it0.tile, nblk, mblk, BN, (int)rank);
+                const Tile t0 = decode_tile<CG>(p, it0.tile, nblk, mblk, BN, (int)rank, mt_table);
                 const int nb0 = t0.n0 + (int)rank * C::BN_LOCAL;
                 npre = min(C::STAGES, it0.kb_hi - it0.kb_lo);
                 for (int k = 0; k < npre; ++k) {   // fresh ring: every slot is free
@@ -278,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool first = true;
             for (long long idx = unit; idx < total && ok; idx += nunits) {
                 const Item item = decode_item(p, idx, num_kb);
-                const Tile t = decode_tile<CG>(p, item.tile, nblk, mblk, BN, (int)rank);
+                const Tile t = decode_tile<CG>(p, item.tile, nblk, mblk, BN, (int)rank, mt_table);
                 const int nb0 = t.n0 + (int)rank * C::BN_LOCAL;
                 for (int kb = item.kb_lo; kb < item.kb_hi; ++kb) {
                     const bool pre = first && kb - item.kb_lo < npre;   // B already issued
@@ -389,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int it = 0;
         for (long long idx = unit; idx < total; idx += nunits, ++it) {
             const Item item = decode_item(p, idx, num_kb);
-            const Tile t = decode_tile<CG>(p, item.tile, nblk, mblk, BN, (int)rank);
+            const Tile t = decode_tile<CG>(p, item.tile, nblk, mblk, BN, (int)rank, mt_table);
             const int acc = it & 1;
             const uint32_t aph = (uint32_t)(it >> 1) & 1u;
             if (!mbar_wait(tfull0 + 8 * acc, aph, wc, SITE_TC_EPILOGUE)) break;
@@ -592,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tempty_leader = CG == 2 ? mapa_shared(tempty0, 0) : tempty0;
         int it = 0;
         for (long long idx = unit; idx < total; idx += nunits, ++it) {
-            const Tile t = decode_tile<CG>(p, idx, nblk, mblk, BN, (int)rank);
+            const Tile t = decode_tile<CG>(p, idx, nblk, mblk, BN, (int)rank, mt_table);
             const int acc = it & 1;
             const uint32_t aph = (uint32_t)(it >> 1) & 1u;
             if (!mbar_wait(tfull0 + 8 * acc, aph, wc, SITE_TC_EPILOGUE)) break;
@@ -821,6 +830,7 @@ static int gemm_tc_pick_bn(int G, int M, int N, int K, bool var_rows, int num_sm
 cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_ns, int num_sms, cudaStream_t s) {
     if (g.K % 8 || g.N % 16 || g.G < 1 || g.M < 0 || g.K < 1) return cudaErrorInvalidValue;
     const bool var = g.grp_cnt != nullptr;
+    if (var && g.G + 1 > kMaxVarGroups) return cudaErrorInvalidValue;
     KParams kp{};
     kp.G = g.G;
     kp.M = g.M;
