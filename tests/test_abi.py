@@ -61,5 +61,20 @@ def test_host_validation_without_gpu(lib_path):
     assert lib.rm_create(ctypes.byref(cfg), ctypes.byref(out)) == rm.RM_ERR_INVALID_ARG
     cfg = rm.rm_config(64, 8, 64, 256, 2, 4, rm.RM_F32, 1e-5, 0)       # MoE needs bf16
     assert lib.rm_create(ctypes.byref(cfg), ctypes.byref(out)) == rm.RM_ERR_UNSUPPORTED
+    # limits of the staged kernels, all rejected before any device call
+    for fields, status in [
+        ((64, 65, 65 * 16, 256, 2, 0, rm.RM_BF16, 1e-5, 0, 1), rm.RM_ERR_UNSUPPORTED),   # T > 64
+        ((64, 8, 128, 256, 2, 33, rm.RM_BF16, 1e-5, 0, 1), rm.RM_ERR_UNSUPPORTED),       # more than 32 experts
+        ((64, 16, 1536, 256, 2, 32, rm.RM_BF16, 1e-5, 0, 1), rm.RM_ERR_UNSUPPORTED),     # router rows beyond 160 KB
+        ((64, 16, 4096, 256, 2, 0, rm.RM_BF16, 1e-5, 0, 1), rm.RM_ERR_UNSUPPORTED),      # D above 2048 (bf16)
+        ((64, 8, 2048, 256, 2, 0, rm.RM_F32, 1e-5, 0, 1), rm.RM_ERR_UNSUPPORTED),        # D above 1024 (fp32)
+        ((64, 64, 2048, 256, 2, 0, rm.RM_BF16, 1e-5, 0, 1), rm.RM_ERR_UNSUPPORTED),      # a sample exceeds shared memory
+        ((64, 8, 64, 256, 2, 0, rm.RM_BF16, 1e-5, 3, 1), rm.RM_ERR_INVALID_ARG),         # unknown activation
+        ((64, 8, 64, 256, 2, 0, rm.RM_BF16, 1e-5, 0, 2), rm.RM_ERR_INVALID_ARG),         # mix_addnorm not 0/1
+        ((64, 8, 64, 256, 2, 0, rm.RM_BF16, 0.0, 0, 1), rm.RM_ERR_INVALID_ARG),          # eps must be > 0
+        ((64, 8, 64, 256, 0, 0, rm.RM_BF16, 1e-5, 0, 1), rm.RM_ERR_INVALID_ARG),         # L < 1
+    ]:
+        cfg = rm.rm_config(*fields)
+        assert lib.rm_create(ctypes.byref(cfg), ctypes.byref(out)) == status, fields
     assert out.value is None
     assert lib.rm_token_mix(None, None, None, 1, None) == rm.RM_ERR_INVALID_ARG

@@ -25,7 +25,9 @@ def _handle(rm, B, T, D, hidden, dtype, n_experts=0, L=1):
 # ------------------------------------------------------------------ token mix
 @pytest.mark.parametrize("dtype,T,dh,B", [
     ("bf16", 8, 8, 3), ("bf16", 16, 48, 5), ("bf16", 16, 20, 7), ("bf16", 32, 48, 2),
-    ("bf16", 1, 64, 4), ("f32", 8, 8, 3), ("f32", 4, 6, 2), ("f32", 2, 4, 9)])
+    ("bf16", 1, 64, 4), ("f32", 8, 8, 3), ("f32", 4, 6, 2), ("f32", 2, 4, 9),
+    ("bf16", 16, 1, 3),     # dh = 1: every output element from a different token
+    ("bf16", 64, 24, 2)])   # T = 64, the largest token count
 def test_token_mix_bitexact(rm, O, dtype, T, dh, B):
     D = T * dh
     X = synth.random_activations((B, T, D), dtype, seed=T + dh)
@@ -173,7 +175,8 @@ def _moe_case(B, T, D, hidden, Ne, seed, router_std=0.1, router_bias=-0.05):
     return blk, S
 
 
-@pytest.mark.parametrize("B,T,D,hidden,Ne", [(300, 4, 64, 128, 8), (129, 2, 256, 256, 3), (1, 4, 64, 64, 2)])
+@pytest.mark.parametrize("B,T,D,hidden,Ne", [(300, 4, 64, 128, 8), (129, 2, 256, 256, 3), (1, 4, 64, 64, 2),
+                                             (40, 2, 1280, 64, 32)])   # 32 experts, router rows at 160 KB
 def test_moe_router_masks_and_output(rm, O, B, T, D, hidden, Ne):
     blk, S = _moe_case(B, T, D, hidden, Ne, seed=B + Ne)
     with _handle(rm, B, T, D, hidden, "bf16", n_experts=Ne) as h:
@@ -258,6 +261,10 @@ def test_argument_errors(rm):
         with pytest.raises(rm.RankMixerError) as e:
             rm.rm_token_mix(h, X, Y, 9)                     # B > B_max
         assert e.value.status == rm.RM_ERR_INVALID_ARG
+        for B in (0, -1):                                   # empty / negative batch
+            with pytest.raises(rm.RankMixerError) as e:
+                rm.rm_token_mix(h, X, Y, B)
+            assert e.value.status == rm.RM_ERR_INVALID_ARG
         with pytest.raises(rm.RankMixerError):
             rm.rm_token_mix(h, X.data_ptr() + 2, Y, 4)      # misaligned
         with pytest.raises(rm.RankMixerError) as e:

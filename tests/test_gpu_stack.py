@@ -54,6 +54,10 @@ def test_small_stack_full(rm, O, name):
     ("bf16", 16, 320, 256, 70, True),   # Pad-Split width: dh = 20 (8-byte pieces)
     ("bf16", 8, 128, 64, 3, True),      # fewer samples than one chunk holds
     ("bf16", 5, 80, 64, 37, False),     # no Add & Norm after mixing
+    ("bf16", 16, 16, 32, 5, True),      # dh = 1
+    ("bf16", 64, 1536, 64, 2, True),    # T = 64 at D = 1536 (a 195 KB staged sample)
+    ("bf16", 32, 2048, 64, 3, True),    # D = 2048, the largest bf16 width
+    ("f32", 16, 1024, 32, 2, True),     # D = 1024, the largest fp32 width
 ])
 def test_stack_small_shapes_full(rm, O, dtype, T, D, hidden, B, mix_addnorm):
     """Two-block stacks compared in full on shapes that exercise the staged
