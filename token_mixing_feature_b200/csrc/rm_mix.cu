@@ -283,7 +283,7 @@ __device__ __forceinline__ void mixed_vec(const E* xs, int rs, int dh, int h, in
     }
 }
 
-template <typename E, bool PRE, int MV, int NV, bool ADDNORM>
+template <typename E, bool PRE, int MV, int NV, bool ADDNORM, int LPR>
 __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
     const E* __restrict__ X, const float* __restrict__ pre_g, const float* __restrict__ pre_b,
     const float2* __restrict__ pstats, int P, const float* __restrict__ g1, const float* __restrict__ b1,
@@ -323,10 +323,13 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
         load_pairs(g1 + c0, g1p);
         load_pairs(b1 + c0, b1p);
     }
-    // statistics pass: lane l of a warp takes vectors l, l + 32, ... of a row
+    // statistics pass: a warp takes 32/LPR rows at a time; lane l of the
+    // row's LPR lanes takes vectors l, l + LPR, ... of it
+    constexpr int RPW = 32 / LPR;
+    const int sl = lane % LPR, sub = lane / LPR;
     MixOff moffA[NV];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) moffA[i] = mix_off<E, MV>((lane + 32 * i) * V, dh, rs);
+    for (int i = 0; i < NV; ++i) moffA[i] = mix_off<E, MV>((sl + LPR * i) * V, dh, rs);
     const int sstride = T * rs;   // elements between the staged samples of a chunk
     int it = 0;
     for (long long c = blockIdx.x; c < nchunks; c += gridDim.x, ++it) {
@@ -345,9 +348,10 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
         }
         E* srow = S + (size_t)row0 * D;
         if (ADDNORM) {
-            // pass A: mean and rstd of Z[h, :] = mix[h, :] + Xh[h, :], one warp
+            // pass A: mean and rstd of Z[h, :] = mix[h, :] + Xh[h, :], LPR lanes
             // per row, sums shifted by the row's first element
-            for (int r = warp; r < R; r += nw) {
+            for (int r0 = warp * RPW; r0 < R; r0 += nw * RPW) {
+                const int r = min(r0 + sub, R - 1);   // lanes past the last row repeat it, unwritten
                 const int s = r / T, h = r - s * T;
                 const E* xsm = xs + (size_t)s * sstride;   // this row's sample
                 const float K = to_f(xsm[h * dh]) + to_f(xs[(size_t)r * rs]);
@@ -355,7 +359,7 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
                 float2 a1 = f2(0.f), a2 = f2(0.f);
 #pragma unroll
                 for (int i = 0; i < NV; ++i) {
-                    const int v = lane + 32 * i;
+                    const int v = sl + LPR * i;
                     if (v < nv) {
                         Vec16<E> xm;
                         mixed_vec<E, MV>(xsm, rs, dh, h, v * V, moffA[i], xm);
@@ -370,9 +374,13 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
                         }
                     }
                 }
-                const float s1 = warp_sum(a1.x + a1.y);
-                const float s2 = warp_sum(a2.x + a2.y);
-                if (lane == 0) {
+                float s1 = a1.x + a1.y, s2 = a2.x + a2.y;
+#pragma unroll
+                for (int o = LPR / 2; o > 0; o >>= 1) {   // within the row's lanes
+                    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+                    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+                }
+                if (sl == 0 && r0 + sub < R) {
                     const float m1 = s1 / D;
                     mean_s[r] = K + m1;
                     rstd_s[r] = rsqrtf(fmaxf(s2 / D - m1 * m1, 0.f) + eps);
@@ -442,7 +450,7 @@ __global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __res
     SampleRing<E> ring;
     // partial sums [spb][groups][D] after the ring and the statistics
     float* part = make_ring<E>(ring, smem, spb * T, D, D, nslots, mean_s, rstd_s);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5;
     const WaitCtx wc{&abort_flag, budget_ns, err};
     if (tid == 0) {
         for (int k = 0; k < nslots; ++k) mbar_init(ring.bar(k), 1);
@@ -587,7 +595,7 @@ inline int mix_groups_cap(int T, int nv, int cap) {
 }
 inline int mix_groups(int T, int nv) { return mix_groups_cap(T, nv, kMixMaxThreads); }
 
-template <typename E, bool PRE, int MV, int NVV, bool ADDNORM>
+template <typename E, bool PRE, int MV, int NVV, bool ADDNORM, int LPR>
 cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps, const float* g1, const float* b1,
                       E* S, int B, int T, int D, float eps, int num_sms, DeviceErr err, uint64_t budget,
                       cudaStream_t s) {
@@ -602,7 +610,7 @@ cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps,
     int nslots;
     size_t smem;
     ring_shape(spb * T, rs, sizeof(E), 0, &nslots, &smem);
-    auto k = mix_ln_kernel<E, PRE, MV, NVV, ADDNORM>;
+    auto k = mix_ln_kernel<E, PRE, MV, NVV, ADDNORM, LPR>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
@@ -618,17 +626,37 @@ cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps,
                       groups, err, budget);
 }
 
+// Lanes per row of the statistics pass: 8 for rows of <= 64 vectors, 16 for
+// <= 128, else 32, so each lane takes at most 8 vectors (NV) and a warp works
+// on 32/LPR rows at once.
 template <typename E, bool PRE, int MV>
-cudaError_t mix_ln_nv(int nvl, int addnorm, const E* X, const float* pg, const float* pb, RowStats ps,
+cudaError_t mix_ln_nv(int nv, int addnorm, const E* X, const float* pg, const float* pb, RowStats ps,
                       const float* g1, const float* b1, E* S, int B, int T, int D, float eps, int num_sms,
                       DeviceErr err, uint64_t budget, cudaStream_t s) {
-    if (!addnorm) return mix_ln_go<E, PRE, MV, 1, false>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
-    if (nvl <= 1) return mix_ln_go<E, PRE, MV, 1, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
-    if (nvl <= 2) return mix_ln_go<E, PRE, MV, 2, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
-    if (nvl <= 3) return mix_ln_go<E, PRE, MV, 3, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
-    if (nvl <= 4) return mix_ln_go<E, PRE, MV, 4, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
-    if (nvl <= 6) return mix_ln_go<E, PRE, MV, 6, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
-    if (nvl <= 8) return mix_ln_go<E, PRE, MV, 8, true>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s);
+#define RM_MIX_GO(NVV, AN, LPRV) \
+    mix_ln_go<E, PRE, MV, NVV, AN, LPRV>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s)
+    if (!addnorm) return RM_MIX_GO(1, false, 32);
+    if (nv <= 64) {
+        const int nvl = (nv + 7) / 8;
+        switch (nvl) {
+            case 1: return RM_MIX_GO(1, true, 8);
+            case 2: return RM_MIX_GO(2, true, 8);
+            case 3: return RM_MIX_GO(3, true, 8);
+            case 4: return RM_MIX_GO(4, true, 8);
+            case 5: return RM_MIX_GO(5, true, 8);
+            case 6: return RM_MIX_GO(6, true, 8);
+            default: return RM_MIX_GO(8, true, 8);
+        }
+    }
+    if (nv <= 128) {
+        const int nvl = (nv + 15) / 16;
+        return nvl <= 5 ? RM_MIX_GO(5, true, 16) : nvl <= 6 ? RM_MIX_GO(6, true, 16) : RM_MIX_GO(8, true, 16);
+    }
+    if (nv <= 256) {
+        const int nvl = (nv + 31) / 32;
+        return nvl <= 5 ? RM_MIX_GO(5, true, 32) : nvl <= 6 ? RM_MIX_GO(6, true, 32) : RM_MIX_GO(8, true, 32);
+    }
+#undef RM_MIX_GO
     return cudaErrorInvalidValue;
 }
 
@@ -637,13 +665,13 @@ cudaError_t mix_ln_typed(const void* X, const float* pg, const float* pb, RowSta
                          const float* b1, void* S, int B, int T, int D, float eps, int addnorm, int num_sms,
                          DeviceErr err, uint64_t budget, cudaStream_t s) {
     constexpr int V = Vec16<E>::N;
-    const int nvl = (D / V + 31) / 32;
+    const int nv = D / V;
     const int dh = D / T;
     const int mv = dh % V == 0 ? V : (dh % (V / 2) == 0 ? V / 2 : 1);
     const E* x = static_cast<const E*>(X);
     E* y = static_cast<E*>(S);
 #define RM_MIX_MV(PREV, MVV) \
-    mix_ln_nv<E, PREV, MVV>(nvl, addnorm, x, pg, pb, ps, g1, b1, y, B, T, D, eps, num_sms, err, budget, s)
+    mix_ln_nv<E, PREV, MVV>(nv, addnorm, x, pg, pb, ps, g1, b1, y, B, T, D, eps, num_sms, err, budget, s)
 #define RM_MIX_PRE(PREV) (mv == V ? RM_MIX_MV(PREV, V) : mv == V / 2 ? RM_MIX_MV(PREV, V / 2) : RM_MIX_MV(PREV, 1))
     const cudaError_t e = pg ? RM_MIX_PRE(true) : RM_MIX_PRE(false);
 #undef RM_MIX_PRE
