@@ -126,6 +126,24 @@ def test_pffn_split_k_tail(rm, O, monkeypatch, T, D, hidden, B):
     assert_close(host64(V0), ref, "bf16", "pffn unsplit", raw=True)
 
 
+@pytest.mark.parametrize("bn", ["256", "192", "128"])
+def test_pffn_dense_tile_widths(rm, O, monkeypatch, bn):
+    """Every dense tile width of the 2-SM kernel on N = 320 (ragged last
+    tile), with the split-K tail (few tiles over K = 1536): 64-column chunks
+    alternate between the epilogue halves, so 192-wide tiles give one half
+    two chunks and the other one."""
+    monkeypatch.setenv("RM_GEMM_BN", bn)
+    T, D, hidden, B = 4, 320, 1536, 300
+    blk = synth.random_like_block(T, D, hidden, "bf16", seed=77)
+    S = synth.random_activations((B, T, D), "bf16", seed=78)
+    with _handle(rm, B, T, D, hidden, "bf16") as h:
+        V = torch.empty(B, T, D, dtype=torch.bfloat16, device="cuda")
+        rm.rm_pffn_forward(h, {k: dev(v) for k, v in blk.items()}, dev(S), V, B)
+        assert rm.rm_sync_status(h) == rm.RM_OK
+    ref = O.pffn(S, blk["W1"], blk["b1"], blk["W2"], blk["b2"])
+    assert_close(host64(V), ref, "bf16", f"pffn BN={bn}", raw=True)
+
+
 # --------------------------------------------------------------------- block
 @pytest.mark.parametrize("dtype,T,D,hidden,B", [
     ("bf16", 16, 768, 3072, 96), ("bf16", 16, 320, 1280, 130), ("bf16", 8, 128, 512, 3),

@@ -92,7 +92,7 @@ struct Cfg {
     static constexpr int NBARS = 2 * STAGES + 5 + kEpiWarps;
     static constexpr int BAR_BYTES = 8 * NBARS + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + TABLE_BYTES;
-    static_assert(BN % 128 == 0 || VAR, "dense tiles leave in 64-column chunks per half");
+    static_assert(BN % 64 == 0 || VAR, "dense tiles leave in 64-column chunks");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
     static_assert(B_BYTES % 1024 == 0, "stage alignment");
     static_assert(CG == 1 || CG == 2, "CTA group");
@@ -387,7 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ew = warp - 2;
         const int quarter = warp & 3;
         const int half = ew >> 2;
-        constexpr int HALF = BN / 2;
+        // 64-column chunks alternate between the two halves (chunk k -> half
+        // k % 2), so every chunk, and the LayerNorm partial of its 64 columns,
+        // belongs to one warp; CH = chunks of the larger share.
+        constexpr int CH = (BN / 64 + 1) / 2;
         const uint32_t tempty_leader = CG == 2 ? mapa_shared(tempty0, 0) : tempty0;
         const uint32_t stg = staging0 + (uint32_t)ew * 4096u;
         const uint32_t rbar = rbar0 + 8u * (uint32_t)ew;
@@ -407,14 +410,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
             const float* bias_g = p.bias + (long long)t.g * p.N;
             const bool split = item.tj >= 0;
-            // this warp's 32 x HALF block of slice s of tail tile tj: [chunk][16 float4][lane]
+            // this warp's block (CH chunks of 32 x 64) of slice s of tail tile tj: [chunk][16 float4][lane]
             const long long wsblk = split ? (((long long)item.tj * p.nsplit) * CG + rank) * kEpiWarps + ew : 0;
-            const long long wstride = (long long)CG * kEpiWarps * (32 * HALF / 4);   // float4s between slices
-            float4* wsw = split ? reinterpret_cast<float4*>(p.sk_ws) + wsblk * (32 * HALF / 4) : nullptr;
+            const long long wstride = (long long)CG * kEpiWarps * (CH * 512);   // float4s between slices
+            float4* wsw = split ? reinterpret_cast<float4*>(p.sk_ws) + wsblk * (CH * 512) : nullptr;
             if (split) {
                 // dump this slice's partial sums, release the accumulator, count the arrival
 #pragma unroll 1
-                for (int c = half * HALF; c < (half + 1) * HALF; c += 64) {
+                for (int c = 64 * half; c < BN; c += 128) {
                     float v[64];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -424,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int e = 0; e < 16; ++e) v[16 * q + e] = w16[e];
                     }
                     tmem_ld_wait();
-                    float4* dst = wsw + (long long)item.slice * wstride + ((c - half * HALF) / 64) * 16 * 32 + lane;
+                    float4* dst = wsw + (long long)item.slice * wstride + ((c - 64 * half) / 128) * 16 * 32 + lane;
 #pragma unroll
                     for (int q = 0; q < 16; ++q) __stcg(dst + q * 32, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
                 }
@@ -447,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             bool ok = true;
 #pragma unroll 1
-            for (int c = half * HALF; c < (half + 1) * HALF; c += 64) {
+            for (int c = 64 * half; c < BN; c += 128) {
                 const int n = t.n0 + c;
                 const bool live = n < p.N;   // warp-uniform
                 if (lane == 0) bulk_wait_read_all();   // the previous store has read the buffer
@@ -460,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float v[64];
                 if (split) {
                     // the tile's sum over its K slices, always in slice order
-                    const float4* src = wsw + ((c - half * HALF) / 64) * 16 * 32 + lane;
+                    const float4* src = wsw + ((c - 64 * half) / 128) * 16 * 32 + lane;
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         const float4 a = __ldcg(src + q * 32);
@@ -490,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tmem_ld_wait();
                 }
-                if (!split && c + 64 >= (half + 1) * HALF) {   // last chunk: the accumulator may be reused
+                if (!split && c + 128 >= BN) {   // this warp's last chunk: the accumulator may be reused
                     tc_fence_before();
                     if (CG == 2 && !leader) mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
                     else mbar_arrive(tempty0 + 8 * acc);
@@ -804,7 +807,7 @@ static int gemm_tc_pick_bn(int G, int M, int N, int K, bool var_rows, int num_sm
     double best_s = -1.0;
     for (int i = 0; i < 4; ++i) {
         const int bn = cands[i];
-        if (!var_rows && bn % 128) continue;   // dense tiles leave in 64-column chunks per half
+        if (!var_rows && bn % 64) continue;   // dense tiles leave in 64-column chunks
         const long long nblk = (N + bn - 1) / bn;
         const double col_fill = (double)N / (double)(nblk * bn);
         double wave_fill = 1.0;
@@ -870,7 +873,7 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     }
     if (const char* e = getenv("RM_GEMM_BN")) {
         const int v = atoi(e);
-        if (v == 256 || v == 128 || (var && (v == 192 || v == 160))) bn = v;
+        if (v == 256 || v == 192 || v == 128 || (var && v == 160)) bn = v;
     }
     Maps m;
     memset(&m, 0, sizeof(m));
@@ -932,9 +935,18 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
             default: return launch_bn<128, 1, true>(g.epi, m, kp, grid, s);
         }
     }
-    if (cg == 2) return bn == 256 ? launch_bn<256, 2, false>(g.epi, m, kp, grid, s)
-                                  : launch_bn<128, 2, false>(g.epi, m, kp, grid, s);
-    return bn == 256 ? launch_bn<256, 1, false>(g.epi, m, kp, grid, s) : launch_bn<128, 1, false>(g.epi, m, kp, grid, s);
+    if (cg == 2) {
+        switch (bn) {
+            case 256: return launch_bn<256, 2, false>(g.epi, m, kp, grid, s);
+            case 192: return launch_bn<192, 2, false>(g.epi, m, kp, grid, s);
+            default: return launch_bn<128, 2, false>(g.epi, m, kp, grid, s);
+        }
+    }
+    switch (bn) {
+        case 256: return launch_bn<256, 1, false>(g.epi, m, kp, grid, s);
+        case 192: return launch_bn<192, 1, false>(g.epi, m, kp, grid, s);
+        default: return launch_bn<128, 1, false>(g.epi, m, kp, grid, s);
+    }
 }
 
 size_t gemm_tc_split_ws_bytes(int num_sms) { return (size_t)num_sms * BM * 256 * sizeof(float); }
