@@ -513,7 +513,9 @@ __global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __res
                     dst[q] = make_float4(acc[2 * q].x, acc[2 * q].y, acc[2 * q + 1].x, acc[2 * q + 1].y);
             }
         }
-        __syncthreads();
+        __syncthreads();   // the slot is free again: refill it before combining the partials
+        const long long nc = c + (long long)nslots * gridDim.x;
+        if (warp == 0 && nc < nchunks) ring.issue(cur, X + (size_t)nc * spb * TD, chunk_samples(nc) * T);
         for (int i = tid; i < ns * D; i += blockDim.x) {
             const int sm = i / D, cc = i - sm * D;
             const float* ps = part + (size_t)sm * groups * D + cc;
@@ -521,9 +523,7 @@ __global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __res
             for (int q = 1; q < groups; ++q) a += ps[(size_t)q * D];
             pooled[(size_t)(c * spb + sm) * D + cc] = fmaf(__ldg(g + cc), a * invT, __ldg(bta + cc));
         }
-        __syncthreads();   // slot, statistics and partials are free again
-        const long long nc = c + (long long)nslots * gridDim.x;
-        if (warp == 0 && nc < nchunks) ring.issue(cur, X + (size_t)nc * spb * TD, chunk_samples(nc) * T);
+        __syncthreads();   // statistics and partials are free again
     }
     if (tid == 0) ring.drain(wc, SITE_LN_POOL);
 }
