@@ -23,7 +23,8 @@ constexpr int kThreads = 256;
 
 // Router logits, ReLU gates and per-expert active counts.  CTA (t, chunk)
 // stages router t's weights Wr_t [Ne][D] in shared memory once and serves
-// kRouteRows samples b.  A warp takes RW = 32 / NE rows (b, t) of S at a time:
+// `rows` samples b (chosen on the host so the grid fills the SMs in one
+// wave).  A warp takes RW = 32 / NE rows (b, t) of S at a time:
 // lane l multiplies columns 4l, 4l+128, ... of all RW rows with all NE
 // experts, so each shared-memory weight vector feeds RW rows and each S
 // vector NE experts, with conflict-free 16-byte shared loads.  The RW x NE =
@@ -31,7 +32,6 @@ constexpr int kThreads = 256;
 // transposing butterfly (31 shuffles in all), after which lane l holds the
 // logit of row l / NE, expert l % NE.  Active counts are summed in shared
 // memory and added to the global counts once per CTA.
-constexpr int kRouteRows = 64;
 
 // acc[i] summed over the warp; afterwards acc[0] of lane l is the sum of
 // everyone's acc[l].
@@ -53,14 +53,15 @@ template <int NE>
 __global__ void __launch_bounds__(kThreads) route_kernel(const __nv_bfloat16* __restrict__ S,
                                                          const float* __restrict__ Wr,
                                                          const float* __restrict__ br, float* __restrict__ gates,
-                                                         int* __restrict__ counts, int B, int T, int D, int Ne) {
+                                                         int* __restrict__ counts, int B, int T, int D, int Ne,
+                                                         int rows) {
     pdl_enter();
     constexpr int RW = 32 / NE;
     extern __shared__ __align__(16) float wsm[];   // [Ne][D]
     __shared__ int cnt[NE];
     const int t = blockIdx.x;
-    const int b0 = blockIdx.y * kRouteRows;
-    const int bend = min(B, b0 + kRouteRows);
+    const int b0 = blockIdx.y * rows;
+    const int bend = min(B, b0 + rows);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     {
         const float4* src = reinterpret_cast<const float4*>(Wr + (size_t)t * Ne * D);
@@ -307,14 +308,30 @@ cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, co
                              int D, int Ne, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(w.counts, 0, sizeof(int) * T * Ne, s);
     if (e != cudaSuccess) return e;
-    const dim3 grid(T, (B + kRouteRows - 1) / kRouteRows);
     const size_t smem = sizeof(float) * (size_t)Ne * D;
     const auto* Sb = static_cast<const __nv_bfloat16*>(S);
+    int num_sms = 0, dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    // Rows per CTA: the (T x chunks) grid fills the resident CTA slots once;
+    // a multiple of the rows a CTA's warps take per pass (8 warps x 32/NE).
 #define RM_ROUTE(NEV)                                                                                    \
     {                                                                                                    \
         e = cudaFuncSetAttribute(route_kernel<NEV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
         if (e != cudaSuccess) return e;                                                                  \
-        e = launch_pdl(route_kernel<NEV>, grid, kThreads, smem, s, Sb, Wr, br, w.gates, w.counts, B, T, D, Ne); \
+        int occ = 0;                                                                                     \
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, route_kernel<NEV>, kThreads, smem);      \
+        if (e != cudaSuccess) return e;                                                                  \
+        const int per_pass = (kThreads / 32) * (32 / NEV);                                               \
+        const long long slots = (long long)num_sms * (occ > 0 ? occ : 1);                                \
+        long long chunks = slots / T;                                                                    \
+        if (chunks < 1) chunks = 1;                                                                      \
+        long long rows = (B + chunks - 1) / chunks;                                                      \
+        rows = (rows + per_pass - 1) / per_pass * per_pass;                                              \
+        const dim3 grid(T, (unsigned)((B + rows - 1) / rows));                                           \
+        e = launch_pdl(route_kernel<NEV>, grid, kThreads, smem, s, Sb, Wr, br, w.gates, w.counts, B, T, D, Ne, \
+                       (int)rows);                                                                       \
         if (e != cudaSuccess) return e;                                                                  \
     }
     if (Ne <= 1) RM_ROUTE(1)
