@@ -9,15 +9,20 @@
 // for every group g, with A rows addressed through strides (so the token-t
 // rows of S [B, T, D] are read in place) and W stored [G][N][K].
 //
-// Structure (one CTA per SM, persistent over 128 x BN output tiles):
+// Structure (persistent; dense problems use CTA pairs, cluster of 2, with
+// 256 x BN tiles and tcgen05.mma.cta_group::2; expert groups use single CTAs
+// with 128 x BN tiles):
 //   warp 0      TMA producer: A and W tiles (64-wide K slices, 128-byte
 //               swizzle) into a STAGES-deep shared-memory ring.
-//   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=BN, K=16)
-//               into a double-buffered fp32 accumulator in tensor memory and
-//               releases ring slots / accumulators with tcgen05.commit.
-//   warps 2..9  epilogue: tcgen05.ld of the accumulator, bias + GELU, bias +
-//               residual, or gate * (acc + bias), bf16 stores.  Two warps per
-//               32-lane TMEM quarter, each taking half of the columns.
+//   warp 1      MMA issuer: one thread issues tcgen05.mma (K=16 per
+//               instruction) into a double-buffered fp32 accumulator in tensor
+//               memory and releases ring slots / accumulators with
+//               tcgen05.commit.
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator, bias + GELU / ReLU,
+//               bias + residual (+ LayerNorm partials), or gate * (acc + bias),
+//               bf16 out (TMA stores of 64-column chunks for dense tiles).
+//               Two warps per 32-lane TMEM quarter.
+// The last partial wave of dense tiles is split along K (split-K tail).
 // Every mbarrier wait is bounded (rm_device.cuh); a wait that runs out records
 // RM_ERR_DEVICE_TIMEOUT, stops the CTA's other roles, drains in-flight copies
 // and MMAs, frees tensor memory and returns.

@@ -4,24 +4,26 @@
 // Token mixing with H = T heads (fun-rec chapter "Rankmixer: 硬件效率优化",
 // section Token Mixing机制) sends chunk h of token t to position t*dh of output
 // token h (dh = D / T).  Every output row of a sample reads a slice of every
-// input row, so the sample is the unit of work: a persistent CTA stages whole
-// samples ([T, D], contiguous) in shared memory with one cp.async.bulk each,
-// into a two-slot ring when two samples fit (the next sample's copy overlaps
-// the current one's arithmetic) and one slot otherwise (then two CTAs per SM
-// overlap each other).  The permutation is applied through shared-memory
-// addressing with 16-byte vectors, so X is read from HBM once and S written
-// once, with no transpose pass; one warp owns one output row.
+// input row, so the sample is the unit of work: persistent CTAs (two per SM)
+// stage whole samples -- or chunks of several small samples -- in a
+// shared-memory ring of 1-4 slots with cp.async.bulk, so the next chunk's
+// copy overlaps the current one's arithmetic.  The permutation is applied
+// through shared-memory addressing with 16-byte vectors (rows padded so the
+// pieces consecutive lanes gather fall in consecutive banks), so X is read
+// from HBM once and S written once, with no transpose pass.  Row statistics
+// take LPR = 8/16/32 lanes per row (pass A); the element-wise pass (pass B)
+// gives each thread one 16-byte column vector of a row group.
 //
 // The previous block's LayerNorm (PRE) uses row statistics produced where the
 // row was written (the grouped GEMM's epilogue, the MoE combine, or
-// row_stats_kernel) as partial (mean, M2) pairs over P column slices, merged
-// here with Chan's pairwise formula -- no extra pass over the rows.
+// row_stats_kernel) as partial (mean, M2) pairs over P equal column slices,
+// merged here in two warp sums -- no extra pass over the rows.
 //
 // mix_ln:  Xh = PRE ? LN_pre(X) : X                       (per token row)
 //          Z[h, t*dh + j] = Xh[t, h*dh + j] + Xh[h, t*dh + j]
-//          S[h, :] = LN1(Z[h, :])             (one warp per output row)
+//          S[h, :] = LN1(Z[h, :])
 //          or, without the Add & Norm after mixing, S[h, t*dh + j] = Xh[t, h*dh + j]
-// ln_pool: pooled[b, :] = (1/T) sum_t LN(X[b, t, :])  (ascending t)
+// ln_pool: pooled[b, :] = (1/T) sum_t LN(X[b, t, :])  (row groups, then groups in order)
 #include <cuda_bf16.h>
 
 #include "rm_device.cuh"
