@@ -109,17 +109,27 @@ class ClockSampler:
                 "power_w_max": pmax, "samples": len(rows), "reasons": reasons}
 
 
+def code_digest(path: str) -> str:
+    """sha256[:16] of a source file with comments and whitespace removed, so a
+    comment-only edit does not count as a change of the kernel."""
+    src = open(path, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    src = re.sub(r"\s+", "", src)
+    return hashlib.sha256(src.encode()).hexdigest()[:16]
+
+
 def traffic_from_profiles(kernel_key: str):
     """Per-launch DRAM bytes of a kernel from a committed ncu summary, if the
-    summary was taken on the current source of the GEMM kernel."""
+    summary was taken on the current code of the GEMM kernel."""
     path = os.path.join(ROOT, "profiles", "ncu_gemm_tc_rm1b.md")
     src = os.path.join(ROOT, "token_mixing_feature_b200", "csrc", "rm_gemm_tc.cu")
     try:
         text = open(path).read()
-        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        digest = code_digest(src)
     except OSError:
         return None
-    m = re.search(r"source sha256\[:16\]:\s*([0-9a-f]{16})", text)
+    m = re.search(r"code sha256\[:16\]:\s*([0-9a-f]{16})", text)
     if not m or m.group(1) != digest:
         return None
     m = re.search(rf"dram_bytes_per_launch\s+{re.escape(kernel_key)}\s*[:=]\s*([0-9.eE+]+)", text)

@@ -50,3 +50,17 @@ def test_moe_flops_need_active_counts():
         roofline.stack_flops(wl)
     f = roofline.stack_flops(wl, [1000, 2000])
     assert f == 3000 * 4 * 768 * 768 + 2 * (2 * 2048 * 16 * 768 * 8)
+
+
+def test_code_digest_ignores_comments_only(tmp_path):
+    """The benchmark reports the committed ncu traffic only while the GEMM's
+    code is the captured one; comment or whitespace edits are not changes."""
+    import bench
+    a = tmp_path / "a.cu"
+    a.write_text("int f(int x) {\n    return x + 1;  // one\n}\n")
+    b = tmp_path / "b.cu"
+    b.write_text("/* header */\nint f(int x) {\n  return x + 1;\n}  // trailing\n")
+    c = tmp_path / "c.cu"
+    c.write_text("int f(int x) {\n    return x + 2;\n}\n")
+    assert bench.code_digest(str(a)) == bench.code_digest(str(b))
+    assert bench.code_digest(str(a)) != bench.code_digest(str(c))
