@@ -180,6 +180,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread may be parked by the hardware
+// until the phase completes or `ns` nanoseconds pass, instead of re-polling,
+// which keeps waiting warps (producers, epilogues between tiles, ring waits)
+// off the issue slots and saves power.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Context of the bounded waits of one CTA: a shared abort flag, the budget and
 // the global error word.  A wait that runs out records RM_ERR_DEVICE_TIMEOUT
 // with its site id and raises the abort flag so the CTA's other roles stop.
@@ -195,15 +211,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
                                           bool honour_abort = true) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    uint32_t n = 0;
-    while (!mbar_try_wait(bar, parity)) {
-        if ((++n & 15u) == 0) {
-            if (honour_abort && *w.abort) return false;
-            if (globaltimer_ns() - t0 > w.budget_ns) {
-                record_error(w.err, RM_ERR_DEVICE_TIMEOUT, site);
-                *w.abort = 1;
-                return false;
-            }
+    while (!mbar_try_wait_sleep(bar, parity, 20000u)) {   // each return: at most ~20 us parked
+        if (honour_abort && *w.abort) return false;
+        if (globaltimer_ns() - t0 > w.budget_ns) {
+            record_error(w.err, RM_ERR_DEVICE_TIMEOUT, site);
+            *w.abort = 1;
+            return false;
         }
     }
     return true;
