@@ -240,7 +240,8 @@ typedef enum {
     RM_K_MOE_COMBINE = 8,
     RM_K_PADSPLIT = 9,
     RM_K_HEAD = 10,
-    RM_K_COUNT = 11
+    RM_K_FFN_FUSED = 11,  /* both FFN projections in one kernel (narrow tokens)      */
+    RM_K_COUNT = 12
 } rm_kernel_kind;
 
 /* Start recording a CUDA event pair around each kernel launch made through h

@@ -93,6 +93,18 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// GELU (tanh form) of a pair: 0.5 x (1 + tanh(u)), u = sqrt(2/pi) x (1 + 0.044715 x^2),
+// written as h + h tanh(u) with h = x/2; paired fp32 arithmetic, tanh from the SFU.
+__device__ __forceinline__ float2 gelu_tanh_pair(float2 x) {
+    const float2 p = f2_fma(f2_mul(x, x), f2(0.7978845608028654f * 0.044715f), f2(0.7978845608028654f));
+    const float2 u = f2_mul(x, p);
+    float2 th;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(u.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(u.y));
+    const float2 hx = f2_mul(x, f2(0.5f));
+    return f2_fma(hx, th, hx);
+}
+
 // ------------------------------------------------------ programmatic launch
 // Every kernel of the library is launched with programmatic stream
 // serialisation (launch_pdl), so it may begin while the previous kernel of

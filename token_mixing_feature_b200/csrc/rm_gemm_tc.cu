@@ -32,9 +32,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
-#include <mutex>
 
 #include "rm_device.cuh"
+#include "rm_tmap.h"
 
 namespace rm {
 namespace {
@@ -177,18 +177,6 @@ __device__ __forceinline__ Item decode_item(const KParams& p, long long idx, int
         it.kb_hi = (int)((long long)(it.slice + 1) * num_kb / p.nsplit);
     }
     return it;
-}
-
-// GELU (tanh form) of a pair: 0.5 x (1 + tanh(u)), u = sqrt(2/pi) x (1 + 0.044715 x^2),
-// written as h + h tanh(u) with h = x/2; paired fp32 arithmetic, tanh from the SFU.
-__device__ __forceinline__ float2 gelu_tanh_pair(float2 x) {
-    const float2 p = f2_fma(f2_mul(x, x), f2(0.7978845608028654f * 0.044715f), f2(0.7978845608028654f));
-    const float2 u = f2_mul(x, p);
-    float2 th;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(u.x));
-    asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(u.y));
-    const float2 hx = f2_mul(x, f2(0.5f));
-    return f2_fma(hx, th, hx);
 }
 
 template <int BN, int EPI, int CG, bool VAR>
@@ -703,39 +691,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------- host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    });
-    return fn;
-}
-
-// 3-D bf16 tensor map: dims d0 (contiguous), d1, d2 with byte strides s1, s2;
-// box (64, b1, b2), 128-byte swizzle, zero fill out of bounds.
-bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
-              uint32_t b1, uint32_t b2) {
-    EncodeTiledFn fn = get_encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {d0, d1, d2};
-    cuuint64_t strides[2] = {s1, s2};
-    cuuint32_t box[3] = {(cuuint32_t)BK, b1, b2};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 struct Maps {
     CUtensorMap a, b, o, r;
 };

@@ -29,7 +29,7 @@ EXPORTED = (
     "rm_stack_forward_host_async", "rm_host_wait",
 )
 RM_STATIC_SCRATCH_BYTES = 16 << 20
-RM_K_COUNT = 11
+RM_K_COUNT = 12
 
 
 class rm_config(ctypes.Structure):
