@@ -3,8 +3,8 @@ activation kept on chip) against the fp64 oracle, through the C ABI.
 
 RM_FFN_FUSED=1 selects the fused kernel (run_pffn uses the two grouped
 GEMMs otherwise).
-Shapes cover every supported width D (one or two second-projection MMAs per
-chunk, D = 64 where one epilogue half has no output slice), one and several
+Shapes cover every supported width D <= 320 (one or two second-projection
+MMAs per chunk, D = 64 where one epilogue half has no output slice), one and several
 hidden chunks, ragged row tails (a partial tile, a CTA with no valid row,
 B = 1), and more tiles than CTA pairs, so that pairs run the cross-tile
 pipeline (the next tile's first hidden chunk before the previous tile's
@@ -45,7 +45,7 @@ def _pffn(rm, blk, S, B, T, D, hidden, act="tanh"):
     (2, 192, 384, 513, "erf"),      # N = 192 second projection, one row in the last tile
     (4, 256, 1024, 256, "tanh"),    # exactly one tile per token, 8 hidden chunks
     (16, 320, 1280, 257, "tanh"),   # the Pad-Split width: two 160-wide MMAs per chunk
-    (8, 384, 512, 130, "tanh"),     # D = 384: acc2 fills columns [0, 384), shallowest ring
+    (8, 256, 384, 130, "tanh"),     # one 256-wide second-projection MMA, 3 hidden chunks
     (2, 320, 128, 1, "tanh"),       # B = 1, a single hidden chunk
     (64, 64, 256, 2048, "tanh"),    # 512 tiles: every CTA pair runs several tiles
     (32, 320, 256, 1024, "relu"),   # 128 tiles over the pairs: some run two
@@ -58,7 +58,7 @@ def test_ffn_fused_parity(rm, O, fused, T, D, hidden, B, act):
     assert_close(host64(V), ref, "bf16", f"fused pffn D={D} kD={hidden} B={B} {act}", raw=True)
 
 
-@pytest.mark.parametrize("T,D,hidden,B", [(16, 320, 1280, 300), (8, 256, 512, 700), (4, 384, 768, 260)])
+@pytest.mark.parametrize("T,D,hidden,B", [(16, 320, 1280, 300), (8, 256, 512, 700), (4, 192, 768, 260)])
 def test_ffn_fused_matches_two_gemm_path(rm, monkeypatch, T, D, hidden, B):
     """Same sums in the same K order as the two grouped GEMMs without their
     split-K tail (both round the hidden activation to bf16 before the second
@@ -122,3 +122,20 @@ def test_ffn_fused_padsplit_size(rm, O, monkeypatch):
             assert rm.rm_sync_status(h) == rm.RM_OK
         assert set(prof) == kinds, prof
         assert_close(host64(V[rows.cuda()]), ref, "bf16", f"pffn {kinds}, Pad-Split size (sampled rows)", raw=True)
+
+
+def test_ffn_fused_unsupported_width_uses_gemms(rm, O, fused):
+    """D = 384 leaves no tensor-memory room for the hidden chunk: even when
+    asked for, the library runs the two grouped GEMMs."""
+    T, D, hidden, B = 8, 384, 512, 130
+    blk = synth.random_like_block(T, D, hidden, "bf16", seed=11)
+    S = synth.random_activations((B, T, D), "bf16", seed=12)
+    with rm.rm_create(B, T, D, hidden, 1, 0, "bf16") as h:
+        V = torch.empty(B, T, D, dtype=torch.bfloat16, device="cuda")
+        rm.rm_profile_begin(h, 8)
+        rm.rm_pffn_forward(h, {k: dev(v) for k, v in blk.items()}, dev(S), V, B)
+        prof = rm.rm_profile_end(h)
+        assert rm.rm_sync_status(h) == rm.RM_OK
+    assert set(prof) == {"gemm1", "gemm2"}, prof
+    ref = O.pffn(S, blk["W1"], blk["b1"], blk["W2"], blk["b2"])
+    assert_close(host64(V), ref, "bf16", "pffn D=384", raw=True)

@@ -6,12 +6,13 @@
 // section Per-Token FFN) gives token t its own two-layer FFN:
 //     V[m, t, :] = GELU(S[m, t, :] W1_t^T + b1_t) W2_t^T + b2_t  (+ S[m, t, :])
 // with W1 stored [T][kD][D] and W2 [T][D][kD].  The two-GEMM path writes
-// the hidden [T, B, kD] to HBM and reads it back.  When D <= 384 the output
-// block of a 256-row tile fits in tensor memory next to one hidden chunk, so
-// this kernel walks the hidden dimension in chunks of 128 columns instead:
+// the hidden [T, B, kD] to HBM and reads it back.  When D <= 320 the output
+// block of a 256-row tile fits in tensor memory next to one hidden chunk and
+// its accumulator, so this kernel walks the hidden dimension in chunks of 128
+// columns instead:
 //     acc1  = S_tile W1_t[chunk]^T                   (tcgen05, tensor memory)
-//     Hc    = bf16(act(acc1 + b1_t[chunk]))          (epilogue warps -> shared memory)
-//     acc2 += Hc W2_t[:, chunk]^T                    (tcgen05, tensor memory)
+//     Hc    = bf16(act(acc1 + b1_t[chunk]))          (epilogue warps -> tensor memory)
+//     acc2 += Hc W2_t[:, chunk]^T                    (tcgen05, A operand in tensor memory)
 // and after the last chunk stores V = bf16(acc2 + b2_t (+ S)) with the
 // LayerNorm partials (mean, M2) of every 64-column slice of each stored row:
 // the same outputs, rounded the same way, as the two-GEMM path.
@@ -25,11 +26,12 @@
 //               works on one while the epilogue turns the other's
 //               accumulator into the next hidden chunk
 //   warps 2..9  epilogue: hidden chunks (tcgen05.ld -> bias + activation ->
-//               bf16 into the 128-byte-swizzled operand layout), then the
-//               previous tile's output rows once the next tile's first
-//               hidden chunk is written
+//               bf16 pairs -> tcgen05.st), then the previous tile's output
+//               rows once the next tile's first hidden chunk is written
 //   warp 10     TMA: W2 chunks through ring 2
-// Tensor memory (512 columns): acc2 in columns [0, D), acc1 in [384, 512).
+// Tensor memory (512 columns): acc2 in columns [0, D), the bf16 hidden chunk
+// in [320, 384) (two values per column: the second projection's A operand),
+// acc1 in [384, 512).  Only the weights pass through shared memory.
 // Every mbarrier wait is bounded (rm_device.cuh); a wait that runs out
 // records RM_ERR_DEVICE_TIMEOUT, stops the CTA's other roles, drains
 // in-flight copies and MMAs, frees tensor memory and returns.
@@ -51,6 +53,7 @@ constexpr int HC = 128;          // hidden columns per chunk
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = (3 + kEpiWarps) * 32;
 constexpr int kW2Warp = 2 + kEpiWarps;
+constexpr int H_COL = 320;       // tensor-memory column of the bf16 hidden chunk (HC / 2 columns)
 constexpr int ACC1_COL = 384;    // tensor-memory column of the hidden-chunk accumulator
 constexpr int TMEM_COLS = 512;
 constexpr int BLK_BYTES = BM * BK * 2;   // one swizzled [128 x 64] operand block
@@ -71,27 +74,26 @@ struct FParams {
 };
 
 // Shared-memory plan for width D.  The second projection's D output columns
-// are one MMA (D <= 256) or two of D/2 (N <= 256 per MMA); for a 2-SM MMA
-// each CTA holds half of the B rows of each, so a ring-2 stage is this CTA's
-// halves of both, one K block deep.
+// are one MMA (D <= 256) or two of D/2 (N <= 256, a multiple of 32 with A in
+// tensor memory); for a 2-SM MMA each CTA holds half of the B rows of each,
+// so a ring-2 stage is this CTA's halves of both, one K block deep.
 template <int D>
 struct FCfg {
     static constexpr int KB1 = D / BK;                        // K blocks of the first projection
     static constexpr int NSUB = D > 256 ? 2 : 1;
     static constexpr int NSUBN = D / NSUB;                    // N of one second-projection MMA
     static constexpr int A_BYTES = KB1 * BLK_BYTES;           // this CTA's 128 S rows
-    static constexpr int H_BYTES = (HC / BK) * BLK_BYTES;     // one hidden chunk (this CTA's rows)
     static constexpr int W1_STAGE = (HC / 2) * BK * 2;        // this CTA's 64 W1 rows, one K block
     static constexpr int W2_SUB = (NSUBN / 2) * BK * 2;       // this CTA's W2 rows of one MMA, one K block
     static constexpr int W2_STAGE = NSUB * W2_SUB;
-    static constexpr int R2 = 2;
+    static constexpr int R2 = 4;
     static constexpr int BAR_BYTES = 512;
-    static constexpr int R1_RAW = (227 * 1024 - 1024 - BAR_BYTES - A_BYTES - H_BYTES - R2 * W2_STAGE) / W1_STAGE;
+    static constexpr int R1_RAW = (227 * 1024 - 1024 - BAR_BYTES - A_BYTES - R2 * W2_STAGE) / W1_STAGE;
     static constexpr int R1 = R1_RAW > 16 ? 16 : R1_RAW;
     static constexpr int NBARS = 2 * R1 + 2 * R2 + 9;
-    static constexpr int SMEM_BYTES = 1024 + A_BYTES + H_BYTES + R1 * W1_STAGE + R2 * W2_STAGE + BAR_BYTES;
-    static_assert(D % 64 == 0 && D >= 64 && D <= ACC1_COL, "D");
-    static_assert(NSUBN % 16 == 0 && NSUBN <= 256 && (NSUBN / 2) % 8 == 0, "second-projection MMA width");
+    static constexpr int SMEM_BYTES = 1024 + A_BYTES + R1 * W1_STAGE + R2 * W2_STAGE + BAR_BYTES;
+    static_assert(D % 64 == 0 && D >= 64 && D <= H_COL, "D");
+    static_assert(NSUBN % 32 == 0 && NSUBN <= 256 && (NSUBN / 2) % 8 == 0, "second-projection MMA width");
     static_assert(W2_SUB % 1024 == 0 && W1_STAGE % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
     static_assert(R1 >= 4, "ring 1 depth");
     static_assert(8 * NBARS + 8 <= BAR_BYTES, "barrier area");
@@ -107,11 +109,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw_addr = smem_u32(smem_raw);
     unsigned char* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
     const uint32_t sA = smem_u32(smem);
-    const uint32_t sH = sA + C::A_BYTES;
-    const uint32_t sW1 = sH + C::H_BYTES;
+    const uint32_t sW1 = sA + C::A_BYTES;
     const uint32_t sW2 = sW1 + C::R1 * C::W1_STAGE;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::A_BYTES + C::H_BYTES + C::R1 * C::W1_STAGE +
-                                                 C::R2 * C::W2_STAGE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::A_BYTES + C::R1 * C::W1_STAGE + C::R2 * C::W2_STAGE);
     const uint32_t full1 = smem_u32(bars);
     const uint32_t empty1 = full1 + 8 * C::R1;
     const uint32_t full2 = empty1 + 8 * C::R1;
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t emptyA = fullA + 8;            // S tile no longer read (both CTAs)
     const uint32_t acc1_full = emptyA + 8;        // hidden-chunk accumulator ready (both CTAs)
     const uint32_t acc1_empty = acc1_full + 8;    // ... read by every epilogue thread (even CTA)
-    const uint32_t h_full = acc1_empty + 8;       // hidden chunk written (even CTA)
+    const uint32_t h_full = acc1_empty + 8;       // hidden chunk stored in tensor memory (even CTA)
     const uint32_t h_empty = h_full + 8;          // ... consumed by the second projection (both CTAs)
     const uint32_t acc2_full = h_empty + 8;       // tile's output accumulator complete (both CTAs)
     const uint32_t acc2_empty = acc2_full + 8;    // ... read by every epilogue thread (even CTA)
@@ -258,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc2 = idesc_bf16_f32(2 * BM, C::NSUBN);
             const uint32_t t_acc1 = tmem_base + ACC1_COL;
             const uint32_t t_acc2 = tmem_base;
+            const uint32_t t_h = tmem_base + H_COL;
             int s1 = 0, s2 = 0;
             uint32_t ph1 = 0, ph2 = 0;
             bool ok = true, any = false;
@@ -269,15 +270,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kb = 0; kb < HC / BK; ++kb) {
                     if (!mbar_wait(full2 + 8 * s2, ph2, wc, SITE_TC_MMA_FULL)) return false;
                     tc_fence_after();
-                    const uint64_t adesc = smem_desc_k_sw128(sH + kb * BLK_BYTES);
                     const uint32_t sb = sW2 + s2 * C::W2_STAGE;
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         const uint32_t accum = (c2 != 0 || kb != 0 || k != 0) ? 1u : 0u;
+                        // hidden columns [64 kb + 16 k, + 16): 8 packed tensor-memory columns
+                        const uint32_t a_tmem = t_h + (uint32_t)(32 * kb + 8 * k);
 #pragma unroll
                         for (int sub = 0; sub < C::NSUB; ++sub)
-                            tc_mma_f16_pair(t_acc2 + (uint32_t)(sub * C::NSUBN), adesc + (uint64_t)(2 * k),
-                                            smem_desc_k_sw128(sb + sub * C::W2_SUB) + (uint64_t)(2 * k), idesc2, accum);
+                            tc_mma_f16_pair_ts(t_acc2 + (uint32_t)(sub * C::NSUBN), a_tmem,
+                                               smem_desc_k_sw128(sb + sub * C::W2_SUB) + (uint64_t)(2 * k), idesc2, accum);
                     }
                     tc_commit_pair_mc(empty2 + 8 * s2, 0x3);
                     if (++s2 == C::R2) { s2 = 0; ph2 ^= 1u; }
@@ -341,31 +343,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         // --------------------------------------------------------- epilogue
         // Warp w reads TMEM lanes 32 (w % 4) .. + 31 (this CTA's rows) and
         // half (w - 2) / 4 of the columns: hidden columns [64 half, 64 half
-        // + 64) of each chunk (= swizzled operand block `half`), and output
-        // slices of 64 columns alternating between the halves.
+        // + 64) of each chunk (stored as tensor-memory columns H_COL + 32 half
+        // .. + 31), and output slices of 64 columns alternating between the
+        // halves.
         const int ew = warp - 2;
         const int quarter = warp & 3;
         const int half = ew >> 2;
         const int rl = quarter * 32 + lane;
         const uint32_t lane_tmem = tmem_base + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t hrow = sH + (uint32_t)(half * BLK_BYTES + rl * 128);
-        const uint32_t swz = (uint32_t)(rl & 7);
         // Waits give one answer per warp (the signals below converge the warp).
         auto warp_wait = [&](uint32_t bar, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc, SITE_TC_EPILOGUE));
         };
-        // One arrival per warp: each lane's fence (tcgen05 reads done, or
-        // shared-memory writes made visible to the async proxy), then the
-        // warp converges and lane 0 signals the pair's even CTA.
+        // One arrival per warp: each lane's tcgen05 loads or stores are
+        // complete and fenced, then the warp converges and lane 0 signals the
+        // pair's even CTA (from the odd CTA without release semantics: the
+        // arrival publishes no memory writes).
         auto arrive_even = [&](uint32_t bar) {
             __syncwarp();
             if (lane == 0) {
                 if (leader) mbar_arrive(bar);
-                else mbar_arrive_cluster(mapa_shared(bar, 0));
+                else mbar_arrive_cluster_relaxed(mapa_shared(bar, 0));
             }
         };
         // hidden chunk c of group g (the k-th chunk of this pair)
         auto hidden_chunk = [&](int g, int c, long long k) -> bool {
+            // the chunk's biases first (weights: no wait needed), then its accumulator
+            const float4* b4 = reinterpret_cast<const float4*>(p.b1 + (long long)g * p.hidden + c * HC + 64 * half);
+            float4 bias[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) bias[r] = __ldg(b4 + r);
             if (!warp_wait(acc1_full, (uint32_t)k & 1u)) return false;
             tc_fence_after();
             float v[64];
@@ -379,10 +386,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld_wait();
             tc_fence_before();
             arrive_even(acc1_empty);
-            const float4* b4 = reinterpret_cast<const float4*>(p.b1 + (long long)g * p.hidden + c * HC + 64 * half);
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                const float4 bb = __ldg(b4 + r);
+                const float4 bb = bias[r];
                 const float2 lo = f2_add(make_float2(v[4 * r], v[4 * r + 1]), make_float2(bb.x, bb.y));
                 const float2 hi = f2_add(make_float2(v[4 * r + 2], v[4 * r + 3]), make_float2(bb.z, bb.w));
                 v[4 * r] = lo.x;
@@ -407,14 +413,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t w[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) w[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-            // the previous chunk's second projection has read the buffer
+            // the previous chunk's second projection has read the operand
             if (!warp_wait(h_empty, ((uint32_t)k & 1u) ^ 1u)) return false;
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(hrow + ((((uint32_t)e) ^ swz) << 4)),
-                             "r"(w[4 * e]), "r"(w[4 * e + 1]), "r"(w[4 * e + 2]), "r"(w[4 * e + 3])
-                             : "memory");
-            fence_proxy_async_shared();   // generic-proxy writes before the MMA's async-proxy reads
+            tmem_st32(lane_tmem + (uint32_t)(H_COL + 32 * half), w);
+            tmem_st_wait();
+            tc_fence_before();
             arrive_even(h_full);
             return true;
         };
@@ -559,7 +562,7 @@ cudaError_t launch_d(const CUtensorMap& mS, const CUtensorMap& mW1, const CUtens
 }  // namespace
 
 bool ffn_fused_supported(int D, int hidden) {
-    return D % 64 == 0 && D >= 64 && D <= ACC1_COL && hidden % HC == 0 && hidden >= HC;
+    return D % 64 == 0 && D >= 64 && D <= H_COL && hidden % HC == 0 && hidden >= HC;
 }
 
 // Opt-in (RM_FFN_FUSED=1).  Measured on B200 at the Pad-Split size (D 320,
@@ -617,8 +620,7 @@ cudaError_t launch_ffn_fused(const FusedFfn& f, DeviceErr err, uint64_t budget_n
         case 128: return launch_d<128>(mS, mW1, mW2, fp, grid, s);
         case 192: return launch_d<192>(mS, mW1, mW2, fp, grid, s);
         case 256: return launch_d<256>(mS, mW1, mW2, fp, grid, s);
-        case 320: return launch_d<320>(mS, mW1, mW2, fp, grid, s);
-        default: return launch_d<384>(mS, mW1, mW2, fp, grid, s);
+        default: return launch_d<320>(mS, mW1, mW2, fp, grid, s);
     }
 }
 

@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int q = 0; q < 16; ++q) __stcg(dst + q * 32, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
                 }
                 tc_fence_before();
-                if (CG == 2 && !leader) mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
+                if (CG == 2 && !leader) mbar_arrive_cluster_relaxed(tempty_leader + 8u * (uint32_t)acc);
                 else mbar_arrive(tempty0 + 8 * acc);
                 __threadfence();
                 __syncwarp();
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!split && c + 128 >= BN) {   // this warp's last chunk: the accumulator may be reused
                     tc_fence_before();
-                    if (CG == 2 && !leader) mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
+                    if (CG == 2 && !leader) mbar_arrive_cluster_relaxed(tempty_leader + 8u * (uint32_t)acc);
                     else mbar_arrive(tempty0 + 8 * acc);
                 }
                 if (!live) continue;
@@ -675,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             tc_fence_before();
-            if (CG == 2 && !leader) mbar_arrive_cluster(tempty_leader + 8u * (uint32_t)acc);
+            if (CG == 2 && !leader) mbar_arrive_cluster_relaxed(tempty_leader + 8u * (uint32_t)acc);
             else mbar_arrive(tempty0 + 8 * acc);
         }
     }

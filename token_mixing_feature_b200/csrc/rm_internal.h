@@ -133,7 +133,7 @@ struct FusedFfn {
     float2* stats;            // may be null
     long long s_gstride, s_ld;
 };
-// Shapes the fused kernel handles: D % 64 == 0, 64 <= D <= 384, hidden % 128 == 0.
+// Shapes the fused kernel handles: D % 64 == 0, 64 <= D <= 320, hidden % 128 == 0.
 bool ffn_fused_supported(int D, int hidden);
 // Whether run_pffn uses the fused kernel: only when supported and asked for
 // with RM_FFN_FUSED=1 (the two grouped GEMMs are faster on B200 today).
