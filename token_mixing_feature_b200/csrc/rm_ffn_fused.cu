@@ -566,12 +566,10 @@ bool ffn_fused_supported(int D, int hidden) {
 }
 
 // Opt-in (RM_FFN_FUSED=1).  Measured on B200 at the Pad-Split size (D 320,
-// kD 1280, 16 tokens x 4096 samples) it takes 190 us per block against 156 us
-// for the two grouped GEMMs: its narrow MMAs (N = 128 and 160) re-read the
-// resident S tile for every hidden chunk and the hidden chunk twice, which
-// with the weight copies needs more shared-memory bandwidth per chunk than
-// the tensor pipe's time for it, and eight epilogue warps take longer for a
-// chunk's GELU than the tensor pipe for its first projection.
+// kD 1280, 16 tokens x 4096 samples) it takes 171 us per block against
+// 78 + 74 us for the two grouped GEMMs: a chunk's first projection (20 MMAs
+// of N = 128) runs at ~60 % of its nominal rate, and 256 tiles fill 3.46
+// waves of the 74 CTA pairs.
 bool ffn_fused_preferred(int G, int M, int D, int hidden, int num_sms) {
     (void)G;
     (void)M;
