@@ -31,7 +31,8 @@
 //   warp 10     TMA: W2 chunks through ring 2
 // Tensor memory (512 columns): acc2 in columns [0, D), the bf16 hidden chunk
 // in [320, 384) (two values per column: the second projection's A operand),
-// acc1 in [384, 512).  Only the weights pass through shared memory.
+// acc1 in [384, 512).  The S tile and the weights sit in shared memory; the
+// hidden chunk never leaves tensor memory.
 // Every mbarrier wait is bounded (rm_device.cuh); a wait that runs out
 // records RM_ERR_DEVICE_TIMEOUT, stops the CTA's other roles, drains
 // in-flight copies and MMAs, frees tensor memory and returns.
