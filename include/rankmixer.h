@@ -115,7 +115,13 @@ rm_status rm_layernorm(rm_handle *h, const void *A, const void *R, const float *
 
 /* Per-token FFN (section Per-Token FFN of the fun-rec chapter):
  *     V[b, t] = W2_t GELU(W1_t S[b, t] + b1_t) + b2_t
- * S, V [B, T, D]; uses w->W1, b1, W2, b2.  No residual, no LayerNorm. */
+ * S, V [B, T, D]; uses w->W1, b1, W2, b2.  No residual, no LayerNorm.
+ * bf16 runs two grouped tcgen05 GEMMs (the hidden [T, B, hidden] in the
+ * handle's workspace).  With the environment variable RM_FFN_FUSED=1 and
+ * D % 64 == 0, D <= 320, hidden % 128 == 0, one kernel computes both
+ * projections with the hidden activation kept on chip instead; its outputs
+ * are bit-identical (it is slower on B200 today, hence off by default).
+ * Blocks and stacks use the same choice. */
 rm_status rm_pffn_forward(rm_handle *h, const rm_block_weights *w, const void *S, void *V,
                           int B, rm_stream_t stream);
 

@@ -120,11 +120,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t fullA = empty2 + 8 * C::R2;    // S tile landed (pair's bytes, on the even CTA)
     const uint32_t emptyA = fullA + 8;            // S tile no longer read (both CTAs)
     const uint32_t acc1_full = emptyA + 8;        // hidden-chunk accumulator ready (both CTAs)
-    const uint32_t acc1_empty = acc1_full + 8;    // ... read by every epilogue thread (even CTA)
+    const uint32_t acc1_empty = acc1_full + 8;    // ... read by every epilogue warp of the pair (even CTA)
     const uint32_t h_full = acc1_empty + 8;       // hidden chunk stored in tensor memory (even CTA)
     const uint32_t h_empty = h_full + 8;          // ... consumed by the second projection (both CTAs)
     const uint32_t acc2_full = h_empty + 8;       // tile's output accumulator complete (both CTAs)
-    const uint32_t acc2_empty = acc2_full + 8;    // ... read by every epilogue thread (even CTA)
+    const uint32_t acc2_empty = acc2_full + 8;    // ... read by every epilogue warp of the pair (even CTA)
     const uint32_t drain_bar = acc2_empty + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
