@@ -219,7 +219,9 @@ rm_status rm_selftest_wait_timeout(rm_handle *h, rm_stream_t stream);
  * library holds until the process exits; the caller passes inputs and outputs
  * only, and the call allocates nothing.
  *   - Returns RM_ERR_INVALID_ARG, before launching anything, if
- *     T * B * hidden * sizeof(element) > RM_STATIC_SCRATCH_BYTES - 256.
+ *     T * B * hidden * sizeof(element) > RM_STATIC_SCRATCH_BYTES - 256,
+ *     unless the fused kernel runs (RM_FFN_FUSED=1, see rm_pffn_forward),
+ *     which keeps the hidden activations on chip.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.

@@ -61,17 +61,20 @@ extern "C" rm_status rm_pffn_forward_static(const rm_block_weights* w, const voi
     if (act != RM_ACT_GELU_TANH && act != RM_ACT_GELU_ERF && act != RM_ACT_RELU) return RM_ERR_INVALID_ARG;
     if (dtype == RM_BF16 && (D % 16 || hidden % 16)) return RM_ERR_UNSUPPORTED;
     if (dtype == RM_F32 && (D % 4 || hidden % 4)) return RM_ERR_UNSUPPORTED;
-    const size_t esz = dtype == RM_BF16 ? 2 : 4;
-    const size_t need = (size_t)T * (size_t)B * (size_t)hidden * esz;
-    if (need > kScratchBytes - kHiddenOffset) return RM_ERR_INVALID_ARG;   // H does not fit the fixed array
-
-    unsigned char* scratch = nullptr;
-    rm_status st = scratch_address(&scratch);
-    if (st != RM_OK) return st;
     int dev = 0, num_sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return RM_ERR_CUDA;
+    // The same kernel choice as rm_pffn_forward; the fused kernel keeps the
+    // hidden activations on chip and needs no scratch for them.
+    const bool fused = dtype == RM_BF16 && rm::ffn_fused_preferred(T, B, D, hidden, num_sms);
+    const size_t esz = dtype == RM_BF16 ? 2 : 4;
+    const size_t need = (size_t)T * (size_t)B * (size_t)hidden * esz;
+    if (!fused && need > kScratchBytes - kHiddenOffset) return RM_ERR_INVALID_ARG;   // H does not fit the array
+
+    unsigned char* scratch = nullptr;
+    rm_status st = scratch_address(&scratch);
+    if (st != RM_OK) return st;
 
     cudaStream_t s = stream;
     int* err_word = reinterpret_cast<int*>(scratch);
@@ -112,7 +115,25 @@ extern "C" rm_status rm_pffn_forward_static(const rm_block_weights* w, const voi
     const rm::DeviceErr err{err_word, err_word + 1};
     const uint64_t budget_ns = 1000000000ull;
     cudaError_t e;
-    if (dtype == RM_BF16) {
+    if (fused) {
+        rm::FusedFfn f{};
+        f.G = T;
+        f.M = B;
+        f.D = D;
+        f.hidden = hidden;
+        f.epi = g1.epi;
+        f.A = S;
+        f.a_gstride = g1.a_gstride;
+        f.a_ld = g1.a_ld;
+        f.W1 = w->W1;
+        f.b1 = g1.bias;
+        f.W2 = w->W2;
+        f.b2 = g2.bias;
+        f.out = V;
+        f.o_gstride = g2.o_gstride;
+        f.o_ld = g2.o_ld;
+        e = rm::launch_ffn_fused(f, err, budget_ns, num_sms, s);
+    } else if (dtype == RM_BF16) {
         e = rm::launch_gemm_tc(g1, err, budget_ns, num_sms, s);
         if (e == cudaSuccess) e = rm::launch_gemm_tc(g2, err, budget_ns, num_sms, s);
     } else {
