@@ -119,11 +119,19 @@ def code_digest(path: str) -> str:
     return hashlib.sha256(src.encode()).hexdigest()[:16]
 
 
-def traffic_from_profiles(kernel_key: str):
-    """Per-launch DRAM bytes of a kernel from a committed ncu summary, if the
-    summary was taken on the current code of the GEMM kernel."""
-    path = os.path.join(ROOT, "profiles", "ncu_gemm_tc_rm1b.md")
-    src = os.path.join(ROOT, "token_mixing_feature_b200", "csrc", "rm_gemm_tc.cu")
+# committed ncu summaries per kernel family: (summary file pattern, kernel source)
+PROFILE_SOURCES = {
+    "gemm_tc": ("ncu_gemm_tc_{workload}.md", "rm_gemm_tc.cu"),
+    "ffn_fused": ("ncu_ffn_fused_{workload}.md", "rm_ffn_fused.cu"),
+}
+
+
+def traffic_from_profiles(family: str, workload: str, kernel_key: str, root: str = ROOT):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary of this
+    workload, if there is one and it was taken on the kernel's current code."""
+    pattern, source = PROFILE_SOURCES[family]
+    path = os.path.join(root, "profiles", pattern.format(workload=workload))
+    src = os.path.join(root, "token_mixing_feature_b200", "csrc", source)
     try:
         text = open(path).read()
         digest = code_digest(src)
@@ -134,6 +142,50 @@ def traffic_from_profiles(kernel_key: str):
         return None
     m = re.search(rf"dram_bytes_per_launch\s+{re.escape(kernel_key)}\s*[:=]\s*([0-9.eE+]+)", text)
     return float(m.group(1)) if m else None
+
+
+# fp32 FFMA lanes per SM (4 sub-partitions x 32): the fp32 path's CUDA-core ceiling
+FP32_LANES_PER_SM = 128
+
+
+def top_kernel_roofline(wl, top: str, ms_avg: float, active, peaks: dict, peak_src: str,
+                        num_sms: int, sm_max_mhz: float, root: str = ROOT) -> dict:
+    """Roofline entry of the kernel with the largest share of the step.
+
+    The FFN kernels are contractions: 2 B T D kD FLOPs per projection (the
+    active expert rows for MoE), against the sustained dense bf16 tensor peak
+    for bf16, or the fp32 FFMA peak of the CUDA cores (SMs x 128 lanes x 2
+    FLOPs x max SM clock) for the fp32 path.  The memory-bound kernels report
+    the HBM peak only."""
+    timing = ("CUDA events around each launch on its stream, over a second timed region of "
+              "the same K steps (about 6 us of event overhead per launch included)")
+    if top not in ("gemm1", "gemm2", "ffn_fused"):
+        return {"kernel": top, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": None, "traffic": None}
+    if wl.n_experts:
+        per_launch = 2.0 * sum(active) * wl.D * wl.hidden / wl.L
+    else:
+        per_launch = 2.0 * wl.B * wl.T * wl.D * wl.hidden
+    if top == "ffn_fused":
+        per_launch *= 2.0   # both projections in one launch
+    achieved = per_launch / (ms_avg / 1e3) / 1e12
+    if wl.dtype == "f32":
+        peak = num_sms * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
+        return {"kernel": f"gemm_simt ({top})", "bound": "alu", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak_source": f"fp32 FFMA: {num_sms} SMs x {FP32_LANES_PER_SM} lanes x 2 x {sm_max_mhz:.0f} MHz",
+                "flops_per_launch": per_launch, "timing": timing}
+    # the GEMM runs inside a long step under the power cap: the sustained
+    # cuBLAS figure is its ceiling (burst given for context)
+    peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+    family = "ffn_fused" if top == "ffn_fused" else "gemm_tc"
+    return {"kernel": f"{family} ({top})" if family == "gemm_tc" else family, "bound": "tensor",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic_from_profiles(family, wl.name, top, root),
+            "peak_source": ("bf16 dense sustained" if peaks.get("bf16_tflops_sustained") else
+                            "bf16 dense burst") + f", of {peak_src}",
+            "burst_peak": peaks["bf16_tflops"], "frac_of_burst": achieved / peaks["bf16_tflops"],
+            "flops_per_launch": per_launch, "timing": timing}
 
 
 # ----------------------------------------------------------- workload steps
@@ -364,28 +416,10 @@ def main():
         kern = {k: {"ms_avg": v[0] / max(v[1], 1), "launches": v[1],
                     "share": v[0] / max(sum(x[0] for x in prof.values()), 1e-9)} for k, v in prof.items()}
         top = max(prof, key=lambda k: prof[k][0])
-        # algorithmic FLOPs per launch of the top kernel (both projections have 2 B T D kD)
-        if top in ("gemm1", "gemm2"):
-            if wl.n_experts:
-                per_launch = 2.0 * sum(active) * wl.D * wl.hidden / wl.L
-            else:
-                per_launch = 2.0 * wl.B * wl.T * wl.D * wl.hidden
-            achieved = per_launch / (kern[top]["ms_avg"] / 1e3) / 1e12
-            # the GEMM runs inside a long step under the power cap: the
-            # sustained cuBLAS figure is its ceiling (burst given for context)
-            peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
-            roof = {"kernel": f"gemm_tc ({top})", "bound": "tensor", "achieved": achieved,
-                    "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                    "traffic": traffic_from_profiles(top),
-                    "peak_source": ("bf16 dense sustained" if peaks.get("bf16_tflops_sustained") else
-                                    "bf16 dense burst") + f", of {peak_src}",
-                    "burst_peak": peaks["bf16_tflops"], "frac_of_burst": achieved / peaks["bf16_tflops"],
-                    "flops_per_launch": per_launch,
-                    "timing": "CUDA events around each launch on its stream, over a second timed region of "
-                              "the same K steps (about 6 us of event overhead per launch included)"}
-        else:
-            roof = {"kernel": top, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s", "frac": None, "traffic": None}
+        props = torch.cuda.get_device_properties(device)
+        sm_max = (clocks or {}).get("sm_max_mhz") or 1965.0
+        roof = top_kernel_roofline(wl, top, kern[top]["ms_avg"], active, peaks, peak_src,
+                                   props.multi_processor_count, float(sm_max))
         line = {
             "metric": METRIC, "value": wl.B * max(world, 1) * a.steps / (ms / 1e3), "unit": "samples/s",
             "n_gpus": max(world, 1), "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps,

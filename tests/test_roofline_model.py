@@ -64,3 +64,55 @@ def test_code_digest_ignores_comments_only(tmp_path):
     c.write_text("int f(int x) {\n    return x + 2;\n}\n")
     assert bench.code_digest(str(a)) == bench.code_digest(str(b))
     assert bench.code_digest(str(a)) != bench.code_digest(str(c))
+
+
+def _fake_tree(tmp_path, workload, family_file, source, digest_of_source=True, bytes_line="gemm1 = 123456"):
+    import bench
+    csrc = tmp_path / "token_mixing_feature_b200" / "csrc"
+    csrc.mkdir(parents=True, exist_ok=True)
+    (csrc / source).write_text("int kernel() { return 1; }  // v1\n")
+    digest = bench.code_digest(str(csrc / source)) if digest_of_source else "0" * 16
+    prof = tmp_path / "profiles"
+    prof.mkdir(exist_ok=True)
+    (prof / family_file.format(workload=workload)).write_text(
+        f"code sha256[:16]: {digest}\n\ndram_bytes_per_launch {bytes_line}\n")
+    return str(tmp_path)
+
+
+PEAKS = {"bf16_tflops": 1617.4, "bf16_tflops_sustained": 1372.7, "hbm_gbs": 6543.4}
+
+
+def test_top_kernel_roofline_tensor_traffic_per_workload(tmp_path):
+    """The GEMM roofline takes its traffic from the summary of the same
+    workload, only while that summary's code digest matches the source."""
+    import bench
+    wl = synth.WORKLOADS["padsplit"]
+    root = _fake_tree(tmp_path, "padsplit", "ncu_gemm_tc_{workload}.md", "rm_gemm_tc.cu")
+    r = bench.top_kernel_roofline(wl, "gemm1", 0.08, None, PEAKS, "measured", 148, 1965.0, root)
+    assert r["bound"] == "tensor" and r["traffic"] == 123456.0
+    flops = 2.0 * wl.B * wl.T * wl.D * wl.hidden
+    assert abs(r["achieved"] - flops / 0.08e-3 / 1e12) < 1e-9
+    assert abs(r["frac"] - r["achieved"] / 1372.7) < 1e-12
+    # another workload has no summary here: no traffic
+    r2 = bench.top_kernel_roofline(synth.WORKLOADS["rm1b"], "gemm1", 0.3, None, PEAKS, "measured", 148, 1965.0, root)
+    assert r2["traffic"] is None
+    # a summary of other code: no traffic
+    root3 = _fake_tree(tmp_path / "stale", "padsplit", "ncu_gemm_tc_{workload}.md", "rm_gemm_tc.cu",
+                       digest_of_source=False)
+    assert bench.top_kernel_roofline(wl, "gemm1", 0.08, None, PEAKS, "m", 148, 1965.0, root3)["traffic"] is None
+
+
+def test_top_kernel_roofline_fused_and_alu_and_hbm(tmp_path):
+    import bench
+    wl = synth.WORKLOADS["padsplit"]
+    root = _fake_tree(tmp_path, "padsplit", "ncu_ffn_fused_{workload}.md", "rm_ffn_fused.cu",
+                      bytes_line="ffn_fused = 777")
+    r = bench.top_kernel_roofline(wl, "ffn_fused", 0.17, None, PEAKS, "measured", 148, 1965.0, root)
+    assert r["flops_per_launch"] == 4.0 * wl.B * wl.T * wl.D * wl.hidden   # both projections
+    assert r["traffic"] == 777.0 and r["bound"] == "tensor"
+    # the fp32 path runs on CUDA cores: FFMA peak of 148 SMs x 128 lanes x 2 x 1965 MHz
+    tiny = synth.WORKLOADS["tiny_f32"]
+    a = bench.top_kernel_roofline(tiny, "gemm2", 0.01, None, PEAKS, "measured", 148, 1965.0, root)
+    assert a["bound"] == "alu" and abs(a["peak"] - 148 * 128 * 2 * 1965e6 / 1e12) < 1e-9
+    h = bench.top_kernel_roofline(wl, "mix_ln", 0.04, None, PEAKS, "measured", 148, 1965.0, root)
+    assert h["bound"] == "hbm" and h["frac"] is None
