@@ -63,9 +63,11 @@ class ClockSampler:
     def __init__(self, device: int):
         self.proc = None
         self.path = None
+        self.power_limit = None
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             gid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.power_limit = self._power_limit(gid)
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.out = open(self.path, "w")
@@ -74,6 +76,16 @@ class ClockSampler:
                                          stdout=self.out, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+
+    @staticmethod
+    def _power_limit(gid: str):
+        """The enforced board power limit in watts (read only), or None."""
+        try:
+            out = subprocess.run(["nvidia-smi", f"--id={gid}", "--query-gpu=enforced.power.limit",
+                                  "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10)
+            return float(out.stdout.strip().splitlines()[0]) if out.returncode == 0 else None
+        except Exception:
+            return None
 
     def stop(self):
         if self.proc is None:
@@ -106,7 +118,8 @@ class ClockSampler:
         reasons = sorted({self.REASONS[i] for r in rows for i in range(4) if "Active" == r[5 + i]
                           or r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(num(r[2]) for r in rows),
-                "power_w_max": pmax, "samples": len(rows), "reasons": reasons}
+                "power_w_max": pmax, "power_limit_w": self.power_limit, "samples": len(rows),
+                "reasons": reasons}
 
 
 def code_digest(path: str) -> str:
