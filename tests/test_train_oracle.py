@@ -1,0 +1,139 @@
+"""Pins of the training-step oracle (oracle/train_oracle.py) against what the
+mathematics fixes, not against itself:
+
+  - its forward equals the C oracle's stack forward (an independent
+    restatement of the block equations, pinned in test_oracle_pins.py);
+  - every gradient equals a central finite difference of the loss;
+  - LayerNorm input gradients sum to zero over a row (LayerNorm ignores a
+    shift of its input row) and, with eps = 0, are orthogonal to the
+    normalised input (it then also ignores a scaling);
+  - the token mixing is its own adjoint (a permutation that is its own
+    inverse), which is what carries the gradient back through it;
+  - degenerate cases: W2 = 0 cuts every first-projection gradient to zero;
+    the head-bias gradient is mean(sigmoid(logit) - y).
+"""
+import numpy as np
+import pytest
+
+from oracle import train_oracle as TO
+from token_mixing_feature_b200 import synth
+
+
+def _stack(T, D, hidden, L, seed=0):
+    blocks = []
+    for l in range(L):
+        blk = synth.random_like_block(T, D, hidden, "f32", seed=seed + 17 * l)
+        # larger LayerNorm perturbations than the default, so their gradients are not near-degenerate
+        rng = np.random.default_rng(seed + l)
+        blk = {k: v.double().numpy() for k, v in blk.items()}
+        for k in ("ln1_g", "ln2_g"):
+            blk[k] = 1.0 + 0.3 * rng.standard_normal(D)
+        for k in ("ln1_b", "ln2_b"):
+            blk[k] = 0.3 * rng.standard_normal(D)
+        blocks.append(blk)
+    return blocks
+
+
+def _inputs(B, T, D, seed=3):
+    rng = np.random.default_rng(seed)
+    X0 = rng.standard_normal((B, T, D))
+    w = 0.5 * rng.standard_normal(D)
+    c = np.array([0.1])
+    y = (rng.random(B) < 0.4).astype(np.float64)
+    return X0, w, c, y
+
+
+def test_forward_matches_c_oracle(O):
+    T, D, hidden, L, B = 4, 16, 24, 2, 5
+    # the C oracle reads parameters and X0 as float: both get the same float values
+    blocks = [{k: v.astype(np.float32).astype(np.float64) for k, v in b.items()} for b in _stack(T, D, hidden, L)]
+    X0, w, c, _ = _inputs(B, T, D)
+    fw = TO.forward(X0, blocks, w, c)
+    ref = O.stack(X0.astype(np.float32), blocks, want_all=True)
+    fw32 = TO.forward(X0.astype(np.float32), blocks, w, c)
+    np.testing.assert_allclose(fw32["pooled"], ref["pooled"], rtol=0, atol=1e-12)
+    for l in range(L):
+        np.testing.assert_allclose(fw32["Xall"][l], ref["Xall"][l], rtol=0, atol=1e-12)
+    assert fw["pooled"].shape == (B, D)
+
+
+def _fd_check(fun_loss, params, grads, name, n_probe=6, h=1e-5, seed=0):
+    rng = np.random.default_rng(seed)
+    flat = params.reshape(-1)
+    gflat = grads.reshape(-1)
+    scale = max(1e-12, float(np.abs(gflat).max()))
+    for i in rng.choice(flat.size, size=min(n_probe, flat.size), replace=False):
+        old = flat[i]
+        flat[i] = old + h
+        lp = fun_loss()
+        flat[i] = old - h
+        lm = fun_loss()
+        flat[i] = old
+        fd = (lp - lm) / (2 * h)
+        assert abs(fd - gflat[i]) <= 1e-6 * scale + 1e-9, f"{name}[{i}]: fd {fd:.10e} vs grad {gflat[i]:.10e}"
+
+
+@pytest.mark.parametrize("act,addnorm", [("tanh", True), ("erf", True), ("relu", True), ("tanh", False)])
+def test_gradients_match_finite_differences(act, addnorm):
+    T, D, hidden, L, B = 4, 8, 12, 2, 3
+    blocks = _stack(T, D, hidden, L, seed=11)
+    X0, w, c, y = _inputs(B, T, D, seed=5)
+
+    def loss():
+        return TO.loss_only(X0, blocks, w, c, y, gelu_mode=act, mix_addnorm=addnorm)
+
+    st = TO.train_step(X0, blocks, w, c, y, gelu_mode=act, mix_addnorm=addnorm)
+    assert abs(st["loss"] - loss()) < 1e-14
+    _fd_check(loss, X0, st["dX0"], "X0")
+    _fd_check(loss, w, st["dhead_w"], "head_w")
+    _fd_check(loss, c, np.array([st["dhead_b"]]), "head_b")
+    for l in range(L):
+        keys = ("W1", "b1", "W2", "b2", "ln2_g", "ln2_b") + (("ln1_g", "ln1_b") if addnorm else ())
+        for k in keys:
+            _fd_check(loss, blocks[l][k], st["blocks"][l][k], f"block{l}.{k}", seed=l)
+
+
+def test_layernorm_input_gradient_is_orthogonal_to_shift_and_scale():
+    """A LayerNorm row is unchanged when a constant is added to its input, so
+    the input gradient sums to zero; with eps = 0 it is also unchanged when the
+    input is scaled, so the gradient is orthogonal to the normalised input
+    (with eps > 0 that holds only up to eps / var)."""
+    rng = np.random.default_rng(7)
+    Z = rng.standard_normal((6, 5, 24)) * 3.0 + 1.5
+    g = 1.0 + 0.5 * rng.standard_normal(24)
+    b = rng.standard_normal(24)
+    dout = rng.standard_normal(Z.shape)
+    for eps in (1e-5, 0.0):
+        _, xhat, rstd = TO.layernorm_fwd(Z, g, b, eps)
+        dZ, _, _ = TO.layernorm_bwd(dout, xhat, rstd, g)
+        np.testing.assert_allclose(dZ.sum(axis=-1), 0.0, atol=1e-12)
+        if eps == 0.0:
+            np.testing.assert_allclose((dZ * xhat).sum(axis=-1), 0.0, atol=1e-11)
+
+
+def test_token_mix_is_its_own_adjoint():
+    rng = np.random.default_rng(9)
+    for T, D in ((4, 16), (8, 40), (1, 8)):
+        x = rng.standard_normal((3, T, D))
+        yv = rng.standard_normal((3, T, D))
+        assert abs(np.sum(TO.token_mix(x) * yv) - np.sum(x * TO.token_mix(yv))) < 1e-10
+        np.testing.assert_array_equal(TO.token_mix(TO.token_mix(x)), x)
+
+
+def test_zero_second_projection_cuts_first_projection_gradients():
+    T, D, hidden, L, B = 4, 8, 12, 1, 4
+    blocks = _stack(T, D, hidden, L, seed=21)
+    blocks[0]["W2"][:] = 0.0
+    X0, w, c, y = _inputs(B, T, D, seed=8)
+    st = TO.train_step(X0, blocks, w, c, y)
+    assert np.all(st["blocks"][0]["W1"] == 0.0) and np.all(st["blocks"][0]["b1"] == 0.0)
+    assert np.abs(st["blocks"][0]["W2"]).max() > 0.0
+
+
+def test_head_bias_gradient_closed_form():
+    T, D, hidden, L, B = 4, 8, 12, 2, 7
+    blocks = _stack(T, D, hidden, L, seed=31)
+    X0, w, c, y = _inputs(B, T, D, seed=4)
+    st = TO.train_step(X0, blocks, w, c, y)
+    p = 1.0 / (1.0 + np.exp(-st["logit"]))
+    assert abs(st["dhead_b"] - float(np.mean(p - y))) < 1e-15
