@@ -1,6 +1,6 @@
-"""fp64 CPU oracle of one training step of a dense RankMixer stack: forward,
-loss, and the gradient of the loss with respect to every parameter and to
-the stack input.
+"""fp64 CPU oracle of one training step of a RankMixer stack (dense or
+sparse-MoE per-token FFN): forward, loss, and the gradient of the loss with
+respect to every parameter and to the stack input.
 
 TEST INFRASTRUCTURE.  Only the test suite may import this module.  It shares
 no code with the CUDA library and never imports it.  Its forward restates the
@@ -17,6 +17,14 @@ What it computes (the pages on RankMixer; primary source the fun-rec chapter
   pooling:   pooled_b = (1/T) sum_t X_L[b, t]
   head:      logit_b = w . pooled_b + c,  p_b = sigmoid(logit_b)
   loss:      L = (1/B) sum_b BCE(p_b, y_b) = (1/B) sum_b [softplus(logit_b) - y_b logit_b]
+             + lambda L_reg
+  sparse MoE in place of the PFFN (section Sparse MoE扩展, ReLU Routing and
+  DTSI-MoE):
+      G_{t,j} = ReLU(h_t(s_t))_j,  v_t = sum_j G_{t,j} e_{t,j}(s_t),  h_t linear
+      L_reg   = sum over the batch's tokens and experts of the regularised gates:
+                those of the routing router itself, or, with a second router
+                h_infer (DTSI), G^infer = ReLU(h_infer(s_t)), which the forward
+                computes beside the routing gates but does not use.
 
 Readings where the pages leave a step open:
   - The task loss.  The pages name L_task without defining it (section Sparse
@@ -29,7 +37,12 @@ Readings where the pages leave a step open:
   - LayerNorm, GELU forms and weight layouts as in rankmixer_oracle.c: LN over
     D with the population variance and eps inside the square root, one
     (gamma, beta) per LN instance shared by all tokens; W1_t stored [kD][D],
-    W2_t [D][kD].
+    W2_t [D][kD]; MoE experts W1 [T][Ne][kD][D], W2 [T][Ne][D][kD], routers
+    Wr [T][Ne][D], br [T][Ne] (h_infer: Wr_infer, br_infer, same shapes).
+  - L_reg's gradient is the plain derivative of the written loss: it reaches
+    the regularised router's parameters and, through the router's input,
+    the tokens s_t.  Under DTSI as written, h_infer receives no other
+    gradient (the task loss does not depend on it).
 
 Each derivative below is the chain rule applied to these definitions, in
 the order the forward computed them; the only library routines are array
@@ -116,8 +129,28 @@ def _sigmoid(x: np.ndarray) -> np.ndarray:
 
 
 # --------------------------------------------------------------- the step
+PARAM_KEYS = ("W1", "b1", "W2", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b", "Wr", "br", "Wr_infer", "br_infer")
+
+
 def _block_params(blk: Dict) -> Dict[str, np.ndarray]:
-    return {k: _f64(blk[k]) for k in ("W1", "b1", "W2", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b")}
+    return {k: _f64(blk[k]) for k in PARAM_KEYS if k in blk}
+
+
+def _moe_forward(S: np.ndarray, p: Dict[str, np.ndarray], gelu_mode: str, c: Dict) -> np.ndarray:
+    """v_t = sum_j ReLU(h_t(s_t))_j e_{t,j}(s_t) for every token; fills the cache."""
+    c["R"] = np.einsum("btd,tjd->btj", S, p["Wr"]) + p["br"][None]
+    c["G"] = np.maximum(c["R"], 0.0)
+    c["U"] = np.einsum("btd,tjkd->btjk", S, p["W1"]) + p["b1"][None]
+    c["Hh"] = gelu(c["U"], gelu_mode)
+    c["E"] = np.einsum("btjk,tjdk->btjd", c["Hh"], p["W2"]) + p["b2"][None]
+    if "Wr_infer" in p:
+        c["R_inf"] = np.einsum("btd,tjd->btj", S, p["Wr_infer"]) + p["br_infer"][None]
+    return np.einsum("btj,btjd->btd", c["G"], c["E"])
+
+
+def _reg_gates(c: Dict) -> np.ndarray:
+    """The gates L_reg sums: h_infer's under DTSI, else the routing gates."""
+    return np.maximum(c["R_inf"], 0.0) if "R_inf" in c else c["G"]
 
 
 def forward(X0, blocks: Sequence[Dict], head_w, head_b, eps: float = 1e-5, gelu_mode: str = "tanh",
@@ -134,11 +167,15 @@ def forward(X0, blocks: Sequence[Dict], head_w, head_b, eps: float = 1e-5, gelu_
             S, xh1, rs1 = layernorm_fwd(M + X, p["ln1_g"], p["ln1_b"], eps)
         else:
             S, xh1, rs1 = M, None, None
-        U = np.einsum("btd,tkd->btk", S, p["W1"]) + p["b1"][None]
-        Hh = gelu(U, gelu_mode)
-        V = np.einsum("btk,tdk->btd", Hh, p["W2"]) + p["b2"][None]
-        Xn, xh2, rs2 = layernorm_fwd(V + S, p["ln2_g"], p["ln2_b"], eps)
-        caches.append({"p": p, "S": S, "U": U, "Hh": Hh, "xh1": xh1, "rs1": rs1, "xh2": xh2, "rs2": rs2})
+        c = {"p": p, "S": S, "xh1": xh1, "rs1": rs1}
+        if "Wr" in p:
+            V = _moe_forward(S, p, gelu_mode, c)
+        else:
+            c["U"] = np.einsum("btd,tkd->btk", S, p["W1"]) + p["b1"][None]
+            c["Hh"] = gelu(c["U"], gelu_mode)
+            V = np.einsum("btk,tdk->btd", c["Hh"], p["W2"]) + p["b2"][None]
+        Xn, c["xh2"], c["rs2"] = layernorm_fwd(V + S, p["ln2_g"], p["ln2_b"], eps)
+        caches.append(c)
         X = Xn
         Xall.append(X)
     pooled = X.mean(axis=1)
@@ -152,18 +189,19 @@ def loss_from_logit(logit: np.ndarray, y: np.ndarray) -> float:
 
 
 def train_step(X0, blocks: Sequence[Dict], head_w, head_b, labels, eps: float = 1e-5,
-               gelu_mode: str = "tanh", mix_addnorm: bool = True):
+               gelu_mode: str = "tanh", mix_addnorm: bool = True, reg_lambda: float = 0.0):
     """Loss and gradients of one training step.
 
     Returns {'loss', 'pooled', 'logit', 'dX0' [B, T, D], 'dhead_w' [D],
-    'dhead_b' (float), 'blocks': [per block {'W1', 'b1', 'W2', 'b2', 'ln1_g',
-    'ln1_b', 'ln2_g', 'ln2_b'} gradients, same shapes as the parameters]}."""
+    'dhead_b' (float), 'l_reg', 'blocks': [per block the gradients of every
+    parameter the block has, same keys and shapes]}."""
     y = _f64(labels).reshape(-1)
     fw = forward(X0, blocks, head_w, head_b, eps, gelu_mode, mix_addnorm)
     pooled, logit = fw["pooled"], fw["logit"]
     B = pooled.shape[0]
     T = fw["caches"][0]["S"].shape[1]
-    loss = loss_from_logit(logit, y)
+    l_reg = sum(float(_reg_gates(c).sum()) for c in fw["caches"] if "G" in c)
+    loss = loss_from_logit(logit, y) + reg_lambda * l_reg
 
     # head and pooling
     dlogit = (_sigmoid(logit) - y) / B                       # d mean(softplus(l) - y l) / dl
@@ -181,15 +219,18 @@ def train_step(X0, blocks: Sequence[Dict], head_w, head_b, labels, eps: float = 
         dZ2, g["ln2_g"], g["ln2_b"] = layernorm_bwd(dX, c["xh2"], c["rs2"], p["ln2_g"])
         dV = dZ2
         dS = dZ2.copy()                                      # residual branch
-        # V = W2_t Hh + b2_t
-        g["W2"] = np.einsum("btd,btk->tdk", dV, c["Hh"])
-        g["b2"] = dV.sum(axis=0)
-        dHh = np.einsum("btd,tdk->btk", dV, p["W2"])
-        # Hh = GELU(U), U = W1_t S + b1_t
-        dU = dHh * gelu_grad(c["U"], gelu_mode)
-        g["W1"] = np.einsum("btk,btd->tkd", dU, c["S"])
-        g["b1"] = dU.sum(axis=0)
-        dS += np.einsum("btk,tkd->btd", dU, p["W1"])
+        if "Wr" in p:
+            dS += _moe_backward(dV, c, p, g, gelu_mode, reg_lambda)
+        else:
+            # V = W2_t Hh + b2_t
+            g["W2"] = np.einsum("btd,btk->tdk", dV, c["Hh"])
+            g["b2"] = dV.sum(axis=0)
+            dHh = np.einsum("btd,tdk->btk", dV, p["W2"])
+            # Hh = GELU(U), U = W1_t S + b1_t
+            dU = dHh * gelu_grad(c["U"], gelu_mode)
+            g["W1"] = np.einsum("btk,btd->tkd", dU, c["S"])
+            g["b1"] = dU.sum(axis=0)
+            dS += np.einsum("btk,tkd->btd", dU, p["W1"])
         # S = LN1(TokenMixing(X) + X)   (or S = TokenMixing(X))
         if mix_addnorm:
             dZ1, g["ln1_g"], g["ln1_b"] = layernorm_bwd(dS, c["xh1"], c["rs1"], p["ln1_g"])
@@ -199,11 +240,43 @@ def train_step(X0, blocks: Sequence[Dict], head_w, head_b, labels, eps: float = 
             g["ln1_b"] = np.zeros_like(p["ln1_b"])
             dX = token_mix(dS)
         grads[l] = g
-    return {"loss": loss, "pooled": pooled, "logit": logit, "dX0": dX, "dhead_w": dhead_w,
+    return {"loss": loss, "l_reg": l_reg, "pooled": pooled, "logit": logit, "dX0": dX, "dhead_w": dhead_w,
             "dhead_b": dhead_b, "blocks": grads}
 
 
+def _moe_backward(dV: np.ndarray, c: Dict, p: Dict[str, np.ndarray], g: Dict, gelu_mode: str,
+                  reg_lambda: float) -> np.ndarray:
+    """Gradients of the MoE FFN (into g) given dL/dV; returns dL/dS from the
+    experts and the routers."""
+    S = c["S"]
+    # v = sum_j G_j e_j
+    dG = np.einsum("btd,btjd->btj", dV, c["E"])
+    dE = c["G"][..., None] * dV[:, :, None, :]
+    # e_j = W2_{t,j} GELU(U_j) + b2_{t,j},  U_j = W1_{t,j} s + b1_{t,j}
+    g["W2"] = np.einsum("btjd,btjk->tjdk", dE, c["Hh"])
+    g["b2"] = dE.sum(axis=0)
+    dU = np.einsum("btjd,tjdk->btjk", dE, p["W2"]) * gelu_grad(c["U"], gelu_mode)
+    g["W1"] = np.einsum("btjk,btd->tjkd", dU, S)
+    g["b1"] = dU.sum(axis=0)
+    dS = np.einsum("btjk,tjkd->btd", dU, p["W1"])
+    # G = ReLU(R), R = Wr s + br; L_reg on these gates unless a second router carries it
+    active = (c["R"] > 0.0).astype(np.float64)
+    dR = dG * active
+    if "R_inf" not in c:
+        dR = dR + reg_lambda * active
+    g["Wr"] = np.einsum("btj,btd->tjd", dR, S)
+    g["br"] = dR.sum(axis=0)
+    dS += np.einsum("btj,tjd->btd", dR, p["Wr"])
+    if "R_inf" in c:
+        dR_inf = reg_lambda * (c["R_inf"] > 0.0).astype(np.float64)
+        g["Wr_infer"] = np.einsum("btj,btd->tjd", dR_inf, S)
+        g["br_infer"] = dR_inf.sum(axis=0)
+        dS += np.einsum("btj,tjd->btd", dR_inf, p["Wr_infer"])
+    return dS
+
+
 def loss_only(X0, blocks: Sequence[Dict], head_w, head_b, labels, eps: float = 1e-5,
-              gelu_mode: str = "tanh", mix_addnorm: bool = True) -> float:
+              gelu_mode: str = "tanh", mix_addnorm: bool = True, reg_lambda: float = 0.0) -> float:
     fw = forward(X0, blocks, head_w, head_b, eps, gelu_mode, mix_addnorm)
-    return loss_from_logit(fw["logit"], _f64(labels).reshape(-1))
+    l_reg = sum(float(_reg_gates(c).sum()) for c in fw["caches"] if "G" in c)
+    return loss_from_logit(fw["logit"], _f64(labels).reshape(-1)) + reg_lambda * l_reg

@@ -10,7 +10,10 @@ mathematics fixes, not against itself:
   - the token mixing is its own adjoint (a permutation that is its own
     inverse), which is what carries the gradient back through it;
   - degenerate cases: W2 = 0 cuts every first-projection gradient to zero;
-    the head-bias gradient is mean(sigmoid(logit) - y).
+    the head-bias gradient is mean(sigmoid(logit) - y);
+  - sparse MoE (ReLU routing, L_reg, DTSI's second router): its forward
+    equals the C oracle's block, every gradient a finite difference, and
+    h_infer's bias gradient is lambda times its count of positive logits.
 """
 import numpy as np
 import pytest
@@ -137,3 +140,69 @@ def test_head_bias_gradient_closed_form():
     st = TO.train_step(X0, blocks, w, c, y)
     p = 1.0 / (1.0 + np.exp(-st["logit"]))
     assert abs(st["dhead_b"] - float(np.mean(p - y))) < 1e-15
+
+
+def _moe_stack(T, D, hidden, Ne, L, seed=0, dtsi=False):
+    blocks = []
+    for l in range(L):
+        blk = synth.random_like_block(T, D, hidden, "f32", seed=seed + 13 * l, n_experts=Ne,
+                                      router_std=0.4, router_bias=0.0)
+        rng = np.random.default_rng(seed + 100 + l)
+        blk = {k: v.double().numpy() for k, v in blk.items()}
+        for k in ("ln1_g", "ln2_g"):
+            blk[k] = 1.0 + 0.3 * rng.standard_normal(D)
+        for k in ("ln1_b", "ln2_b"):
+            blk[k] = 0.3 * rng.standard_normal(D)
+        if dtsi:
+            blk["Wr_infer"] = 0.4 * rng.standard_normal((T, Ne, D))
+            blk["br_infer"] = 0.1 * rng.standard_normal((T, Ne))
+        blocks.append({k: v.astype(np.float32).astype(np.float64) for k, v in blk.items()})
+    return blocks
+
+
+def test_moe_forward_matches_c_oracle(O):
+    T, D, hidden, Ne, B = 4, 16, 12, 3, 5
+    blocks = _moe_stack(T, D, hidden, Ne, 1, seed=2)
+    X0, w, c, _ = _inputs(B, T, D)
+    X0 = X0.astype(np.float32).astype(np.float64)
+    fw = TO.forward(X0, blocks, w, c)
+    ref = O.block(X0, blocks[0])
+    np.testing.assert_allclose(fw["Xall"][0], ref, rtol=0, atol=1e-12)
+    G = fw["caches"][0]["G"]
+    assert 0 < np.count_nonzero(G) < G.size     # some experts open, some closed
+
+
+@pytest.mark.parametrize("dtsi", [False, True])
+def test_moe_gradients_match_finite_differences(dtsi):
+    T, D, hidden, Ne, L, B = 4, 8, 6, 3, 2, 3
+    lam = 0.05
+    blocks = _moe_stack(T, D, hidden, Ne, L, seed=5, dtsi=dtsi)
+    X0, w, c, y = _inputs(B, T, D, seed=6)
+
+    def loss():
+        return TO.loss_only(X0, blocks, w, c, y, reg_lambda=lam)
+
+    st = TO.train_step(X0, blocks, w, c, y, reg_lambda=lam)
+    assert abs(st["loss"] - loss()) < 1e-14 and st["l_reg"] > 0.0
+    _fd_check(loss, X0, st["dX0"], "X0")
+    for l in range(L):
+        keys = ["W1", "b1", "W2", "b2", "Wr", "br", "ln1_g", "ln1_b", "ln2_g", "ln2_b"]
+        if dtsi:
+            keys += ["Wr_infer", "br_infer"]
+        for k in keys:
+            _fd_check(loss, blocks[l][k], st["blocks"][l][k], f"block{l}.{k}", seed=l)
+
+
+def test_dtsi_inference_router_gradient_is_the_regulariser_count():
+    """Under DTSI the task loss does not depend on h_infer, so its bias
+    gradient is lambda times the number of the batch's positive h_infer
+    logits for that (token, expert), and zero without the regulariser."""
+    T, D, hidden, Ne, B = 4, 8, 6, 3, 9
+    blocks = _moe_stack(T, D, hidden, Ne, 1, seed=8, dtsi=True)
+    X0, w, c, y = _inputs(B, T, D, seed=9)
+    for lam in (0.0, 0.25):
+        st = TO.train_step(X0, blocks, w, c, y, reg_lambda=lam)
+        R_inf = TO.forward(X0, blocks, w, c)["caches"][0]["R_inf"]
+        np.testing.assert_array_equal(st["blocks"][0]["br_infer"], lam * (R_inf > 0).sum(axis=0))
+        if lam == 0.0:
+            assert not np.any(st["blocks"][0]["Wr_infer"])
