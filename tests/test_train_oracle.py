@@ -3,7 +3,9 @@ mathematics fixes, not against itself:
 
   - its forward equals the C oracle's stack forward (an independent
     restatement of the block equations, pinned in test_oracle_pins.py);
-  - every gradient equals a central finite difference of the loss;
+  - every gradient equals a central finite difference of the loss, and every
+    entry equals torch autograd (float64, CPU) of a forward written here
+    with torch ops;
   - LayerNorm input gradients sum to zero over a row (LayerNorm ignores a
     shift of its input row) and, with eps = 0, are orthogonal to the
     normalised input (it then also ignores a scaling);
@@ -206,3 +208,77 @@ def test_dtsi_inference_router_gradient_is_the_regulariser_count():
         np.testing.assert_array_equal(st["blocks"][0]["br_infer"], lam * (R_inf > 0).sum(axis=0))
         if lam == 0.0:
             assert not np.any(st["blocks"][0]["Wr_infer"])
+
+
+def _torch_loss(X0, blocks, w, c, y, act, addnorm, lam, eps=1e-5):
+    """The stack's loss written with torch ops in float64, for autograd."""
+    import torch
+    import torch.nn.functional as F
+
+    def mix(X):
+        B, T, D = X.shape
+        return X.reshape(B, T, T, D // T).transpose(1, 2).reshape(B, T, D)
+
+    def ln(Z, g, b):
+        mu = Z.mean(-1, keepdim=True)
+        var = ((Z - mu) ** 2).mean(-1, keepdim=True)
+        return (Z - mu) / torch.sqrt(var + eps) * g + b
+
+    def act_fn(u):
+        if act == "tanh":
+            return F.gelu(u, approximate="tanh")
+        if act == "erf":
+            return F.gelu(u)
+        return torch.relu(u)
+
+    X = X0
+    l_reg = X0.new_zeros(())
+    for p in blocks:
+        S = ln(mix(X) + X, p["ln1_g"], p["ln1_b"]) if addnorm else mix(X)
+        if "Wr" in p:
+            G = torch.relu(torch.einsum("btd,tjd->btj", S, p["Wr"]) + p["br"])
+            E = torch.einsum("btjk,tjdk->btjd", act_fn(torch.einsum("btd,tjkd->btjk", S, p["W1"]) + p["b1"]),
+                             p["W2"]) + p["b2"]
+            V = torch.einsum("btj,btjd->btd", G, E)
+            if "Wr_infer" in p:
+                l_reg = l_reg + torch.relu(torch.einsum("btd,tjd->btj", S, p["Wr_infer"]) + p["br_infer"]).sum()
+            else:
+                l_reg = l_reg + G.sum()
+        else:
+            H = act_fn(torch.einsum("btd,tkd->btk", S, p["W1"]) + p["b1"])
+            V = torch.einsum("btk,tdk->btd", H, p["W2"]) + p["b2"]
+        X = ln(V + S, p["ln2_g"], p["ln2_b"])
+    logit = X.mean(1) @ w + c[0]
+    return F.binary_cross_entropy_with_logits(logit, y) + lam * l_reg
+
+
+@pytest.mark.parametrize("kind,act,addnorm", [("dense", "tanh", True), ("dense", "erf", False),
+                                              ("dense", "relu", True), ("moe", "tanh", True),
+                                              ("dtsi", "tanh", True)])
+def test_gradients_match_autograd(kind, act, addnorm):
+    """Every entry of every gradient against torch autograd (float64, CPU) of
+    a forward written separately with torch ops."""
+    import torch
+    T, D, hidden, L, B = 4, 8, 6, 2, 5
+    lam = 0.05 if kind != "dense" else 0.0
+    if kind == "dense":
+        blocks = _stack(T, D, hidden, L, seed=41)
+    else:
+        blocks = _moe_stack(T, D, hidden, 3, L, seed=43, dtsi=kind == "dtsi")
+    X0, w, c, y = _inputs(B, T, D, seed=44)
+    st = TO.train_step(X0, blocks, w, c, y, gelu_mode=act, mix_addnorm=addnorm, reg_lambda=lam)
+    tt = lambda a: torch.tensor(a, dtype=torch.float64, requires_grad=True)   # noqa: E731
+    tb = [{k: tt(v) for k, v in b.items()} for b in blocks]
+    tX, tw, tc = tt(X0), tt(w), tt(c)
+    loss = _torch_loss(tX, tb, tw, tc, torch.tensor(y, dtype=torch.float64), act, addnorm, lam)
+    loss.backward()
+    assert abs(loss.item() - st["loss"]) < 1e-12
+    np.testing.assert_allclose(st["dX0"], tX.grad.numpy(), rtol=1e-9, atol=1e-13)
+    np.testing.assert_allclose(st["dhead_w"], tw.grad.numpy(), rtol=1e-9, atol=1e-13)
+    assert abs(st["dhead_b"] - tc.grad.item()) < 1e-12
+    for l in range(L):
+        for k, v in tb[l].items():
+            if not addnorm and k in ("ln1_g", "ln1_b"):
+                continue   # unused without the Add & Norm (the oracle reports zeros)
+            np.testing.assert_allclose(st["blocks"][l][k], v.grad.numpy(), rtol=1e-9, atol=1e-13,
+                                       err_msg=f"block{l}.{k}")
