@@ -201,6 +201,29 @@ def top_kernel_roofline(wl, top: str, ms_avg: float, active, peaks: dict, peak_s
             "flops_per_launch": per_launch, "timing": timing}
 
 
+def per_kernel_rooflines(wl, kern: dict, active, peaks: dict, num_sms: int, sm_max_mhz: float) -> dict:
+    """Every kernel's achieved rate against its own bound: algorithmic bytes per
+    launch (roofline.kernel_work) over the measured launch time against the
+    HBM peak, or FLOPs against the sustained dense bf16 tensor peak (the fp32
+    FFMA peak for the fp32 path).  Adds 'achieved', 'unit', 'bound', 'frac'
+    to each entry of kern (times include ~6 us of event overhead per launch)."""
+    active_mean = sum(active) / len(active) if active else None
+    tensor_peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+    fp32_peak = num_sms * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
+    for kind, e in kern.items():
+        what, n = roofline.kernel_work(wl, kind, active_mean)
+        sec = e["ms_avg"] / 1e3
+        if what == "bytes":
+            e.update(achieved=n / sec / 1e9, unit="GB/s", bound="hbm", algorithmic=n)
+            e["frac"] = e["achieved"] / peaks["hbm_gbs"]
+        else:
+            peak = fp32_peak if wl.dtype == "f32" else tensor_peak
+            e.update(achieved=n / sec / 1e12, unit="TFLOP/s", bound="alu" if wl.dtype == "f32" else "tensor",
+                     algorithmic=n)
+            e["frac"] = e["achieved"] / peak
+    return kern
+
+
 # ----------------------------------------------------------- workload steps
 class Runner:
     def __init__(self, wl: synth.Workload, device):
@@ -433,6 +456,7 @@ def main():
         sm_max = (clocks or {}).get("sm_max_mhz") or 1965.0
         roof = top_kernel_roofline(wl, top, kern[top]["ms_avg"], active, peaks, peak_src,
                                    props.multi_processor_count, float(sm_max))
+        kern = per_kernel_rooflines(wl, kern, active, peaks, props.multi_processor_count, float(sm_max))
         line = {
             "metric": METRIC, "value": wl.B * max(world, 1) * a.steps / (ms / 1e3), "unit": "samples/s",
             "n_gpus": max(world, 1), "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps,

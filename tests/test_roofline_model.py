@@ -116,3 +116,48 @@ def test_top_kernel_roofline_fused_and_alu_and_hbm(tmp_path):
     assert a["bound"] == "alu" and abs(a["peak"] - 148 * 128 * 2 * 1965e6 / 1e12) < 1e-9
     h = bench.top_kernel_roofline(wl, "mix_ln", 0.04, None, PEAKS, "measured", 148, 1965.0, root)
     assert h["bound"] == "hbm" and h["frac"] is None
+
+
+KERNELS_BY_WORKLOAD = {
+    "rm1b": ["mix_ln", "gemm1", "gemm2", "ln_pool"],
+    "rm100m": ["mix_ln", "gemm1", "gemm2", "ln_pool"],
+    "padsplit": ["mix_ln", "gemm1", "gemm2", "ln_pool", "padsplit", "head"],
+    "moe": ["mix_ln", "gemm1", "gemm2", "ln_pool", "moe_route", "moe_gather", "moe_combine"],
+    "appendix_b": ["mix_ln", "gemm1", "gemm2", "ln_pool"],
+    "tiny_f32": ["mix_ln", "gemm1", "gemm2", "ln_pool"],
+}
+
+
+@pytest.mark.parametrize("name", sorted(KERNELS_BY_WORKLOAD))
+def test_per_kernel_rooflines_cover_every_kernel(name):
+    """Every kernel kind the stack launches gets an achieved rate against its
+    own bound (HBM for the memory-bound kinds, tensor or fp32 FFMA for the
+    FFN contractions)."""
+    import bench
+    wl = synth.WORKLOADS[name]
+    kinds = KERNELS_BY_WORKLOAD[name] + (["ffn_fused"] if name == "padsplit" else [])
+    kern = {k: {"ms_avg": 0.05, "launches": 2, "share": 0.1} for k in kinds}
+    active = [wl.B * wl.T * 2, wl.B * wl.T * 2] if wl.n_experts else None
+    out = bench.per_kernel_rooflines(wl, kern, active, PEAKS, 148, 1965.0)
+    for k, e in out.items():
+        assert e["frac"] > 0 and e["achieved"] > 0, k
+        if k in ("gemm1", "gemm2", "ffn_fused"):
+            assert e["unit"] == "TFLOP/s" and e["bound"] == ("alu" if wl.dtype == "f32" else "tensor")
+        else:
+            assert e["unit"] == "GB/s" and e["bound"] == "hbm"
+
+
+def test_kernel_work_figures():
+    """Algorithmic bytes of the memory-bound kinds at the 1B-scale and
+    Pad-Split sizes, by hand: X in + S out, plus half the launches reading
+    the previous block's 24 LayerNorm partials per row."""
+    rm1b = synth.WORKLOADS["rm1b"]
+    act = 512 * 32 * 1536 * 2
+    assert roofline.kernel_work(rm1b, "mix_ln") == ("bytes", 2 * act + 512 * 32 * 24 * 8 * 0.5)
+    assert roofline.kernel_work(rm1b, "ln_pool") == ("bytes", act + 512 * 32 * 24 * 8 + 512 * 1536 * 4)
+    ps = synth.WORKLOADS["padsplit"]
+    assert roofline.kernel_work(ps, "padsplit") == ("bytes", 4096 * 4800 * 2 + 4096 * 16 * 320 * 2)
+    assert roofline.kernel_work(ps, "gemm1") == ("flops", 2.0 * 4096 * 16 * 320 * 1280)
+    assert roofline.kernel_work(ps, "ffn_fused") == ("flops", 4.0 * 4096 * 16 * 320 * 1280)
+    with pytest.raises(KeyError):
+        roofline.kernel_work(ps, "no_such_kernel")

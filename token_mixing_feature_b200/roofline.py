@@ -82,3 +82,45 @@ def stack_bytes(wl: Workload, experts_touched_per_block: Optional[Sequence[int]]
 def roofline_seconds(flops: float, nbytes: float, peak_flops: float, peak_bw: float) -> float:
     """Lower bound on time: the slower of compute at peak and traffic at bandwidth."""
     return max(flops / peak_flops, nbytes / peak_bw)
+
+
+def stat_slices(wl: Workload) -> int:
+    """LayerNorm partials per row that the FFN stage writes: one per 64
+    columns from the dense bf16 second projection, else one per row."""
+    return wl.D // 64 if (wl.dtype == "bf16" and wl.n_experts == 0 and wl.D % 64 == 0) else 1
+
+
+def kernel_work(wl: Workload, kind: str, active_mean: Optional[float] = None):
+    """Algorithmic work of one launch of a kernel kind of the stack:
+    ("bytes", n) for memory-bound kernels (what the kernel must read and write
+    at least once), ("flops", n) for the FFN contractions.  For MoE kinds,
+    active_mean is the mean number of active (sample, token, expert) entries
+    per block."""
+    es = ELEM_BYTES[wl.dtype]
+    B, T, D, Hd, L = wl.B, wl.T, wl.D, wl.hidden, wl.L
+    act = B * T * D * es
+    stats = B * T * stat_slices(wl) * 8              # (mean, M2) float pairs
+    A = active_mean or 0.0
+    if kind == "mix_ln":        # X in, S out; blocks after the first also read the previous LN2 statistics
+        return "bytes", 2 * act + stats * (L - 1) / L
+    if kind == "ln_pool":       # Y and its statistics in, pooled (fp32) out
+        return "bytes", act + stats + B * D * 4
+    if kind == "padsplit":      # feature groups in, tokens out
+        return "bytes", B * sum(wl.group_widths) * es + act
+    if kind == "head":
+        return "bytes", B * D * 4 + D * es + B * 4
+    if kind == "token_mix":
+        return "bytes", 2 * act
+    if kind == "layernorm":     # in a stack: row statistics of the FFN output (fp32 path), V in, (mean, M2) out
+        return "bytes", act + B * T * 8
+    if kind == "moe_route":     # S and the routers in, gates out
+        return "bytes", act + T * wl.n_experts * (D + 1) * 4 + B * T * wl.n_experts * 4
+    if kind == "moe_gather":    # active rows copied
+        return "bytes", 2 * A * D * es
+    if kind == "moe_combine":   # expert rows and the residual in, block output and its statistics out
+        return "bytes", A * D * es + 2 * act + B * T * 8
+    if kind in ("gemm1", "gemm2"):
+        return "flops", (2.0 * A * D * Hd) if wl.n_experts else (2.0 * B * T * D * Hd)
+    if kind == "ffn_fused":
+        return "flops", 4.0 * B * T * D * Hd
+    raise KeyError(kind)
