@@ -146,6 +146,20 @@ def moe(S, blk: Dict, gelu: str = "tanh"):
     return V, logits
 
 
+def router(S, Wr, br) -> np.ndarray:
+    """Router logits h_t(s) = Wr_t s + br_t of every token row, [B, T, Ne]
+    (before the ReLU; an expert is active iff its logit is > 0)."""
+    S = _np(S, np.float64)
+    B, T, D = S.shape
+    Wr, br = _np(Wr, np.float32), _np(br, np.float32)
+    Ne = Wr.shape[1]
+    assert Wr.shape == (T, Ne, D) and br.shape == (T, Ne)
+    logits = np.empty((B, T, Ne), dtype=np.float64)
+    _load().orc_router(ctypes.c_long(B), ctypes.c_int(T), ctypes.c_int(D), ctypes.c_int(Ne), _p(S), _p(Wr),
+                       _p(br), _p(logits))
+    return logits
+
+
 def _dims(blk: Dict, T: int, D: int):
     W1 = blk["W1"]
     if len(W1.shape) == 3:

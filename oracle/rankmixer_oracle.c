@@ -243,6 +243,17 @@ void orc_moe(long B, int T, int D, int Hd, int Ne, const double *S, const orc_bl
     }
 }
 
+/* Router logits alone: logits[b][t][j] = Wr_t[j] . S[b][t] + br_t[j]
+ * (the linear router h_t of the ReLU routing equation, before the ReLU). */
+void orc_router(long B, int T, int D, int Ne, const double *S, const float *Wr, const float *br,
+                double *logits) {
+    #pragma omp parallel for schedule(static)
+    for (long b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            router_vec(D, Ne, S + ((size_t)b * T + t) * D, Wr + (size_t)t * Ne * D, br + (size_t)t * Ne,
+                       logits + ((size_t)b * T + t) * Ne);
+}
+
 /* One block over B samples. logits [B][T][Ne] (MoE only, may be NULL). */
 void orc_block(long B, int T, int D, int Hd, int Ne, const double *X, const orc_block_params *p,
                double eps, int gelu, int mix_addnorm, double *Y, double *logits) {

@@ -218,16 +218,45 @@ def test_cuda_graph_replay_equals_direct_launch(rm, name, B):
     st.close()
 
 
-def test_moe_active_rate_is_reported(rm):
-    """The MoE workload's routing statistics: fraction of active experts."""
-    wl = synth.WORKLOADS["moe"].with_batch(512)
+def test_moe_router_masks_at_workload_constants(rm, O, record_property):
+    """Router masks of the sparse-MoE workload at its own constants (B 2048,
+    T 16, D 768, 8 experts per token, router weights N(0, 0.02), bias -0.5),
+    on the S the library's LayerNorm produces for every block of the stack.
+    The ReLU routing equation (fun-rec "Rankmixer: 硬件效率优化", section
+    Sparse MoE扩展) opens expert j iff its logit is > 0: the masks must equal
+    the oracle's wherever |logit| >= 1e-3 (the kernel decides in fp32, the
+    oracle in fp64), the undecided band must stay small, the gates must equal
+    ReLU(logit), and the expert output V must match on sampled rows."""
+    wl = synth.WORKLOADS["moe"]
     d = synth.make_inputs(wl)
     st = _stack(wl, d)
-    S = dev(d["X0"])
-    V = torch.empty_like(S)
+    x = dev(d["X0"])
     G = torch.empty(wl.B, wl.T, wl.n_experts, dtype=torch.float32, device="cuda")
-    rm.rm_moe_forward(st.h, st.blocks[0], S, V, G, wl.B)
-    assert rm.rm_sync_status(st.h) == rm.RM_OK
-    rate = (G > 0).float().mean().item()
-    assert 0.0 < rate < 1.0
+    V = torch.empty_like(x)
+    idx = sample_rows(wl.B, 16)
+    for l in range(wl.L):
+        blk = st.blocks[l]
+        M = torch.empty_like(x)
+        rm.rm_token_mix(st.h, x, M, wl.B)
+        S = torch.empty_like(x)
+        rm.rm_layernorm(st.h, M, x, blk["ln1_g"], blk["ln1_b"], S, wl.B * wl.T)
+        rm.rm_moe_forward(st.h, blk, S, V, G, wl.B)
+        assert rm.rm_sync_status(st.h) == rm.RM_OK
+        S_h = S.cpu()
+        logits = O.router(S_h, d["blocks"][l]["Wr"], d["blocks"][l]["br"])
+        g = host64(G)
+        decided = np.abs(logits) >= 1e-3
+        excluded = int((~decided).sum())
+        rate = float((g > 0).mean())
+        record_property(f"block{l}_undecided_entries", excluded)
+        record_property(f"block{l}_active_rate", rate)
+        print(f"block {l}: {excluded} of {logits.size} router entries within 1e-3 of zero, "
+              f"active rate {rate:.4f}")
+        assert excluded < 0.005 * logits.size
+        np.testing.assert_array_equal((g > 0)[decided], (logits > 0)[decided])
+        np.testing.assert_allclose(g, np.maximum(logits, 0), rtol=0, atol=1e-4)
+        assert 0.1 < rate < 0.3          # about 18 % for logits ~ N(-0.5, 0.55^2)
+        Vref, _ = O.moe(S_h[idx], d["blocks"][l])
+        assert_close(host64(V[idx.to("cuda")]), Vref, "bf16", f"moe V, block {l}", raw=True)
+        x = st.block(l, x)
     st.close()

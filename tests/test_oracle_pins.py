@@ -239,6 +239,27 @@ def test_moe_skipping_equals_dense_evaluation(O):
     np.testing.assert_allclose(V, ref.numpy(), rtol=0, atol=1e-12)
 
 
+def test_router_logits_alone(O):
+    """The router-only entry equals the logits the MoE forward reports, and a
+    router that reads one input column per expert returns that column plus the
+    bias (a hand-checkable case of the linear router h_t)."""
+    B, T, D, Hd, Ne = 6, 3, 16, 8, 5
+    blk = _moe_block(T, D, Hd, Ne, 60, router_std=0.4, router_bias=-0.1)
+    S = synth.random_activations((B, T, D), seed=61)
+    _, logits = O.moe(S, blk)
+    np.testing.assert_array_equal(O.router(S, blk["Wr"], blk["br"]), logits)
+    Wr = torch.zeros(T, Ne, D)
+    for t in range(T):
+        for j in range(Ne):
+            Wr[t, j, (3 * t + j) % D] = 1.0          # expert j of token t reads column 3t + j
+    br = torch.arange(T * Ne, dtype=torch.float32).reshape(T, Ne) * 0.25
+    got = O.router(S, Wr, br)
+    Sd = S.double().numpy()
+    for t in range(T):
+        for j in range(Ne):
+            np.testing.assert_array_equal(got[:, t, j], Sd[:, t, (3 * t + j) % D] + float(br[t, j]))
+
+
 def test_moe_gate_scales_second_bias(O):
     """W2 = 0: every active expert returns its b2, scaled by its gate."""
     B, T, D, Hd, Ne = 5, 2, 8, 8, 3

@@ -92,7 +92,10 @@ def test_top_kernel_roofline_tensor_traffic_per_workload(tmp_path):
     assert r["bound"] == "tensor" and r["traffic"] == 123456.0
     flops = 2.0 * wl.B * wl.T * wl.D * wl.hidden
     assert abs(r["achieved"] - flops / 0.08e-3 / 1e12) < 1e-9
-    assert abs(r["frac"] - r["achieved"] / 1372.7) < 1e-12
+    # a short timed region: the burst peak is the ceiling, sustained and spec beside it
+    assert abs(r["frac"] - r["achieved"] / 1617.4) < 1e-12
+    assert abs(r["frac_of_sustained"] - r["achieved"] / 1372.7) < 1e-12
+    assert abs(r["frac_of_spec"] - r["achieved"] / 2250.0) < 1e-12
     # another workload has no summary here: no traffic
     r2 = bench.top_kernel_roofline(synth.WORKLOADS["rm1b"], "gemm1", 0.3, None, PEAKS, "measured", 148, 1965.0, root)
     assert r2["traffic"] is None
@@ -115,7 +118,9 @@ def test_top_kernel_roofline_fused_and_alu_and_hbm(tmp_path):
     a = bench.top_kernel_roofline(tiny, "gemm2", 0.01, None, PEAKS, "measured", 148, 1965.0, root)
     assert a["bound"] == "alu" and abs(a["peak"] - 148 * 128 * 2 * 1965e6 / 1e12) < 1e-9
     h = bench.top_kernel_roofline(wl, "mix_ln", 0.04, None, PEAKS, "measured", 148, 1965.0, root)
-    assert h["bound"] == "hbm" and h["frac"] is None
+    nbytes = roofline.kernel_work(wl, "mix_ln")[1]
+    assert h["bound"] == "hbm" and abs(h["achieved"] - nbytes / 0.04e-3 / 1e9) < 1e-6
+    assert abs(h["frac"] - h["achieved"] / 6543.4) < 1e-12
 
 
 KERNELS_BY_WORKLOAD = {

@@ -57,6 +57,7 @@ extern "C" rm_status rm_pffn_forward_static(const rm_block_weights* w, const voi
         !aligned16(w->b2))
         return RM_ERR_INVALID_ARG;
     if (B < 1 || T < 1 || D < 1 || hidden < 1) return RM_ERR_INVALID_ARG;
+    if (T > 64) return RM_ERR_UNSUPPORTED;   // the token limit of rm_create
     if (dtype != RM_BF16 && dtype != RM_F32) return RM_ERR_INVALID_ARG;
     if (act != RM_ACT_GELU_TANH && act != RM_ACT_GELU_ERF && act != RM_ACT_RELU) return RM_ERR_INVALID_ARG;
     if (dtype == RM_BF16 && (D % 16 || hidden % 16)) return RM_ERR_UNSUPPORTED;
@@ -68,9 +69,13 @@ extern "C" rm_status rm_pffn_forward_static(const rm_block_weights* w, const voi
     // The same kernel choice as rm_pffn_forward; the fused kernel keeps the
     // hidden activations on chip and needs no scratch for them.
     const bool fused = dtype == RM_BF16 && rm::ffn_fused_preferred(T, B, D, hidden, num_sms);
+    // H [T, B, hidden] must fit the array; each factor is checked against the
+    // room left, so no product of the int arguments can wrap around.
     const size_t esz = dtype == RM_BF16 ? 2 : 4;
-    const size_t need = (size_t)T * (size_t)B * (size_t)hidden * esz;
-    if (!fused && need > kScratchBytes - kHiddenOffset) return RM_ERR_INVALID_ARG;   // H does not fit the array
+    const size_t room = kScratchBytes - kHiddenOffset;
+    const size_t row = (size_t)hidden * esz;   // < 2^33, no wrap
+    if (!fused && (row > room || (size_t)B > room / row || (size_t)T > room / (row * (size_t)B)))
+        return RM_ERR_INVALID_ARG;
 
     unsigned char* scratch = nullptr;
     rm_status st = scratch_address(&scratch);
