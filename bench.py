@@ -380,6 +380,8 @@ def main():
                     help="only the warm-up and the K timed steps (for profiler launch lists)")
     ap.add_argument("--no-graph", action="store_true",
                     help="time direct launches instead of replaying the step captured in a CUDA graph")
+    ap.add_argument("--train", action="store_true",
+                    help="time one training step (forward, loss, every gradient) of the dense workload instead")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -396,6 +398,8 @@ def main():
 
     if a.impl == "reference":
         return run_reference(a, wl, cfg, rank, world)
+    if a.train:
+        return run_train(a, wl, cfg, rank, world, local)
 
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
@@ -548,6 +552,97 @@ def main():
         print(json.dumps(line), flush=True)
     del graph, step_fn
     runner.st.close()
+    if pg:
+        pg.barrier(device_ids=[local])
+        pg.destroy_process_group()
+
+
+def run_train(a, wl, cfg, rank, world, local):
+    """K training steps (rm_train_step: forward keeping the backward's inputs,
+    mean BCE loss of the sigmoid head, every gradient) on the workload's
+    synthetic inputs with seeded 0/1 labels; device time with CUDA events on
+    the launch stream, max over ranks.  FLOPs: the forward's 4 B T D kD L
+    plus the backward's activation and weight gradients, 8 B T D kD L."""
+    if wl.n_experts or wl.dtype != "bf16" or not wl.mix_addnorm:
+        raise SystemExit("the training step covers dense bf16 stacks with the Add & Norm after mixing")
+    from token_mixing_feature_b200 import rankmixer as rm
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        pg = dist
+    d = synth.make_inputs(wl)
+    head = synth.make_head(wl)
+    B, T, D, Hd, L = wl.B, wl.T, wl.D, wl.hidden, wl.L
+    blocks = [{k: v.to(device) for k, v in blk.items()} for blk in d["blocks"]]
+    g = torch.Generator().manual_seed(1)
+    labels = (torch.rand(B, generator=g) < 0.5).float().to(device)
+    X0 = d["X0"].to(device)
+    hw, hb = head["w"].to(device), head["b"].to(device)
+    grads = [{"W1": torch.empty(T, Hd, D, device=device), "b1": torch.empty(T, Hd, device=device),
+              "W2": torch.empty(T, D, Hd, device=device), "b2": torch.empty(T, D, device=device),
+              **{k: torch.empty(D, device=device) for k in ("ln1_g", "ln1_b", "ln2_g", "ln2_b")}}
+             for _ in range(L)]
+    dX0 = torch.empty(B, T, D, dtype=torch.bfloat16, device=device)
+    dhw, dhb, loss = torch.empty(D, device=device), torch.empty(1, device=device), torch.empty(1, device=device)
+    tr = rm.rm_train_create(B, T, D, Hd, L, act=wl.act)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        rm.rm_train_step(tr, blocks, X0, hw, hb, labels, grads, dX0, dhw, dhb, loss, None, B, stream)
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if rm.rm_train_sync_status(tr) != rm.RM_OK:
+        raise SystemExit("device error during warm-up")
+
+    def barrier():
+        if pg:
+            pg.barrier(device_ids=[local])
+        torch.cuda.synchronize(device)
+    barrier()
+    wall0 = time.time()
+    ms = time_steps(step, a.steps, stream)
+    barrier()
+    wall1 = time.time()
+    ms = replicas.max_over_ranks(ms, device)
+    if rm.rm_train_sync_status(tr) != rm.RM_OK:
+        raise SystemExit("device error during timing")
+    clocks = None
+    if sampler:
+        sampler.stop()
+        clocks = sampler.summary(wall0 - 0.05, wall1 + 0.05)
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        flops = 12.0 * B * T * D * Hd * L
+        es = 2
+        wbytes = L * (2 * T * D * Hd * es)
+        # weights read by the forward and by the activation-gradient products,
+        # weight gradients written in float, the stack input read once
+        nbytes = 2 * wbytes + L * (2 * T * D * Hd * 4) + B * T * D * es
+        sec = ms / 1e3 / a.steps
+        t_roof = roofline.roofline_seconds(flops, nbytes, peaks["bf16_tflops"] * 1e12, peaks["hbm_gbs"] * 1e9)
+        line = {
+            "metric": "RankMixer stack training step samples/s and TFLOP/s as % of bf16 roofline on 1\u00d7B200",
+            "value": B * max(world, 1) * a.steps / (ms / 1e3), "unit": "samples/s", "n_gpus": max(world, 1),
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms / a.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) inputs, Xavier-normal weights, seeded 0/1 labels)",
+            "config": dict(cfg, mode="train", launch="direct"),
+            "tflops": flops / sec / 1e12,
+            "train_roofline": {"flops": flops, "bytes": nbytes, "t_roof_ms": t_roof * 1e3, "frac": t_roof / sec,
+                               "peaks": f"bf16 {peaks['bf16_tflops']} TFLOP/s (burst), HBM {peaks['hbm_gbs']} "
+                                        f"GB/s, of {peak_src}"},
+            "loss": float(loss.item()),
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    tr.close()
     if pg:
         pg.barrier(device_ids=[local])
         pg.destroy_process_group()

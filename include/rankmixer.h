@@ -31,8 +31,8 @@
  *   - Requirements: D % T == 0 (H = T heads of width D/T), D % 16 == 0 and
  *     hidden % 16 == 0 for RM_BF16 (D % 4 == 0 for RM_F32), 1 <= B <= B_max,
  *     1 <= T <= 64, n_experts <= 32, n_experts * D <= 40960, D <= 2048 (bf16) or 1024 (fp32), and
- *     one sample (T * D elements, rows padded by < 128 bytes) plus T * 8 + D * 4 bytes within
- *     226 KB of shared memory.  Violations return RM_ERR_INVALID_ARG or RM_ERR_UNSUPPORTED.
+ *     one sample (T * D elements, rows padded by < 128 bytes) plus T * (8 + 8 * P) + D * 8 bytes
+ *     within 226 KB of shared memory (P = D / 64 for RM_BF16 when D % 64 == 0, else 1).  Violations return RM_ERR_INVALID_ARG or RM_ERR_UNSUPPORTED.
  *   - RM_F32 handles compute on CUDA cores only (no tensor cores).  RM_BF16
  *     handles run the FFN products on tcgen05 tensor cores with fp32
  *     accumulation; S, the FFN hidden and the pre-LN rows are stored bf16.
@@ -233,6 +233,55 @@ rm_status rm_selftest_wait_timeout(rm_handle *h, rm_stream_t stream);
 rm_status rm_pffn_forward_static(const rm_block_weights *w, const void *S, void *V, int B, int T,
                                  int D, int hidden, rm_dtype dtype, int act, int *device_status,
                                  rm_stream_t stream);
+
+/* ---- training step (dense bf16 stacks) -----------------------------------
+ * One training step of a stack of L dense RankMixer blocks with the sigmoid
+ * head: the forward pass (keeping what the backward pass needs), the task loss
+ * and the gradient of the loss with respect to every parameter and to the
+ * stack input.  The pages give the FLOPs of a RankMixer training step
+ * ("重新理解 RankMixer", Table 1) and name the task loss without defining it
+ * (fun-rec "Rankmixer: 硬件效率优化", section Sparse MoE扩展: L = L_task +
+ * lambda L_reg); this library takes the mean binary cross-entropy of the
+ * sigmoid head,
+ *     L = (1/B) sum_b [softplus(logit_b) - y_b logit_b],
+ *     logit_b = head_w . mean_t X_L[b, t] + head_b,
+ * and the gradients are the chain rule through the block equations (the
+ * token mixing with H = T is its own transpose).
+ *
+ * A trainer owns its device workspace (per block: S, the normalised mixed
+ * rows, their 1/sqrt(var + eps), the FFN activation input and output, the
+ * pre-LN rows and their statistics; plus the backward buffers), allocated by
+ * rm_train_create for batches up to cfg->B_max.  Supported: dtype RM_BF16,
+ * n_experts 0, mix_addnorm 1, D % 64 == 0, hidden % 64 == 0, (D / T) % 8 == 0,
+ * D <= 2048, plus the forward's limits.  Otherwise RM_ERR_UNSUPPORTED. */
+typedef struct rm_trainer rm_trainer;
+
+/* Gradient outputs of one block (device pointers, float, the parameters'
+ * shapes and layouts): W1 [T][kD][D], b1 [T][kD], W2 [T][D][kD], b2 [T][D],
+ * ln1_g, ln1_b, ln2_g, ln2_b [D].  Every entry is overwritten (not added to). */
+typedef struct {
+    float *W1, *b1, *W2, *b2;
+    float *ln1_g, *ln1_b, *ln2_g, *ln2_b;
+} rm_block_grads;
+
+rm_status rm_train_create(const rm_config *cfg, rm_trainer **out);
+rm_status rm_train_destroy(rm_trainer *t);
+size_t rm_train_workspace_bytes(const rm_trainer *t);
+
+/* One step on B samples (8 <= B <= B_max, B % 8 == 0):
+ *   X0 [B, T, D] bf16 input; head_w [D] bf16, head_b [1] float; labels [B]
+ *   float (0 or 1); grads [L] outputs; dX0 [B, T, D] bf16 (may be NULL):
+ *   dL/dX0; dhead_w [D], dhead_b [1], loss [1] float outputs; pooled_out
+ *   [B, D] float (may be NULL): the forward's pooled output.
+ * Asynchronous on the stream; device-side faults (a bounded wait that ran
+ * out) set the trainer's error word, read by rm_train_sync_status. */
+rm_status rm_train_step(rm_trainer *t, const rm_block_weights *blocks, const void *X0, const void *head_w,
+                        const float *head_b, const float *labels, const rm_block_grads *grads, void *dX0,
+                        float *dhead_w, float *dhead_b, float *loss, float *pooled_out, int B,
+                        rm_stream_t stream);
+
+/* Synchronise the stream and return the trainer's device error word. */
+rm_status rm_train_sync_status(rm_trainer *t, rm_stream_t stream);
 
 /* ---- launch profiling ----------------------------------------------------
  * Kernel kinds launched by the forward entry points: */

@@ -70,6 +70,9 @@ struct KParams {
     int nsplit;
     float* sk_ws;
     int* sk_cnt;
+    int save_pre;             // activation epilogues: also store bf16(acc + bias), the activation's input, via tmR
+    int w_from_kernel;        // W (B operand) written by an earlier kernel: no loads before the launch wait
+    int w_g_inner;            // W map coordinate order (k|n, g, n|k) if 1, else (k|n, n|k, g)
     DeviceErr err;
     unsigned long long budget_ns;
 };
@@ -179,12 +182,72 @@ __device__ __forceinline__ Item decode_item(const KParams& p, long long idx, int
     return it;
 }
 
-template <int BN, int EPI, int CG, bool VAR>
+// Operand layouts in shared memory (one ring stage): K-major operands are
+// single TMA boxes of 64 K x rows (128-byte swizzled rows of K); M- or
+// N-major operands (AMN / BMN, the backward products) are boxes of 64 rows x
+// 64 K, one 8 KB box per 64 rows, each K row a 128-byte swizzled run of 64
+// rows.
+constexpr uint32_t kMnChunkBytes = 64 * BK * 2;
+
+// A ring stage's operand tile of `rows` rows starting at row r0 and K column
+// kc, from map tm whose coordinate order is (k|r, g, r|k) with g_inner, else
+// (k|r, r|k, g).  pair: completion counted on the even CTA's barrier.
+template <bool MN, int ROWS, bool PAIR>
+__device__ __forceinline__ void load_operand(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int kc, int r0, int g,
+                                             int g_inner) {
+    if constexpr (!MN) {
+        if (PAIR) {
+            if (g_inner) tma_load_3d_pair(dst, tm, bar, kc, g, r0);
+            else tma_load_3d_pair(dst, tm, bar, kc, r0, g);
+        } else {
+            if (g_inner) tma_load_3d(dst, tm, bar, kc, g, r0);
+            else tma_load_3d(dst, tm, bar, kc, r0, g);
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < ROWS / 64; ++c) {
+            const uint32_t d = dst + (uint32_t)c * kMnChunkBytes;
+            const int r = r0 + 64 * c;
+            if (PAIR) {
+                if (g_inner) tma_load_3d_pair(d, tm, bar, r, g, kc);
+                else tma_load_3d_pair(d, tm, bar, r, kc, g);
+            } else {
+                if (g_inner) tma_load_3d(d, tm, bar, r, g, kc);
+                else tma_load_3d(d, tm, bar, r, kc, g);
+            }
+        }
+    }
+}
+
+// Derivative of the FFN activation at u (the backward products' epilogue).
+template <int EPI>
+__device__ __forceinline__ float dact(float u) {
+    if constexpr (EPI == EPI_DACT_RELU) {
+        return u > 0.f ? 1.f : 0.f;
+    } else if constexpr (EPI == EPI_DACT_ERF) {
+        // d/du [u Phi(u)] = Phi(u) + u phi(u)
+        return 0.5f * (1.0f + erff(u * 0.7071067811865476f)) + u * 0.3989422804014327f * __expf(-0.5f * u * u);
+    } else {
+        // tanh form: g(u) = u/2 (1 + tanh(a)), a = c (u + 0.044715 u^3), c = sqrt(2/pi)
+        // g'(u) = (1 + tanh(a))/2 + u/2 (1 - tanh(a)^2) c (1 + 3 * 0.044715 u^2)
+        const float c = 0.7978845608028654f;
+        const float a = c * fmaf(0.044715f * u * u, u, u);
+        float th;
+        asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(a));
+        return fmaf(0.5f * u * c * fmaf(3.0f * 0.044715f, u * u, 1.0f), 1.0f - th * th, 0.5f * (1.0f + th));
+    }
+}
+
+template <int BN, int EPI, int CG, bool VAR, bool AMN = false, bool BMN = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
                    const KParams p) {
     using C = Cfg<BN, CG, VAR>;
+    static_assert(!(VAR && (AMN || BMN)), "variable-row groups read K-major operands");
+    static_assert(!BMN || C::BN_LOCAL % 64 == 0, "N-major W tiles are whole 64-row boxes");
+    constexpr bool DACT = EPI == EPI_DACT_TANH || EPI == EPI_DACT_ERF || EPI == EPI_DACT_RELU;
+    constexpr bool F32OUT = EPI == EPI_F32;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     unsigned char* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -262,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             // Weight (B) tiles of the first tile's first stages, before the wait.
             int npre = 0;
-            if (!VAR && unit < total) {
+            if (!VAR && !p.w_from_kernel && unit < total) {
                 const Item it0 = decode_item(p, unit, num_kb);
                 const Tile t0 = decode_tile<CG>(p, it0.tile, nblk, mblk, BN, (int)rank, mt_table);
                 const int nb0 = t0.n0 + (int)rank * C::BN_LOCAL;
@@ -272,8 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (leader) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
                     const uint32_t sb = sbase + k * C::STAGE_BYTES + C::A_BYTES;
                     const int kc = (it0.kb_lo + k) * BK;
-                    if (CG == 2) tma_load_3d_pair(sb, &tmB, mapa_shared(fb, 0), kc, nb0, t0.g);
-                    else tma_load_3d(sb, &tmB, fb, kc, nb0, t0.g);
+                    load_operand<BMN, C::BN_LOCAL, CG == 2>(sb, &tmB, CG == 2 ? mapa_shared(fb, 0) : fb, kc, nb0,
+                                                            t0.g, p.w_g_inner);
                 }
             }
             pdl_wait();
@@ -292,16 +355,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (leader && !pre) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
                     const uint32_t sa = sbase + stage * C::STAGE_BYTES;
                     const int kc = kb * BK;
-                    if (CG == 2) {
-                        const uint32_t fbl = mapa_shared(fb, 0);   // the pair counts bytes on the even CTA
-                        if (p.a_g_inner) tma_load_3d_pair(sa, &tmA, fbl, kc, t.ag, t.arow);
-                        else tma_load_3d_pair(sa, &tmA, fbl, kc, t.arow, t.ag);
-                        if (!pre) tma_load_3d_pair(sa + C::A_BYTES, &tmB, fbl, kc, nb0, t.g);
-                    } else {
-                        if (p.a_g_inner) tma_load_3d(sa, &tmA, fb, kc, t.ag, t.arow);
-                        else tma_load_3d(sa, &tmA, fb, kc, t.arow, t.ag);
-                        if (!pre) tma_load_3d(sa + C::A_BYTES, &tmB, fb, kc, nb0, t.g);
-                    }
+                    // the pair counts bytes on the even CTA's barrier
+                    const uint32_t fbl = CG == 2 ? mapa_shared(fb, 0) : fb;
+                    load_operand<AMN, BM, CG == 2>(sa, &tmA, fbl, kc, t.arow, t.ag, p.a_g_inner);
+                    if (!pre) load_operand<BMN, C::BN_LOCAL, CG == 2>(sa + C::A_BYTES, &tmB, fbl, kc, nb0, t.g, p.w_g_inner);
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -320,7 +377,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         pdl_wait();   // (reads no global memory; keeps every thread ordered after the previous kernel)
         if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = idesc_bf16_f32(C::TM, BN);
+            constexpr uint32_t idesc = idesc_bf16_f32(C::TM, BN, AMN, BMN);
+            // per K = 16 step: 32 bytes along a K-major row, or 16 K rows (2 KB)
+            // of an M/N-major tile; descriptors count 16-byte units
+            constexpr uint64_t a_step = AMN ? 128 : 2, b_step = BMN ? 128 : 2;
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true, any = false;
@@ -339,17 +399,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint32_t sa = sbase + stage * C::STAGE_BYTES;
-                    const uint64_t adesc = smem_desc_k_sw128(sa);
-                    const uint64_t bdesc = smem_desc_k_sw128(sa + C::A_BYTES);
+                    const uint64_t adesc = AMN ? smem_desc_mn_sw128(sa, kMnChunkBytes) : smem_desc_k_sw128(sa);
+                    const uint64_t bdesc = BMN ? smem_desc_mn_sw128(sa + C::A_BYTES, kMnChunkBytes)
+                                               : smem_desc_k_sw128(sa + C::A_BYTES);
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
-                        // advance the start address by k * 32 bytes (16-byte units)
                         const uint32_t accum = (kb != item.kb_lo || k != 0) ? 1u : 0u;
                         if (CG == 2)
-                            tc_mma_f16_pair(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
-                                            accum);
+                            tc_mma_f16_pair(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, accum);
                         else
-                            tc_mma_f16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc, accum);
+                            tc_mma_f16(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, accum);
                     }
                     if (CG == 2) tc_commit_pair_mc(empty0 + 8 * stage, 0x3);
                     else tc_commit(empty0 + 8 * stage);
@@ -388,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t stg = staging0 + (uint32_t)ew * 4096u;
         const uint32_t rbar = rbar0 + 8u * (uint32_t)ew;
         uint32_t rphase = 0;
-        const bool has_resid = EPI == EPI_BIAS_RESID && p.resid != nullptr;
+        const bool has_resid = (EPI == EPI_BIAS_RESID || DACT) && p.resid != nullptr;
         const uint32_t my_row = stg + (uint32_t)lane * 128u;
         const uint32_t swz = (uint32_t)(lane & 7);
         int it = 0;
@@ -401,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int wrow0 = (int)t.orow0 + quarter * 32;
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-            const float* bias_g = p.bias + (long long)t.g * p.N;
+            const float* bias_g = p.bias ? p.bias + (long long)t.g * p.N : nullptr;
             const bool split = item.tj >= 0;
             // this warp's block (CH chunks of 32 x 64) of slice s of tail tile tj: [chunk][16 float4][lane]
             const long long wsblk = split ? (((long long)item.tj * p.nsplit) * CG + rank) * kEpiWarps + ew : 0;
@@ -494,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!live) continue;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    if (n + 16 * q < p.N) {
+                    if (bias_g && n + 16 * q < p.N) {
                         const float4* b4 = reinterpret_cast<const float4*>(bias_g + n + 16 * q);
 #pragma unroll
                         for (int r = 0; r < 4; ++r) {
@@ -509,6 +568,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
+                if ((EPI == EPI_RELU || EPI == EPI_GELU_TANH || EPI == EPI_GELU_ERF) && p.save_pre) {
+                    // the activation's input, kept for the backward pass: its own
+                    // store through the staging buffer, before the activation
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(my_row + ((((uint32_t)j) ^ swz) << 4)),
+                                     "r"(pack_bf16x2(v[8 * j], v[8 * j + 1])), "r"(pack_bf16x2(v[8 * j + 2], v[8 * j + 3])),
+                                     "r"(pack_bf16x2(v[8 * j + 4], v[8 * j + 5])), "r"(pack_bf16x2(v[8 * j + 6], v[8 * j + 7]))
+                                     : "memory");
+                    fence_proxy_async_shared();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (p.o_g_inner) tma_store_3d(&tmR, stg, n, t.g, wrow0);
+                        else tma_store_3d(&tmR, stg, n, wrow0, t.g);
+                        bulk_commit_group();
+                        bulk_wait_read_all();
+                    }
+                    __syncwarp();
+                }
                 if (EPI == EPI_RELU) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e) v[e] = fmaxf(v[e], 0.0f);
@@ -522,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else if (EPI == EPI_GELU_ERF) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e) v[e] = 0.5f * v[e] * (1.0f + erff(v[e] * 0.7071067811865476f));
-                } else if (EPI == EPI_BIAS_RESID) {
+                } else if (EPI == EPI_BIAS_RESID || DACT) {
                     if (has_resid) {
                         if (!mbar_wait(rbar, rphase, wc, SITE_TC_EPILOGUE)) {
                             ok = false;
@@ -539,12 +617,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                             unpack_pairs(u, rp);
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                const float2 y = f2_add(make_float2(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]), rp[e]);
+                                const float2 a = make_float2(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
+                                const float2 y = DACT ? f2_mul(a, make_float2(dact<EPI>(rp[e].x), dact<EPI>(rp[e].y)))
+                                                      : f2_add(a, rp[e]);
                                 v[8 * j + 2 * e] = y.x;
                                 v[8 * j + 2 * e + 1] = y.y;
                             }
                         }
                     }
+                }
+                if constexpr (F32OUT) {
+                    // two 32-column float halves through the staging buffer
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (hh) {
+                            if (lane == 0) bulk_wait_read_all();
+                            __syncwarp();
+                        }
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float* q = v + 32 * hh + 4 * j;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                             my_row + ((((uint32_t)j) ^ swz) << 4)),
+                                         "r"(__float_as_uint(q[0])), "r"(__float_as_uint(q[1])),
+                                         "r"(__float_as_uint(q[2])), "r"(__float_as_uint(q[3]))
+                                         : "memory");
+                        }
+                        fence_proxy_async_shared();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (p.o_g_inner) tma_store_3d(&tmO, stg, n + 32 * hh, t.g, wrow0);
+                            else tma_store_3d(&tmO, stg, n + 32 * hh, wrow0, t.g);
+                            bulk_commit_group();
+                        }
+                    }
+                    continue;
                 }
                 uint32_t w[32];
 #pragma unroll
@@ -695,10 +802,10 @@ struct Maps {
     CUtensorMap a, b, o, r;
 };
 
-template <int BN, int EPI, int CG, bool VAR>
+template <int BN, int EPI, int CG, bool VAR, bool AMN = false, bool BMN = false>
 cudaError_t launch_typed(const Maps& m, const KParams& kp, int grid, cudaStream_t s) {
     using C = Cfg<BN, CG, VAR>;
-    auto k = gemm_tc_kernel<BN, EPI, CG, VAR>;
+    auto k = gemm_tc_kernel<BN, EPI, CG, VAR, AMN, BMN>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -716,6 +823,27 @@ cudaError_t launch_typed(const Maps& m, const KParams& kp, int grid, cudaStream_
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, k, m.a, m.b, m.o, m.r, kp);
+}
+
+// Operand layouts of the backward products: (K-major A, N-major W) for the
+// activation gradients, (M-major A, N-major W) for the weight gradients.
+template <int BN, int CG>
+cudaError_t launch_bn_mn(int epi, bool a_mn, const Maps& m, const KParams& kp, int grid, cudaStream_t s) {
+    if constexpr ((BN / CG) % 64 != 0) {
+        return cudaErrorInvalidValue;
+    } else {
+        if (a_mn) {
+            if (epi == EPI_F32) return launch_typed<BN, EPI_F32, CG, false, true, true>(m, kp, grid, s);
+            return cudaErrorInvalidValue;
+        }
+        switch (epi) {
+            case EPI_DACT_TANH: return launch_typed<BN, EPI_DACT_TANH, CG, false, false, true>(m, kp, grid, s);
+            case EPI_DACT_ERF: return launch_typed<BN, EPI_DACT_ERF, CG, false, false, true>(m, kp, grid, s);
+            case EPI_DACT_RELU: return launch_typed<BN, EPI_DACT_RELU, CG, false, false, true>(m, kp, grid, s);
+            case EPI_BIAS_RESID: return launch_typed<BN, EPI_BIAS_RESID, CG, false, false, true>(m, kp, grid, s);
+        }
+        return cudaErrorInvalidValue;
+    }
 }
 
 template <int BN, int CG, bool VAR>
@@ -760,7 +888,8 @@ static cudaError_t launch_gemm_tc_nosplit(const GroupedGemm& g, DeviceErr err, u
     return launch_gemm_tc(h, err, budget_ns, num_sms, s);
 }
 
-static int gemm_tc_pick_bn(int G, int M, int N, int K, bool var_rows, int num_sms, int cg, bool split) {
+static int gemm_tc_pick_bn(int G, int M, int N, int K, bool var_rows, int num_sms, int cg, bool split,
+                           bool w_mn = false) {
     const int cands[4] = {256, 192, 160, 128};
     const double mma_eff[4] = {1.0, 0.88, 0.8, 0.74};
     int best = 256;
@@ -768,6 +897,7 @@ static int gemm_tc_pick_bn(int G, int M, int N, int K, bool var_rows, int num_sm
     for (int i = 0; i < 4; ++i) {
         const int bn = cands[i];
         if (!var_rows && bn % 64) continue;   // dense tiles leave in 64-column chunks
+        if (w_mn && (bn / cg) % 64) continue;  // N-major W tiles are whole 64-row boxes
         const long long nblk = (N + bn - 1) / bn;
         const double col_fill = (double)N / (double)(nblk * bn);
         double wave_fill = 1.0;
@@ -794,6 +924,16 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     if (g.K % 8 || g.N % 16 || g.G < 1 || g.M < 0 || g.K < 1) return cudaErrorInvalidValue;
     const bool var = g.grp_cnt != nullptr;
     if (var && g.G + 1 > kMaxVarGroups) return cudaErrorInvalidValue;
+    const bool dact = g.epi == EPI_DACT_TANH || g.epi == EPI_DACT_ERF || g.epi == EPI_DACT_RELU;
+    const bool f32out = g.epi == EPI_F32;
+    const bool mn = g.a_mn || g.w_mn;
+    // layouts the kernel is instantiated for
+    if (mn && (var || !g.w_mn || (g.a_mn != f32out) || (!g.a_mn && !dact && g.epi != EPI_BIAS_RESID)))
+        return cudaErrorInvalidValue;
+    if ((dact || f32out) && !mn) return cudaErrorInvalidValue;
+    if (dact && !g.resid) return cudaErrorInvalidValue;
+    if (g.a_mn && g.M % 8) return cudaErrorInvalidValue;   // 16-byte rows of an M-major A
+    if (f32out && g.N % 32) return cudaErrorInvalidValue;
     KParams kp{};
     kp.G = g.G;
     kp.M = g.M;
@@ -819,13 +959,18 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     kp.nsplit = 1;
     kp.sk_ws = g.sk_ws;
     kp.sk_cnt = g.sk_cnt;
+    kp.w_from_kernel = g.w_from_kernel ? 1 : 0;
+    // activation epilogues with resid set: resid receives the pre-activation values
+    kp.save_pre = (g.resid && (g.epi == EPI_GELU_TANH || g.epi == EPI_GELU_ERF || g.epi == EPI_RELU)) ? 1 : 0;
+    if (kp.save_pre && var) return cudaErrorInvalidValue;
+    kp.w_g_inner = 0;
     kp.err = err;
     kp.budget_ns = budget_ns;
 
     // 2-SM (256-row) tiles for dense problems with more than one 128-row block;
     // the variable-row (MoE) groups keep 128-row tiles.
     int cg = (!var && g.M > BM) ? 2 : 1;
-    int bn = gemm_tc_pick_bn(g.G, g.M, g.N, g.K, var, num_sms, cg, g.sk_ws && g.sk_cnt);
+    int bn = gemm_tc_pick_bn(g.G, g.M, g.N, g.K, var, num_sms, cg, g.sk_ws && g.sk_cnt, g.w_mn);
     // Tuning overrides (same kernel, other tile shape): RM_GEMM_CG=1|2, RM_GEMM_BN=256|192|160|128.
     if (const char* e = getenv("RM_GEMM_CG")) {
         const int v = atoi(e);
@@ -835,6 +980,7 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
         const int v = atoi(e);
         if (v == 256 || v == 192 || v == 128 || (var && v == 160)) bn = v;
     }
+    if (g.w_mn && (bn / cg) % 64) bn = 128 * cg > 256 ? 256 : 128 * cg;
     Maps m;
     memset(&m, 0, sizeof(m));
     bool ok;
@@ -842,6 +988,15 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
         // compacted rows [rows_total, K]
         ok = make_map(&m.a, g.A, g.K, g.a_rows_total, 1, g.a_ld * 2, g.a_rows_total * g.a_ld * 2, BM, 1);
         kp.a_g_inner = 0;
+    } else if (g.a_mn) {
+        // M-major A: element (g, m, k) at g*a_gstride + k*a_ld + m; boxes of 64 rows x 64 K
+        if (g.a_gstride <= g.a_ld) {
+            ok = make_map(&m.a, g.A, g.M, g.G, g.K, g.a_gstride * 2, g.a_ld * 2, 1, BK);
+            kp.a_g_inner = 1;
+        } else {
+            ok = make_map(&m.a, g.A, g.M, g.K, g.G, g.a_ld * 2, g.a_gstride * 2, BK, 1);
+            kp.a_g_inner = 0;
+        }
     } else if (g.a_gstride <= g.a_ld) {
         // group stride inside the row stride, e.g. S [B, T, D]: dims (K, G, M)
         ok = make_map(&m.a, g.A, g.K, g.G, g.M, g.a_gstride * 2, g.a_ld * 2, 1, BM);
@@ -851,17 +1006,30 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
         ok = make_map(&m.a, g.A, g.K, g.M, g.G, g.a_ld * 2, g.a_gstride * 2, BM, 1);
         kp.a_g_inner = 0;
     }
-    ok = ok && make_map(&m.b, g.W, g.K, g.N, g.G, (uint64_t)g.K * 2, (uint64_t)g.N * g.K * 2, (uint32_t)(bn / cg), 1);
+    const long long w_ld = g.w_ld ? g.w_ld : g.K, w_gs = g.w_ld ? g.w_gstride : (long long)g.N * g.K;
+    if (g.w_mn) {
+        // N-major W: element (g, n, k) at g*w_gstride + k*w_ld + n; boxes of 64 rows x 64 K
+        if (w_gs <= w_ld) {
+            ok = ok && make_map(&m.b, g.W, g.N, g.G, g.K, w_gs * 2, w_ld * 2, 1, BK);
+            kp.w_g_inner = 1;
+        } else {
+            ok = ok && make_map(&m.b, g.W, g.N, g.K, g.G, w_ld * 2, w_gs * 2, BK, 1);
+        }
+    } else {
+        ok = ok && make_map(&m.b, g.W, g.K, g.N, g.G, w_ld * 2, w_gs * 2, (uint32_t)(bn / cg), 1);
+    }
     if (!var) {
-        // output (and residual) tiles of 32 rows x 64 columns, same orientation as A
+        // output (and residual) tiles of 32 rows x 64 columns (32 for float
+        // output), same orientation as A
+        const uint64_t osz = f32out ? 4 : 2;
         if (g.o_gstride <= g.o_ld) {
-            ok = ok && make_map(&m.o, g.out, g.N, g.G, g.M, g.o_gstride * 2, g.o_ld * 2, 1, 32);
+            ok = ok && make_map(&m.o, g.out, g.N, g.G, g.M, g.o_gstride * osz, g.o_ld * osz, 1, 32, f32out);
             kp.o_g_inner = 1;
         } else {
-            ok = ok && make_map(&m.o, g.out, g.N, g.M, g.G, g.o_ld * 2, g.o_gstride * 2, 32, 1);
+            ok = ok && make_map(&m.o, g.out, g.N, g.M, g.G, g.o_ld * osz, g.o_gstride * osz, 32, 1, f32out);
             kp.o_g_inner = 0;
         }
-        if (g.resid) {
+        if (g.resid) {   // residual / activation input tile (loaded), or the pre-activation output (stored)
             if ((g.r_gstride <= g.r_ld) != (kp.o_g_inner == 1)) return cudaErrorInvalidValue;
             ok = ok && (kp.o_g_inner ? make_map(&m.r, g.resid, g.N, g.G, g.M, g.r_gstride * 2, g.r_ld * 2, 1, 32)
                                      : make_map(&m.r, g.resid, g.N, g.M, g.G, g.r_ld * 2, g.r_gstride * 2, 32, 1));
@@ -893,6 +1061,15 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
             case 192: return launch_bn<192, 1, true>(g.epi, m, kp, grid, s);
             case 160: return launch_bn<160, 1, true>(g.epi, m, kp, grid, s);
             default: return launch_bn<128, 1, true>(g.epi, m, kp, grid, s);
+        }
+    }
+    if (mn) {
+        if (cg == 2) return bn == 256 ? launch_bn_mn<256, 2>(g.epi, g.a_mn, m, kp, grid, s)
+                                      : launch_bn_mn<128, 2>(g.epi, g.a_mn, m, kp, grid, s);
+        switch (bn) {
+            case 256: return launch_bn_mn<256, 1>(g.epi, g.a_mn, m, kp, grid, s);
+            case 192: return launch_bn_mn<192, 1>(g.epi, g.a_mn, m, kp, grid, s);
+            default: return launch_bn_mn<128, 1>(g.epi, g.a_mn, m, kp, grid, s);
         }
     }
     if (cg == 2) {

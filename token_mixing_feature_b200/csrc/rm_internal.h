@@ -23,6 +23,7 @@ enum WaitSite : int {
     SITE_TC_DRAIN = 5,
     SITE_MIX_LN = 6,
     SITE_LN_POOL = 7,
+    SITE_TRAIN_MIX = 8,
     SITE_SELFTEST = 9,
 };
 
@@ -39,9 +40,12 @@ struct RowStats {
 };
 // S = LN1(TokenMixing(Xh) + Xh), Xh = pre_g ? LN_pre(X) : X (per token row,
 // statistics from pre_stats); with addnorm == 0, S = TokenMixing(Xh).
+// Training (addnorm only): xhat_out [B, T, D] receives the normalised rows
+// (Z - mean) * rstd and rstd_out [B*T] the rows' 1/sqrt(var + eps).
 cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const float* pre_b, RowStats pre_stats,
                           const float* g1, const float* b1, void* S, int B, int T, int D, float eps, int addnorm,
-                          int num_sms, DeviceErr err, uint64_t budget_ns, cudaStream_t s);
+                          int num_sms, DeviceErr err, uint64_t budget_ns, cudaStream_t s, void* xhat_out = nullptr,
+                          float* rstd_out = nullptr);
 // pooled[b] = mean_t LN(X[b, t]) (statistics given); Xout (optional) = LN(X).
 cudaError_t launch_ln_pool(int dtype, const void* X, RowStats stats, const float* g, const float* b, float* pooled,
                            void* Xout, int B, int T, int D, float eps, int num_sms, DeviceErr err,
@@ -66,25 +70,47 @@ cudaError_t launch_selftest_wait(DeviceErr err, uint64_t budget_ns, cudaStream_t
 enum Epilogue : int {
     EPI_GELU_TANH = 0,   // bf16( GELU_tanh(acc + bias) )
     EPI_GELU_ERF = 1,    // bf16( GELU_erf(acc + bias) )
-    EPI_BIAS_RESID = 2,  // bf16( acc + bias [+ resid] )
+    EPI_BIAS_RESID = 2,  // bf16( acc [+ bias] [+ resid] )
     EPI_BIAS_GATE = 3,   // bf16( gate[row] * (acc + bias) )
     EPI_RELU = 4,        // bf16( max(acc + bias, 0) )
+    // backward products (dense only): resid holds the activation's input U
+    EPI_DACT_TANH = 5,   // bf16( acc * GELU_tanh'(U) )
+    EPI_DACT_ERF = 6,    // bf16( acc * GELU_erf'(U) )
+    EPI_DACT_RELU = 7,   // bf16( acc * [U > 0] )
+    EPI_F32 = 8,         // float( acc )   (out is float)
 };
 inline int epi_for_act(int act) { return act == RM_ACT_GELU_ERF ? EPI_GELU_ERF : act == RM_ACT_RELU ? EPI_RELU : EPI_GELU_TANH; }
+inline int dact_epi_for_act(int act) {
+    return act == RM_ACT_GELU_ERF ? EPI_DACT_ERF : act == RM_ACT_RELU ? EPI_DACT_RELU : EPI_DACT_TANH;
+}
 
 struct GroupedGemm {
     int G, M, N, K;
-    // A operand: element (g, m, k) at A + g*a_gstride + m*a_ld + k (elements).
+    // A operand: element (g, m, k) at A + g*a_gstride + m*a_ld + k (elements),
+    // or, with a_mn (M-major A, dense only), at A + g*a_gstride + k*a_ld + m.
     const void* A;
     long long a_gstride, a_ld;
     long long a_rows_total;   // variable-row mode: rows allocated in A (and out)
-    // W operand [G][N][K] contiguous.
+    bool a_mn;
+    // W operand: [G][N][K] contiguous when w_ld == 0; else element (g, n, k)
+    // at W + g*w_gstride + n*w_ld + k, or, with w_mn (N-major, dense only),
+    // at W + g*w_gstride + k*w_ld + n.
     const void* W;
-    // out element (g, m, n) at out + g*o_gstride + m*o_ld + n.
+    long long w_gstride, w_ld;
+    bool w_mn;
+    // W was written by an earlier kernel on the stream (activations in a
+    // weight-gradient product): its tiles are loaded only after the
+    // programmatic-launch wait.  False for model weights.
+    bool w_from_kernel;
+    // out element (g, m, n) at out + g*o_gstride + m*o_ld + n (bf16; float
+    // for EPI_F32).
     void* out;
     long long o_gstride, o_ld;
-    const float* bias;        // [G][N]
-    const void* resid;        // EPI_BIAS_RESID (may be null): same indexing as out, strides below
+    const float* bias;        // [G][N]; may be null for EPI_BIAS_RESID; unused by EPI_DACT_* / EPI_F32
+    // bf16, same indexing as out, strides below: EPI_BIAS_RESID the residual
+    // (may be null); EPI_DACT_* the activation input U; activation epilogues
+    // (dense, may be null): receives bf16(acc + bias), the activation input.
+    const void* resid;
     long long r_gstride, r_ld;
     const float* gate;        // EPI_BIAS_GATE: [rows] in variable-row mode
     int epi;
@@ -156,10 +182,10 @@ struct MoeWork {
 };
 cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, const MoeWork& w, int B,
                              int T, int D, int Ne, cudaStream_t s);
-cudaError_t launch_moe_gather(const void* S, const MoeWork& w, int B, int T, int D, int Ne,
-                              cudaStream_t s);
 // out[r] = resid[r] + sum_j Eg[slot_of[r, j]]; stats (may be null) = (mean, M2)
 // of each stored row (P = 1).
+cudaError_t launch_moe_gather(const void* S, const MoeWork& w, int B, int T, int D, int Ne,
+                              cudaStream_t s);
 cudaError_t launch_moe_combine(const MoeWork& w, const void* resid, void* out, float2* stats, int B, int T, int D,
                                int Ne, cudaStream_t s);
 

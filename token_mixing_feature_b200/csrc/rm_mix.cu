@@ -10,21 +10,26 @@
 // copy overlaps the current one's arithmetic.  The permutation is applied
 // through shared-memory addressing with 16-byte vectors (rows padded so the
 // pieces consecutive lanes gather fall in consecutive banks), so X is read
-// from HBM once and S written once, with no transpose pass.  Row statistics
-// take LPR = 8/16/32 lanes per row (pass A); the element-wise pass (pass B)
-// gives each thread one 16-byte column vector of a row group.
+// from HBM once and S written once, with no transpose pass.
 //
-// The previous block's LayerNorm (PRE) uses row statistics produced where the
-// row was written (the grouped GEMM's epilogue, the MoE combine, or
-// row_stats_kernel) as partial (mean, M2) pairs over P equal column slices,
-// merged here in two warp sums -- no extra pass over the rows.
+// The mixing kernel computes each output row's LN1 statistics with LPR =
+// 8/16/32 lanes per row (pass A), then writes the normalised rows with one
+// thread per (row group, 16-byte column vector) that keeps gamma / beta in
+// registers (pass B).  The previous block's LayerNorm (PRE) uses row
+// statistics produced where the row was written (the grouped GEMM's epilogue,
+// the MoE combine, or row_stats_kernel) as partial (mean, M2) pairs over P
+// equal column slices; those partials travel into the ring slot with the rows
+// (one more bulk copy), so no thread waits on a global load for them.
 //
 // mix_ln:  Xh = PRE ? LN_pre(X) : X                       (per token row)
 //          Z[h, t*dh + j] = Xh[t, h*dh + j] + Xh[h, t*dh + j]
 //          S[h, :] = LN1(Z[h, :])
 //          or, without the Add & Norm after mixing, S[h, t*dh + j] = Xh[t, h*dh + j]
-// ln_pool: pooled[b, :] = (1/T) sum_t LN(X[b, t, :])  (row groups, then groups in order)
+// ln_pool: pooled[b, :] = (1/T) sum_t LN(X[b, t, :])  (one thread per sample
+//          and 16-byte column vector, rows summed in ascending t)
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 #include "rm_device.cuh"
 
@@ -63,10 +68,18 @@ __device__ __forceinline__ void load_params(const float* __restrict__ p, float (
     }
 }
 
-// Ring of whole samples in shared memory.  Slot s holds one sample's T rows
-// at a row stride of rs >= D elements; it fills from one cp.async.bulk copy
-// (rs == D) or T row copies issued by the lanes of warp 0, on the slot's
-// mbarrier.  Slot bookkeeping lives in bit masks in lane 0 of warp 0.
+// Ring of whole samples in shared memory.  Slot s holds one chunk's rows at a
+// row stride of rs >= D elements, and (when the kernel merges LayerNorm
+// partials) the chunk's partial statistics after them; it fills from one
+// cp.async.bulk copy of the rows (rs == D) or one copy per row issued by the
+// lanes of warp 0, plus one copy of the partials, all on the slot's mbarrier.
+// Slot bookkeeping lives in bit masks in lane 0 of warp 0.
+//
+// Partials: the chunk's P * rows float2 pairs are contiguous in global memory
+// but need not start on a 16-byte boundary, so the copy starts at the
+// boundary below and ends at the one above; the partial array must be
+// readable up to the 16-byte boundary past its end (its workspace region is
+// padded to 256 bytes).  stats() returns the chunk's first pair in the slot.
 constexpr int kMaxSlots = 4;
 
 template <typename E>
@@ -75,23 +88,41 @@ struct SampleRing {
     uint32_t bar0;         // mbarrier of slot s at bar0 + 8 * s
     int nslots, D, rs;
     uint32_t slot_bytes;
+    uint32_t stats_off;    // byte offset of the staged partials in a slot; 0: none staged
+    const float2* part;    // partials [rows][P] in global memory (stats_off != 0)
+    int P;
     uint32_t outstanding;  // bit s: a copy into slot s was issued and not yet waited for
     uint32_t parity;       // bit s: parity of slot s's next completion
 
     __device__ __forceinline__ E* buf(int slot) const { return reinterpret_cast<E*>(base + (size_t)slot * slot_bytes); }
     __device__ __forceinline__ uint32_t bar(int slot) const { return bar0 + 8u * (uint32_t)slot; }
+    __device__ __forceinline__ const float2* stats(int slot, long long row0) const {
+        const uintptr_t a = reinterpret_cast<uintptr_t>(part + row0 * P);
+        return reinterpret_cast<const float2*>(base + (size_t)slot * slot_bytes + stats_off + (a & 15u));
+    }
 
-    // all lanes of warp 0: `rows` contiguous rows [rows, D] from src into `slot`
-    __device__ void issue(int slot, const E* src, int rows) {
+    // all lanes of warp 0: `rows` contiguous rows [rows, D] from src (global
+    // rows row0 ...) into `slot`, with their partials if staged
+    __device__ void issue(int slot, const E* src, int rows, long long row0) {
         const int lane = threadIdx.x & 31;
         const uint32_t row_bytes = (uint32_t)(D * sizeof(E));
+        uint32_t sbytes = 0;
+        const void* ssrc = nullptr;
+        if (stats_off) {
+            const uintptr_t a = reinterpret_cast<uintptr_t>(part + row0 * P);
+            const uintptr_t e = a + (uintptr_t)rows * (uintptr_t)P * sizeof(float2);
+            const uintptr_t a16 = a & ~static_cast<uintptr_t>(15), e16 = (e + 15) & ~static_cast<uintptr_t>(15);
+            ssrc = reinterpret_cast<const void*>(a16);
+            sbytes = (uint32_t)(e16 - a16);
+        }
         if (lane == 0) {
-            mbar_arrive_expect_tx(bar(slot), row_bytes * (uint32_t)rows);
+            mbar_arrive_expect_tx(bar(slot), row_bytes * (uint32_t)rows + sbytes);
             outstanding |= 1u << slot;
         }
         __syncwarp();
         fence_proxy_async_smem();   // earlier generic accesses to the slot come first
         const uint32_t dst = smem_u32(buf(slot));
+        if (sbytes && lane == 31) bulk_load(dst + stats_off, ssrc, sbytes, bar(slot));
         if (rs == D) {   // unpadded rows: one contiguous copy
             if (lane == 0) bulk_load(dst, src, row_bytes * (uint32_t)rows, bar(slot));
             return;
@@ -115,18 +146,29 @@ struct SampleRing {
     }
 };
 
-// Bytes of one ring slot (128-byte multiple).
-inline __host__ __device__ size_t slot_bytes_of(int T, int rs, size_t esz) {
-    return ((size_t)T * rs * esz + 127) / 128 * 128;
+// Bytes of the rows part of a slot (128-byte multiple) and of its staged
+// partials (rows * P pairs plus 16 bytes of alignment slack, 16-byte multiple).
+inline __host__ __device__ size_t rows_bytes_of(int rows, int rs, size_t esz) {
+    return ((size_t)rows * rs * esz + 127) / 128 * 128;
+}
+inline __host__ __device__ size_t stats_bytes_of(int rows, int P) {
+    return P > 0 ? ((size_t)rows * P * 8 + 16 + 15) / 16 * 16 : 0;
+}
+inline __host__ __device__ size_t slot_bytes_of(int rows, int rs, size_t esz, int P) {
+    return (rows_bytes_of(rows, rs, esz) + stats_bytes_of(rows, P) + 127) / 128 * 128;
 }
 
-// Carves the ring (nslots slots of `rows` rows), its barriers and the
-// per-row statistics (mean_s[rows], rstd_s[rows]) out of dynamic shared
-// memory; returns the first float after them.
+// Carves the ring (nslots slots of `rows` rows, with partials when P > 0), its
+// barriers and the per-row statistics (mean_s[rows], rstd_s[rows]) out of
+// dynamic shared memory.
 template <typename E>
-__device__ __forceinline__ float* make_ring(SampleRing<E>& r, unsigned char* smem, int rows, int D, int rs,
-                                            int nslots, float*& mean_s, float*& rstd_s) {
-    r.slot_bytes = (uint32_t)slot_bytes_of(rows, rs, sizeof(E));
+__device__ __forceinline__ void make_ring(SampleRing<E>& r, unsigned char* smem, int rows, int D, int rs,
+                                          int nslots, const float2* part, int P, float*& mean_s,
+                                          float*& rstd_s) {
+    r.slot_bytes = (uint32_t)slot_bytes_of(rows, rs, sizeof(E), part ? P : 0);
+    r.stats_off = part ? (uint32_t)rows_bytes_of(rows, rs, sizeof(E)) : 0u;
+    r.part = part;
+    r.P = P;
     r.nslots = nslots;
     r.D = D;
     r.rs = rs;
@@ -137,7 +179,6 @@ __device__ __forceinline__ float* make_ring(SampleRing<E>& r, unsigned char* sme
     r.parity = 0;
     mean_s = reinterpret_cast<float*>(bars + kMaxSlots);
     rstd_s = mean_s + rows;
-    return reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(rstd_s + rows) + 15) & ~static_cast<uintptr_t>(15));
 }
 
 // Row stride of the staged sample for the mixing kernel: D plus a pad that
@@ -157,32 +198,20 @@ inline int mix_row_stride(int D, int dh, size_t esz) {
 // (Chan et al.) combination reduces to mean = (1/P) sum_p mean_p and
 // M2 = sum_p M2_p + n sum_p (mean_p - mean)^2: two warp sums in a fixed
 // butterfly order (deterministic), no divisions; P <= 32.
-// Row statistics of rows row0 .. row0+R-1 into mean_s/rstd_s, all warps of
-// the CTA: each warp loads the partials of up to four rows before reducing
-// them, so the loads' latency is paid once per four rows.
-__device__ __forceinline__ void chunk_stats(const float2* __restrict__ part, int P, int D, long long row0, int R,
-                                            float eps, float* mean_s, float* rstd_s) {
+// Row statistics of the R rows of a chunk into mean_s/rstd_s, all warps of
+// the CTA, from the partials staged in shared memory with the chunk.
+__device__ __forceinline__ void chunk_stats(const float2* part, int P, int D, int R, float eps, float* mean_s,
+                                            float* rstd_s) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const float n = (float)D / (float)P;
-    for (int r = warp; r < R; r += 4 * nw) {
-        float2 v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int rr = r + k * nw;
-            v[k] = (rr < R && lane < P) ? __ldcg(part + (row0 + rr) * P + lane) : make_float2(0.f, 0.f);
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int rr = r + k * nw;
-            if (rr < R) {   // warp-uniform
-                const float mean = warp_sum(v[k].x) / (float)P;
-                const float d = v[k].x - mean;
-                const float q = warp_sum(lane < P ? fmaf(n * d, d, v[k].y) : 0.f);
-                if (lane == 0) {
-                    mean_s[rr] = mean;
-                    rstd_s[rr] = rsqrtf(q / D + eps);
-                }
-            }
+    for (int r = warp; r < R; r += nw) {
+        const float2 v = lane < P ? part[(size_t)r * P + lane] : make_float2(0.f, 0.f);
+        const float mean = warp_sum(v.x) / (float)P;
+        const float d = v.x - mean;
+        const float q = warp_sum(lane < P ? fmaf(n * d, d, v.y) : 0.f);
+        if (lane == 0) {
+            mean_s[r] = mean;
+            rstd_s[r] = rsqrtf(q / D + eps);
         }
     }
 }
@@ -233,23 +262,24 @@ constexpr int kMixMaxThreads = 384;
 // In-place LayerNorm of the staged sample (row statistics in shared memory),
 // in fp32 pairs: y = ((x r) - m r) gamma + beta.
 template <typename E>
-__device__ __forceinline__ void normalize_in_place(E* xs, int rows, int rs, int c0, int grp, int groups,
+__device__ __forceinline__ void normalize_in_place(uint32_t xs_a, int rows, int rs, int c0, int grp, int groups,
                                                    const float* __restrict__ g, const float* __restrict__ bta,
-                                                   const float* mean_s, const float* rstd_s) {
+                                                   uint32_t mean_a, uint32_t rstd_a) {
     constexpr int NP = Vec16<E>::N / 2;
     float2 gp[NP], bp[NP];
     load_pairs(g + c0, gp);
     load_pairs(bta + c0, bp);
-#pragma unroll 2
-    for (int t = grp; t < rows; t += groups) {
-        uint4* p = reinterpret_cast<uint4*>(xs + (size_t)t * rs + c0);
+    uint32_t pa = xs_a + (uint32_t)((grp * rs + c0) * (int)sizeof(E));
+    const uint32_t pstep = (uint32_t)(groups * rs * (int)sizeof(E));
+#pragma unroll 4
+    for (int t = grp; t < rows; t += groups, pa += pstep) {
         float2 x[NP];
-        unpack_pairs(*p, x);
-        const float r = rstd_s[t];
-        const float2 r2 = f2(r), mr2 = f2(-mean_s[t] * r);
+        unpack_pairs(lds128(pa), x);
+        const float r = lds_f32(rstd_a + 4u * (uint32_t)t);
+        const float2 r2 = f2(r), mr2 = f2(-lds_f32(mean_a + 4u * (uint32_t)t) * r);
 #pragma unroll
         for (int j = 0; j < NP; ++j) x[j] = f2_fma(f2_fma(x[j], r2, mr2), gp[j], bp[j]);
-        *p = pack_pairs(x);
+        sts128(pa, pack_pairs(x));
     }
 }
 
@@ -290,7 +320,7 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
     const E* __restrict__ X, const float* __restrict__ pre_g, const float* __restrict__ pre_b,
     const float2* __restrict__ pstats, int P, const float* __restrict__ g1, const float* __restrict__ b1,
     E* __restrict__ S, int B, int T, int D, float eps, int rs, int spb, int nslots, int groups, DeviceErr err,
-    uint64_t budget_ns) {
+    uint64_t budget_ns, E* __restrict__ xhat_out, float* __restrict__ rstd_out) {
     pdl_enter();
     constexpr int V = Vec16<E>::N;
     extern __shared__ __align__(128) unsigned char smem[];
@@ -299,7 +329,7 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
     const int nchunks = (B + spb - 1) / spb;   // chunk c: samples [c*spb, c*spb + spb) in one slot
     float *mean_s, *rstd_s;
     SampleRing<E> ring;
-    make_ring<E>(ring, smem, spb * T, D, rs, nslots, mean_s, rstd_s);
+    make_ring<E>(ring, smem, spb * T, D, rs, nslots, PRE ? pstats : nullptr, P, mean_s, rstd_s);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const WaitCtx wc{&abort_flag, budget_ns, err};
     if (tid == 0) {
@@ -312,7 +342,7 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
     if (warp == 0)
         for (int k = 0; k < nslots; ++k) {
             const long long ck = blockIdx.x + (long long)k * gridDim.x;
-            if (ck < nchunks) ring.issue(k, X + (size_t)ck * spb * TD, chunk_rows(ck));
+            if (ck < nchunks) ring.issue(k, X + (size_t)ck * spb * TD, chunk_rows(ck), ck * spb * T);
         }
     const int dh = D / T;
     const int nv = D / V;
@@ -338,14 +368,18 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
         const int cur = it % nslots;
         const int R = chunk_rows(c);
         const long long row0 = c * spb * T;   // global row of the chunk's first row
-        if (PRE) chunk_stats(pstats, P, D, row0, R, eps, mean_s, rstd_s);   // from the producer's partials
         if (tid == 0) s_ok = ring.wait(cur, wc, SITE_MIX_LN);
         __syncthreads();
         if (!s_ok) break;
         E* xs = ring.buf(cur);
         if (PRE) {
-            // the previous block's LayerNorm, applied once per element, in place
-            if (active) normalize_in_place(xs, R, rs, c0, grp, groups, pre_g, pre_b, mean_s, rstd_s);
+            // the previous block's LayerNorm, from the partials staged with the
+            // chunk, applied once per element, in place
+            chunk_stats(ring.stats(cur, row0), P, D, R, eps, mean_s, rstd_s);
+            __syncthreads();
+            if (active)
+                normalize_in_place<E>(smem_u32(xs), R, rs, c0, grp, groups, pre_g, pre_b, smem_u32(mean_s),
+                                      smem_u32(rstd_s));
             __syncthreads();
         }
         E* srow = S + (size_t)row0 * D;
@@ -384,8 +418,10 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
                 }
                 if (sl == 0 && r0 + sub < R) {
                     const float m1 = s1 / D;
+                    const float rstd = rsqrtf(fmaxf(s2 / D - m1 * m1, 0.f) + eps);
                     mean_s[r] = K + m1;
-                    rstd_s[r] = rsqrtf(fmaxf(s2 / D - m1 * m1, 0.f) + eps);
+                    rstd_s[r] = rstd;
+                    if (rstd_out) rstd_out[row0 + r] = rstd;
                 }
             }
             __syncthreads();
@@ -407,7 +443,11 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
                     const float rr = rstd_s[r];
                     const float2 r2 = f2(rr), mr2 = f2(-mean_s[r] * rr);
 #pragma unroll
-                    for (int j = 0; j < NP; ++j) pm[j] = f2_fma(f2_fma(f2_add(pm[j], pr[j]), r2, mr2), g1p[j], b1p[j]);
+                    for (int j = 0; j < NP; ++j) pm[j] = f2_fma(f2_add(pm[j], pr[j]), r2, mr2);   // xhat
+                    if (xhat_out)   // training: the normalised row, kept for the backward pass
+                        *reinterpret_cast<uint4*>(xhat_out + (size_t)(row0 + r) * D + c0) = pack_pairs(pm);
+#pragma unroll
+                    for (int j = 0; j < NP; ++j) pm[j] = f2_fma(pm[j], g1p[j], b1p[j]);
                     o = pack_pairs(pm);
                 }
                 *reinterpret_cast<uint4*>(srow + (size_t)r * D + c0) = o;
@@ -420,18 +460,19 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
         }
         __syncthreads();   // the slot and the statistics are free again
         const long long nc = c + (long long)nslots * gridDim.x;
-        if (warp == 0 && nc < nchunks) ring.issue(cur, X + (size_t)nc * spb * TD, chunk_rows(nc));
+        if (warp == 0 && nc < nchunks) ring.issue(cur, X + (size_t)nc * spb * TD, chunk_rows(nc), nc * spb * T);
     }
     if (tid == 0) ring.drain(wc, SITE_MIX_LN);
 }
 
 // pooled[b, c] = gamma[c] * (1/T) sum_t (x[t, c] - m_t) r_t + beta[c]; Xout
 // (optional) receives LN(x).  Persistent CTAs stream chunks of spb whole
-// samples through the shared-memory ring.  The threads form `groups` row
-// groups (groups divides T) of nv = D/V column-vector threads; group q sums
-// rows q, q + groups, ... of each sample, and the groups' partial sums are
-// added in ascending q (deterministic).
-constexpr int kPoolThreads = 512;
+// samples, with their partial statistics, through the shared-memory ring.
+// After the chunk's row statistics are merged, thread u takes (sample
+// u / nv, 16-byte column vector u % nv) and sums that column over the
+// sample's T rows in ascending t (deterministic), so no partial sums cross
+// threads.
+constexpr int kPoolThreads = 384;
 constexpr size_t kMaxSmemPerCta = 227 * 1024;
 
 template <typename E>
@@ -441,7 +482,7 @@ __global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __res
                                                                  const float* __restrict__ bta,
                                                                  float* __restrict__ pooled, E* __restrict__ Xout,
                                                                  int B, int T, int D, float eps, int spb, int nslots,
-                                                                 int groups, DeviceErr err, uint64_t budget_ns) {
+                                                                 DeviceErr err, uint64_t budget_ns) {
     pdl_enter();
     constexpr int V = Vec16<E>::N;
     extern __shared__ __align__(128) unsigned char smem[];
@@ -450,8 +491,7 @@ __global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __res
     const int nchunks = (B + spb - 1) / spb;
     float *mean_s, *rstd_s;
     SampleRing<E> ring;
-    // partial sums [spb][groups][D] after the ring and the statistics
-    float* part = make_ring<E>(ring, smem, spb * T, D, D, nslots, mean_s, rstd_s);
+    make_ring<E>(ring, smem, spb * T, D, D, nslots, pstats, P, mean_s, rstd_s);
     const int tid = threadIdx.x, warp = tid >> 5;
     const WaitCtx wc{&abort_flag, budget_ns, err};
     if (tid == 0) {
@@ -464,68 +504,62 @@ __global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __res
     if (warp == 0)
         for (int k = 0; k < nslots; ++k) {
             const long long ck = blockIdx.x + (long long)k * gridDim.x;
-            if (ck < nchunks) ring.issue(k, X + (size_t)ck * spb * TD, chunk_samples(ck) * T);
+            if (ck < nchunks) ring.issue(k, X + (size_t)ck * spb * TD, chunk_samples(ck) * T, ck * spb * T);
         }
     const int nv = D / V;
-    const int grp = tid / nv, c0 = (tid - grp * nv) * V;
     const float invT = 1.0f / T;
     constexpr int NP = V / 2;
-    float2 gp[NP], bp[NP];
-    if (Xout && grp < groups) {
-        load_pairs(g + c0, gp);
-        load_pairs(bta + c0, bp);
-    }
     int it = 0;
     for (long long c = blockIdx.x; c < nchunks; c += gridDim.x, ++it) {
         const int cur = it % nslots;
         const int ns = chunk_samples(c);
         const int R = ns * T;
         const long long row0 = c * spb * T;
-        chunk_stats(pstats, P, D, row0, R, eps, mean_s, rstd_s);
         if (tid == 0) s_ok = ring.wait(cur, wc, SITE_LN_POOL);
         __syncthreads();
         if (!s_ok) break;
+        chunk_stats(ring.stats(cur, row0), P, D, R, eps, mean_s, rstd_s);
+        __syncthreads();
         const E* xs = ring.buf(cur);
-        if (grp < groups) {
-            for (int sm = 0; sm < ns; ++sm) {
-                float2 acc[NP];
+        for (int u = tid; u < ns * nv; u += blockDim.x) {
+            const int sm = u / nv, c0 = (u - sm * nv) * V;
+            float2 gp[NP], bp[NP];
+            load_pairs(g + c0, gp);
+            load_pairs(bta + c0, bp);
+            float2 acc[NP];
 #pragma unroll
-                for (int j = 0; j < NP; ++j) acc[j] = f2(0.f);
-#pragma unroll 2
-                for (int h = grp; h < T; h += groups) {
-                    const int r = sm * T + h;
-                    float2 x[NP];
-                    unpack_pairs(*reinterpret_cast<const uint4*>(xs + (size_t)r * D + c0), x);
-                    const float rt = rstd_s[r];
-                    const float2 r2 = f2(rt), mr2 = f2(-mean_s[r] * rt);
+            for (int j = 0; j < NP; ++j) acc[j] = f2(0.f);
+            const uint32_t col_a = smem_u32(xs) + (uint32_t)((sm * TD + c0) * (int)sizeof(E));
+            const uint32_t mean_a = smem_u32(mean_s) + 4u * (uint32_t)(sm * T), rstd_a = smem_u32(rstd_s) + 4u * (uint32_t)(sm * T);
+#pragma unroll 4
+            for (int t = 0; t < T; ++t) {
+                const int r = sm * T + t;
+                float2 x[NP];
+                unpack_pairs(lds128(col_a + (uint32_t)(t * D * (int)sizeof(E))), x);
+                const float rt = lds_f32(rstd_a + 4u * (uint32_t)t);
+                const float2 r2 = f2(rt), mr2 = f2(-lds_f32(mean_a + 4u * (uint32_t)t) * rt);
 #pragma unroll
-                    for (int j = 0; j < NP; ++j) {
-                        x[j] = f2_fma(x[j], r2, mr2);   // (x - m_t) r_t
-                        acc[j] = f2_add(acc[j], x[j]);
-                    }
-                    if (Xout) {
-#pragma unroll
-                        for (int j = 0; j < NP; ++j) x[j] = f2_fma(x[j], gp[j], bp[j]);
-                        *reinterpret_cast<uint4*>(Xout + (size_t)(row0 + r) * D + c0) = pack_pairs(x);
-                    }
+                for (int j = 0; j < NP; ++j) {
+                    x[j] = f2_fma(x[j], r2, mr2);   // (x - m_t) r_t
+                    acc[j] = f2_add(acc[j], x[j]);
                 }
-                float4* dst = reinterpret_cast<float4*>(part + ((size_t)sm * groups + grp) * D + c0);
+                if (Xout) {
 #pragma unroll
-                for (int q = 0; q < NP / 2; ++q)
-                    dst[q] = make_float4(acc[2 * q].x, acc[2 * q].y, acc[2 * q + 1].x, acc[2 * q + 1].y);
+                    for (int j = 0; j < NP; ++j) x[j] = f2_fma(x[j], gp[j], bp[j]);
+                    *reinterpret_cast<uint4*>(Xout + (size_t)(row0 + r) * D + c0) = pack_pairs(x);
+                }
+            }
+            float4* dst = reinterpret_cast<float4*>(pooled + (size_t)(c * spb + sm) * D + c0);
+#pragma unroll
+            for (int q = 0; q < NP / 2; ++q) {
+                const float2 p0 = f2_fma(gp[2 * q], f2_mul(acc[2 * q], f2(invT)), bp[2 * q]);
+                const float2 p1 = f2_fma(gp[2 * q + 1], f2_mul(acc[2 * q + 1], f2(invT)), bp[2 * q + 1]);
+                dst[q] = make_float4(p0.x, p0.y, p1.x, p1.y);
             }
         }
-        __syncthreads();   // the slot is free again: refill it before combining the partials
+        __syncthreads();   // the slot and the statistics are free again
         const long long nc = c + (long long)nslots * gridDim.x;
-        if (warp == 0 && nc < nchunks) ring.issue(cur, X + (size_t)nc * spb * TD, chunk_samples(nc) * T);
-        for (int i = tid; i < ns * D; i += blockDim.x) {
-            const int sm = i / D, cc = i - sm * D;
-            const float* ps = part + (size_t)sm * groups * D + cc;
-            float a = ps[0];
-            for (int q = 1; q < groups; ++q) a += ps[(size_t)q * D];
-            pooled[(size_t)(c * spb + sm) * D + cc] = fmaf(__ldg(g + cc), a * invT, __ldg(bta + cc));
-        }
-        __syncthreads();   // statistics and partials are free again
+        if (warp == 0 && nc < nchunks) ring.issue(cur, X + (size_t)nc * spb * TD, chunk_samples(nc) * T, nc * spb * T);
     }
     if (tid == 0) ring.drain(wc, SITE_LN_POOL);
 }
@@ -570,16 +604,18 @@ inline int samples_per_chunk(int T, int rs, size_t esz, int B) {
 }
 
 // Ring slots (up to kMaxSlots, at least 1) and dynamic shared memory for
-// chunks of `rows` rows at row stride rs, plus extra_floats floats after the
-// per-row statistics.  Two CTAs share an SM whenever one slot each fits:
-// measured in the stack, two independent CTAs (one computes while the other
-// waits for its copy) beat one CTA with a deeper ring.
-inline void ring_shape(int rows, int rs, size_t esz, size_t extra_floats, int* nslots, size_t* smem) {
-    const size_t one = slot_bytes_of(rows, rs, esz);
-    const size_t fixed = 8 * kMaxSlots + sizeof(float) * (2 * (size_t)rows + extra_floats) + 16;
+// chunks of `rows` rows at row stride rs, with P staged partials per row (P =
+// 0: none), plus the per-row statistics and extra_floats floats, for `per_sm`
+// CTAs per SM (two, each with as many slots as fit, whenever one slot each
+// fits: measured in the stack, two independent CTAs -- one computes while the
+// other waits for its copy -- beat one CTA with a deeper ring).
+inline void ring_shape(int rows, int rs, size_t esz, int P, int per_sm, int* nslots, size_t* smem,
+                       size_t extra_floats = 0) {
+    const size_t one = slot_bytes_of(rows, rs, esz, P);
+    const size_t fixed = 8 * kMaxSlots + sizeof(float) * (2 * (size_t)rows + extra_floats) + 32;
     const size_t full = 227 * 1024 - 1024;    // static shared memory and slack
     const size_t half = full / 2 - 1024;
-    const size_t avail = one + fixed <= half ? half : full;
+    const size_t avail = per_sm > 1 && one + fixed <= half ? half : full;
     long long n = avail > fixed ? (long long)((avail - fixed) / one) : 0;
     if (n > kMaxSlots) n = kMaxSlots;
     if (n < 1) n = 1;
@@ -600,7 +636,7 @@ inline int mix_groups(int T, int nv) { return mix_groups_cap(T, nv, kMixMaxThrea
 template <typename E, bool PRE, int MV, int NVV, bool ADDNORM, int LPR>
 cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps, const float* g1, const float* b1,
                       E* S, int B, int T, int D, float eps, int num_sms, DeviceErr err, uint64_t budget,
-                      cudaStream_t s) {
+                      cudaStream_t s, E* xhat_out, float* rstd_out) {
     constexpr int V = Vec16<E>::N;
     const int nv = D / V;
     if (nv < 1 || nv > kMixMaxThreads) return cudaErrorInvalidValue;
@@ -611,7 +647,7 @@ cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps,
     const int spb = samples_per_chunk(T, rs, sizeof(E), B);
     int nslots;
     size_t smem;
-    ring_shape(spb * T, rs, sizeof(E), 0, &nslots, &smem);
+    ring_shape(spb * T, rs, sizeof(E), PRE ? ps.P : 0, 2, &nslots, &smem);
     auto k = mix_ln_kernel<E, PRE, MV, NVV, ADDNORM, LPR>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
@@ -625,7 +661,7 @@ cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps,
     const long long g = (long long)num_sms * per_sm;
     const int grid = (int)(g < nchunks ? g : nchunks);
     return launch_pdl(k, grid, threads, smem, s, X, pg, pb, ps.part, ps.P, g1, b1, S, B, T, D, eps, rs, spb, nslots,
-                      groups, err, budget);
+                      groups, err, budget, xhat_out, rstd_out);
 }
 
 // Lanes per row of the statistics pass: 8 for rows of <= 64 vectors, 16 for
@@ -634,9 +670,9 @@ cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps,
 template <typename E, bool PRE, int MV>
 cudaError_t mix_ln_nv(int nv, int addnorm, const E* X, const float* pg, const float* pb, RowStats ps,
                       const float* g1, const float* b1, E* S, int B, int T, int D, float eps, int num_sms,
-                      DeviceErr err, uint64_t budget, cudaStream_t s) {
+                      DeviceErr err, uint64_t budget, cudaStream_t s, E* xo, float* ro) {
 #define RM_MIX_GO(NVV, AN, LPRV) \
-    mix_ln_go<E, PRE, MV, NVV, AN, LPRV>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s)
+    mix_ln_go<E, PRE, MV, NVV, AN, LPRV>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s, xo, ro)
     if (!addnorm) return RM_MIX_GO(1, false, 32);
     if (nv <= 64) {
         const int nvl = (nv + 7) / 8;
@@ -665,7 +701,7 @@ cudaError_t mix_ln_nv(int nv, int addnorm, const E* X, const float* pg, const fl
 template <typename E>
 cudaError_t mix_ln_typed(const void* X, const float* pg, const float* pb, RowStats ps, const float* g1,
                          const float* b1, void* S, int B, int T, int D, float eps, int addnorm, int num_sms,
-                         DeviceErr err, uint64_t budget, cudaStream_t s) {
+                         DeviceErr err, uint64_t budget, cudaStream_t s, void* xhat_out, float* rstd_out) {
     constexpr int V = Vec16<E>::N;
     const int nv = D / V;
     const int dh = D / T;
@@ -673,7 +709,8 @@ cudaError_t mix_ln_typed(const void* X, const float* pg, const float* pb, RowSta
     const E* x = static_cast<const E*>(X);
     E* y = static_cast<E*>(S);
 #define RM_MIX_MV(PREV, MVV) \
-    mix_ln_nv<E, PREV, MVV>(nv, addnorm, x, pg, pb, ps, g1, b1, y, B, T, D, eps, num_sms, err, budget, s)
+    mix_ln_nv<E, PREV, MVV>(nv, addnorm, x, pg, pb, ps, g1, b1, y, B, T, D, eps, num_sms, err, budget, s, \
+                            static_cast<E*>(xhat_out), rstd_out)
 #define RM_MIX_PRE(PREV) (mv == V ? RM_MIX_MV(PREV, V) : mv == V / 2 ? RM_MIX_MV(PREV, V / 2) : RM_MIX_MV(PREV, 1))
     const cudaError_t e = pg ? RM_MIX_PRE(true) : RM_MIX_PRE(false);
 #undef RM_MIX_PRE
@@ -687,31 +724,27 @@ cudaError_t ln_pool_go(const void* X, RowStats stats, const float* g, const floa
     constexpr int V = Vec16<E>::N;
     const int nv = D / V;
     if (nv < 1 || nv > kPoolThreads) return cudaErrorInvalidValue;
-    int groups = mix_groups_cap(T, nv, kPoolThreads);   // divides T
-    // chunk partials [spb][groups][D] stay within 32 KB
-    int spb = samples_per_chunk(T, D, sizeof(E), B);
-    while (spb > 1 && (size_t)spb * groups * D * sizeof(float) > kChunkTargetBytes) --spb;
+    const int spb = samples_per_chunk(T, D, sizeof(E), B);
+    int threads = (int)std::min<long long>(kPoolThreads, ((long long)spb * nv + 31) / 32 * 32);
+    if (threads < 64) threads = 64;
     int nslots;
     size_t smem;
-    ring_shape(spb * T, D, sizeof(E), (size_t)spb * groups * D, &nslots, &smem);
-    while (groups > 1 && smem > kMaxSmemPerCta - 1024) {   // large samples: fewer row groups
-        groups = mix_groups_cap(T, nv, groups * nv - 1);
-        ring_shape(spb * T, D, sizeof(E), (size_t)spb * groups * D, &nslots, &smem);
-    }
+    ring_shape(spb * T, D, sizeof(E), stats.P, 2, &nslots, &smem);
+    if (smem > kMaxSmemPerCta - 1024) return cudaErrorInvalidValue;
     auto k = ln_pool_kernel<E>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kPoolThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const long long nchunks = (B + spb - 1) / spb;
     const long long gr = (long long)num_sms * per_sm;
     const int grid = (int)(gr < nchunks ? gr : nchunks);
-    return launch_pdl(k, grid, kPoolThreads, smem, s, static_cast<const E*>(X), stats.part, stats.P, g, b, pooled,
-                      static_cast<E*>(Xout), B, T, D, eps, spb, nslots, groups, err, budget);
+    return launch_pdl(k, grid, threads, smem, s, static_cast<const E*>(X), stats.part, stats.P, g, b, pooled,
+                      static_cast<E*>(Xout), B, T, D, eps, spb, nslots, err, budget);
 }
 
 }  // namespace
@@ -720,26 +753,30 @@ cudaError_t ln_pool_go(const void* X, RowStats stats, const float* g, const floa
 // statistics pass).
 int mix_ln_max_d(int dtype) { return 32 * 8 * (dtype == RM_BF16 ? 8 : 4); }
 
-// Whether one staged sample (padded for the mixing gather) plus the kernels'
-// per-row and pooling scratch fits a CTA's shared memory.
+// Whether one staged sample (padded for the mixing gather) with its staged
+// LayerNorm partials (D/64 per row for bf16 rows of a multiple of 64 columns,
+// else 1) and per-row statistics fits a CTA's shared memory.
 bool mix_ln_sample_fits(int dtype, int T, int D) {
     const size_t esz = dtype == RM_BF16 ? 2 : 4;
     const int V = (int)(16 / esz);
     const int dh = D / T;
     const int rs = dh % V == 0 ? mix_row_stride(D, dh, esz) : D;
-    const size_t fixed = 8 * kMaxSlots + sizeof(float) * (2 * (size_t)T + (size_t)D);   // one pooling group
-    return slot_bytes_of(T, rs, esz) + fixed <= 227 * 1024 - 1024;
+    const int P = (dtype == RM_BF16 && D % 64 == 0) ? D / 64 : 1;   // LayerNorm partials per row
+    const size_t fixed = 8 * kMaxSlots + sizeof(float) * 2 * (size_t)T + 32;
+    return slot_bytes_of(T, rs, esz, P) + fixed <= 227 * 1024 - 1024;
 }
 
 cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const float* pre_b, RowStats pre_stats,
                           const float* g1, const float* b1, void* S, int B, int T, int D, float eps, int addnorm,
-                          int num_sms, DeviceErr err, uint64_t budget_ns, cudaStream_t s) {
+                          int num_sms, DeviceErr err, uint64_t budget_ns, cudaStream_t s, void* xhat_out,
+                          float* rstd_out) {
     if (pre_g && (!pre_stats.part || pre_stats.P < 1 || pre_stats.P > 32)) return cudaErrorInvalidValue;
+    if ((xhat_out || rstd_out) && !addnorm) return cudaErrorInvalidValue;
     if (dtype == RM_BF16)
         return mix_ln_typed<__nv_bfloat16>(X, pre_g, pre_b, pre_stats, g1, b1, S, B, T, D, eps, addnorm, num_sms,
-                                           err, budget_ns, s);
+                                           err, budget_ns, s, xhat_out, rstd_out);
     return mix_ln_typed<float>(X, pre_g, pre_b, pre_stats, g1, b1, S, B, T, D, eps, addnorm, num_sms, err,
-                               budget_ns, s);
+                               budget_ns, s, xhat_out, rstd_out);
 }
 
 cudaError_t launch_ln_pool(int dtype, const void* X, RowStats stats, const float* g, const float* b, float* pooled,

@@ -27,6 +27,7 @@ EXPORTED = (
     "rm_last_error_site", "rm_set_wait_budget", "rm_selftest_wait_timeout", "rm_status_string",
     "rm_profile_begin", "rm_profile_end", "rm_kernel_name", "rm_pffn_forward_static",
     "rm_stack_forward_host_async", "rm_host_wait",
+    "rm_train_create", "rm_train_destroy", "rm_train_workspace_bytes", "rm_train_step", "rm_train_sync_status",
 )
 RM_STATIC_SCRATCH_BYTES = 16 << 20
 RM_K_COUNT = 12
@@ -42,6 +43,10 @@ class rm_config(ctypes.Structure):
 class rm_block_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("W1", "b1", "W2", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b", "Wr", "br")]
+
+
+class rm_block_grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W1", "b1", "W2", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b")]
 
 
 class RankMixerError(RuntimeError):
@@ -80,6 +85,12 @@ def _load() -> ctypes.CDLL:
         "rm_kernel_name": (ctypes.c_char_p, [ci]),
         "rm_pffn_forward_static": (st, [ctypes.POINTER(rm_block_weights), vp, vp, ci, ci, ci, ci, ci, ci,
                                         vp, vp]),
+        "rm_train_create": (st, [ctypes.POINTER(rm_config), ctypes.POINTER(vp)]),
+        "rm_train_destroy": (st, [vp]),
+        "rm_train_workspace_bytes": (ctypes.c_size_t, [vp]),
+        "rm_train_step": (st, [vp, ctypes.POINTER(rm_block_weights), vp, vp, vp, vp, ctypes.POINTER(rm_block_grads),
+                               vp, vp, vp, vp, vp, ci, vp]),
+        "rm_train_sync_status": (st, [vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -285,3 +296,65 @@ def rm_pffn_forward_static(w: Dict, S, V, B: int, T: int, D: int, hidden: int, d
     _check(_lib.rm_pffn_forward_static(ctypes.byref(bw), _ptr(S), _ptr(V), B, T, D, hidden, DTYPES[dtype],
                                        ACTS[act], _ptr(device_status), _stream(stream)),
            "rm_pffn_forward_static")
+
+
+# ------------------------------------------------------------- training step
+class Trainer:
+    """Owns one rm_trainer.  Call close() (or use as a context manager)."""
+
+    def __init__(self, ptr: int, cfg: rm_config):
+        self.ptr = ptr
+        self.cfg = cfg
+
+    def close(self) -> None:
+        if self.ptr:
+            p, self.ptr = self.ptr, None
+            _check(_lib.rm_train_destroy(p), "rm_train_destroy")
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def rm_train_create(B_max: int, T: int, D: int, hidden: int, L: int, ln_eps: float = 1e-5,
+                    act: str = "tanh") -> Trainer:
+    cfg = rm_config(B_max, T, D, hidden, L, 0, RM_BF16, ln_eps, ACTS[act], 1)
+    out = ctypes.c_void_p()
+    _check(_lib.rm_train_create(ctypes.byref(cfg), ctypes.byref(out)), "rm_train_create")
+    return Trainer(out.value, cfg)
+
+
+def rm_train_destroy(t: Trainer) -> None:
+    t.close()
+
+
+def rm_train_workspace_bytes(t: Trainer) -> int:
+    return _lib.rm_train_workspace_bytes(t.ptr)
+
+
+def block_grads(g: Dict) -> rm_block_grads:
+    return rm_block_grads(**{n: _ptr(g.get(n)) for n, _ in rm_block_grads._fields_})
+
+
+def rm_train_step(t: Trainer, blocks: Sequence[Dict], X0, head_w, head_b, labels, grads: Sequence[Dict], dX0,
+                  dhead_w, dhead_b, loss, pooled, B: int, stream=None) -> None:
+    """grads: one dict of float device tensors per block (keys of rm_block_grads)."""
+    arr = _block_array(blocks)
+    garr = (rm_block_grads * len(grads))()
+    for i, g in enumerate(grads):
+        garr[i] = block_grads(g)
+    _check(_lib.rm_train_step(t.ptr, arr, _ptr(X0), _ptr(head_w), _ptr(head_b), _ptr(labels), garr, _ptr(dX0),
+                              _ptr(dhead_w), _ptr(dhead_b), _ptr(loss), _ptr(pooled), B, _stream(stream)),
+           "rm_train_step")
+
+
+def rm_train_sync_status(t: Trainer, stream=None) -> int:
+    return _lib.rm_train_sync_status(t.ptr, _stream(stream))
