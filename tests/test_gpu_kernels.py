@@ -245,6 +245,39 @@ def test_moe_block(rm, O):
     assert_close(host64(Xout), O.block(X, blk), "bf16", "moe block")
 
 
+def test_moe_pair_tiles_match(rm, O, tmp_path):
+    """Expert GEMMs on CTA pairs with 256-row tiles (tuning override
+    RM_MOE_PAIR=1, read once per process: a child process) give the MoE block
+    within the bf16 bounds of the oracle; a group's odd CTA past the group's
+    end computes nothing it stores."""
+    import os
+    import subprocess
+    import sys
+    B, T, D, hidden, Ne = 300, 4, 128, 128, 8
+    blk = synth.random_like_block(T, D, hidden, "bf16", seed=33, n_experts=Ne, router_std=0.1,
+                                  router_bias=-0.05)
+    X = synth.random_activations((B, T, D), "bf16", seed=34)
+    torch.save({"blk": blk, "X": X}, tmp_path / "in.pt")
+    script = tmp_path / "run.py"
+    script.write_text(
+        "import sys, torch\n"
+        "sys.path.insert(0, %r)\n"
+        "from token_mixing_feature_b200 import rankmixer as rm\n"
+        "d = torch.load(sys.argv[1])\n"
+        "blk = {k: v.cuda().contiguous() for k, v in d['blk'].items()}\n"
+        "X = d['X'].cuda()\n"
+        "with rm.rm_create(%d, %d, %d, %d, 1, %d, 'bf16') as h:\n"
+        "    out = torch.empty_like(X)\n"
+        "    rm.rm_block_forward(h, blk, X, out, %d)\n"
+        "    assert rm.rm_sync_status(h) == rm.RM_OK\n"
+        "torch.save(out.cpu(), sys.argv[2])\n" % (os.getcwd(), B, T, D, hidden, Ne, B))
+    env = dict(os.environ, RM_MOE_PAIR="1")
+    subprocess.run([sys.executable, str(script), str(tmp_path / "in.pt"), str(tmp_path / "out.pt")], check=True,
+                   env=env, timeout=600)
+    got = torch.load(tmp_path / "out.pt")
+    assert_close(host64(got), O.block(X, blk), "bf16", "moe block, pair tiles")
+
+
 # ------------------------------------------------------ robustness / checks
 def test_deterministic(rm):
     T, D, hidden, B = 16, 256, 1024, 200

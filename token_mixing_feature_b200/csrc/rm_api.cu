@@ -203,6 +203,16 @@ rm_status run_pffn(rm_handle* h, const rm_block_weights* w, const void* S, void*
     return cuda_status(e);
 }
 
+// Expert tiles: single CTAs with 128-row tiles, or CTA pairs with 256-row
+// tiles (tuning override RM_MOE_PAIR=1; the routing's tile prefix follows).
+bool moe_pair_tiles() {
+    static const bool on = [] {
+        const char* e = getenv("RM_MOE_PAIR");
+        return e && atoi(e) == 1;
+    }();
+    return on;
+}
+
 // V = sum_j ReLU-gate * expert(S) (+ resid); gates_out optional copy of G;
 // stats (optional) receives the LayerNorm statistics of V (one slice per row).
 rm_status run_moe(rm_handle* h, const rm_block_weights* w, const void* S, void* V, const void* resid,
@@ -214,7 +224,7 @@ rm_status run_moe(rm_handle* h, const rm_block_weights* w, const void* S, void* 
     cudaError_t e;
     {
         ProfScope ps(h, RM_K_MOE_ROUTE, s);
-        e = rm::launch_moe_route(S, w->Wr, w->br, h->moe, B, c.T, c.D, Ne, s);
+        e = rm::launch_moe_route(S, w->Wr, w->br, h->moe, B, c.T, c.D, Ne, s, moe_pair_tiles() ? 256 : 128);
     }
     if (e == cudaSuccess) {
         ProfScope ps(h, RM_K_MOE_GATHER, s);
@@ -233,6 +243,7 @@ rm_status run_moe(rm_handle* h, const rm_block_weights* w, const void* S, void* 
     g1.o_ld = c.hidden;
     g1.bias = static_cast<const float*>(w->b1);
     g1.epi = rm::epi_for_act(c.act);
+    g1.var_cg = moe_pair_tiles() ? 2 : 1;
     g1.grp_cnt = h->moe.counts;
     g1.grp_off = h->moe.offsets;
     g1.mtile_prefix = h->moe.mtile_prefix;

@@ -132,7 +132,7 @@ __device__ __forceinline__ Tile decode_tile(const KParams& p, long long idx, int
         t.rows = min(BM, p.M - m0);
         t.n0 = nb * bn;
         t.orow0 = m0;
-    } else {   // CG == 1 only
+    } else {   // tiles of BM * CG rows; rank r of a pair takes rows [r*BM, r*BM + BM) of it
         int lo = 0, hi = p.G;
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
@@ -142,12 +142,12 @@ __device__ __forceinline__ Tile decode_tile(const KParams& p, long long idx, int
         const int nt = mt[lo + 1] - p0;
         const int local = (int)(idx - (long long)p0 * nblk);
         const int nb = local / nt, mb = local - nb * nt;
-        const int m0 = mb * BM;
+        const int m0 = mb * (BM * CG) + rank * BM;
         const int off = __ldcg(p.grp_off + lo);
         t.g = lo;
         t.ag = 0;
         t.arow = off + m0;
-        t.rows = min(BM, __ldcg(p.grp_cnt + lo) - m0);
+        t.rows = min(BM, __ldcg(p.grp_cnt + lo) - m0);   // <= 0: the odd CTA of a pair past the group's end
         t.n0 = nb * bn;
         t.orow0 = off + m0;
     }
@@ -505,8 +505,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 64 * half; c < BN; c += 128) {
                 const int n = t.n0 + c;
                 const bool live = n < p.N;   // warp-uniform
-                if (lane == 0) bulk_wait_read_all();   // the previous store has read the buffer
-                __syncwarp();
+                if (!F32OUT) {   // (float output alternates two buffers below)
+                    if (lane == 0) bulk_wait_read_all();   // the previous store has read the buffer
+                    __syncwarp();
+                }
                 if (has_resid && live && lane == 0) {
                     mbar_arrive_expect_tx(rbar, 4096);
                     if (p.o_g_inner) tma_load_3d(stg, &tmR, rbar, n, t.g, wrow0);
@@ -630,10 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // two 32-column float halves through the staging buffer
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
-                        if (hh) {
-                            if (lane == 0) bulk_wait_read_all();
-                            __syncwarp();
-                        }
+                        if (lane == 0) bulk_wait_read_all();   // the previous store has read the buffer
+                        __syncwarp();
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             const float* q = v + 32 * hh + 4 * j;
@@ -969,7 +969,7 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
 
     // 2-SM (256-row) tiles for dense problems with more than one 128-row block;
     // the variable-row (MoE) groups keep 128-row tiles.
-    int cg = (!var && g.M > BM) ? 2 : 1;
+    int cg = var ? (g.var_cg == 2 ? 2 : 1) : (g.M > BM ? 2 : 1);
     int bn = gemm_tc_pick_bn(g.G, g.M, g.N, g.K, var, num_sms, cg, g.sk_ws && g.sk_cnt, g.w_mn);
     // Tuning overrides (same kernel, other tile shape): RM_GEMM_CG=1|2, RM_GEMM_BN=256|192|160|128.
     if (const char* e = getenv("RM_GEMM_CG")) {
@@ -1056,6 +1056,14 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     }
     const int grid = units * cg;
     if (var) {
+        if (cg == 2) {
+            switch (bn) {
+                case 256: return launch_bn<256, 2, true>(g.epi, m, kp, grid, s);
+                case 192: return launch_bn<192, 2, true>(g.epi, m, kp, grid, s);
+                case 160: return launch_bn<160, 2, true>(g.epi, m, kp, grid, s);
+                default: return launch_bn<128, 2, true>(g.epi, m, kp, grid, s);
+            }
+        }
         switch (bn) {
             case 256: return launch_bn<256, 1, true>(g.epi, m, kp, grid, s);
             case 192: return launch_bn<192, 1, true>(g.epi, m, kp, grid, s);

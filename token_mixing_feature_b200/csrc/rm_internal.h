@@ -120,7 +120,9 @@ struct GroupedGemm {
     float2* stats;
     long long s_gstride, s_ld;
     // Variable-row mode (sparse MoE): group g owns rows [grp_off[g], grp_off[g] + grp_cnt[g])
-    // of A and out (g strides unused); mtile_prefix[g] = sum_{g' < g} ceil(cnt / 128).
+    // of A and out (g strides unused); mtile_prefix[g] = sum_{g' < g} ceil(cnt / (128 var_cg)).
+    // var_cg = 2: CTA pairs with 256-row tiles (each CTA 128 rows); else 1.
+    int var_cg;
     const int* grp_cnt;
     const int* grp_off;
     const int* mtile_prefix;  // [G + 1]
@@ -171,7 +173,7 @@ struct MoeWork {
     float* gates;          // [B, T, Ne]
     int* counts;           // [T*Ne]
     int* offsets;          // [T*Ne]
-    int* mtile_prefix;     // [T*Ne + 1]
+    int* mtile_prefix;     // [T*Ne + 1]: prefix of ceil(count / tile rows) over the experts
     int* totals;           // [2]: active entries, m-tiles
     int* slot_row;         // [B*T*Ne]: slot -> row b*T + t of S
     float* slot_gate;      // [B*T*Ne]
@@ -181,7 +183,7 @@ struct MoeWork {
     void* Eg;              // [B*T*Ne, D] bf16 gate-scaled expert outputs
 };
 cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, const MoeWork& w, int B,
-                             int T, int D, int Ne, cudaStream_t s);
+                             int T, int D, int Ne, cudaStream_t s, int tile_rows = 128);
 // out[r] = resid[r] + sum_j Eg[slot_of[r, j]]; stats (may be null) = (mean, M2)
 // of each stored row (P = 1).
 cudaError_t launch_moe_gather(const void* S, const MoeWork& w, int B, int T, int D, int Ne,

@@ -139,7 +139,8 @@ __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__
                                                        const int* __restrict__ counts, int* __restrict__ offsets,
                                                        int* __restrict__ mtile_prefix, int* __restrict__ totals,
                                                        int* __restrict__ slot_row, float* __restrict__ slot_gate,
-                                                       int* __restrict__ slot_of, int B, int T, int Ne) {
+                                                       int* __restrict__ slot_of, int B, int T, int Ne,
+                                                       int tile_rows) {
     pdl_enter();
     __shared__ int s_off;
     __shared__ int s_warp[32];
@@ -152,7 +153,7 @@ __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__
         for (int q = lane; q < g; q += 32) {
             const int c = __ldcg(counts + q);
             off += c;
-            mt += (c + 127) / 128;
+            mt += (c + tile_rows - 1) / tile_rows;
         }
         off = warp_isum(off);
         mt = warp_isum(mt);
@@ -162,9 +163,9 @@ __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__
             mtile_prefix[g] = mt;
             if (g == G - 1) {
                 const int c = __ldcg(counts + g);
-                mtile_prefix[G] = mt + (c + 127) / 128;
+                mtile_prefix[G] = mt + (c + tile_rows - 1) / tile_rows;
                 totals[0] = off + c;
-                totals[1] = mt + (c + 127) / 128;
+                totals[1] = mt + (c + tile_rows - 1) / tile_rows;
             }
         }
     }
@@ -305,7 +306,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const __nv_bfloat16* 
 }  // namespace
 
 cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, const MoeWork& w, int B, int T,
-                             int D, int Ne, cudaStream_t s) {
+                             int D, int Ne, cudaStream_t s, int tile_rows) {
     cudaError_t e = cudaMemsetAsync(w.counts, 0, sizeof(int) * T * Ne, s);
     if (e != cudaSuccess) return e;
     const size_t smem = sizeof(float) * (size_t)Ne * D;
@@ -342,7 +343,7 @@ cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, co
     else RM_ROUTE(32)
 #undef RM_ROUTE
     return launch_pdl(compact_kernel, T * Ne, 1024, 0, s, w.gates, w.counts, w.offsets, w.mtile_prefix, w.totals,
-                      w.slot_row, w.slot_gate, w.slot_of, B, T, Ne);
+                      w.slot_row, w.slot_gate, w.slot_of, B, T, Ne, tile_rows);
 }
 
 cudaError_t launch_moe_gather(const void* S, const MoeWork& w, int B, int T, int D, int Ne, cudaStream_t s) {

@@ -41,9 +41,10 @@ namespace rm {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kLnRows = 4;          // rows per block-wide reduction in the LayerNorm backward
+constexpr int kLnRows = 8;          // rows per block-wide reduction in the LayerNorm backward
 constexpr int kMaxSampleBlock = 64; // samples per CTA of the LayerNorm backward
-constexpr int kColRows = 64;        // rows per partial of the column sums
+constexpr int kColRows = 16;        // rows per partial of the column sums
+constexpr int kRedWarps = 8;        // sample / slice warps of the ordered column reductions
 
 __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -97,24 +98,36 @@ __global__ void __launch_bounds__(kThreads) head_logit_kernel(const float* poole
     }
 }
 
-// Thread per column n: dw[n] = sum_b dlogit_b pooled[b, n] (ascending b) and
-// gpool[b, n] = dlogit_b w[n] / T, the gradient of every token row of the last
-// block's output; one thread adds up the loss and dc in ascending b.
-__global__ void __launch_bounds__(kThreads) head_grad_kernel(const float* pooled, const __nv_bfloat16* __restrict__ w,
-                                                            const float* dlogit, const float* lterm, float* dw,
-                                                            float* dc, float* loss, float* gpool, int B, int D,
-                                                            float invT) {
+// dw[n] = sum_b dlogit_b pooled[b, n] and gpool[b, n] = dlogit_b w[n] / T,
+// the gradient of every token row of the last block's output.  CTA = 32
+// columns; warp w takes samples b = w, w + 8, ... in ascending order and the
+// eight warp sums are added in warp order.  One thread adds up the loss and
+// dc in ascending b.
+__global__ void __launch_bounds__(32 * kRedWarps) head_grad_kernel(const float* pooled,
+                                                                  const __nv_bfloat16* __restrict__ w,
+                                                                  const float* dlogit, const float* lterm, float* dw,
+                                                                  float* dc, float* loss, float* gpool, int B, int D,
+                                                                  float invT) {
     pdl_enter();
-    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    __shared__ float red[kRedWarps][33];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n = blockIdx.x * 32 + lane;
+    float acc = 0.f;
     if (n < D) {
         const float wn = __bfloat162float(w[n]) * invT;
-        float acc = 0.f;
-        for (int b = 0; b < B; ++b) {
+        for (int b = warp; b < B; b += kRedWarps) {
             const float g = __ldcg(dlogit + b);
             acc = fmaf(g, __ldcg(pooled + (long long)b * D + n), acc);
             gpool[(long long)b * D + n] = g * wn;
         }
-        dw[n] = acc;
+    }
+    red[warp][lane] = acc;
+    __syncthreads();
+    if (warp == 0 && n < D) {
+        float t = 0.f;
+#pragma unroll
+        for (int q = 0; q < kRedWarps; ++q) t += red[q][lane];
+        dw[n] = t;
     }
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         float l = 0.f, c = 0.f;
@@ -133,8 +146,18 @@ __global__ void __launch_bounds__(kThreads) head_grad_kernel(const float* pooled
 // recomputed from Y and its partial statistics.  Thread v owns the 8 columns
 // [8v, 8v + 8) of every row and accumulates, over its rows, the partial
 // column sums of G * xhat (dgamma), G (dbeta) and dY (the token's second
-// bias).  G is dX' [B, T, D] (bf16), or with FROM_POOL gpool [B, D] (fp32,
+// bias).  Rows go in groups of kLnRows: one pass for the rows' sums (one
+// block-wide reduction per group), a second pass, reading the rows again,
+// for dY.  G is dX' [B, T, D] (bf16), or with FROM_POOL gpool [B, D] (fp32,
 // the same row for every token).
+template <bool FROM_POOL>
+__device__ __forceinline__ void ln2_bwd_load(const __nv_bfloat16* G, const float* gpool, const __nv_bfloat16* Y,
+                                             long long b, long long row, int D, int c0, float (&g)[8], float (&y)[8]) {
+    if (FROM_POOL) load8f(gpool + b * D + c0, g);
+    else unpack8(__ldcg(reinterpret_cast<const uint4*>(G + row * D + c0)), g);
+    unpack8(__ldcg(reinterpret_cast<const uint4*>(Y + row * D + c0)), y);
+}
+
 template <bool FROM_POOL>
 __global__ void __launch_bounds__(kThreads) ln2_bwd_kernel(const __nv_bfloat16* G, const float* gpool,
                                                           const __nv_bfloat16* Y, const float2* ystats, int P,
@@ -170,30 +193,25 @@ __global__ void __launch_bounds__(kThreads) ln2_bwd_kernel(const __nv_bfloat16* 
     const float invD = 1.0f / (float)D;
     int par = 0;
     for (int i0 = 0; i0 < nb; i0 += kLnRows, par ^= 1) {
-        float gx[kLnRows][8], xh[kLnRows][8], cs[2 * kLnRows];
+        // pass 1: the rows' sums of g*G and g*G*xhat, and the column partials
+        float cs[2 * kLnRows];
 #pragma unroll
         for (int k = 0; k < kLnRows; ++k) {
             const int i = i0 + k;
             float s1 = 0.f, s2 = 0.f;
             if (active && i < nb) {
-                const long long row = (long long)(b0 + i) * T + t;
                 float g[8], y[8];
-                if (FROM_POOL) load8f(gpool + (long long)(b0 + i) * D + c0, g);
-                else unpack8(__ldcg(reinterpret_cast<const uint4*>(G + row * D + c0)), g);
-                unpack8(__ldcg(reinterpret_cast<const uint4*>(Y + row * D + c0)), y);
+                ln2_bwd_load<FROM_POOL>(G, gpool, Y, b0 + i, (long long)(b0 + i) * T + t, D, c0, g, y);
                 const float m = mean_s[i], r = rstd_s[i];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    xh[k][e] = (y[e] - m) * r;
-                    gx[k][e] = g[e] * gm[e];
-                    s1 += gx[k][e];
-                    s2 = fmaf(gx[k][e], xh[k][e], s2);
-                    ag[e] = fmaf(g[e], xh[k][e], ag[e]);
+                    const float xh = (y[e] - m) * r;
+                    const float gx = g[e] * gm[e];
+                    s1 += gx;
+                    s2 = fmaf(gx, xh, s2);
+                    ag[e] = fmaf(g[e], xh, ag[e]);
                     ab[e] += g[e];
                 }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) xh[k][e] = gx[k][e] = 0.f;
             }
             cs[2 * k] = s1;
             cs[2 * k + 1] = s2;
@@ -210,16 +228,19 @@ __global__ void __launch_bounds__(kThreads) ln2_bwd_kernel(const __nv_bfloat16* 
             for (int w = 0; w < nw; ++w) a += red[par][w][q];
             cs[q] = a * invD;
         }
+        // pass 2: the rows again (from L1 / L2), dY out
 #pragma unroll
         for (int k = 0; k < kLnRows; ++k) {
             const int i = i0 + k;
             if (active && i < nb) {
                 const long long row = (long long)(b0 + i) * T + t;
-                const float r = rstd_s[i];
-                float dy[8];
+                float g[8], y[8], dy[8];
+                ln2_bwd_load<FROM_POOL>(G, gpool, Y, b0 + i, row, D, c0, g, y);
+                const float m = mean_s[i], r = rstd_s[i];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    dy[e] = r * (gx[k][e] - cs[2 * k] - xh[k][e] * cs[2 * k + 1]);
+                    const float xh = (y[e] - m) * r;
+                    dy[e] = r * (g[e] * gm[e] - cs[2 * k] - xh * cs[2 * k + 1]);
                     adb[e] += dy[e];
                 }
                 *reinterpret_cast<uint4*>(dY + row * D + c0) = pack8(dy);
@@ -249,33 +270,70 @@ __global__ void __launch_bounds__(kThreads) colsum_kernel(const __nv_bfloat16* A
     float a[8], a2[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) a[e] = a2[e] = 0.f;
-    for (int r = r0; r < r1; ++r) {
-        const long long off = g * gs + r * ld + 8 * v;
-        float x[8];
-        unpack8(__ldcg(reinterpret_cast<const uint4*>(A + off)), x);
-        if (X2) {
-            float y[8];
-            unpack8(__ldcg(reinterpret_cast<const uint4*>(X2 + off)), y);
+    for (int r = r0; r < r1; r += 4) {   // up to four rows' loads in flight, summed in row order
+        uint4 xa[4], xb[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a2[e] = fmaf(x[e], y[e], a2[e]);
+        for (int q = 0; q < 4; ++q) {
+            if (r + q < r1) {
+                const long long off = g * gs + (long long)(r + q) * ld + 8 * v;
+                xa[q] = __ldcg(reinterpret_cast<const uint4*>(A + off));
+                if (X2) xb[q] = __ldcg(reinterpret_cast<const uint4*>(X2 + off));
+            }
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a[e] += x[e];
+        for (int q = 0; q < 4; ++q) {
+            if (r + q < r1) {
+                float x[8];
+                unpack8(xa[q], x);
+                if (X2) {
+                    float y[8];
+                    unpack8(xb[q], y);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) a2[e] = fmaf(x[e], y[e], a2[e]);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) a[e] += x[e];
+            }
+        }
     }
     const long long o = ((long long)g * nrb + rb) * N + 8 * v;
     store8f(part + o, a);
     if (X2) store8f(part2 + o, a2);
 }
 
-// out[g * N + n] = sum_{j < J} part[(g * J + j) * N + n], ascending j.
-__global__ void __launch_bounds__(kThreads) reduce_parts_kernel(const float* part, float* out, int G, int J, int N) {
+// out[g * N + n] = sum_{j < J} part[(g * J + j) * N + n].  CTA = (32
+// columns, group g); warp w sums the slices j = w, w + 8, ... of its lane's
+// column in ascending j, then one warp adds the eight warp sums in warp order
+// (a fixed order: deterministic).
+__global__ void __launch_bounds__(32 * kRedWarps) reduce_parts_kernel(const float* part, float* out, int G, int J,
+                                                                      int N) {
     pdl_enter();
-    const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-    if (i >= (long long)G * N) return;
-    const long long g = i / N, n = i - g * N;
+    __shared__ float red[kRedWarps][33];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n = blockIdx.x * 32 + lane, g = blockIdx.y;
     float a = 0.f;
-    for (int j = 0; j < J; ++j) a += __ldcg(part + (g * J + j) * N + n);
-    out[i] = a;
+    if (n < N) {
+        const float* p = part + (long long)g * J * N + n;
+        int j = warp;
+        for (; j + 3 * kRedWarps < J; j += 4 * kRedWarps) {   // four loads in flight
+            const float x0 = __ldcg(p + (long long)j * N), x1 = __ldcg(p + (long long)(j + kRedWarps) * N);
+            const float x2 = __ldcg(p + (long long)(j + 2 * kRedWarps) * N);
+            const float x3 = __ldcg(p + (long long)(j + 3 * kRedWarps) * N);
+            a += x0;
+            a += x1;
+            a += x2;
+            a += x3;
+        }
+        for (; j < J; j += kRedWarps) a += __ldcg(p + (long long)j * N);
+    }
+    red[warp][lane] = a;
+    __syncthreads();
+    if (warp == 0 && n < N) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < kRedWarps; ++w) t += red[w][lane];
+        out[(long long)g * N + n] = t;
+    }
 }
 
 // ---------------------------------------------- LN1 backward + mixing transpose
@@ -636,7 +694,7 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
     const __nv_bfloat16* hw = static_cast<const __nv_bfloat16*>(head_w);
     RM_TRY(rm::launch_pdl(rm::head_logit_kernel, dim3((B + 7) / 8), dim3(rm::kThreads), 0, s,
                           (const float*)t->pooled, hw, head_b, labels, t->dlogit, t->lterm, B, D));
-    RM_TRY(rm::launch_pdl(rm::head_grad_kernel, dim3((D + rm::kThreads - 1) / rm::kThreads), dim3(rm::kThreads), 0, s,
+    RM_TRY(rm::launch_pdl(rm::head_grad_kernel, dim3((D + 31) / 32), dim3(32 * rm::kRedWarps), 0, s,
                           (const float*)t->pooled, hw, (const float*)t->dlogit, (const float*)t->lterm, dhead_w,
                           dhead_b, loss, t->gpool, B, D, 1.0f / T));
 
@@ -660,12 +718,11 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
             RM_TRY(rm::launch_pdl(rm::ln2_bwd_kernel<false>, dim3(nsb, T), dim3(lnb_threads), 0, s,
                                   (const __nv_bfloat16*)t->dX, (const float*)nullptr, Yl, (const float2*)t->ystats[l],
                                   P, w.ln2_g, c.ln_eps, dY, t->pg, t->pb, t->pdb, B, T, D, t->SB));
-        const int rthreads = rm::kThreads;
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + rthreads - 1) / rthreads), dim3(rthreads), 0, s,
+        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + 31) / 32, 1), dim3(32 * rm::kRedWarps), 0, s,
                               (const float*)t->pg, gr.ln2_g, 1, T * nsb, D));
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + rthreads - 1) / rthreads), dim3(rthreads), 0, s,
+        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + 31) / 32, 1), dim3(32 * rm::kRedWarps), 0, s,
                               (const float*)t->pb, gr.ln2_b, 1, T * nsb, D));
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((T * D + rthreads - 1) / rthreads), dim3(rthreads), 0, s,
+        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + 31) / 32, T), dim3(32 * rm::kRedWarps), 0, s,
                               (const float*)t->pdb, gr.b2, T, nsb, D));
         // dU = (dY W2_t) * act'(U)
         rm::GroupedGemm gh{};
@@ -691,7 +748,7 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
         RM_TRY(rm::launch_pdl(rm::colsum_kernel, dim3((Hd / 8 + rm::kThreads - 1) / rm::kThreads, nrb_b, T),
                               dim3(rm::kThreads), 0, s, (const __nv_bfloat16*)t->dU, (const __nv_bfloat16*)nullptr,
                               t->pcol, (float*)nullptr, B, Hd, (long long)B * Hd, (long long)Hd, rm::kColRows));
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((T * Hd + rthreads - 1) / rthreads), dim3(rthreads), 0, s,
+        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((Hd + 31) / 32, T), dim3(32 * rm::kRedWarps), 0, s,
                               (const float*)t->pcol, gr.b1, T, nrb_b, Hd));
         // dS = dU W1_t + dY
         rm::GroupedGemm gs{};
@@ -718,9 +775,9 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
                               dim3(rm::kThreads), 0, s, (const __nv_bfloat16*)t->dS,
                               (const __nv_bfloat16*)t->XH1[l], t->pcol, t->pcol2, B * T, D, 0LL, (long long)D,
                               rm::kColRows));
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + rthreads - 1) / rthreads), dim3(rthreads), 0, s,
+        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + 31) / 32, 1), dim3(32 * rm::kRedWarps), 0, s,
                               (const float*)t->pcol2, gr.ln1_g, 1, nrb, D));
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + rthreads - 1) / rthreads), dim3(rthreads), 0, s,
+        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + 31) / 32, 1), dim3(32 * rm::kRedWarps), 0, s,
                               (const float*)t->pcol, gr.ln1_b, 1, nrb, D));
         // LN1 backward and the mixing's transpose: dX (the stack input's gradient for l = 0)
         __nv_bfloat16* dXo = (l == 0 && dX0) ? static_cast<__nv_bfloat16*>(dX0)
