@@ -315,7 +315,9 @@ __device__ __forceinline__ void mixed_vec(const E* xs, int rs, int dh, int h, in
     }
 }
 
-template <typename E, bool PRE, int MV, int NV, bool ADDNORM, int LPR>
+// SAVE (training): also write the normalised rows xhat_out and the rows'
+// 1/sqrt(var + eps) rstd_out, the LN1 backward's inputs.
+template <typename E, bool PRE, int MV, int NV, bool ADDNORM, int LPR, bool SAVE>
 __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
     const E* __restrict__ X, const float* __restrict__ pre_g, const float* __restrict__ pre_b,
     const float2* __restrict__ pstats, int P, const float* __restrict__ g1, const float* __restrict__ b1,
@@ -421,7 +423,7 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
                     const float rstd = rsqrtf(fmaxf(s2 / D - m1 * m1, 0.f) + eps);
                     mean_s[r] = K + m1;
                     rstd_s[r] = rstd;
-                    if (rstd_out) rstd_out[row0 + r] = rstd;
+                    if (SAVE) rstd_out[row0 + r] = rstd;
                 }
             }
             __syncthreads();
@@ -444,7 +446,7 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
                     const float2 r2 = f2(rr), mr2 = f2(-mean_s[r] * rr);
 #pragma unroll
                     for (int j = 0; j < NP; ++j) pm[j] = f2_fma(f2_add(pm[j], pr[j]), r2, mr2);   // xhat
-                    if (xhat_out)   // training: the normalised row, kept for the backward pass
+                    if (SAVE)   // training: the normalised row, kept for the backward pass
                         *reinterpret_cast<uint4*>(xhat_out + (size_t)(row0 + r) * D + c0) = pack_pairs(pm);
 #pragma unroll
                     for (int j = 0; j < NP; ++j) pm[j] = f2_fma(pm[j], g1p[j], b1p[j]);
@@ -633,7 +635,7 @@ inline int mix_groups_cap(int T, int nv, int cap) {
 }
 inline int mix_groups(int T, int nv) { return mix_groups_cap(T, nv, kMixMaxThreads); }
 
-template <typename E, bool PRE, int MV, int NVV, bool ADDNORM, int LPR>
+template <typename E, bool PRE, int MV, int NVV, bool ADDNORM, int LPR, bool SAVE>
 cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps, const float* g1, const float* b1,
                       E* S, int B, int T, int D, float eps, int num_sms, DeviceErr err, uint64_t budget,
                       cudaStream_t s, E* xhat_out, float* rstd_out) {
@@ -648,7 +650,7 @@ cudaError_t mix_ln_go(const E* X, const float* pg, const float* pb, RowStats ps,
     int nslots;
     size_t smem;
     ring_shape(spb * T, rs, sizeof(E), PRE ? ps.P : 0, 2, &nslots, &smem);
-    auto k = mix_ln_kernel<E, PRE, MV, NVV, ADDNORM, LPR>;
+    auto k = mix_ln_kernel<E, PRE, MV, NVV, ADDNORM, LPR, SAVE>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
@@ -671,8 +673,14 @@ template <typename E, bool PRE, int MV>
 cudaError_t mix_ln_nv(int nv, int addnorm, const E* X, const float* pg, const float* pb, RowStats ps,
                       const float* g1, const float* b1, E* S, int B, int T, int D, float eps, int num_sms,
                       DeviceErr err, uint64_t budget, cudaStream_t s, E* xo, float* ro) {
-#define RM_MIX_GO(NVV, AN, LPRV) \
-    mix_ln_go<E, PRE, MV, NVV, AN, LPRV>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, s, xo, ro)
+    // the training outputs exist for bf16 rows of whole 16-byte pieces only
+    constexpr bool kSaveOk = sizeof(E) == 2 && MV == Vec16<E>::N;
+#define RM_MIX_GO(NVV, AN, LPRV)                                                                                    \
+    ((kSaveOk && AN && xo)                                                                                          \
+         ? mix_ln_go<E, PRE, MV, NVV, AN, LPRV, kSaveOk && AN>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, \
+                                                              budget, s, xo, ro)                                   \
+         : mix_ln_go<E, PRE, MV, NVV, AN, LPRV, false>(X, pg, pb, ps, g1, b1, S, B, T, D, eps, num_sms, err, budget, \
+                                                      s, nullptr, nullptr))
     if (!addnorm) return RM_MIX_GO(1, false, 32);
     if (nv <= 64) {
         const int nvl = (nv + 7) / 8;
@@ -771,7 +779,8 @@ cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const fl
                           int num_sms, DeviceErr err, uint64_t budget_ns, cudaStream_t s, void* xhat_out,
                           float* rstd_out) {
     if (pre_g && (!pre_stats.part || pre_stats.P < 1 || pre_stats.P > 32)) return cudaErrorInvalidValue;
-    if ((xhat_out || rstd_out) && !addnorm) return cudaErrorInvalidValue;
+    if ((xhat_out || rstd_out) && (!addnorm || !xhat_out || !rstd_out || dtype != RM_BF16 || (D / T) % 8))
+        return cudaErrorInvalidValue;
     if (dtype == RM_BF16)
         return mix_ln_typed<__nv_bfloat16>(X, pre_g, pre_b, pre_stats, g1, b1, S, B, T, D, eps, addnorm, num_sms,
                                            err, budget_ns, s, xhat_out, rstd_out);

@@ -44,7 +44,7 @@ constexpr int kThreads = 256;
 constexpr int kLnRows = 8;          // rows per block-wide reduction in the LayerNorm backward
 constexpr int kMaxSampleBlock = 64; // samples per CTA of the LayerNorm backward
 constexpr int kColRows = 16;        // rows per partial of the column sums
-constexpr int kRedWarps = 8;        // sample / slice warps of the ordered column reductions
+constexpr int kRedWarps = 32;       // sample / slice warps of the ordered column reductions
 
 __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -100,8 +100,8 @@ __global__ void __launch_bounds__(kThreads) head_logit_kernel(const float* poole
 
 // dw[n] = sum_b dlogit_b pooled[b, n] and gpool[b, n] = dlogit_b w[n] / T,
 // the gradient of every token row of the last block's output.  CTA = 32
-// columns; warp w takes samples b = w, w + 8, ... in ascending order and the
-// eight warp sums are added in warp order.  One thread adds up the loss and
+// columns; warp w takes samples b = w, w + kRedWarps, ... in ascending order
+// and the warp sums are added in warp order.  One thread adds up the loss and
 // dc in ascending b.
 __global__ void __launch_bounds__(32 * kRedWarps) head_grad_kernel(const float* pooled,
                                                                   const __nv_bfloat16* __restrict__ w,
@@ -302,8 +302,8 @@ __global__ void __launch_bounds__(kThreads) colsum_kernel(const __nv_bfloat16* A
 }
 
 // out[g * N + n] = sum_{j < J} part[(g * J + j) * N + n].  CTA = (32
-// columns, group g); warp w sums the slices j = w, w + 8, ... of its lane's
-// column in ascending j, then one warp adds the eight warp sums in warp order
+// columns, group g); warp w sums the slices j = w, w + kRedWarps, ... of its
+// lane's column in ascending j, then one warp adds the warp sums in warp order
 // (a fixed order: deterministic).
 __global__ void __launch_bounds__(32 * kRedWarps) reduce_parts_kernel(const float* part, float* out, int G, int J,
                                                                       int N) {
@@ -337,17 +337,18 @@ __global__ void __launch_bounds__(32 * kRedWarps) reduce_parts_kernel(const floa
 }
 
 // ---------------------------------------------- LN1 backward + mixing transpose
-// Per sample (persistent CTAs): stage dS [T, D] (rows padded for the mixing
-// gather) and xhat1 [T, D]; one warp per row computes
+// Per sample (persistent CTAs, two per SM): one warp per row h reads the
+// row's dS and xhat1 from global memory and computes
 //     dZ = rstd1 * (g1*dS - mean(g1*dS) - xhat1 * mean(g1*dS*xhat1))
-// and writes it over the row's dS in shared memory; then
+// into shared memory (rows padded for the mixing gather); then
 //     dX[t] = dZ[t] + TokenMixing(dZ)[t]
-// leaves through the same gather the forward mixing uses (thread = row group
-// x 16-byte column vector).
-constexpr int kBwdMixThreads = 512;
+// leaves through the same 16-byte gather as the forward mixing (thread =
+// row group x 16-byte column vector).  Only dZ is staged, since every other
+// input is row-local.
+constexpr int kBwdMixThreads = 256;
 
 template <int NV>
-__global__ void __launch_bounds__(kBwdMixThreads, 1) ln1_bwd_mix_kernel(const __nv_bfloat16* dS,
+__global__ void __launch_bounds__(kBwdMixThreads, 2) ln1_bwd_mix_kernel(const __nv_bfloat16* dS,
                                                                        const __nv_bfloat16* xhat, const float* rstd1,
                                                                        const float* __restrict__ gamma,
                                                                        __nv_bfloat16* dX, int B, int T, int D, int rs,
@@ -355,20 +356,9 @@ __global__ void __launch_bounds__(kBwdMixThreads, 1) ln1_bwd_mix_kernel(const __
                                                                        uint64_t budget_ns) {
     pdl_enter();
     extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ __align__(8) uint64_t bar;
-    __shared__ int abort_flag, s_ok;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const int TD = T * D, dh = D / T, nv = D / 8;
-    const uint32_t ds_a = smem_u32(smem);                                       // [T][rs] bf16
-    const uint32_t xh_a = ds_a + (uint32_t)(((size_t)T * rs * 2 + 127) / 128 * 128);   // [T][D] bf16
-    const uint32_t bar_a = smem_u32(&bar);
-    const WaitCtx wc{&abort_flag, budget_ns, err};
-    if (tid == 0) {
-        mbar_init(bar_a, 1);
-        abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
+    const uint32_t dz_a = smem_u32(smem);   // [T][rs] bf16
     const float invD = 1.0f / (float)D;
     // element pass layout: thread (grp, v) over rows grp, grp + groups, ...
     const int grp = tid / nv, c0 = (tid - grp * nv) * 8;
@@ -376,46 +366,33 @@ __global__ void __launch_bounds__(kBwdMixThreads, 1) ln1_bwd_mix_kernel(const __
     // source of the mixed vector at column c0 of output row h: token t = c0 / dh,
     // element t*rs + h*dh + (c0 - t*dh) of the staged sample (16-byte pieces: dh % 8 == 0)
     const int msrc = (c0 / dh) * (rs - dh) + c0;
-    uint32_t parity = 0;
     for (int b = blockIdx.x; b < B; b += gridDim.x) {
-        if (warp == 0) {
-            if (lane == 0) mbar_arrive_expect_tx(bar_a, (uint32_t)(2 * TD * 2));
-            __syncwarp();
-            fence_proxy_async_shared();
-            const __nv_bfloat16* src = dS + (size_t)b * TD;
-            for (int r = lane; r < T; r += 32)
-                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                                 ds_a + (uint32_t)(r * rs * 2)),
-                             "l"(src + (size_t)r * D), "r"((uint32_t)(D * 2)), "r"(bar_a)
-                             : "memory");
-            if (lane == 0)
-                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                                 xh_a),
-                             "l"(xhat + (size_t)b * TD), "r"((uint32_t)(TD * 2)), "r"(bar_a)
-                             : "memory");
-        }
-        if (tid == 0) s_ok = mbar_wait(bar_a, parity, wc, SITE_TRAIN_MIX, false);
-        __syncthreads();
-        if (!s_ok) break;
-        parity ^= 1u;
-        // dZ of each row, in place
+        const __nv_bfloat16* dsb = dS + (size_t)b * TD;
+        const __nv_bfloat16* xhb = xhat + (size_t)b * TD;
         for (int h = warp; h < T; h += nw) {
+            uint4 du[NV], xu[NV];
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {   // every load of the row in flight at once
+                const int v = lane + 32 * i;
+                if (v < nv) {
+                    du[i] = __ldcg(reinterpret_cast<const uint4*>(dsb + (size_t)h * D) + v);
+                    xu[i] = __ldcg(reinterpret_cast<const uint4*>(xhb + (size_t)h * D) + v);
+                }
+            }
             const float r = __ldcg(rstd1 + (long long)b * T + h);
-            float gx[NV][8], xv[NV][8];
             float s1 = 0.f, s2 = 0.f;
 #pragma unroll
             for (int i = 0; i < NV; ++i) {
-                const int v = lane + 32 * i;
-                if (v < nv) {
-                    float d[8], g[8];
-                    unpack8(lds128(ds_a + (uint32_t)((h * rs + 8 * v) * 2)), d);
-                    unpack8(lds128(xh_a + (uint32_t)((h * D + 8 * v) * 2)), xv[i]);
-                    load8_param(gamma + 8 * v, g);
+                if (lane + 32 * i < nv) {
+                    float d[8], x[8], g[8];
+                    unpack8(du[i], d);
+                    unpack8(xu[i], x);
+                    load8_param(gamma + 8 * (lane + 32 * i), g);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        gx[i][e] = d[e] * g[e];
-                        s1 += gx[i][e];
-                        s2 = fmaf(gx[i][e], xv[i][e], s2);
+                        const float gx = d[e] * g[e];
+                        s1 += gx;
+                        s2 = fmaf(gx, x[e], s2);
                     }
                 }
             }
@@ -425,10 +402,13 @@ __global__ void __launch_bounds__(kBwdMixThreads, 1) ln1_bwd_mix_kernel(const __
             for (int i = 0; i < NV; ++i) {
                 const int v = lane + 32 * i;
                 if (v < nv) {
-                    float dz[8];
+                    float d[8], x[8], g[8], dz[8];
+                    unpack8(du[i], d);
+                    unpack8(xu[i], x);
+                    load8_param(gamma + 8 * v, g);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) dz[e] = r * (gx[i][e] - s1 - xv[i][e] * s2);
-                    sts128(ds_a + (uint32_t)((h * rs + 8 * v) * 2), pack8(dz));
+                    for (int e = 0; e < 8; ++e) dz[e] = r * (d[e] * g[e] - s1 - x[e] * s2);
+                    sts128(dz_a + (uint32_t)((h * rs + 8 * v) * 2), pack8(dz));
                 }
             }
         }
@@ -437,15 +417,17 @@ __global__ void __launch_bounds__(kBwdMixThreads, 1) ln1_bwd_mix_kernel(const __
             __nv_bfloat16* out = dX + (size_t)b * TD;
             for (int r = grp; r < T; r += groups) {
                 float a[8], m[8];
-                unpack8(lds128(ds_a + (uint32_t)((r * rs + c0) * 2)), a);
-                unpack8(lds128(ds_a + (uint32_t)((msrc + r * dh) * 2)), m);
+                unpack8(lds128(dz_a + (uint32_t)((r * rs + c0) * 2)), a);
+                unpack8(lds128(dz_a + (uint32_t)((msrc + r * dh) * 2)), m);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) a[e] += m[e];
                 *reinterpret_cast<uint4*>(out + (size_t)r * D + c0) = pack8(a);
             }
         }
-        __syncthreads();   // the staged sample is free again
+        __syncthreads();   // the staged dZ is free again
     }
+    (void)err;
+    (void)budget_ns;
 }
 
 int mix_pad_stride(int D, int dh) {
@@ -457,7 +439,8 @@ int mix_pad_stride(int D, int dh) {
 }
 
 size_t ln1_bwd_smem(int T, int D, int rs) {
-    return ((size_t)T * rs * 2 + 127) / 128 * 128 + (size_t)T * D * 2;
+    (void)D;
+    return ((size_t)T * rs * 2 + 127) / 128 * 128;
 }
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -794,7 +777,7 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
         auto go = [&](auto kern) -> cudaError_t {
             cudaError_t ee = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (ee != cudaSuccess) return ee;
-            const int grid = std::min(B, t->num_sms);
+            const int grid = std::min(B, 2 * t->num_sms);
             return rm::launch_pdl(kern, dim3(grid), dim3(rm::kBwdMixThreads), smem, s, (const __nv_bfloat16*)t->dS,
                                   (const __nv_bfloat16*)t->XH1[l], (const float*)t->RS1[l], w.ln1_g, dXo, B, T, D, rs,
                                   groups, err, budget);
