@@ -162,7 +162,6 @@ def code_digest(path: str) -> str:
 # committed ncu summaries per kernel family: (summary file pattern, kernel source)
 PROFILE_SOURCES = {
     "gemm_tc": ("ncu_gemm_tc_{workload}.md", "rm_gemm_tc.cu"),
-    "ffn_fused": ("ncu_ffn_fused_{workload}.md", "rm_ffn_fused.cu"),
 }
 
 
@@ -199,7 +198,7 @@ def top_kernel_roofline(wl, top: str, ms_avg: float, active, peaks: dict, peak_s
     the HBM peak only."""
     timing = ("CUDA events around each launch on its stream, over a second timed region of "
               "the same K steps (about 6 us of event overhead per launch included)")
-    if top not in ("gemm1", "gemm2", "ffn_fused"):
+    if top not in ("gemm1", "gemm2"):
         active_mean = sum(active) / len(active) if active else None
         what, n = roofline.kernel_work(wl, top, active_mean)
         achieved = n / (ms_avg / 1e3) / 1e9
@@ -210,8 +209,6 @@ def top_kernel_roofline(wl, top: str, ms_avg: float, active, peaks: dict, peak_s
         per_launch = 2.0 * sum(active) * wl.D * wl.hidden / wl.L
     else:
         per_launch = 2.0 * wl.B * wl.T * wl.D * wl.hidden
-    if top == "ffn_fused":
-        per_launch *= 2.0   # both projections in one launch
     achieved = per_launch / (ms_avg / 1e3) / 1e12
     if wl.dtype == "f32":
         peak = num_sms * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
@@ -224,8 +221,8 @@ def top_kernel_roofline(wl, top: str, ms_avg: float, active, peaks: dict, peak_s
     # given beside it
     peak = peaks["bf16_tflops"]
     sustained = peaks.get("bf16_tflops_sustained")
-    family = "ffn_fused" if top == "ffn_fused" else "gemm_tc"
-    return {"kernel": f"{family} ({top})" if family == "gemm_tc" else family, "bound": "tensor",
+    family = "gemm_tc"
+    return {"kernel": f"{family} ({top})", "bound": "tensor",
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": traffic_from_profiles(family, wl.name, top, root),
             "peak_source": f"bf16 dense burst, of {peak_src}",

@@ -117,11 +117,7 @@ rm_status rm_layernorm(rm_handle *h, const void *A, const void *R, const float *
  *     V[b, t] = W2_t GELU(W1_t S[b, t] + b1_t) + b2_t
  * S, V [B, T, D]; uses w->W1, b1, W2, b2.  No residual, no LayerNorm.
  * bf16 runs two grouped tcgen05 GEMMs (the hidden [T, B, hidden] in the
- * handle's workspace).  With the environment variable RM_FFN_FUSED=1 and
- * D % 64 == 0, D <= 320, hidden % 128 == 0, one kernel computes both
- * projections with the hidden activation kept on chip instead; its outputs
- * are bit-identical (it is slower on B200 today, hence off by default).
- * Blocks and stacks use the same choice. */
+ * handle's workspace). */
 rm_status rm_pffn_forward(rm_handle *h, const rm_block_weights *w, const void *S, void *V,
                           int B, rm_stream_t stream);
 
@@ -219,9 +215,8 @@ rm_status rm_selftest_wait_timeout(rm_handle *h, rm_stream_t stream);
  * library holds until the process exits; the caller passes inputs and outputs
  * only, and the call allocates nothing.
  *   - Returns RM_ERR_INVALID_ARG, before launching anything, if
- *     T * B * hidden * sizeof(element) > RM_STATIC_SCRATCH_BYTES - 256,
- *     unless the fused kernel runs (RM_FFN_FUSED=1, see rm_pffn_forward),
- *     which keeps the hidden activations on chip.
+ *     T * B * hidden * sizeof(element) > RM_STATIC_SCRATCH_BYTES - 256, and
+ *     RM_ERR_UNSUPPORTED if T > 64.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.
@@ -297,8 +292,7 @@ typedef enum {
     RM_K_MOE_COMBINE = 8,
     RM_K_PADSPLIT = 9,
     RM_K_HEAD = 10,
-    RM_K_FFN_FUSED = 11,  /* both FFN projections in one kernel (narrow tokens)      */
-    RM_K_COUNT = 12
+    RM_K_COUNT = 11
 } rm_kernel_kind;
 
 /* Start recording a CUDA event pair around each kernel launch made through h

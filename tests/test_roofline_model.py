@@ -105,14 +105,10 @@ def test_top_kernel_roofline_tensor_traffic_per_workload(tmp_path):
     assert bench.top_kernel_roofline(wl, "gemm1", 0.08, None, PEAKS, "m", 148, 1965.0, root3)["traffic"] is None
 
 
-def test_top_kernel_roofline_fused_and_alu_and_hbm(tmp_path):
+def test_top_kernel_roofline_alu_and_hbm(tmp_path):
     import bench
     wl = synth.WORKLOADS["padsplit"]
-    root = _fake_tree(tmp_path, "padsplit", "ncu_ffn_fused_{workload}.md", "rm_ffn_fused.cu",
-                      bytes_line="ffn_fused = 777")
-    r = bench.top_kernel_roofline(wl, "ffn_fused", 0.17, None, PEAKS, "measured", 148, 1965.0, root)
-    assert r["flops_per_launch"] == 4.0 * wl.B * wl.T * wl.D * wl.hidden   # both projections
-    assert r["traffic"] == 777.0 and r["bound"] == "tensor"
+    root = _fake_tree(tmp_path, "padsplit", "ncu_gemm_tc_{workload}.md", "rm_gemm_tc.cu")
     # the fp32 path runs on CUDA cores: FFMA peak of 148 SMs x 128 lanes x 2 x 1965 MHz
     tiny = synth.WORKLOADS["tiny_f32"]
     a = bench.top_kernel_roofline(tiny, "gemm2", 0.01, None, PEAKS, "measured", 148, 1965.0, root)
@@ -140,13 +136,13 @@ def test_per_kernel_rooflines_cover_every_kernel(name):
     FFN contractions)."""
     import bench
     wl = synth.WORKLOADS[name]
-    kinds = KERNELS_BY_WORKLOAD[name] + (["ffn_fused"] if name == "padsplit" else [])
+    kinds = KERNELS_BY_WORKLOAD[name]
     kern = {k: {"ms_avg": 0.05, "launches": 2, "share": 0.1} for k in kinds}
     active = [wl.B * wl.T * 2, wl.B * wl.T * 2] if wl.n_experts else None
     out = bench.per_kernel_rooflines(wl, kern, active, PEAKS, 148, 1965.0)
     for k, e in out.items():
         assert e["frac"] > 0 and e["achieved"] > 0, k
-        if k in ("gemm1", "gemm2", "ffn_fused"):
+        if k in ("gemm1", "gemm2"):
             assert e["unit"] == "TFLOP/s" and e["bound"] == ("alu" if wl.dtype == "f32" else "tensor")
         else:
             assert e["unit"] == "GB/s" and e["bound"] == "hbm"
@@ -163,6 +159,5 @@ def test_kernel_work_figures():
     ps = synth.WORKLOADS["padsplit"]
     assert roofline.kernel_work(ps, "padsplit") == ("bytes", 4096 * 4800 * 2 + 4096 * 16 * 320 * 2)
     assert roofline.kernel_work(ps, "gemm1") == ("flops", 2.0 * 4096 * 16 * 320 * 1280)
-    assert roofline.kernel_work(ps, "ffn_fused") == ("flops", 4.0 * 4096 * 16 * 320 * 1280)
     with pytest.raises(KeyError):
         roofline.kernel_work(ps, "no_such_kernel")

@@ -66,25 +66,3 @@ def test_static_scratch_rejects_oversize():
     with pytest.raises(rm.RankMixerError) as e:
         rm.rm_pffn_forward_static(blk, S, torch.empty_like(S), 2 ** 31 - 1, T, D, 2 ** 31 - 16)
     assert e.value.status == rm.RM_ERR_INVALID_ARG
-
-
-def test_static_scratch_fused_ffn(monkeypatch):
-    """With RM_FFN_FUSED=1 the static entry point runs the fused kernel like
-    rm_pffn_forward (identical outputs) and needs no scratch for the hidden
-    activations: a batch whose hidden would not fit the array is accepted."""
-    from token_mixing_feature_b200 import rankmixer as rm
-    monkeypatch.setenv("RM_FFN_FUSED", "1")
-    T, D, hidden = 16, 320, 1280
-    B = rm.RM_STATIC_SCRATCH_BYTES // (T * hidden * 2) + 1     # H would not fit: 16.0 MB + one sample
-    blk = {k: dev(v) for k, v in synth.random_like_block(T, D, hidden, "bf16", seed=81).items()}
-    S = dev(synth.random_activations((B, T, D), "bf16", seed=82))
-    ref = torch.empty_like(S)
-    with rm.rm_create(B, T, D, hidden, 1, 0, "bf16") as h:
-        rm.rm_pffn_forward(h, blk, S, ref, B)
-        assert rm.rm_sync_status(h) == rm.RM_OK
-    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
-    V = torch.full_like(S, float("nan"))
-    rm.rm_pffn_forward_static(blk, S, V, B, T, D, hidden, "bf16", "tanh", status)
-    torch.cuda.synchronize()
-    assert int(status.item()) == rm.RM_OK
-    assert torch.equal(V, ref)

@@ -163,33 +163,6 @@ rm_status run_pffn(rm_handle* h, const rm_block_weights* w, const void* S, void*
     if (stats_done) *stats_done = gemm_stats;
 
     cudaError_t e;
-    if (c.dtype == RM_BF16 && rm::ffn_fused_preferred(c.T, B, c.D, c.hidden, h->num_sms)) {
-        // narrow tokens: both projections in one kernel, the hidden stays on chip
-        rm::FusedFfn f{};
-        f.G = c.T;
-        f.M = B;
-        f.D = c.D;
-        f.hidden = c.hidden;
-        f.epi = g1.epi;
-        f.A = S;
-        f.a_gstride = g1.a_gstride;
-        f.a_ld = g1.a_ld;
-        f.W1 = w->W1;
-        f.b1 = g1.bias;
-        f.W2 = w->W2;
-        f.b2 = g2.bias;
-        f.out = V;
-        f.o_gstride = g2.o_gstride;
-        f.o_ld = g2.o_ld;
-        f.resid = resid;
-        f.r_gstride = g2.r_gstride;
-        f.r_ld = g2.r_ld;
-        f.stats = g2.stats;
-        f.s_gstride = g2.s_gstride;
-        f.s_ld = g2.s_ld;
-        ProfScope ps(h, RM_K_FFN_FUSED, s);
-        return cuda_status(rm::launch_ffn_fused(f, derr(h), h->budget_ns, h->num_sms, s));
-    }
     {
         ProfScope ps(h, RM_K_GEMM1, s);
         e = c.dtype == RM_BF16 ? rm::launch_gemm_tc(g1, derr(h), h->budget_ns, h->num_sms, s)
@@ -686,8 +659,7 @@ rm_status rm_profile_end(rm_handle* h, float* ms_by_kind, int* launches_by_kind,
 
 const char* rm_kernel_name(int kind) {
     static const char* names[RM_K_COUNT] = {"mix_ln", "gemm1", "gemm2", "ln_pool", "layernorm", "token_mix",
-                                            "moe_route", "moe_gather", "moe_combine", "padsplit", "head",
-                                            "ffn_fused"};
+                                            "moe_route", "moe_gather", "moe_combine", "padsplit", "head"};
     return kind >= 0 && kind < RM_K_COUNT ? names[kind] : "unknown";
 }
 

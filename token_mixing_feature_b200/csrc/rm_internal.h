@@ -141,33 +141,6 @@ cudaError_t launch_gemm_tc(const GroupedGemm& p, DeviceErr err, uint64_t budget_
                            cudaStream_t s);
 cudaError_t launch_gemm_simt(const GroupedGemm& p, cudaStream_t s);   // fp32, CUDA cores
 
-// ---- fused per-token FFN for narrow tokens (rm_ffn_fused.cu) -------------
-// out[g, m, :] = act(A[g, m, :] W1_g^T + b1_g) W2_g^T + b2_g (+ resid), with
-// the hidden activation rounded to bf16 as the two-GEMM path stores it, but
-// never written to memory; optional LayerNorm partials as GroupedGemm::stats.
-struct FusedFfn {
-    int G, M, D, hidden;
-    int epi;                  // EPI_GELU_TANH, EPI_GELU_ERF or EPI_RELU
-    const void* A;            // element (g, m, k) at A + g*a_gstride + m*a_ld + k, a_gstride <= a_ld
-    long long a_gstride, a_ld;
-    const void* W1;           // [G][hidden][D]
-    const float* b1;          // [G][hidden]
-    const void* W2;           // [G][D][hidden]
-    const float* b2;          // [G][D]
-    void* out;
-    long long o_gstride, o_ld;
-    const void* resid;        // may be null
-    long long r_gstride, r_ld;
-    float2* stats;            // may be null
-    long long s_gstride, s_ld;
-};
-// Shapes the fused kernel handles: D % 64 == 0, 64 <= D <= 320, hidden % 128 == 0.
-bool ffn_fused_supported(int D, int hidden);
-// Whether run_pffn uses the fused kernel: only when supported and asked for
-// with RM_FFN_FUSED=1 (the two grouped GEMMs are faster on B200 today).
-bool ffn_fused_preferred(int G, int M, int D, int hidden, int num_sms);
-cudaError_t launch_ffn_fused(const FusedFfn& f, DeviceErr err, uint64_t budget_ns, int num_sms, cudaStream_t s);
-
 // ---- sparse MoE routing (rm_moe.cu) ----------------------------------------
 struct MoeWork {
     float* gates;          // [B, T, Ne]

@@ -468,102 +468,100 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
 }
 
 // pooled[b, c] = gamma[c] * (1/T) sum_t (x[t, c] - m_t) r_t + beta[c]; Xout
-// (optional) receives LN(x).  Persistent CTAs stream chunks of spb whole
-// samples, with their partial statistics, through the shared-memory ring.
-// After the chunk's row statistics are merged, thread u takes (sample
-// u / nv, 16-byte column vector u % nv) and sums that column over the
-// sample's T rows in ascending t (deterministic), so no partial sums cross
-// threads.
-constexpr int kPoolThreads = 384;
-constexpr size_t kMaxSmemPerCta = 227 * 1024;
+// (optional) receives LN(x).  CTA = spc samples: its rows' statistics are
+// merged from the producer's partials (one warp per row) into shared memory;
+// then thread u takes (sample u / nv, 16-byte column vector u % nv) and sums
+// that column over the sample's T rows in ascending t (deterministic), with
+// eight rows' loads in flight at a time straight from global memory (no
+// staging: each element is read once, and many small CTAs keep enough loads
+// in flight to cover the memory latency).
+constexpr int kPoolThreads = 256;
+constexpr int kPoolRowsInFlight = 8;
 
 template <typename E>
-__global__ void __launch_bounds__(kPoolThreads, 2) ln_pool_kernel(const E* __restrict__ X,
-                                                                 const float2* __restrict__ pstats, int P,
-                                                                 const float* __restrict__ g,
-                                                                 const float* __restrict__ bta,
-                                                                 float* __restrict__ pooled, E* __restrict__ Xout,
-                                                                 int B, int T, int D, float eps, int spb, int nslots,
-                                                                 DeviceErr err, uint64_t budget_ns) {
+__global__ void __launch_bounds__(kPoolThreads, 3) ln_pool_kernel(const E* X, const float2* pstats, int P,
+                                                              const float* __restrict__ g,
+                                                              const float* __restrict__ bta, float* __restrict__ pooled,
+                                                              E* __restrict__ Xout, int B, int T, int D, float eps,
+                                                              int spc) {
     pdl_enter();
     constexpr int V = Vec16<E>::N;
-    extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ int abort_flag, s_ok;
-    const int TD = T * D;
-    const int nchunks = (B + spb - 1) / spb;
-    float *mean_s, *rstd_s;
-    SampleRing<E> ring;
-    make_ring<E>(ring, smem, spb * T, D, D, nslots, pstats, P, mean_s, rstd_s);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const WaitCtx wc{&abort_flag, budget_ns, err};
-    if (tid == 0) {
-        for (int k = 0; k < nslots; ++k) mbar_init(ring.bar(k), 1);
-        abort_flag = 0;
-        fence_mbar_init();
+    constexpr int NP = V / 2;
+    extern __shared__ float rowstat[];   // mean [spc * T], rstd [spc * T]
+    float* mean_s = rowstat;
+    float* rstd_s = rowstat + spc * T;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const long long b0 = (long long)blockIdx.x * spc;
+    const int ns = (int)min((long long)spc, B - b0);
+    const int R = ns * T;
+    const float n = (float)D / (float)P;
+    for (int r = warp; r < R; r += 8 * nw) {   // eight rows' partials in flight per warp
+        float2 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int rr = r + k * nw;
+            v[k] = (rr < R && lane < P) ? __ldcg(pstats + (b0 * T + rr) * P + lane) : make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int rr = r + k * nw;
+            if (rr < R) {   // warp-uniform
+                const float mean = warp_sum(v[k].x) / (float)P;
+                const float d = v[k].x - mean;
+                const float q = warp_sum(lane < P ? fmaf(n * d, d, v[k].y) : 0.f);
+                if (lane == 0) {
+                    mean_s[rr] = mean;
+                    rstd_s[rr] = rsqrtf(q / D + eps);
+                }
+            }
+        }
     }
     __syncthreads();
-    auto chunk_samples = [&](long long c) { return (int)min((long long)spb, B - c * spb); };
-    if (warp == 0)
-        for (int k = 0; k < nslots; ++k) {
-            const long long ck = blockIdx.x + (long long)k * gridDim.x;
-            if (ck < nchunks) ring.issue(k, X + (size_t)ck * spb * TD, chunk_samples(ck) * T, ck * spb * T);
-        }
     const int nv = D / V;
     const float invT = 1.0f / T;
-    constexpr int NP = V / 2;
-    int it = 0;
-    for (long long c = blockIdx.x; c < nchunks; c += gridDim.x, ++it) {
-        const int cur = it % nslots;
-        const int ns = chunk_samples(c);
-        const int R = ns * T;
-        const long long row0 = c * spb * T;
-        if (tid == 0) s_ok = ring.wait(cur, wc, SITE_LN_POOL);
-        __syncthreads();
-        if (!s_ok) break;
-        chunk_stats(ring.stats(cur, row0), P, D, R, eps, mean_s, rstd_s);
-        __syncthreads();
-        const E* xs = ring.buf(cur);
-        for (int u = tid; u < ns * nv; u += blockDim.x) {
-            const int sm = u / nv, c0 = (u - sm * nv) * V;
-            float2 gp[NP], bp[NP];
-            load_pairs(g + c0, gp);
-            load_pairs(bta + c0, bp);
-            float2 acc[NP];
+    for (int u = tid; u < ns * nv; u += blockDim.x) {
+        const int sm = u / nv, c0 = (u - sm * nv) * V;
+        const E* col = X + (size_t)(b0 + sm) * T * D + c0;
+        float2 gp[NP], bp[NP];
+        load_pairs(g + c0, gp);
+        load_pairs(bta + c0, bp);
+        float2 acc[NP];
 #pragma unroll
-            for (int j = 0; j < NP; ++j) acc[j] = f2(0.f);
-            const uint32_t col_a = smem_u32(xs) + (uint32_t)((sm * TD + c0) * (int)sizeof(E));
-            const uint32_t mean_a = smem_u32(mean_s) + 4u * (uint32_t)(sm * T), rstd_a = smem_u32(rstd_s) + 4u * (uint32_t)(sm * T);
-#pragma unroll 4
-            for (int t = 0; t < T; ++t) {
-                const int r = sm * T + t;
-                float2 x[NP];
-                unpack_pairs(lds128(col_a + (uint32_t)(t * D * (int)sizeof(E))), x);
-                const float rt = lds_f32(rstd_a + 4u * (uint32_t)t);
-                const float2 r2 = f2(rt), mr2 = f2(-lds_f32(mean_a + 4u * (uint32_t)t) * rt);
+        for (int j = 0; j < NP; ++j) acc[j] = f2(0.f);
+        for (int t0 = 0; t0 < T; t0 += kPoolRowsInFlight) {
+            uint4 xv[kPoolRowsInFlight];
 #pragma unroll
-                for (int j = 0; j < NP; ++j) {
-                    x[j] = f2_fma(x[j], r2, mr2);   // (x - m_t) r_t
-                    acc[j] = f2_add(acc[j], x[j]);
+            for (int k = 0; k < kPoolRowsInFlight; ++k)
+                if (t0 + k < T) xv[k] = __ldcg(reinterpret_cast<const uint4*>(col + (size_t)(t0 + k) * D));
+#pragma unroll
+            for (int k = 0; k < kPoolRowsInFlight; ++k) {
+                const int t = t0 + k;
+                if (t < T) {
+                    float2 x[NP];
+                    unpack_pairs(xv[k], x);
+                    const float rt = rstd_s[sm * T + t];
+                    const float2 r2 = f2(rt), mr2 = f2(-mean_s[sm * T + t] * rt);
+#pragma unroll
+                    for (int j = 0; j < NP; ++j) {
+                        x[j] = f2_fma(x[j], r2, mr2);   // (x - m_t) r_t
+                        acc[j] = f2_add(acc[j], x[j]);
+                    }
+                    if (Xout) {
+#pragma unroll
+                        for (int j = 0; j < NP; ++j) x[j] = f2_fma(x[j], gp[j], bp[j]);
+                        *reinterpret_cast<uint4*>(Xout + ((size_t)(b0 + sm) * T + t) * D + c0) = pack_pairs(x);
+                    }
                 }
-                if (Xout) {
-#pragma unroll
-                    for (int j = 0; j < NP; ++j) x[j] = f2_fma(x[j], gp[j], bp[j]);
-                    *reinterpret_cast<uint4*>(Xout + (size_t)(row0 + r) * D + c0) = pack_pairs(x);
-                }
-            }
-            float4* dst = reinterpret_cast<float4*>(pooled + (size_t)(c * spb + sm) * D + c0);
-#pragma unroll
-            for (int q = 0; q < NP / 2; ++q) {
-                const float2 p0 = f2_fma(gp[2 * q], f2_mul(acc[2 * q], f2(invT)), bp[2 * q]);
-                const float2 p1 = f2_fma(gp[2 * q + 1], f2_mul(acc[2 * q + 1], f2(invT)), bp[2 * q + 1]);
-                dst[q] = make_float4(p0.x, p0.y, p1.x, p1.y);
             }
         }
-        __syncthreads();   // the slot and the statistics are free again
-        const long long nc = c + (long long)nslots * gridDim.x;
-        if (warp == 0 && nc < nchunks) ring.issue(cur, X + (size_t)nc * spb * TD, chunk_samples(nc) * T, nc * spb * T);
+        float4* dst = reinterpret_cast<float4*>(pooled + (size_t)(b0 + sm) * D + c0);
+#pragma unroll
+        for (int q = 0; q < NP / 2; ++q) {
+            const float2 p0 = f2_fma(gp[2 * q], f2_mul(acc[2 * q], f2(invT)), bp[2 * q]);
+            const float2 p1 = f2_fma(gp[2 * q + 1], f2_mul(acc[2 * q + 1], f2(invT)), bp[2 * q + 1]);
+            dst[q] = make_float4(p0.x, p0.y, p1.x, p1.y);
+        }
     }
-    if (tid == 0) ring.drain(wc, SITE_LN_POOL);
 }
 
 // (mean, M2) of every row over all D columns (P = 1), one warp per row, one
@@ -728,31 +726,18 @@ cudaError_t mix_ln_typed(const void* X, const float* pg, const float* pb, RowSta
 
 template <typename E>
 cudaError_t ln_pool_go(const void* X, RowStats stats, const float* g, const float* b, float* pooled, void* Xout, int B,
-                       int T, int D, float eps, int num_sms, DeviceErr err, uint64_t budget, cudaStream_t s) {
+                       int T, int D, float eps, cudaStream_t s) {
     constexpr int V = Vec16<E>::N;
     const int nv = D / V;
     if (nv < 1 || nv > kPoolThreads) return cudaErrorInvalidValue;
-    const int spb = samples_per_chunk(T, D, sizeof(E), B);
-    int threads = (int)std::min<long long>(kPoolThreads, ((long long)spb * nv + 31) / 32 * 32);
-    if (threads < 64) threads = 64;
-    int nslots;
-    size_t smem;
-    ring_shape(spb * T, D, sizeof(E), stats.P, 2, &nslots, &smem);
-    if (smem > kMaxSmemPerCta - 1024) return cudaErrorInvalidValue;
-    auto k = ln_pool_kernel<E>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    const long long nchunks = (B + spb - 1) / spb;
-    const long long gr = (long long)num_sms * per_sm;
-    const int grid = (int)(gr < nchunks ? gr : nchunks);
-    return launch_pdl(k, grid, threads, smem, s, static_cast<const E*>(X), stats.part, stats.P, g, b, pooled,
-                      static_cast<E*>(Xout), B, T, D, eps, spb, nslots, err, budget);
+    int spc = kPoolThreads / nv;   // samples per CTA
+    if (spc > B) spc = B;
+    if (spc < 1) spc = 1;
+    const int threads = std::max(64, (spc * nv + 31) / 32 * 32);
+    const size_t smem = sizeof(float) * 2 * (size_t)spc * T;
+    const int grid = (B + spc - 1) / spc;
+    return launch_pdl(ln_pool_kernel<E>, grid, threads, smem, s, static_cast<const E*>(X), stats.part, stats.P, g,
+                      b, pooled, static_cast<E*>(Xout), B, T, D, eps, spc);
 }
 
 }  // namespace
@@ -791,10 +776,13 @@ cudaError_t launch_mix_ln(int dtype, const void* X, const float* pre_g, const fl
 cudaError_t launch_ln_pool(int dtype, const void* X, RowStats stats, const float* g, const float* b, float* pooled,
                            void* Xout, int B, int T, int D, float eps, int num_sms, DeviceErr err, uint64_t budget_ns,
                            cudaStream_t s) {
+    (void)num_sms;   // (a grid of ceil(B / samples per CTA) small CTAs; no waits)
+    (void)err;
+    (void)budget_ns;
     if (!stats.part || stats.P < 1 || stats.P > 32) return cudaErrorInvalidValue;
     if (dtype == RM_BF16)
-        return ln_pool_go<__nv_bfloat16>(X, stats, g, b, pooled, Xout, B, T, D, eps, num_sms, err, budget_ns, s);
-    return ln_pool_go<float>(X, stats, g, b, pooled, Xout, B, T, D, eps, num_sms, err, budget_ns, s);
+        return ln_pool_go<__nv_bfloat16>(X, stats, g, b, pooled, Xout, B, T, D, eps, s);
+    return ln_pool_go<float>(X, stats, g, b, pooled, Xout, B, T, D, eps, s);
 }
 
 cudaError_t launch_row_stats(int dtype, const void* X, float2* out, long long rows, int D, cudaStream_t s) {

@@ -66,15 +66,12 @@ extern "C" rm_status rm_pffn_forward_static(const rm_block_weights* w, const voi
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return RM_ERR_CUDA;
-    // The same kernel choice as rm_pffn_forward; the fused kernel keeps the
-    // hidden activations on chip and needs no scratch for them.
-    const bool fused = dtype == RM_BF16 && rm::ffn_fused_preferred(T, B, D, hidden, num_sms);
     // H [T, B, hidden] must fit the array; each factor is checked against the
     // room left, so no product of the int arguments can wrap around.
     const size_t esz = dtype == RM_BF16 ? 2 : 4;
     const size_t room = kScratchBytes - kHiddenOffset;
     const size_t row = (size_t)hidden * esz;   // < 2^33, no wrap
-    if (!fused && (row > room || (size_t)B > room / row || (size_t)T > room / (row * (size_t)B)))
+    if (row > room || (size_t)B > room / row || (size_t)T > room / (row * (size_t)B))
         return RM_ERR_INVALID_ARG;
 
     unsigned char* scratch = nullptr;
@@ -120,25 +117,7 @@ extern "C" rm_status rm_pffn_forward_static(const rm_block_weights* w, const voi
     const rm::DeviceErr err{err_word, err_word + 1};
     const uint64_t budget_ns = 1000000000ull;
     cudaError_t e;
-    if (fused) {
-        rm::FusedFfn f{};
-        f.G = T;
-        f.M = B;
-        f.D = D;
-        f.hidden = hidden;
-        f.epi = g1.epi;
-        f.A = S;
-        f.a_gstride = g1.a_gstride;
-        f.a_ld = g1.a_ld;
-        f.W1 = w->W1;
-        f.b1 = g1.bias;
-        f.W2 = w->W2;
-        f.b2 = g2.bias;
-        f.out = V;
-        f.o_gstride = g2.o_gstride;
-        f.o_ld = g2.o_ld;
-        e = rm::launch_ffn_fused(f, err, budget_ns, num_sms, s);
-    } else if (dtype == RM_BF16) {
+    if (dtype == RM_BF16) {
         e = rm::launch_gemm_tc(g1, err, budget_ns, num_sms, s);
         if (e == cudaSuccess) e = rm::launch_gemm_tc(g2, err, budget_ns, num_sms, s);
     } else {

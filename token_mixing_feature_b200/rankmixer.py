@@ -30,7 +30,7 @@ EXPORTED = (
     "rm_train_create", "rm_train_destroy", "rm_train_workspace_bytes", "rm_train_step", "rm_train_sync_status",
 )
 RM_STATIC_SCRATCH_BYTES = 16 << 20
-RM_K_COUNT = 12
+RM_K_COUNT = 11
 
 
 class rm_config(ctypes.Structure):

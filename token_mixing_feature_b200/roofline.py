@@ -121,6 +121,4 @@ def kernel_work(wl: Workload, kind: str, active_mean: Optional[float] = None):
         return "bytes", A * D * es + 2 * act + B * T * 8
     if kind in ("gemm1", "gemm2"):
         return "flops", (2.0 * A * D * Hd) if wl.n_experts else (2.0 * B * T * D * Hd)
-    if kind == "ffn_fused":
-        return "flops", 4.0 * B * T * D * Hd
     raise KeyError(kind)
