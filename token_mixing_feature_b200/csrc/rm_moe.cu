@@ -22,23 +22,28 @@ namespace {
 constexpr int kThreads = 256;
 
 // Router logits, ReLU gates and per-expert active counts.  CTA (t, chunk)
-// stages router t's weights Wr_t [Ne][D] in shared memory once and serves
-// `rows` samples b (chosen on the host so the grid fills the SMs in one
-// wave).  A warp takes RW = 32 / NE rows (b, t) of S at a time:
-// lane l multiplies columns 4l, 4l+128, ... of all RW rows with all NE
-// experts, so each shared-memory weight vector feeds RW rows and each S
-// vector NE experts, with conflict-free 16-byte shared loads.  The RW x NE =
-// 32 partial dot products per lane are reduced across the warp by a
-// transposing butterfly (31 shuffles in all), after which lane l holds the
-// logit of row l / NE, expert l % NE.  Active counts are summed in shared
-// memory and added to the global counts once per CTA.
+// stages router t's weights Wr_t [Ne][D] in shared memory once (before the
+// launch wait: no kernel of the forward pass writes router weights) and
+// serves `rows` samples b (chosen on the host so the grid fills the SMs in
+// one wave).  A warp takes RW = max(1, 16 / NE) rows (b, t) of S at a time:
+// lane l multiplies the 8-column vectors l, l + 32, ... of those rows (all
+// their 16-byte loads issued before the first multiply) with all NE experts,
+// in paired fp32 accumulators, so each staged weight vector feeds RW rows and
+// each S vector NE experts.  The weights are staged split by halves of each
+// 8-column vector ([Ne][2][D/8] float4s), so the lanes' 16-byte shared loads
+// are consecutive (conflict-free).  The NA = RW x NE partial dot products per
+// lane (16 or 32) are reduced across the warp by a transposing butterfly,
+// after which lane l holds the logit of entry l % NA (row (l % NA) / NE,
+// expert l % NE).  Active counts are summed in shared memory and added to the
+// global counts once per CTA.
 
-// acc[i] summed over the warp; afterwards acc[0] of lane l is the sum of
-// everyone's acc[l].
-__device__ __forceinline__ void warp_reduce_transpose32(float (&acc)[32]) {
+// acc[i] summed over the warp (N = 16 or 32); afterwards acc[0] of lane l
+// is the sum of everyone's acc[l % N].
+template <int N>
+__device__ __forceinline__ void warp_reduce_transpose(float (&acc)[N]) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
+    for (int o = N / 2; o >= 1; o >>= 1) {
         const bool upper = (lane & o) != 0;
 #pragma unroll
         for (int i = 0; i < o; ++i) {
@@ -47,75 +52,89 @@ __device__ __forceinline__ void warp_reduce_transpose32(float (&acc)[32]) {
             acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
         }
     }
+    if constexpr (N == 16) acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 16);
 }
 
+// 16-byte S vectors per row and lane per pass: two for up to two rows per
+// warp pass, else one; three CTAs per SM for NE = 8 or 16 (two for 32).
 template <int NE>
-__global__ void __launch_bounds__(kThreads) route_kernel(const __nv_bfloat16* __restrict__ S,
-                                                         const float* __restrict__ Wr,
-                                                         const float* __restrict__ br, float* __restrict__ gates,
-                                                         int* __restrict__ counts, int B, int T, int D, int Ne,
-                                                         int rows) {
-    pdl_enter();
-    constexpr int RW = 32 / NE;
-    extern __shared__ __align__(16) float wsm[];   // [Ne][D]
+__global__ void __launch_bounds__(kThreads, NE == 32 ? 2 : (NE >= 8 ? 3 : 1)) route_kernel(const __nv_bfloat16* __restrict__ S,
+                                                            const float* __restrict__ Wr,
+                                                            const float* __restrict__ br, float* __restrict__ gates,
+                                                            int* __restrict__ counts, int B, int T, int D, int Ne,
+                                                            int rows) {
+    pdl_trigger();
+    constexpr int RW = NE < 16 ? 16 / NE : 1;   // rows per warp pass
+    constexpr int NA = RW * NE;                 // dot products per lane: 16 or 32
+    constexpr int KV = RW <= 2 ? 2 : 1;
+    extern __shared__ __align__(16) float4 wsm4[];   // [Ne][2][D/8]
     __shared__ int cnt[NE];
     const int t = blockIdx.x;
     const int b0 = blockIdx.y * rows;
     const int bend = min(B, b0 + rows);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int nv = D / 8;   // 8-column vectors per row
     {
         const float4* src = reinterpret_cast<const float4*>(Wr + (size_t)t * Ne * D);
-        float4* dst = reinterpret_cast<float4*>(wsm);
-        for (int i = threadIdx.x; i < Ne * D / 4; i += blockDim.x) dst[i] = __ldg(src + i);
+        const int nq = D / 4;
+        for (int i = threadIdx.x; i < Ne * nq; i += blockDim.x) {
+            const int j = i / nq, q = i - j * nq;   // columns 4q .. 4q+3 of expert j: half q & 1 of vector q / 2
+            wsm4[(2 * j + (q & 1)) * nv + (q >> 1)] = __ldg(src + i);
+        }
         if (threadIdx.x < NE) cnt[threadIdx.x] = 0;
     }
-    __syncthreads();
-    const int nv = D / 4;
-    const int jl = lane % NE, rl = lane / NE;   // this lane's (row, expert) after the reduction
+    const int ia = lane % NA;
+    const int jl = ia % NE, rl = ia / NE;   // this lane's (row, expert) after the reduction
     const float bias = jl < Ne ? __ldg(br + (long long)t * Ne + jl) : 0.f;
+    pdl_wait();
+    __syncthreads();
     for (int bw = b0 + warp * RW; bw < bend; bw += nw * RW) {
-        float2 acc2[32];   // paired partial dot products (even / odd columns)
+        float2 acc2[NA];   // [row q][expert j], even / odd columns
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc2[i] = f2(0.f);
-#pragma unroll 2
-        for (int v = lane; v < nv; v += 32) {
-            float xf[RW][4];
+        for (int i = 0; i < NA; ++i) acc2[i] = f2(0.f);
+        for (int v0 = 0; v0 < nv; v0 += 32 * KV) {
+            uint4 xs[RW][KV];
 #pragma unroll
             for (int q = 0; q < RW; ++q) {
                 const int b = bw + q;
-                if (b < bend) {
-                    const uint2 u = __ldcg(reinterpret_cast<const uint2*>(S + ((long long)b * T + t) * D) + v);
-                    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-                    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-                    xf[q][0] = lo.x;
-                    xf[q][1] = lo.y;
-                    xf[q][2] = hi.x;
-                    xf[q][3] = hi.y;
-                } else {
-                    xf[q][0] = xf[q][1] = xf[q][2] = xf[q][3] = 0.f;
+                const uint4* row = reinterpret_cast<const uint4*>(S + ((long long)b * T + t) * D);
+#pragma unroll
+                for (int k = 0; k < KV; ++k) {
+                    const int v = v0 + lane + 32 * k;
+                    xs[q][k] = (b < bend && v < nv) ? __ldcg(row + v) : make_uint4(0u, 0u, 0u, 0u);
                 }
             }
 #pragma unroll
-            for (int j = 0; j < NE; ++j) {
-                if (j < Ne) {
-                    const float4 w = *reinterpret_cast<const float4*>(wsm + (size_t)j * D + 4 * v);
-                    const float2 wl = make_float2(w.x, w.y), wh = make_float2(w.z, w.w);
+            for (int k = 0; k < KV; ++k) {
+                const int v = v0 + lane + 32 * k;
+                if (v < nv) {
+                    float2 xf[RW][4];
 #pragma unroll
-                    for (int q = 0; q < RW; ++q) {
-                        float2 a = acc2[q * NE + j];
-                        a = f2_fma(make_float2(xf[q][0], xf[q][1]), wl, a);
-                        a = f2_fma(make_float2(xf[q][2], xf[q][3]), wh, a);
-                        acc2[q * NE + j] = a;
+                    for (int q = 0; q < RW; ++q) unpack_pairs(xs[q][k], xf[q]);
+#pragma unroll
+                    for (int j = 0; j < NE; ++j) {
+                        if (j < Ne) {
+                            const float4 w0 = wsm4[(2 * j) * nv + v], w1 = wsm4[(2 * j + 1) * nv + v];
+                            const float2 wp[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w),
+                                                  make_float2(w1.x, w1.y), make_float2(w1.z, w1.w)};
+#pragma unroll
+                            for (int q = 0; q < RW; ++q) {
+                                float2 a = acc2[q * NE + j];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) a = f2_fma(xf[q][e], wp[e], a);
+                                acc2[q * NE + j] = a;
+                            }
+                        }
                     }
                 }
             }
         }
-        float acc[32];
+        float acc[NA];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] = acc2[i].x + acc2[i].y;
-        warp_reduce_transpose32(acc);
+        for (int i = 0; i < NA; ++i) acc[i] = acc2[i].x + acc2[i].y;
+        warp_reduce_transpose<NA>(acc);
         const int b = bw + rl;
-        if (jl < Ne && b < bend) {
+        if (lane < NA && jl < Ne && b < bend) {
             const float logit = acc[0] + bias;
             const float gate = logit > 0.f ? logit : 0.f;
             gates[((long long)b * T + t) * Ne + jl] = gate;
@@ -316,7 +335,7 @@ cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, co
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     // Rows per CTA: the (T x chunks) grid fills the resident CTA slots once;
-    // a multiple of the rows a CTA's warps take per pass (8 warps x 32/NE).
+    // a multiple of the rows a CTA's warps take per pass (8 warps x max(1, 16/NE)).
 #define RM_ROUTE(NEV)                                                                                    \
     {                                                                                                    \
         e = cudaFuncSetAttribute(route_kernel<NEV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
@@ -324,7 +343,7 @@ cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, co
         int occ = 0;                                                                                     \
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, route_kernel<NEV>, kThreads, smem);      \
         if (e != cudaSuccess) return e;                                                                  \
-        const int per_pass = (kThreads / 32) * (32 / NEV);                                               \
+        const int per_pass = (kThreads / 32) * (NEV < 16 ? 16 / NEV : 1);                                \
         const long long slots = (long long)num_sms * (occ > 0 ? occ : 1);                                \
         long long chunks = slots / T;                                                                    \
         if (chunks < 1) chunks = 1;                                                                      \
