@@ -302,38 +302,44 @@ __global__ void __launch_bounds__(kThreads) colsum_kernel(const __nv_bfloat16* A
 }
 
 // out[g * N + n] = sum_{j < J} part[(g * J + j) * N + n].  CTA = (32
-// columns, group g); warp w sums the slices j = w, w + kRedWarps, ... of its
+// columns, group g) x W warps (W = blockDim.x / 32, about J / 8 from the
+// host, at most kRedWarps); warp w sums the slices j = w, w + W, ... of its
 // lane's column in ascending j, then one warp adds the warp sums in warp order
-// (a fixed order: deterministic).
+// (a fixed order for a given shape: deterministic).
 __global__ void __launch_bounds__(32 * kRedWarps) reduce_parts_kernel(const float* part, float* out, int G, int J,
                                                                       int N) {
     pdl_enter();
     __shared__ float red[kRedWarps][33];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, W = blockDim.x >> 5;
     const int n = blockIdx.x * 32 + lane, g = blockIdx.y;
     float a = 0.f;
     if (n < N) {
         const float* p = part + (long long)g * J * N + n;
         int j = warp;
-        for (; j + 3 * kRedWarps < J; j += 4 * kRedWarps) {   // four loads in flight
-            const float x0 = __ldcg(p + (long long)j * N), x1 = __ldcg(p + (long long)(j + kRedWarps) * N);
-            const float x2 = __ldcg(p + (long long)(j + 2 * kRedWarps) * N);
-            const float x3 = __ldcg(p + (long long)(j + 3 * kRedWarps) * N);
+        for (; j + 3 * W < J; j += 4 * W) {   // four loads in flight
+            const float x0 = __ldcg(p + (long long)j * N), x1 = __ldcg(p + (long long)(j + W) * N);
+            const float x2 = __ldcg(p + (long long)(j + 2 * W) * N);
+            const float x3 = __ldcg(p + (long long)(j + 3 * W) * N);
             a += x0;
             a += x1;
             a += x2;
             a += x3;
         }
-        for (; j < J; j += kRedWarps) a += __ldcg(p + (long long)j * N);
+        for (; j < J; j += W) a += __ldcg(p + (long long)j * N);
     }
     red[warp][lane] = a;
     __syncthreads();
     if (warp == 0 && n < N) {
         float t = 0.f;
-#pragma unroll
-        for (int w = 0; w < kRedWarps; ++w) t += red[w][lane];
+        for (int w = 0; w < W; ++w) t += red[w][lane];
         out[(long long)g * N + n] = t;
     }
+}
+
+// Ordered reduction of J slices per column: about eight slices per warp.
+inline cudaError_t launch_reduce_parts(const float* part, float* out, int G, int J, int N, cudaStream_t s) {
+    const int W = std::min(kRedWarps, std::max(1, (J + 7) / 8));
+    return launch_pdl(reduce_parts_kernel, dim3((N + 31) / 32, G), dim3(32 * W), 0, s, part, out, G, J, N);
 }
 
 // ---------------------------------------------- LN1 backward + mixing transpose
@@ -701,12 +707,9 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
             RM_TRY(rm::launch_pdl(rm::ln2_bwd_kernel<false>, dim3(nsb, T), dim3(lnb_threads), 0, s,
                                   (const __nv_bfloat16*)t->dX, (const float*)nullptr, Yl, (const float2*)t->ystats[l],
                                   P, w.ln2_g, c.ln_eps, dY, t->pg, t->pb, t->pdb, B, T, D, t->SB));
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + 31) / 32, 1), dim3(32 * rm::kRedWarps), 0, s,
-                              (const float*)t->pg, gr.ln2_g, 1, T * nsb, D));
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + 31) / 32, 1), dim3(32 * rm::kRedWarps), 0, s,
-                              (const float*)t->pb, gr.ln2_b, 1, T * nsb, D));
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + 31) / 32, T), dim3(32 * rm::kRedWarps), 0, s,
-                              (const float*)t->pdb, gr.b2, T, nsb, D));
+        RM_TRY(rm::launch_reduce_parts((const float*)t->pg, gr.ln2_g, 1, T * nsb, D, s));
+        RM_TRY(rm::launch_reduce_parts((const float*)t->pb, gr.ln2_b, 1, T * nsb, D, s));
+        RM_TRY(rm::launch_reduce_parts((const float*)t->pdb, gr.b2, T, nsb, D, s));
         // dU = (dY W2_t) * act'(U)
         rm::GroupedGemm gh{};
         gh.G = T; gh.M = B; gh.N = Hd; gh.K = D;
@@ -731,8 +734,7 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
         RM_TRY(rm::launch_pdl(rm::colsum_kernel, dim3((Hd / 8 + rm::kThreads - 1) / rm::kThreads, nrb_b, T),
                               dim3(rm::kThreads), 0, s, (const __nv_bfloat16*)t->dU, (const __nv_bfloat16*)nullptr,
                               t->pcol, (float*)nullptr, B, Hd, (long long)B * Hd, (long long)Hd, rm::kColRows));
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((Hd + 31) / 32, T), dim3(32 * rm::kRedWarps), 0, s,
-                              (const float*)t->pcol, gr.b1, T, nrb_b, Hd));
+        RM_TRY(rm::launch_reduce_parts((const float*)t->pcol, gr.b1, T, nrb_b, Hd, s));
         // dS = dU W1_t + dY
         rm::GroupedGemm gs{};
         gs.G = T; gs.M = B; gs.N = D; gs.K = Hd;
@@ -758,10 +760,8 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
                               dim3(rm::kThreads), 0, s, (const __nv_bfloat16*)t->dS,
                               (const __nv_bfloat16*)t->XH1[l], t->pcol, t->pcol2, B * T, D, 0LL, (long long)D,
                               rm::kColRows));
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + 31) / 32, 1), dim3(32 * rm::kRedWarps), 0, s,
-                              (const float*)t->pcol2, gr.ln1_g, 1, nrb, D));
-        RM_TRY(rm::launch_pdl(rm::reduce_parts_kernel, dim3((D + 31) / 32, 1), dim3(32 * rm::kRedWarps), 0, s,
-                              (const float*)t->pcol, gr.ln1_b, 1, nrb, D));
+        RM_TRY(rm::launch_reduce_parts((const float*)t->pcol2, gr.ln1_g, 1, nrb, D, s));
+        RM_TRY(rm::launch_reduce_parts((const float*)t->pcol, gr.ln1_b, 1, nrb, D, s));
         // LN1 backward and the mixing's transpose: dX (the stack input's gradient for l = 0)
         __nv_bfloat16* dXo = (l == 0 && dX0) ? static_cast<__nv_bfloat16*>(dX0)
                                              : reinterpret_cast<__nv_bfloat16*>(t->dX);
