@@ -43,6 +43,7 @@ FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_g
 # datasheet figures of one B200: dense bf16 tensor throughput and HBM3e bandwidth
 SPEC_PEAKS = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 SUSTAINED_S = 1.5   # length of the repeat of the headline steps (clock record, sustained time)
+MOE_REG_LAMBDA = 1e-4   # L_reg weight of the sparse-MoE training step (the pages give no value)
 
 
 # ---------------------------------------------------------------- utilities
@@ -559,9 +560,12 @@ def run_train(a, wl, cfg, rank, world, local):
     mean BCE loss of the sigmoid head, every gradient) on the workload's
     synthetic inputs with seeded 0/1 labels; device time with CUDA events on
     the launch stream, max over ranks.  FLOPs: the forward's 4 B T D kD L
-    plus the backward's activation and weight gradients, 8 B T D kD L."""
-    if wl.n_experts or wl.dtype != "bf16" or not wl.mix_addnorm:
-        raise SystemExit("the training step covers dense bf16 stacks with the Add & Norm after mixing")
+    plus the backward's activation and weight gradients, 8 B T D kD L; for a
+    sparse-MoE stack 12 D kD per active (sample, token, expert) entry, the
+    active entries counted by routing every block's S through the library,
+    with L_reg weight MOE_REG_LAMBDA on the routing gates."""
+    if wl.dtype != "bf16" or not wl.mix_addnorm:
+        raise SystemExit("the training step covers bf16 stacks with the Add & Norm after mixing")
     from token_mixing_feature_b200 import rankmixer as rm
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
@@ -579,13 +583,25 @@ def run_train(a, wl, cfg, rank, world, local):
     labels = (torch.rand(B, generator=g) < 0.5).float().to(device)
     X0 = d["X0"].to(device)
     hw, hb = head["w"].to(device), head["b"].to(device)
-    grads = [{"W1": torch.empty(T, Hd, D, device=device), "b1": torch.empty(T, Hd, device=device),
-              "W2": torch.empty(T, D, Hd, device=device), "b2": torch.empty(T, D, device=device),
-              **{k: torch.empty(D, device=device) for k in ("ln1_g", "ln1_b", "ln2_g", "ln2_b")}}
+    Ne = wl.n_experts
+    TE = (T, Ne) if Ne else (T,)
+    grads = [{"W1": torch.empty(*TE, Hd, D, device=device), "b1": torch.empty(*TE, Hd, device=device),
+              "W2": torch.empty(*TE, D, Hd, device=device), "b2": torch.empty(*TE, D, device=device),
+              **{k: torch.empty(D, device=device) for k in ("ln1_g", "ln1_b", "ln2_g", "ln2_b")},
+              **({"Wr": torch.empty(T, Ne, D, device=device), "br": torch.empty(T, Ne, device=device)} if Ne else {})}
              for _ in range(L)]
     dX0 = torch.empty(B, T, D, dtype=torch.bfloat16, device=device)
     dhw, dhb, loss = torch.empty(D, device=device), torch.empty(1, device=device), torch.empty(1, device=device)
-    tr = rm.rm_train_create(B, T, D, Hd, L, act=wl.act)
+    active = None
+    if Ne and rank == 0:   # active entries per block, from the library's own routing of each block's S
+        runner = Runner(wl, device)
+        active = moe_active_counts(runner)
+        runner.st.close()
+        del runner
+        torch.cuda.synchronize(device)
+    tr = rm.rm_train_create(B, T, D, Hd, L, act=wl.act, n_experts=Ne)
+    if Ne:
+        rm.rm_train_set_reg(tr, MOE_REG_LAMBDA)
     stream = torch.cuda.current_stream(device)
 
     def step():
@@ -616,12 +632,13 @@ def run_train(a, wl, cfg, rank, world, local):
         clocks = sampler.summary(wall0 - 0.05, wall1 + 0.05)
     if rank == 0:
         peaks, peak_src = load_peaks()
-        flops = 12.0 * B * T * D * Hd * L
+        flops = 12.0 * D * Hd * (sum(active) if Ne else B * T * L)
         es = 2
-        wbytes = L * (2 * T * D * Hd * es)
+        TN = T * max(Ne, 1)
+        wbytes = L * (2 * TN * D * Hd * es)
         # weights read by the forward and by the activation-gradient products,
         # weight gradients written in float, the stack input read once
-        nbytes = 2 * wbytes + L * (2 * T * D * Hd * 4) + B * T * D * es
+        nbytes = 2 * wbytes + L * (2 * TN * D * Hd * 4) + B * T * D * es
         sec = ms / 1e3 / a.steps
         t_roof = roofline.roofline_seconds(flops, nbytes, peaks["bf16_tflops"] * 1e12, peaks["hbm_gbs"] * 1e9)
         line = {
@@ -638,6 +655,9 @@ def run_train(a, wl, cfg, rank, world, local):
             "loss": float(loss.item()),
             "clocks": clocks,
         }
+        if Ne:
+            line["moe_active_fraction"] = [c / (B * T * Ne) for c in active]
+            line["reg_lambda"] = MOE_REG_LAMBDA
         print(json.dumps(line), flush=True)
     tr.close()
     if pg:

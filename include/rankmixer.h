@@ -86,6 +86,9 @@ typedef struct {
     const float *ln1_g, *ln1_b;                /* LN after token mixing [D]      */
     const float *ln2_g, *ln2_b;                /* LN after the FFN [D]           */
     const float *Wr, *br;                      /* MoE router (NULL when dense)   */
+    /* DTSI's second router h_infer (training only, may be NULL): its gates
+     * carry L_reg; the forward routes with Wr, br.  Same shapes as Wr, br. */
+    const float *Wr_infer, *br_infer;
 } rm_block_weights;
 
 typedef struct rm_handle rm_handle;
@@ -247,19 +250,38 @@ rm_status rm_pffn_forward_static(const rm_block_weights *w, const void *S, void 
  * rows, their 1/sqrt(var + eps), the FFN activation input and output, the
  * pre-LN rows and their statistics; plus the backward buffers), allocated by
  * rm_train_create for batches up to cfg->B_max.  Supported: dtype RM_BF16,
- * n_experts 0, mix_addnorm 1, D % 64 == 0, hidden % 64 == 0, (D / T) % 8 == 0,
- * D <= 2048, plus the forward's limits.  Otherwise RM_ERR_UNSUPPORTED. */
+ * n_experts 0 (dense) or 1..32 (sparse MoE with ReLU routing), mix_addnorm 1,
+ * D % 64 == 0, hidden % 64 == 0, (D / T) % 8 == 0, D <= 2048, plus the
+ * forward's limits.  Otherwise RM_ERR_UNSUPPORTED.  Sparse-MoE blocks keep
+ * their routing, their compacted expert rows (each expert's slot list padded
+ * to a multiple of 64 with zero rows) and the experts' activation inputs, and
+ * the backward pass computes, per active (sample, token, expert) entry,
+ * dG = dV . e_j and de_j = G_j dV, the experts' gradients over their slots
+ * (the weight gradients as products whose K runs over the expert's slots),
+ * and the routers' gradients through ReLU (fun-rec "Rankmixer: 硬件效率优化",
+ * section Sparse MoE扩展). */
 typedef struct rm_trainer rm_trainer;
 
 /* Gradient outputs of one block (device pointers, float, the parameters'
  * shapes and layouts): W1 [T][kD][D], b1 [T][kD], W2 [T][D][kD], b2 [T][D],
- * ln1_g, ln1_b, ln2_g, ln2_b [D].  Every entry is overwritten (not added to). */
+ * ln1_g, ln1_b, ln2_g, ln2_b [D]; sparse MoE: W1 [T][Ne][kD][D], b1
+ * [T][Ne][kD], W2 [T][Ne][D][kD], b2 [T][Ne][D], the router's Wr [T][Ne][D]
+ * and br [T][Ne], and DTSI's second router's Wr_infer, br_infer (when the
+ * block's weights give one; else unused, may be NULL).  Every entry is
+ * overwritten (not added to). */
 typedef struct {
     float *W1, *b1, *W2, *b2;
     float *ln1_g, *ln1_b, *ln2_g, *ln2_b;
+    float *Wr, *br, *Wr_infer, *br_infer;
 } rm_block_grads;
 
 rm_status rm_train_create(const rm_config *cfg, rm_trainer **out);
+/* Weight lambda of L_reg (default 0; lambda >= 0, else RM_ERR_INVALID_ARG):
+ * the loss becomes L_task + lambda * (sum over the batch's tokens and experts
+ * of the regularised gates of every MoE block: DTSI's second router's where a
+ * block gives one, else the routing gates).  fun-rec "Rankmixer: 硬件效率优化",
+ * section Sparse MoE扩展 (L = L_task + lambda L_reg, DTSI-MoE). */
+rm_status rm_train_set_reg(rm_trainer *t, float lambda);
 rm_status rm_train_destroy(rm_trainer *t);
 size_t rm_train_workspace_bytes(const rm_trainer *t);
 

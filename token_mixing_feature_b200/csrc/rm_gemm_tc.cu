@@ -73,6 +73,11 @@ struct KParams {
     int save_pre;             // activation epilogues: also store bf16(acc + bias), the activation's input, via tmR
     int w_from_kernel;        // W (B operand) written by an earlier kernel: no loads before the launch wait
     int w_g_inner;            // W map coordinate order (k|n, g, n|k) if 1, else (k|n, n|k, g)
+    // Variable-K groups (weight gradients of the sparse-MoE experts): dense
+    // G x M x N tiles whose K rows are rows [grp_off[g], grp_off[g] + grp_cnt[g])
+    // of the compacted A and W operands (grp_cnt a multiple of 64, the padding
+    // rows zero); group coordinate 0 in both maps.
+    int vark;
     DeviceErr err;
     unsigned long long budget_ns;
 };
@@ -127,7 +132,7 @@ __device__ __forceinline__ Tile decode_tile(const KParams& p, long long idx, int
         const int r = (int)(idx - (long long)t.g * per_g);
         const int nb = r / mblk, mb = r - nb * mblk;
         const int m0 = mb * (BM * CG) + rank * BM;
-        t.ag = t.g;
+        t.ag = p.vark ? 0 : t.g;
         t.arow = m0;
         t.rows = min(BM, p.M - m0);
         t.n0 = nb * bn;
@@ -159,18 +164,25 @@ __device__ __forceinline__ Tile decode_tile(const KParams& p, long long idx, int
 struct Item {
     long long tile;
     int kb_lo, kb_hi;
+    int koff;    // K offset of the tile's group (variable-K groups), else 0
     int tj;      // tail tile ordinal (split items), else -1
     int slice;
 };
 
-__device__ __forceinline__ Item decode_item(const KParams& p, long long idx, int num_kb) {
+__device__ __forceinline__ Item decode_item(const KParams& p, long long idx, int num_kb, long long per_g = 1) {
     Item it;
+    it.koff = 0;
     if (idx < p.full_tiles || p.nsplit == 1) {
         it.tile = idx;
         it.kb_lo = 0;
         it.kb_hi = num_kb;
         it.tj = -1;
         it.slice = 0;
+        if (p.vark) {   // this group's K rows
+            const int g = (int)(idx / per_g);
+            it.kb_hi = __ldcg(p.grp_cnt + g) / BK;
+            it.koff = __ldcg(p.grp_off + g);
+        }
     } else {
         const long long j = idx - p.full_tiles;
         it.tj = (int)(j / p.nsplit);
@@ -244,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
                    const KParams p) {
     using C = Cfg<BN, CG, VAR>;
-    static_assert(!(VAR && (AMN || BMN)), "variable-row groups read K-major operands");
+    static_assert(!(VAR && AMN), "variable-row groups read a K-major A");
     static_assert(!BMN || C::BN_LOCAL % 64 == 0, "N-major W tiles are whole 64-row boxes");
     constexpr bool DACT = EPI == EPI_DACT_TANH || EPI == EPI_DACT_ERF || EPI == EPI_DACT_RELU;
     constexpr bool F32OUT = EPI == EPI_F32;
@@ -316,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long total = p.var_rows ? (long long)mt_table[p.G] * nblk
                                        : p.full_tiles + ((long long)p.G * nblk * mblk - p.full_tiles) * p.nsplit;
     const long long unit = blockIdx.x / CG, nunits = gridDim.x / CG;
+    const long long per_g = (long long)nblk * mblk;   // tiles per group (dense decode)
 
     if (warp == 0) {
         if (lane == 0) {
@@ -325,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             // Weight (B) tiles of the first tile's first stages, before the wait.
             int npre = 0;
-            if (!VAR && !p.w_from_kernel && unit < total) {
+            if (!VAR && !p.w_from_kernel && !p.vark && unit < total) {
                 const Item it0 = decode_item(p, unit, num_kb);
                 const Tile t0 = decode_tile<CG>(p, it0.tile, nblk, mblk, BN, (int)rank, mt_table);
                 const int nb0 = t0.n0 + (int)rank * C::BN_LOCAL;
@@ -342,9 +355,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             pdl_wait();
             bool first = true;
             for (long long idx = unit; idx < total && ok; idx += nunits) {
-                const Item item = decode_item(p, idx, num_kb);
+                const Item item = decode_item(p, idx, num_kb, per_g);
                 const Tile t = decode_tile<CG>(p, item.tile, nblk, mblk, BN, (int)rank, mt_table);
                 const int nb0 = t.n0 + (int)rank * C::BN_LOCAL;
+                const int wg = p.vark ? 0 : t.g;   // W map group coordinate
                 for (int kb = item.kb_lo; kb < item.kb_hi; ++kb) {
                     const bool pre = first && kb - item.kb_lo < npre;   // B already issued
                     if (!pre && !mbar_wait(empty0 + 8 * stage, phase ^ 1u, wc, SITE_TC_PRODUCER)) {
@@ -354,11 +368,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t fb = full0 + 8 * stage;
                     if (leader && !pre) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
                     const uint32_t sa = sbase + stage * C::STAGE_BYTES;
-                    const int kc = kb * BK;
+                    const int kc = kb * BK + item.koff;
                     // the pair counts bytes on the even CTA's barrier
                     const uint32_t fbl = CG == 2 ? mapa_shared(fb, 0) : fb;
                     load_operand<AMN, BM, CG == 2>(sa, &tmA, fbl, kc, t.arow, t.ag, p.a_g_inner);
-                    if (!pre) load_operand<BMN, C::BN_LOCAL, CG == 2>(sa + C::A_BYTES, &tmB, fbl, kc, nb0, t.g, p.w_g_inner);
+                    if (!pre) load_operand<BMN, C::BN_LOCAL, CG == 2>(sa + C::A_BYTES, &tmB, fbl, kc, nb0, wg, p.w_g_inner);
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -391,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(tempty0 + 8 * acc, aph ^ 1u, wc, SITE_TC_MMA_TMEM)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                const Item item = decode_item(p, idx, num_kb);
+                const Item item = decode_item(p, idx, num_kb, per_g);
                 for (int kb = item.kb_lo; kb < item.kb_hi; ++kb) {
                     if (!mbar_wait(full0 + 8 * stage, phase, wc, SITE_TC_MMA_FULL)) {
                         ok = false;
@@ -712,10 +726,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_ok = row < t.rows;
             const long long orow = t.orow0 + row;
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-            const float* bias_g = p.bias + (long long)t.g * p.N;
+            const float* bias_g = p.bias ? p.bias + (long long)t.g * p.N : nullptr;
             __nv_bfloat16* out_row = p.out + (long long)t.g * p.o_gstride + orow * p.o_ld;
-            float gate = 0.f;
-            if (EPI == EPI_BIAS_GATE && row_ok) gate = __ldcg(p.gate + orow);
+            // bf16 row of the same shape as out: the activation input (DACT, loaded)
+            // or the pre-activation values (save_pre, stored)
+            const long long rrow = orow * p.r_ld;
+            float gate = 1.f;
+            if (EPI == EPI_BIAS_GATE && row_ok && p.gate) gate = __ldcg(p.gate + orow);
 #pragma unroll 1
             for (int c = half * HALF; c < (half + 1) * HALF; c += 16) {
                 float v[16];
@@ -723,16 +740,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_wait();
                 const int n = t.n0 + c;
                 if (row_ok && n < p.N) {
-                    const float4* b4 = reinterpret_cast<const float4*>(bias_g + n);
+                    if (bias_g) {
+                        const float4* b4 = reinterpret_cast<const float4*>(bias_g + n);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float4 bb = __ldg(b4 + q);
-                        const float2 lo = f2_add(make_float2(v[4 * q], v[4 * q + 1]), make_float2(bb.x, bb.y));
-                        const float2 hi = f2_add(make_float2(v[4 * q + 2], v[4 * q + 3]), make_float2(bb.z, bb.w));
-                        v[4 * q] = lo.x;
-                        v[4 * q + 1] = lo.y;
-                        v[4 * q + 2] = hi.x;
-                        v[4 * q + 3] = hi.y;
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 bb = __ldg(b4 + q);
+                            const float2 lo = f2_add(make_float2(v[4 * q], v[4 * q + 1]), make_float2(bb.x, bb.y));
+                            const float2 hi = f2_add(make_float2(v[4 * q + 2], v[4 * q + 3]), make_float2(bb.z, bb.w));
+                            v[4 * q] = lo.x;
+                            v[4 * q + 1] = lo.y;
+                            v[4 * q + 2] = hi.x;
+                            v[4 * q + 3] = hi.y;
+                        }
+                    }
+                    if ((EPI == EPI_RELU || EPI == EPI_GELU_TANH || EPI == EPI_GELU_ERF) && p.save_pre) {
+                        uint4* pre = reinterpret_cast<uint4*>(const_cast<__nv_bfloat16*>(p.resid) + rrow + n);
+                        pre[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                            pack_bf16x2(v[6], v[7]));
+                        pre[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                                            pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
                     }
                     if (EPI == EPI_RELU) {
 #pragma unroll
@@ -747,19 +773,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else if (EPI == EPI_GELU_ERF) {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = 0.5f * v[e] * (1.0f + erff(v[e] * 0.7071067811865476f));
-                    } else if (EPI == EPI_BIAS_RESID) {
-                        if (p.resid) {
-                            const uint4* r4 = reinterpret_cast<const uint4*>(
-                                p.resid + (long long)t.g * p.r_gstride + orow * p.r_ld + n);
+                    } else if (DACT) {   // acc * act'(U), U the stored activation input of the row
+                        const uint4* u4 = reinterpret_cast<const uint4*>(p.resid + rrow + n);
 #pragma unroll
-                            for (int q = 0; q < 2; ++q) {
-                                Vec16<__nv_bfloat16> r;
-                                r.u = __ldcg(r4 + q);
+                        for (int q = 0; q < 2; ++q) {
+                            float2 up[4];
+                            unpack_pairs(__ldcg(u4 + q), up);
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) v[8 * q + e] += __bfloat162float(r.e[e]);
+                            for (int e = 0; e < 4; ++e) {
+                                v[8 * q + 2 * e] *= dact<EPI>(up[e].x);
+                                v[8 * q + 2 * e + 1] *= dact<EPI>(up[e].y);
                             }
                         }
-                    } else {  // EPI_BIAS_GATE
+                    } else if (EPI == EPI_BIAS_GATE) {
 #pragma unroll
                         for (int e = 0; e < 16; e += 2) {
                             const float2 y = f2_mul(make_float2(v[e], v[e + 1]), f2(gate));
@@ -846,6 +872,23 @@ cudaError_t launch_bn_mn(int epi, bool a_mn, const Maps& m, const KParams& kp, i
     }
 }
 
+// Variable-row groups with an N-major W (the sparse-MoE experts' activation
+// gradients): acc x act'(U), or plain acc (EPI_BIAS_GATE without bias and gate).
+template <int BN>
+cudaError_t launch_bn_var_mn(int epi, const Maps& m, const KParams& kp, int grid, cudaStream_t s) {
+    if constexpr (BN % 64 != 0) {
+        return cudaErrorInvalidValue;
+    } else {
+        switch (epi) {
+            case EPI_DACT_TANH: return launch_typed<BN, EPI_DACT_TANH, 1, true, false, true>(m, kp, grid, s);
+            case EPI_DACT_ERF: return launch_typed<BN, EPI_DACT_ERF, 1, true, false, true>(m, kp, grid, s);
+            case EPI_DACT_RELU: return launch_typed<BN, EPI_DACT_RELU, 1, true, false, true>(m, kp, grid, s);
+            case EPI_BIAS_GATE: return launch_typed<BN, EPI_BIAS_GATE, 1, true, false, true>(m, kp, grid, s);
+        }
+        return cudaErrorInvalidValue;
+    }
+}
+
 template <int BN, int CG, bool VAR>
 cudaError_t launch_bn(int epi, const Maps& m, const KParams& kp, int grid, cudaStream_t s) {
     switch (epi) {
@@ -927,10 +970,15 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     const bool dact = g.epi == EPI_DACT_TANH || g.epi == EPI_DACT_ERF || g.epi == EPI_DACT_RELU;
     const bool f32out = g.epi == EPI_F32;
     const bool mn = g.a_mn || g.w_mn;
+    const bool vark = g.vark;
     // layouts the kernel is instantiated for
-    if (mn && (var || !g.w_mn || (g.a_mn != f32out) || (!g.a_mn && !dact && g.epi != EPI_BIAS_RESID)))
+    if (var && (vark || g.a_mn || (g.w_mn && !dact && g.epi != EPI_BIAS_GATE) || (dact && !g.w_mn)))
         return cudaErrorInvalidValue;
-    if ((dact || f32out) && !mn) return cudaErrorInvalidValue;
+    if (!var && mn && (!g.w_mn || (g.a_mn != f32out) || (!g.a_mn && !dact && g.epi != EPI_BIAS_RESID)))
+        return cudaErrorInvalidValue;
+    if (vark && (!g.a_mn || !g.w_mn || !f32out || !g.grp_off || !g.vark_cnt)) return cudaErrorInvalidValue;
+    if (f32out && !mn) return cudaErrorInvalidValue;
+    if (dact && !mn) return cudaErrorInvalidValue;
     if (dact && !g.resid) return cudaErrorInvalidValue;
     if (g.a_mn && g.M % 8) return cudaErrorInvalidValue;   // 16-byte rows of an M-major A
     if (f32out && g.N % 32) return cudaErrorInvalidValue;
@@ -940,6 +988,7 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     kp.N = g.N;
     kp.K = g.K;
     kp.var_rows = var ? 1 : 0;
+    kp.vark = vark ? 1 : 0;
     kp.out = static_cast<__nv_bfloat16*>(g.out);
     kp.o_gstride = var ? 0 : g.o_gstride;
     kp.o_ld = g.o_ld;
@@ -948,7 +997,7 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     kp.r_gstride = var ? 0 : g.r_gstride;
     kp.r_ld = g.r_ld;
     kp.gate = g.gate;
-    kp.grp_cnt = g.grp_cnt;
+    kp.grp_cnt = vark ? g.vark_cnt : g.grp_cnt;
     kp.grp_off = g.grp_off;
     kp.mtile_prefix = g.mtile_prefix;
     kp.stats = g.stats;
@@ -959,17 +1008,16 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     kp.nsplit = 1;
     kp.sk_ws = g.sk_ws;
     kp.sk_cnt = g.sk_cnt;
-    kp.w_from_kernel = g.w_from_kernel ? 1 : 0;
+    kp.w_from_kernel = (g.w_from_kernel || vark) ? 1 : 0;
     // activation epilogues with resid set: resid receives the pre-activation values
     kp.save_pre = (g.resid && (g.epi == EPI_GELU_TANH || g.epi == EPI_GELU_ERF || g.epi == EPI_RELU)) ? 1 : 0;
-    if (kp.save_pre && var) return cudaErrorInvalidValue;
     kp.w_g_inner = 0;
     kp.err = err;
     kp.budget_ns = budget_ns;
 
     // 2-SM (256-row) tiles for dense problems with more than one 128-row block;
     // the variable-row (MoE) groups keep 128-row tiles.
-    int cg = var ? (g.var_cg == 2 ? 2 : 1) : (g.M > BM ? 2 : 1);
+    int cg = var ? (g.var_cg == 2 && !g.w_mn ? 2 : 1) : (g.M > BM ? 2 : 1);
     int bn = gemm_tc_pick_bn(g.G, g.M, g.N, g.K, var, num_sms, cg, g.sk_ws && g.sk_cnt, g.w_mn);
     // Tuning overrides (same kernel, other tile shape): RM_GEMM_CG=1|2, RM_GEMM_BN=256|192|160|128.
     if (const char* e = getenv("RM_GEMM_CG")) {
@@ -987,6 +1035,10 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     if (var) {
         // compacted rows [rows_total, K]
         ok = make_map(&m.a, g.A, g.K, g.a_rows_total, 1, g.a_ld * 2, g.a_rows_total * g.a_ld * 2, BM, 1);
+        kp.a_g_inner = 0;
+    } else if (vark) {
+        // compacted rows [rows_total, M], M-major: K runs over the rows (group coordinate 0)
+        ok = make_map(&m.a, g.A, g.M, g.a_rows_total, 1, g.a_ld * 2, g.a_rows_total * g.a_ld * 2, BK, 1);
         kp.a_g_inner = 0;
     } else if (g.a_mn) {
         // M-major A: element (g, m, k) at g*a_gstride + k*a_ld + m; boxes of 64 rows x 64 K
@@ -1007,7 +1059,10 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
         kp.a_g_inner = 0;
     }
     const long long w_ld = g.w_ld ? g.w_ld : g.K, w_gs = g.w_ld ? g.w_gstride : (long long)g.N * g.K;
-    if (g.w_mn) {
+    if (vark) {
+        // compacted rows [rows_total, N], N-major: K runs over the rows (group coordinate 0)
+        ok = ok && make_map(&m.b, g.W, g.N, g.a_rows_total, 1, w_ld * 2, g.a_rows_total * w_ld * 2, BK, 1);
+    } else if (g.w_mn) {
         // N-major W: element (g, n, k) at g*w_gstride + k*w_ld + n; boxes of 64 rows x 64 K
         if (w_gs <= w_ld) {
             ok = ok && make_map(&m.b, g.W, g.N, g.G, g.K, w_gs * 2, w_ld * 2, 1, BK);
@@ -1042,7 +1097,7 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
         const long long tiles = (long long)g.G * ((g.M + BM * cg - 1) / (BM * cg)) * ((g.N + bn - 1) / bn);
         if (tiles == 0) return cudaSuccess;
         const int num_kb = (g.K + BK - 1) / BK;
-        const int S = (g.sk_ws && g.sk_cnt) ? split_slices(tiles, units, num_kb) : 1;
+        const int S = (g.sk_ws && g.sk_cnt && !vark) ? split_slices(tiles, units, num_kb) : 1;
         if (const char* e = getenv("RM_GEMM_SPLIT"))   // tuning override: 0 disables the split tail
             if (atoi(e) == 0 && S > 1) return launch_gemm_tc_nosplit(g, err, budget_ns, num_sms, s);
         const long long tail = S > 1 ? tiles % units : 0;
@@ -1055,6 +1110,13 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
                     g.G, g.M, g.N, g.K, g.epi, cg, bn, tiles, tail, S, units * cg);
     }
     const int grid = units * cg;
+    if (var && g.w_mn) {
+        switch (bn) {
+            case 256: return launch_bn_var_mn<256>(g.epi, m, kp, grid, s);
+            case 192: return launch_bn_var_mn<192>(g.epi, m, kp, grid, s);
+            default: return launch_bn_var_mn<128>(g.epi, m, kp, grid, s);
+        }
+    }
     if (var) {
         if (cg == 2) {
             switch (bn) {

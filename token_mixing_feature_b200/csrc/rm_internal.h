@@ -126,6 +126,13 @@ struct GroupedGemm {
     const int* grp_cnt;
     const int* grp_off;
     const int* mtile_prefix;  // [G + 1]
+    // Variable-K mode (the sparse-MoE experts' weight gradients, a_mn and w_mn,
+    // EPI_F32): dense G x M x N output tiles; group g's K runs over rows
+    // [grp_off[g], grp_off[g] + vark_cnt[g]) of the compacted A [rows][M] and
+    // W [rows][N] (a_ld, w_ld their row strides; vark_cnt a multiple of 64,
+    // at least 64, the padding rows zero).  grp_cnt must be null.
+    bool vark;
+    const int* vark_cnt;
     // Optional split-K workspace for the dense tcgen05 path (both null: no
     // split).  sk_ws holds gemm_tc_split_ws_bytes(num_sms) bytes; sk_cnt holds
     // gemm_tc_split_cnt_ints(num_sms) ints, zero before the first use (the
@@ -154,6 +161,9 @@ struct MoeWork {
     void* Sg;              // [B*T*Ne, D] bf16 gathered rows
     void* Hg;              // [B*T*Ne, hidden] bf16
     void* Eg;              // [B*T*Ne, D] bf16 gate-scaled expert outputs
+    // training: every expert's slot list padded to a multiple of 64, at least
+    // 64 (padded counts here; rows -1 and gates 0 in the padding); null: none
+    int* cnt_pad = nullptr;    // [T*Ne]
 };
 cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, const MoeWork& w, int B,
                              int T, int D, int Ne, cudaStream_t s, int tile_rows = 128);
@@ -163,5 +173,23 @@ cudaError_t launch_moe_gather(const void* S, const MoeWork& w, int B, int T, int
                               cudaStream_t s);
 cudaError_t launch_moe_combine(const MoeWork& w, const void* resid, void* out, float2* stats, int B, int T, int D,
                                int Ne, cudaStream_t s);
+// Training (sparse-MoE backward).  Gates of a router alone (no compaction);
+// counts_scratch [T*Ne] ints.
+cudaError_t launch_moe_route_only(const void* S, const float* Wr, const float* br, float* gates, int* counts_scratch,
+                                  int B, int T, int D, int Ne, cudaStream_t s);
+// dEg[slot] = G dV[row], dR[r, j] = dV . e_j [active] (+ lambda unless gates_inf),
+// dRinf[r, j] = lambda [gates_inf > 0] (gates_inf / dRinf may be null); the
+// padding slots' rows of dEg are zeroed.
+cudaError_t launch_moe_bwd_gate(const void* dV, const MoeWork& w, const float* gates_inf, float lambda, void* dEg,
+                                float* dR, float* dRinf, int B, int T, int D, int Ne, cudaStream_t s);
+// dS[r] = dZ[r] + sum_j dSg[slot(r, j)] + sum_j dR[r, j] Wr[t, j] + sum_j dRinf[r, j] Wrinf[t, j].
+cudaError_t launch_moe_bwd_combine(const void* dZ, const void* dSg, const MoeWork& w, const float* dR, const float* Wr,
+                                   const float* dRinf, const float* Wrinf, void* dS, int B, int T, int D, int Ne,
+                                   cudaStream_t s);
+// Router weight-gradient partials over blocks of RB samples (see rm_moe.cu).
+cudaError_t launch_router_grad(const void* S, const float* dR, float* part, float* part_b, int B, int T, int D, int Ne,
+                               int RB, cudaStream_t s);
+// loss[0] += lambda * sum of x[0 .. n), in a fixed order.
+cudaError_t launch_add_scaled_sum(const float* x, long long n, float lambda, float* loss, cudaStream_t s);
 
 }  // namespace rm

@@ -153,13 +153,19 @@ __device__ __forceinline__ int warp_isum(int v) {
 
 // One CTA of 1024 threads per expert g = t * Ne + j: its slot offset and
 // m-tile prefix (sums over the experts before it), then the list of samples
-// b (ascending) whose gate is > 0.
+// b (ascending) whose gate is > 0.  With cnt_pad (training), every expert's
+// list is padded to a multiple of 64 slots, at least 64 (the expert's
+// K range in the weight-gradient products): offsets, m-tiles and totals count
+// the padded lists, cnt_pad receives the padded counts, and the padding slots
+// get row -1 and gate 0.
+__device__ __forceinline__ int padded_count(int c) { return c < 64 ? 64 : (c + 63) / 64 * 64; }
+
 __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__ gates,
                                                        const int* __restrict__ counts, int* __restrict__ offsets,
                                                        int* __restrict__ mtile_prefix, int* __restrict__ totals,
                                                        int* __restrict__ slot_row, float* __restrict__ slot_gate,
-                                                       int* __restrict__ slot_of, int B, int T, int Ne,
-                                                       int tile_rows) {
+                                                       int* __restrict__ slot_of, int* __restrict__ cnt_pad, int B,
+                                                       int T, int Ne, int tile_rows) {
     pdl_enter();
     __shared__ int s_off;
     __shared__ int s_warp[32];
@@ -167,10 +173,12 @@ __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__
     const int g = blockIdx.x;
     const int t = g / Ne, j = g - t * Ne;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const bool pad = cnt_pad != nullptr;
+    auto rows_of = [&](int c) { return pad ? padded_count(c) : c; };
     if (warp == 0) {
         int off = 0, mt = 0;
         for (int q = lane; q < g; q += 32) {
-            const int c = __ldcg(counts + q);
+            const int c = rows_of(__ldcg(counts + q));
             off += c;
             mt += (c + tile_rows - 1) / tile_rows;
         }
@@ -180,8 +188,9 @@ __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__
             s_off = off;
             offsets[g] = off;
             mtile_prefix[g] = mt;
+            if (pad) cnt_pad[g] = rows_of(__ldcg(counts + g));
             if (g == G - 1) {
-                const int c = __ldcg(counts + g);
+                const int c = rows_of(__ldcg(counts + g));
                 mtile_prefix[G] = mt + (c + tile_rows - 1) / tile_rows;
                 totals[0] = off + c;
                 totals[1] = mt + (c + tile_rows - 1) / tile_rows;
@@ -190,6 +199,13 @@ __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__
     }
     __syncthreads();
     const int off = s_off;
+    if (pad) {   // the padding slots after the expert's active entries
+        const int c = __ldcg(counts + g);
+        for (int q = c + threadIdx.x; q < padded_count(c); q += blockDim.x) {
+            slot_row[off + q] = -1;
+            slot_gate[off + q] = 0.f;
+        }
+    }
     int base = 0;
     for (int b0 = 0; b0 < B; b0 += 1024) {
         const int b = b0 + threadIdx.x;
@@ -221,7 +237,8 @@ __global__ void __launch_bounds__(1024) compact_kernel(const float* __restrict__
     }
 }
 
-// Sg[slot] = S[slot_row[slot]]: one warp per active slot, 16-byte vectors.
+// Sg[slot] = S[slot_row[slot]] (zeros for a padding slot, row -1): one warp
+// per slot, 16-byte vectors.
 __global__ void __launch_bounds__(kThreads) gather_kernel(const __nv_bfloat16* __restrict__ S,
                                                           const int* __restrict__ slot_row,
                                                           const int* __restrict__ totals,
@@ -232,8 +249,13 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const __nv_bfloat16* _
     const int nv = D / 8;
     for (long long s = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); s < n;
          s += (long long)gridDim.x * (blockDim.x >> 5)) {
-        const uint4* src = reinterpret_cast<const uint4*>(S + (long long)__ldcg(slot_row + s) * D);
+        const int row = __ldcg(slot_row + s);
         uint4* dst = reinterpret_cast<uint4*>(Sg + s * D);
+        if (row < 0) {
+            for (int v = lane; v < nv; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+            continue;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(S + (long long)row * D);
         for (int v0 = lane; v0 < nv; v0 += 128) {   // up to four loads in flight per lane
             uint4 t[4];
 #pragma unroll
@@ -361,8 +383,9 @@ cudaError_t launch_moe_route(const void* S, const float* Wr, const float* br, co
     else if (Ne <= 16) RM_ROUTE(16)
     else RM_ROUTE(32)
 #undef RM_ROUTE
+    if (tile_rows == 0) return cudaSuccess;   // gates only (DTSI's second router)
     return launch_pdl(compact_kernel, T * Ne, 1024, 0, s, w.gates, w.counts, w.offsets, w.mtile_prefix, w.totals,
-                      w.slot_row, w.slot_gate, w.slot_of, B, T, Ne, tile_rows);
+                      w.slot_row, w.slot_gate, w.slot_of, w.cnt_pad, B, T, Ne, tile_rows);
 }
 
 cudaError_t launch_moe_gather(const void* S, const MoeWork& w, int B, int T, int D, int Ne, cudaStream_t s) {
@@ -386,6 +409,301 @@ cudaError_t launch_moe_combine(const MoeWork& w, const void* resid, void* out, f
     if (nvl <= 4) return launch_pdl(combine_kernel<4>, grid, kThreads, 0, s, eg, w.slot_of, rs, o, stats, rows, D, Ne);
     if (nvl <= 8) return launch_pdl(combine_kernel<8>, grid, kThreads, 0, s, eg, w.slot_of, rs, o, stats, rows, D, Ne);
     return cudaErrorInvalidValue;
+}
+
+}  // namespace rm
+
+// ------------------------------------------------------ training (backward)
+// Gradients of v = sum_j G_j e_j (fun-rec "Rankmixer: 硬件效率优化", section
+// Sparse MoE扩展, ReLU routing) for the active entries, and of the routers
+// G = ReLU(Wr s + br): dG_j = dV . e_j, de_j = G_j dV, dR_j = dG_j [R_j > 0]
+// (+ lambda for L_reg on these gates), DTSI's second router dR_inf_j =
+// lambda [R_inf_j > 0].
+namespace rm {
+namespace {
+
+// One warp per row r = (b, t): dV's vectors stay in registers; for each
+// active expert j (ascending) the gated output row Eg = G_j e_j gives
+// dG_j = dV . Eg / G_j (a fixed-order warp sum), and de_j = G_j dV is
+// written to the expert's slot.  Lane j writes dR[r, j] (0 when inactive)
+// and, under DTSI, dRinf[r, j].
+template <int NVL>
+__global__ void __launch_bounds__(kThreads) moe_bwd_gate_kernel(
+    const __nv_bfloat16* __restrict__ dV, const __nv_bfloat16* __restrict__ Eg, const int* __restrict__ slot_of,
+    const float* __restrict__ slot_gate, const float* __restrict__ gates_inf, float lambda,
+    __nv_bfloat16* __restrict__ dEg, float* __restrict__ dR, float* __restrict__ dRinf, long long rows, int D,
+    int Ne) {
+    pdl_enter();
+    const int lane = threadIdx.x & 31;
+    const long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (r >= rows) return;   // warp-uniform
+    const int nv = D / 8;
+    const int myslot = lane < Ne ? __ldcg(slot_of + r * Ne + lane) : -1;
+    const unsigned act = __ballot_sync(0xffffffffu, myslot >= 0);
+    float2 dv[NVL][4];
+#pragma unroll
+    for (int i = 0; i < NVL; ++i) {
+        const int v = lane + 32 * i;
+        if (v < nv) unpack_pairs(__ldcg(reinterpret_cast<const uint4*>(dV + r * D) + v), dv[i]);
+    }
+    float my_dr = 0.f;
+    for (unsigned m = act; m; m &= m - 1) {   // active experts, ascending j
+        const int j = __ffs(m) - 1;
+        const int slot = __shfl_sync(0xffffffffu, myslot, j);
+        const float gate = __ldcg(slot_gate + slot);
+        const uint4* src = reinterpret_cast<const uint4*>(Eg + (long long)slot * D);
+        uint4 x[NVL];
+#pragma unroll
+        for (int i = 0; i < NVL; ++i)
+            if (lane + 32 * i < nv) x[i] = __ldcg(src + lane + 32 * i);
+        float2 a = f2(0.f);
+        uint4* dst = reinterpret_cast<uint4*>(dEg + (long long)slot * D);
+#pragma unroll
+        for (int i = 0; i < NVL; ++i) {
+            if (lane + 32 * i < nv) {
+                float2 e[4], de[4];
+                unpack_pairs(x[i], e);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    a = f2_fma(dv[i][q], e[q], a);
+                    de[q] = f2_mul(dv[i][q], f2(gate));
+                }
+                dst[lane + 32 * i] = pack_pairs(de);
+            }
+        }
+        const float dG = warp_sum(a.x + a.y) / gate;
+        if (lane == j) my_dr = dG + (gates_inf ? 0.f : lambda);
+    }
+    if (lane < Ne) {
+        dR[r * Ne + lane] = my_dr;
+        if (dRinf) dRinf[r * Ne + lane] = __ldcg(gates_inf + r * Ne + lane) > 0.f ? lambda : 0.f;
+    }
+}
+
+// Zero the rows of the padding slots (row -1) of a compacted [slots, D] array.
+__global__ void __launch_bounds__(kThreads) zero_pad_rows_kernel(__nv_bfloat16* __restrict__ dst,
+                                                                 const int* __restrict__ slot_row,
+                                                                 const int* __restrict__ totals, int D) {
+    pdl_enter();
+    const int lane = threadIdx.x & 31;
+    const int n = __ldcg(totals);
+    const int nv = D / 8;
+    for (long long s = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); s < n;
+         s += (long long)gridDim.x * (blockDim.x >> 5)) {
+        if (__ldcg(slot_row + s) >= 0) continue;   // warp-uniform
+        uint4* d = reinterpret_cast<uint4*>(dst + s * D);
+        for (int v = lane; v < nv; v += 32) d[v] = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// dS[r] = dZ[r] + sum over active j (ascending) of dSg[slot(r, j)]
+//         + sum_j dR[r, j] Wr[t, j, :] + sum_j dRinf[r, j] Wrinf[t, j, :]
+// (one warp per row, fp32 pairs, fixed order; zero router terms skipped).
+template <int NVL>
+__global__ void __launch_bounds__(kThreads) moe_bwd_combine_kernel(
+    const __nv_bfloat16* __restrict__ dZ, const __nv_bfloat16* __restrict__ dSg, const int* __restrict__ slot_of,
+    const float* __restrict__ dR, const float* __restrict__ Wr, const float* __restrict__ dRinf,
+    const float* __restrict__ Wrinf, __nv_bfloat16* __restrict__ dS, long long rows, int T, int D, int Ne) {
+    pdl_enter();
+    const int lane = threadIdx.x & 31;
+    const long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (r >= rows) return;   // warp-uniform
+    const int t = (int)(r % T);
+    const int nv = D / 8;
+    const int myslot = lane < Ne ? __ldcg(slot_of + r * Ne + lane) : -1;
+    const unsigned act = __ballot_sync(0xffffffffu, myslot >= 0);
+    float2 acc[NVL][4];
+#pragma unroll
+    for (int i = 0; i < NVL; ++i) {
+        const int v = lane + 32 * i;
+        if (v < nv) unpack_pairs(__ldcg(reinterpret_cast<const uint4*>(dZ + r * D) + v), acc[i]);
+    }
+    for (unsigned m = act; m; m &= m - 1) {
+        const int slot = __shfl_sync(0xffffffffu, myslot, __ffs(m) - 1);
+        const uint4* src = reinterpret_cast<const uint4*>(dSg + (long long)slot * D);
+        uint4 x[NVL];
+#pragma unroll
+        for (int i = 0; i < NVL; ++i)
+            if (lane + 32 * i < nv) x[i] = __ldcg(src + lane + 32 * i);
+#pragma unroll
+        for (int i = 0; i < NVL; ++i) {
+            if (lane + 32 * i < nv) {
+                float2 p[4];
+                unpack_pairs(x[i], p);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[i][q] = f2_add(acc[i][q], p[q]);
+            }
+        }
+    }
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {   // the routing router, then DTSI's second router
+        const float* d = pass ? dRinf : dR;
+        const float* W = pass ? Wrinf : Wr;
+        if (!d) continue;
+        const float my = lane < Ne ? __ldcg(d + r * Ne + lane) : 0.f;
+        for (int j = 0; j < Ne; ++j) {
+            const float dr = __shfl_sync(0xffffffffu, my, j);
+            if (dr == 0.f) continue;   // warp-uniform
+            const float* w = W + ((long long)t * Ne + j) * D;
+#pragma unroll
+            for (int i = 0; i < NVL; ++i) {
+                const int v = lane + 32 * i;
+                if (v < nv) {
+                    const float4 w0 = __ldg(reinterpret_cast<const float4*>(w) + 2 * v);
+                    const float4 w1 = __ldg(reinterpret_cast<const float4*>(w) + 2 * v + 1);
+                    const float2 wp[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w), make_float2(w1.x, w1.y),
+                                          make_float2(w1.z, w1.w)};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[i][q] = f2_fma(f2(dr), wp[q], acc[i][q]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NVL; ++i)
+        if (lane + 32 * i < nv) reinterpret_cast<uint4*>(dS + r * D)[lane + 32 * i] = pack_pairs(acc[i]);
+}
+
+// Router weight-gradient partials over blocks of RB samples: part[((t * nrb +
+// rb) * Ne + j) * D + d] = sum_{b in block rb} dR[b, t, j] S[b, t, d], and
+// part_b[(t * nrb + rb) * Ne + j] = sum_b dR[b, t, j] (both in ascending b).
+// Thread = 8 columns; experts in passes of 8; rows whose dR is zero skipped.
+__global__ void __launch_bounds__(kThreads) router_grad_kernel(const __nv_bfloat16* __restrict__ S,
+                                                               const float* __restrict__ dR, float* __restrict__ part,
+                                                               float* __restrict__ part_b, int B, int T, int D, int Ne,
+                                                               int RB) {
+    pdl_enter();
+    const int v = blockIdx.x * blockDim.x + threadIdx.x;
+    const int rb = blockIdx.y, nrb = gridDim.y, t = blockIdx.z;
+    const int b0 = rb * RB, b1 = min(B, b0 + RB);
+    const bool col = 8 * v < D;
+    for (int j0 = 0; j0 < Ne; j0 += 8) {
+        float a[8][8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a[jj][e] = 0.f;
+        for (int b = b0; b < b1; ++b) {
+            const long long row = (long long)b * T + t;
+            float dr[8];
+            bool any = false;
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                dr[jj] = j0 + jj < Ne ? __ldg(dR + row * Ne + j0 + jj) : 0.f;
+                any |= dr[jj] != 0.f;
+            }
+            if (!any || !col) continue;
+            float2 sp[4];
+            unpack_pairs(__ldcg(reinterpret_cast<const uint4*>(S + row * D) + v), sp);
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                if (dr[jj] != 0.f) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        a[jj][2 * q] = fmaf(dr[jj], sp[q].x, a[jj][2 * q]);
+                        a[jj][2 * q + 1] = fmaf(dr[jj], sp[q].y, a[jj][2 * q + 1]);
+                    }
+                }
+            }
+        }
+        if (col) {
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                if (j0 + jj < Ne) {
+                    float4* o = reinterpret_cast<float4*>(part + (((long long)t * nrb + rb) * Ne + j0 + jj) * D + 8 * v);
+                    o[0] = make_float4(a[jj][0], a[jj][1], a[jj][2], a[jj][3]);
+                    o[1] = make_float4(a[jj][4], a[jj][5], a[jj][6], a[jj][7]);
+                }
+            }
+        }
+    }
+    if (blockIdx.x == 0 && threadIdx.x < Ne) {
+        float sb = 0.f;
+        for (int b = b0; b < b1; ++b) sb += __ldg(dR + ((long long)b * T + t) * Ne + threadIdx.x);
+        part_b[((long long)t * nrb + rb) * Ne + threadIdx.x] = sb;
+    }
+}
+
+// loss[0] += lambda * sum of x[0 .. n) (one CTA, a fixed order: thread i sums
+// x[i], x[i + 1024], ...; then a fixed tree).
+__global__ void __launch_bounds__(1024) add_scaled_sum_kernel(const float* __restrict__ x, long long n, float lambda,
+                                                              float* __restrict__ loss) {
+    pdl_enter();
+    __shared__ float red[32];
+    float a = 0.f;
+    for (long long i = threadIdx.x; i < n; i += blockDim.x) a += __ldcg(x + i);
+    a = warp_sum(a);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = red[threadIdx.x];
+        v = warp_sum(v);
+        if (threadIdx.x == 0) loss[0] += lambda * v;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_moe_route_only(const void* S, const float* Wr, const float* br, float* gates, int* counts_scratch,
+                                  int B, int T, int D, int Ne, cudaStream_t s) {
+    MoeWork w{};
+    w.gates = gates;
+    w.counts = counts_scratch;
+    return launch_moe_route(S, Wr, br, w, B, T, D, Ne, s, 0);
+}
+
+cudaError_t launch_moe_bwd_gate(const void* dV, const MoeWork& w, const float* gates_inf, float lambda, void* dEg,
+                                float* dR, float* dRinf, int B, int T, int D, int Ne, cudaStream_t s) {
+    const long long rows = (long long)B * T;
+    const int grid = (int)((rows + kThreads / 32 - 1) / (kThreads / 32));
+    const int nvl = (D / 8 + 31) / 32;
+    const auto* dv = static_cast<const __nv_bfloat16*>(dV);
+    const auto* eg = static_cast<const __nv_bfloat16*>(w.Eg);
+    auto* de = static_cast<__nv_bfloat16*>(dEg);
+    cudaError_t e;
+#define RM_GATE(N)                                                                                                  \
+    e = launch_pdl(moe_bwd_gate_kernel<N>, grid, kThreads, 0, s, dv, eg, w.slot_of, w.slot_gate, gates_inf, lambda, \
+                   de, dR, dRinf, rows, D, Ne)
+    if (nvl <= 1) RM_GATE(1);
+    else if (nvl <= 2) RM_GATE(2);
+    else if (nvl <= 4) RM_GATE(4);
+    else if (nvl <= 8) RM_GATE(8);
+    else return cudaErrorInvalidValue;
+#undef RM_GATE
+    if (e != cudaSuccess) return e;
+    return launch_pdl(zero_pad_rows_kernel, 148 * 8, kThreads, 0, s, de, w.slot_row, w.totals, D);
+}
+
+cudaError_t launch_moe_bwd_combine(const void* dZ, const void* dSg, const MoeWork& w, const float* dR, const float* Wr,
+                                   const float* dRinf, const float* Wrinf, void* dS, int B, int T, int D, int Ne,
+                                   cudaStream_t s) {
+    const long long rows = (long long)B * T;
+    const int grid = (int)((rows + kThreads / 32 - 1) / (kThreads / 32));
+    const int nvl = (D / 8 + 31) / 32;
+    const auto* dz = static_cast<const __nv_bfloat16*>(dZ);
+    const auto* dsg = static_cast<const __nv_bfloat16*>(dSg);
+    auto* ds = static_cast<__nv_bfloat16*>(dS);
+#define RM_CMB(N)                                                                                                  \
+    return launch_pdl(moe_bwd_combine_kernel<N>, grid, kThreads, 0, s, dz, dsg, w.slot_of, dR, Wr, dRinf, Wrinf, ds, \
+                      rows, T, D, Ne)
+    if (nvl <= 1) RM_CMB(1);
+    if (nvl <= 2) RM_CMB(2);
+    if (nvl <= 4) RM_CMB(4);
+    if (nvl <= 8) RM_CMB(8);
+#undef RM_CMB
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_router_grad(const void* S, const float* dR, float* part, float* part_b, int B, int T, int D, int Ne,
+                               int RB, cudaStream_t s) {
+    const int nrb = (B + RB - 1) / RB;
+    const dim3 grid((unsigned)((D / 8 + kThreads - 1) / kThreads), (unsigned)nrb, (unsigned)T);
+    return launch_pdl(router_grad_kernel, grid, kThreads, 0, s, static_cast<const __nv_bfloat16*>(S), dR, part, part_b,
+                      B, T, D, Ne, RB);
+}
+
+cudaError_t launch_add_scaled_sum(const float* x, long long n, float lambda, float* loss, cudaStream_t s) {
+    return launch_pdl(add_scaled_sum_kernel, 1, 1024, 0, s, x, n, lambda, loss);
 }
 
 }  // namespace rm

@@ -301,6 +301,41 @@ __global__ void __launch_bounds__(kThreads) colsum_kernel(const __nv_bfloat16* A
     if (X2) store8f(part2 + o, a2);
 }
 
+// The same over variable row ranges: part[(g * nrb + rb) * N + n] = sum over
+// rows r of block rb of [0, cnt[g]) of A[(off[g] + r) * ld + n] (the
+// sparse-MoE experts' compacted rows; blocks past cnt[g] write zeros).
+__global__ void __launch_bounds__(kThreads) colsum_var_kernel(const __nv_bfloat16* A, float* part,
+                                                             const int* __restrict__ off,
+                                                             const int* __restrict__ cnt, int N, long long ld,
+                                                             int RB) {
+    pdl_enter();
+    const int v = blockIdx.x * blockDim.x + threadIdx.x;
+    if (8 * v >= N) return;
+    const int rb = blockIdx.y, nrb = gridDim.y, g = blockIdx.z;
+    const int c = __ldcg(cnt + g);
+    const long long base = __ldcg(off + g);
+    const int r0 = rb * RB, r1 = min(c, r0 + RB);
+    float a[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) a[e] = 0.f;
+    for (int r = r0; r < r1; r += 4) {   // up to four rows' loads in flight, summed in row order
+        uint4 xa[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if (r + q < r1) xa[q] = __ldcg(reinterpret_cast<const uint4*>(A + (base + r + q) * ld + 8 * v));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (r + q < r1) {
+                float x[8];
+                unpack8(xa[q], x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) a[e] += x[e];
+            }
+        }
+    }
+    store8f(part + ((long long)g * nrb + rb) * N + 8 * v, a);
+}
+
 // out[g * N + n] = sum_{j < J} part[(g * J + j) * N + n].  CTA = (32
 // columns, group g) x W warps (W = blockDim.x / 32, about J / 8 from the
 // host, at most kRedWarps); warp w sums the slices j = w, w + W, ... of its
@@ -468,12 +503,24 @@ struct rm_trainer {
     unsigned char **S, **XH1, **U, **H, **Y;
     float** RS1;
     float2** ystats;
+    // per block, sparse MoE (Ne > 0): routing and compaction (slot lists
+    // padded per expert to a multiple of 64), DTSI's second router's gates,
+    // and the compacted expert rows (S, activation input U, hidden H, gated
+    // output)
+    rm::MoeWork* moe;
+    float** gates_inf;
+    long long rows_max;      // compacted rows allocated per array
+    float lambda;            // L_reg weight
     // shared
     float *pooled, *dlogit, *lterm, *gpool;
     unsigned char *dY, *dU, *dS, *dX;
     float *pg, *pb, *pdb, *pcol, *pcol2;
     float* sk_ws;
     int* sk_cnt;
+    // shared, sparse MoE backward
+    unsigned char *dEg, *dUg, *dSg;
+    float *dR, *dRinf, *prt, *prt_b;
+    int* cnt_scratch;
 };
 
 namespace {
@@ -495,44 +542,154 @@ rm_status cuda_st(cudaError_t e) { return e == cudaSuccess ? RM_OK : RM_ERR_CUDA
 
 }  // namespace
 
+namespace {
+
+// Backward of one sparse-MoE FFN given dL/dY in t->dY (fun-rec "Rankmixer:
+// 硬件效率优化", section Sparse MoE扩展): the gates' and the experts'
+// gradients over the compacted (padded) slot lists, the experts' weight
+// gradients as variable-K grouped products, the routers' gradients (L_reg on
+// the routing gates, or on DTSI's second router), and dL/dS into t->dS.
+cudaError_t moe_backward(rm_trainer* t, const rm_block_weights& w, const rm_block_grads& gr, int l, int B,
+                         cudaStream_t s) {
+    const rm_config& c = t->cfg;
+    const int T = c.T, D = c.D, Hd = c.hidden, Ne = c.n_experts, G = T * Ne;
+    const rm::DeviceErr err = terr(t);
+    const uint64_t budget = t->budget_ns;
+    const rm::MoeWork& mw = t->moe[l];
+    const float* ginf = w.Wr_infer ? t->gates_inf[l] : nullptr;
+    float* dRinf = ginf ? t->dRinf : nullptr;
+    cudaError_t e = rm::launch_moe_bwd_gate(t->dY, mw, ginf, t->lambda, t->dEg, t->dR, dRinf, B, T, D, Ne, s);
+    if (e != cudaSuccess) return e;
+    // dU_j = (de_j W2_j) * act'(U_j) over the expert's slots
+    rm::GroupedGemm gh{};
+    gh.G = G; gh.M = 0; gh.N = Hd; gh.K = D;
+    gh.A = t->dEg; gh.a_ld = D; gh.a_rows_total = t->rows_max;
+    gh.W = w.W2; gh.w_mn = true; gh.w_gstride = (long long)D * Hd; gh.w_ld = Hd;
+    gh.out = t->dUg; gh.o_ld = Hd;
+    gh.resid = t->U[l]; gh.r_ld = Hd;
+    gh.epi = rm::dact_epi_for_act(c.act);
+    gh.var_cg = 1;
+    gh.grp_cnt = mw.cnt_pad; gh.grp_off = mw.offsets; gh.mtile_prefix = mw.mtile_prefix;
+    if ((e = rm::launch_gemm_tc(gh, err, budget, t->num_sms, s)) != cudaSuccess) return e;
+    // dW2_j = de_j^T H_j (fp32), K = the expert's padded slot count
+    rm::GroupedGemm gw2{};
+    gw2.G = G; gw2.M = D; gw2.N = Hd; gw2.K = 64;
+    gw2.A = t->dEg; gw2.a_mn = true; gw2.a_ld = D; gw2.a_rows_total = t->rows_max;
+    gw2.W = mw.Hg; gw2.w_mn = true; gw2.w_ld = Hd;
+    gw2.out = gr.W2; gw2.o_gstride = (long long)D * Hd; gw2.o_ld = Hd;
+    gw2.epi = rm::EPI_F32;
+    gw2.vark = true; gw2.vark_cnt = mw.cnt_pad; gw2.grp_off = mw.offsets;
+    if ((e = rm::launch_gemm_tc(gw2, err, budget, t->num_sms, s)) != cudaSuccess) return e;
+    // db2_j, db1_j: column sums over the expert's slots (padding rows are zero)
+    const int nrb_g = (B + 64 + rm::kColRows - 1) / rm::kColRows;
+    e = rm::launch_pdl(rm::colsum_var_kernel, dim3((D / 8 + rm::kThreads - 1) / rm::kThreads, nrb_g, G),
+                       dim3(rm::kThreads), 0, s, (const __nv_bfloat16*)t->dEg, t->pcol, (const int*)mw.offsets,
+                       (const int*)mw.cnt_pad, D, (long long)D, rm::kColRows);
+    if (e != cudaSuccess) return e;
+    if ((e = rm::launch_reduce_parts((const float*)t->pcol, gr.b2, G, nrb_g, D, s)) != cudaSuccess) return e;
+    // dS_j = dU_j W1_j (plain bf16 rows)
+    rm::GroupedGemm gs{};
+    gs.G = G; gs.M = 0; gs.N = D; gs.K = Hd;
+    gs.A = t->dUg; gs.a_ld = Hd; gs.a_rows_total = t->rows_max;
+    gs.W = w.W1; gs.w_mn = true; gs.w_gstride = (long long)Hd * D; gs.w_ld = D;
+    gs.out = t->dSg; gs.o_ld = D;
+    gs.epi = rm::EPI_BIAS_GATE;   // no bias, no gate: the product itself
+    gs.var_cg = 1;
+    gs.grp_cnt = mw.cnt_pad; gs.grp_off = mw.offsets; gs.mtile_prefix = mw.mtile_prefix;
+    if ((e = rm::launch_gemm_tc(gs, err, budget, t->num_sms, s)) != cudaSuccess) return e;
+    // dW1_j = dU_j^T S_j (fp32)
+    rm::GroupedGemm gw1{};
+    gw1.G = G; gw1.M = Hd; gw1.N = D; gw1.K = 64;
+    gw1.A = t->dUg; gw1.a_mn = true; gw1.a_ld = Hd; gw1.a_rows_total = t->rows_max;
+    gw1.W = mw.Sg; gw1.w_mn = true; gw1.w_ld = D;
+    gw1.out = gr.W1; gw1.o_gstride = (long long)Hd * D; gw1.o_ld = D;
+    gw1.epi = rm::EPI_F32;
+    gw1.vark = true; gw1.vark_cnt = mw.cnt_pad; gw1.grp_off = mw.offsets;
+    if ((e = rm::launch_gemm_tc(gw1, err, budget, t->num_sms, s)) != cudaSuccess) return e;
+    e = rm::launch_pdl(rm::colsum_var_kernel, dim3((Hd / 8 + rm::kThreads - 1) / rm::kThreads, nrb_g, G),
+                       dim3(rm::kThreads), 0, s, (const __nv_bfloat16*)t->dUg, t->pcol, (const int*)mw.offsets,
+                       (const int*)mw.cnt_pad, Hd, (long long)Hd, rm::kColRows);
+    if (e != cudaSuccess) return e;
+    if ((e = rm::launch_reduce_parts((const float*)t->pcol, gr.b1, G, nrb_g, Hd, s)) != cudaSuccess) return e;
+    // router gradients: dWr[t, j] = sum_b dR[b, t, j] s_bt, dbr[t, j] = sum_b dR[b, t, j]
+    const int nrb_b = (B + rm::kColRows - 1) / rm::kColRows;
+    for (int pass = 0; pass < (ginf ? 2 : 1); ++pass) {
+        const float* dR = pass ? dRinf : t->dR;
+        e = rm::launch_router_grad(t->S[l], dR, t->prt, t->prt_b, B, T, D, Ne, rm::kColRows, s);
+        if (e != cudaSuccess) return e;
+        if ((e = rm::launch_reduce_parts((const float*)t->prt, pass ? gr.Wr_infer : gr.Wr, T, nrb_b, Ne * D, s)) !=
+            cudaSuccess)
+            return e;
+        if ((e = rm::launch_reduce_parts((const float*)t->prt_b, pass ? gr.br_infer : gr.br, T, nrb_b, Ne, s)) !=
+            cudaSuccess)
+            return e;
+    }
+    // dS = dY (the residual) + sum_j dS_j + the routers' terms
+    return rm::launch_moe_bwd_combine(t->dY, t->dSg, mw, t->dR, w.Wr, dRinf, w.Wr_infer, t->dS, B, T, D, Ne, s);
+}
+
+}  // namespace
+
 extern "C" {
+
+static void free_trainer(rm_trainer* t) {
+    if (!t) return;
+    if (t->ws) cudaFree(t->ws);
+    delete[] t->S;
+    delete[] t->RS1;
+    delete[] t->ystats;
+    delete[] t->moe;
+    delete[] t->gates_inf;
+    delete t;
+}
 
 rm_status rm_train_create(const rm_config* cfg, rm_trainer** out) {
     if (!cfg || !out) return RM_ERR_INVALID_ARG;
     *out = nullptr;
     const rm_config c = *cfg;
-    if (c.B_max < 8 || c.T < 1 || c.D < 1 || c.hidden < 1 || c.L < 1) return RM_ERR_INVALID_ARG;
-    if (c.dtype != RM_BF16 || c.n_experts != 0 || !c.mix_addnorm) return RM_ERR_UNSUPPORTED;
+    if (c.B_max < 8 || c.T < 1 || c.D < 1 || c.hidden < 1 || c.L < 1 || c.n_experts < 0) return RM_ERR_INVALID_ARG;
+    if (c.dtype != RM_BF16 || !c.mix_addnorm || c.n_experts > 32) return RM_ERR_UNSUPPORTED;
     if (c.act != RM_ACT_GELU_TANH && c.act != RM_ACT_GELU_ERF && c.act != RM_ACT_RELU) return RM_ERR_INVALID_ARG;
     if (c.T > 64 || c.D % c.T || c.D % 64 || c.hidden % 64 || c.D > 2048 || (c.D / c.T) % 8) return RM_ERR_UNSUPPORTED;
     if (!rm::mix_ln_sample_fits(RM_BF16, c.T, c.D)) return RM_ERR_UNSUPPORTED;
     const int rs = rm::mix_pad_stride(c.D, c.D / c.T);
     if (rm::ln1_bwd_smem(c.T, c.D, rs) > 227 * 1024 - 1024) return RM_ERR_UNSUPPORTED;
+    const int Ne = c.n_experts;
+    const int G = c.T * Ne;
+    // (T <= 64 and Ne <= 32: at most 2048 expert groups, the grouped GEMM's limit)
     rm_trainer* t = new (std::nothrow) rm_trainer();
     if (!t) return RM_ERR_OOM;
     t->cfg = c;
     t->budget_ns = 1000000000ull;
+    t->lambda = 0.f;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&t->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-        delete t;
+        free_trainer(t);
         return RM_ERR_CUDA;
     }
-    t->stat_P = c.D / 64;
+    // the sparse-MoE combine writes whole-row statistics; the dense second
+    // projection writes one partial per 64 columns
+    t->stat_P = Ne ? 1 : c.D / 64;
     t->SB = 32;
     t->nsb = (c.B_max + t->SB - 1) / t->SB;
-    const size_t L = (size_t)c.L, BTD = (size_t)c.B_max * c.T * c.D, TBH = (size_t)c.T * c.B_max * c.hidden;
+    const size_t L = (size_t)c.L, BTD = (size_t)c.B_max * c.T * c.D;
+    const size_t TBH = Ne ? 0 : (size_t)c.T * c.B_max * c.hidden;
+    const size_t BTN = (size_t)c.B_max * c.T * Ne;                 // (sample, token, expert) entries
+    t->rows_max = (long long)BTN + 64LL * G;                        // padded slot lists
+    const size_t RM = (size_t)t->rows_max;
     const size_t nrb_rows = (size_t)((c.B_max * c.T + rm::kColRows - 1) / rm::kColRows);
     const size_t nrb_b = (size_t)((c.B_max + rm::kColRows - 1) / rm::kColRows);
-    const size_t col_parts = std::max(nrb_rows * c.D, nrb_b * (size_t)c.T * c.hidden);
+    const size_t nrb_g = (size_t)((c.B_max + 64 + rm::kColRows - 1) / rm::kColRows);   // rows per expert <= B + 63
+    size_t col_parts = std::max(nrb_rows * c.D, nrb_b * (size_t)c.T * c.hidden);
+    if (Ne) col_parts = std::max(col_parts, nrb_g * (size_t)G * std::max(c.D, c.hidden));
     t->S = new (std::nothrow) unsigned char*[5 * L];
     t->RS1 = new (std::nothrow) float*[L];
     t->ystats = new (std::nothrow) float2*[L];
-    if (!t->S || !t->RS1 || !t->ystats) {
-        delete[] t->S;
-        delete[] t->RS1;
-        delete[] t->ystats;
-        delete t;
+    t->moe = new (std::nothrow) rm::MoeWork[L];
+    t->gates_inf = new (std::nothrow) float*[L];
+    if (!t->S || !t->RS1 || !t->ystats || !t->moe || !t->gates_inf) {
+        free_trainer(t);
         return RM_ERR_OOM;
     }
     t->XH1 = t->S + L;
@@ -552,6 +709,25 @@ rm_status rm_train_create(const rm_config* cfg, rm_trainer** out) {
             t->H[l] = carve<unsigned char>(base, off, TBH * 2);
             t->Y[l] = carve<unsigned char>(base, off, BTD * 2);
             t->ystats[l] = carve<float2>(base, off, (size_t)c.B_max * c.T * t->stat_P * 8);
+            rm::MoeWork& m = t->moe[l];
+            m = rm::MoeWork{};
+            t->gates_inf[l] = nullptr;
+            if (Ne) {
+                m.gates = carve<float>(base, off, BTN * 4);
+                m.counts = carve<int>(base, off, (size_t)G * 4);
+                m.offsets = carve<int>(base, off, (size_t)G * 4);
+                m.cnt_pad = carve<int>(base, off, (size_t)G * 4);
+                m.mtile_prefix = carve<int>(base, off, (size_t)(G + 1) * 4);
+                m.totals = carve<int>(base, off, 2 * 4);
+                m.slot_row = carve<int>(base, off, RM * 4);
+                m.slot_gate = carve<float>(base, off, RM * 4);
+                m.slot_of = carve<int>(base, off, BTN * 4);
+                m.Sg = carve<unsigned char>(base, off, RM * c.D * 2);
+                m.Hg = carve<unsigned char>(base, off, RM * c.hidden * 2);
+                m.Eg = carve<unsigned char>(base, off, RM * c.D * 2);
+                t->U[l] = carve<unsigned char>(base, off, RM * c.hidden * 2);   // the experts' activation input
+                t->gates_inf[l] = carve<float>(base, off, BTN * 4);
+            }
         }
         t->pooled = carve<float>(base, off, (size_t)c.B_max * c.D * 4);
         t->dlogit = carve<float>(base, off, (size_t)c.B_max * 4);
@@ -568,24 +744,28 @@ rm_status rm_train_create(const rm_config* cfg, rm_trainer** out) {
         t->pcol2 = carve<float>(base, off, col_parts * 4);
         t->sk_cnt = carve<int>(base, off, rm::gemm_tc_split_cnt_ints(t->num_sms) * sizeof(int));
         t->sk_ws = carve<float>(base, off, rm::gemm_tc_split_ws_bytes(t->num_sms));
+        if (Ne) {
+            t->dEg = carve<unsigned char>(base, off, RM * c.D * 2);
+            t->dUg = carve<unsigned char>(base, off, RM * c.hidden * 2);
+            t->dSg = carve<unsigned char>(base, off, RM * c.D * 2);
+            t->dR = carve<float>(base, off, BTN * 4);
+            t->dRinf = carve<float>(base, off, BTN * 4);
+            t->prt = carve<float>(base, off, (size_t)c.T * nrb_b * Ne * c.D * 4);
+            t->prt_b = carve<float>(base, off, (size_t)c.T * nrb_b * Ne * 4);
+            t->cnt_scratch = carve<int>(base, off, (size_t)G * 4);
+        }
         if (pass == 0) {
             t->ws_bytes = off;
             if (cudaMalloc(&t->ws, off) != cudaSuccess) {
                 cudaGetLastError();
-                delete[] t->S;
-                delete[] t->RS1;
-                delete[] t->ystats;
-                delete t;
+                t->ws = nullptr;
+                free_trainer(t);
                 return RM_ERR_OOM;
             }
         }
     }
     if (cudaMemset(t->ws, 0, t->ws_bytes) != cudaSuccess) {
-        cudaFree(t->ws);
-        delete[] t->S;
-        delete[] t->RS1;
-        delete[] t->ystats;
-        delete t;
+        free_trainer(t);
         return RM_ERR_CUDA;
     }
     *out = t;
@@ -595,11 +775,13 @@ rm_status rm_train_create(const rm_config* cfg, rm_trainer** out) {
 rm_status rm_train_destroy(rm_trainer* t) {
     if (!t) return RM_ERR_INVALID_ARG;
     cudaDeviceSynchronize();
-    cudaFree(t->ws);
-    delete[] t->S;
-    delete[] t->RS1;
-    delete[] t->ystats;
-    delete t;
+    free_trainer(t);
+    return RM_OK;
+}
+
+rm_status rm_train_set_reg(rm_trainer* t, float lambda) {
+    if (!t || !(lambda >= 0.f)) return RM_ERR_INVALID_ARG;
+    t->lambda = lambda;
     return RM_OK;
 }
 
@@ -632,9 +814,14 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
         if (!aligned16(g.W1) || !aligned16(g.b1) || !aligned16(g.W2) || !aligned16(g.b2) || !aligned16(g.ln1_g) ||
             !aligned16(g.ln1_b) || !aligned16(g.ln2_g) || !aligned16(g.ln2_b))
             return RM_ERR_INVALID_ARG;
+        if (c.n_experts) {   // routers (and DTSI's second router, when given)
+            if (!aligned16(w.Wr) || !w.br || !aligned16(g.Wr) || !g.br) return RM_ERR_INVALID_ARG;
+            if (w.Wr_infer && (!aligned16(w.Wr_infer) || !w.br_infer || !aligned16(g.Wr_infer) || !g.br_infer))
+                return RM_ERR_INVALID_ARG;
+        }
     }
     cudaStream_t s = stream;
-    const int T = c.T, D = c.D, Hd = c.hidden, L = c.L, P = t->stat_P;
+    const int T = c.T, D = c.D, Hd = c.hidden, L = c.L, P = t->stat_P, Ne = c.n_experts, G = T * Ne;
     const rm::DeviceErr err = terr(t);
     const uint64_t budget = t->budget_ns;
     cudaError_t e = cudaSuccess;
@@ -652,6 +839,40 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
                                  prev ? prev->ln2_b : nullptr, rm::RowStats{l ? t->ystats[l - 1] : nullptr, P},
                                  w.ln1_g, w.ln1_b, t->S[l], B, T, D, c.ln_eps, 1, t->num_sms, err, budget, s,
                                  t->XH1[l], t->RS1[l]));
+        if (Ne) {
+            // sparse MoE: route (slot lists padded per expert to a multiple of
+            // 64), DTSI's second router, gather, the expert projections (the
+            // first also stores its activation input), combine
+            rm::MoeWork& mw = t->moe[l];
+            RM_TRY(rm::launch_moe_route(t->S[l], w.Wr, w.br, mw, B, T, D, Ne, s, 128));
+            if (w.Wr_infer)
+                RM_TRY(rm::launch_moe_route_only(t->S[l], w.Wr_infer, w.br_infer, t->gates_inf[l], t->cnt_scratch, B, T,
+                                                 D, Ne, s));
+            RM_TRY(rm::launch_moe_gather(t->S[l], mw, B, T, D, Ne, s));
+            rm::GroupedGemm e1{};
+            e1.G = G; e1.M = 0; e1.N = Hd; e1.K = D;
+            e1.A = mw.Sg; e1.a_ld = D; e1.a_rows_total = t->rows_max;
+            e1.W = w.W1;
+            e1.out = mw.Hg; e1.o_ld = Hd;
+            e1.resid = t->U[l]; e1.r_ld = Hd;   // the activation input, stored
+            e1.bias = static_cast<const float*>(w.b1);
+            e1.epi = rm::epi_for_act(c.act);
+            e1.var_cg = 1;
+            e1.grp_cnt = mw.cnt_pad; e1.grp_off = mw.offsets; e1.mtile_prefix = mw.mtile_prefix;
+            RM_TRY(rm::launch_gemm_tc(e1, err, budget, t->num_sms, s));
+            rm::GroupedGemm e2 = e1;
+            e2.N = D; e2.K = Hd;
+            e2.A = mw.Hg; e2.a_ld = Hd;
+            e2.W = w.W2;
+            e2.out = mw.Eg; e2.o_ld = D;
+            e2.resid = nullptr; e2.r_ld = 0;
+            e2.bias = static_cast<const float*>(w.b2);
+            e2.gate = mw.slot_gate;
+            e2.epi = rm::EPI_BIAS_GATE;
+            RM_TRY(rm::launch_gemm_tc(e2, err, budget, t->num_sms, s));
+            RM_TRY(rm::launch_moe_combine(mw, t->S[l], t->Y[l], t->ystats[l], B, T, D, Ne, s));
+            continue;
+        }
         rm::GroupedGemm g1{};
         g1.G = T; g1.M = B; g1.N = Hd; g1.K = D;
         g1.A = t->S[l]; g1.a_gstride = D; g1.a_ld = (long long)T * D;
@@ -686,6 +907,10 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
     RM_TRY(rm::launch_pdl(rm::head_grad_kernel, dim3((D + 31) / 32), dim3(32 * rm::kRedWarps), 0, s,
                           (const float*)t->pooled, hw, (const float*)t->dlogit, (const float*)t->lterm, dhead_w,
                           dhead_b, loss, t->gpool, B, D, 1.0f / T));
+    if (Ne && t->lambda > 0.f)   // + lambda L_reg: the regularised gates of every MoE block, in block order
+        for (int l = 0; l < L; ++l)
+            RM_TRY(rm::launch_add_scaled_sum(blocks[l].Wr_infer ? t->gates_inf[l] : t->moe[l].gates,
+                                             (long long)B * T * Ne, t->lambda, loss, s));
 
     // ------------------------------------------------------------ backward
     const int nsb = (B + t->SB - 1) / t->SB;
@@ -709,6 +934,9 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
                                   P, w.ln2_g, c.ln_eps, dY, t->pg, t->pb, t->pdb, B, T, D, t->SB));
         RM_TRY(rm::launch_reduce_parts((const float*)t->pg, gr.ln2_g, 1, T * nsb, D, s));
         RM_TRY(rm::launch_reduce_parts((const float*)t->pb, gr.ln2_b, 1, T * nsb, D, s));
+        if (Ne) {
+            RM_TRY(moe_backward(t, w, gr, l, B, s));
+        } else {
         RM_TRY(rm::launch_reduce_parts((const float*)t->pdb, gr.b2, T, nsb, D, s));
         // dU = (dY W2_t) * act'(U)
         rm::GroupedGemm gh{};
@@ -754,6 +982,7 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
         gw1.epi = rm::EPI_F32;
         gw1.sk_ws = t->sk_ws; gw1.sk_cnt = t->sk_cnt;
         RM_TRY(rm::launch_gemm_tc(gw1, err, budget, t->num_sms, s));
+        }
         // dgamma1 = sum dS * xhat1, dbeta1 = sum dS over every row
         const int nrb = (B * T + rm::kColRows - 1) / rm::kColRows;
         RM_TRY(rm::launch_pdl(rm::colsum_kernel, dim3((D / 8 + rm::kThreads - 1) / rm::kThreads, nrb, 1),

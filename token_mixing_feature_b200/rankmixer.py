@@ -28,6 +28,7 @@ EXPORTED = (
     "rm_profile_begin", "rm_profile_end", "rm_kernel_name", "rm_pffn_forward_static",
     "rm_stack_forward_host_async", "rm_host_wait",
     "rm_train_create", "rm_train_destroy", "rm_train_workspace_bytes", "rm_train_step", "rm_train_sync_status",
+    "rm_train_set_reg",
 )
 RM_STATIC_SCRATCH_BYTES = 16 << 20
 RM_K_COUNT = 11
@@ -42,11 +43,12 @@ class rm_config(ctypes.Structure):
 
 class rm_block_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("W1", "b1", "W2", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b", "Wr", "br")]
+                ("W1", "b1", "W2", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b", "Wr", "br", "Wr_infer", "br_infer")]
 
 
 class rm_block_grads(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("W1", "b1", "W2", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b")]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W1", "b1", "W2", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b",
+                                                "Wr", "br", "Wr_infer", "br_infer")]
 
 
 class RankMixerError(RuntimeError):
@@ -91,6 +93,7 @@ def _load() -> ctypes.CDLL:
         "rm_train_step": (st, [vp, ctypes.POINTER(rm_block_weights), vp, vp, vp, vp, ctypes.POINTER(rm_block_grads),
                                vp, vp, vp, vp, vp, ci, vp]),
         "rm_train_sync_status": (st, [vp, vp]),
+        "rm_train_set_reg": (st, [vp, ctypes.c_float]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -325,8 +328,8 @@ class Trainer:
 
 
 def rm_train_create(B_max: int, T: int, D: int, hidden: int, L: int, ln_eps: float = 1e-5,
-                    act: str = "tanh") -> Trainer:
-    cfg = rm_config(B_max, T, D, hidden, L, 0, RM_BF16, ln_eps, ACTS[act], 1)
+                    act: str = "tanh", n_experts: int = 0) -> Trainer:
+    cfg = rm_config(B_max, T, D, hidden, L, n_experts, RM_BF16, ln_eps, ACTS[act], 1)
     out = ctypes.c_void_p()
     _check(_lib.rm_train_create(ctypes.byref(cfg), ctypes.byref(out)), "rm_train_create")
     return Trainer(out.value, cfg)
@@ -334,6 +337,10 @@ def rm_train_create(B_max: int, T: int, D: int, hidden: int, L: int, ln_eps: flo
 
 def rm_train_destroy(t: Trainer) -> None:
     t.close()
+
+
+def rm_train_set_reg(t: Trainer, reg_lambda: float) -> None:
+    _check(_lib.rm_train_set_reg(t.ptr, float(reg_lambda)), "rm_train_set_reg")
 
 
 def rm_train_workspace_bytes(t: Trainer) -> int:
