@@ -232,7 +232,7 @@ rm_status rm_pffn_forward_static(const rm_block_weights *w, const void *S, void 
                                  int D, int hidden, rm_dtype dtype, int act, int *device_status,
                                  rm_stream_t stream);
 
-/* ---- training step (dense bf16 stacks) -----------------------------------
+/* ---- training step (dense and sparse-MoE bf16 stacks) ---------------------
  * One training step of a stack of L dense RankMixer blocks with the sigmoid
  * head: the forward pass (keeping what the backward pass needs), the task loss
  * and the gradient of the loss with respect to every parameter and to the
