@@ -733,8 +733,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const long long rrow = orow * p.r_ld;
             float gate = 1.f;
             if (EPI == EPI_BIAS_GATE && row_ok && p.gate) gate = __ldcg(p.gate + orow);
+            // DACT: the activation input of the row, one 16-column chunk ahead
+            uint4 un[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+            if (DACT && row_ok && t.n0 + half * HALF < p.N) {
+                const uint4* u4 = reinterpret_cast<const uint4*>(p.resid + rrow + t.n0 + half * HALF);
+                un[0] = __ldcg(u4);
+                un[1] = __ldcg(u4 + 1);
+            }
 #pragma unroll 1
             for (int c = half * HALF; c < (half + 1) * HALF; c += 16) {
+                const uint4 uc[2] = {un[0], un[1]};
+                if (DACT && row_ok && c + 16 < (half + 1) * HALF && t.n0 + c + 16 < p.N) {
+                    const uint4* u4 = reinterpret_cast<const uint4*>(p.resid + rrow + t.n0 + c + 16);
+                    un[0] = __ldcg(u4);
+                    un[1] = __ldcg(u4 + 1);
+                }
                 float v[16];
                 tmem_ld16(tbase + (uint32_t)c, v);
                 tmem_ld_wait();
@@ -774,11 +787,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = 0.5f * v[e] * (1.0f + erff(v[e] * 0.7071067811865476f));
                     } else if (DACT) {   // acc * act'(U), U the stored activation input of the row
-                        const uint4* u4 = reinterpret_cast<const uint4*>(p.resid + rrow + n);
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {
                             float2 up[4];
-                            unpack_pairs(__ldcg(u4 + q), up);
+                            unpack_pairs(uc[q], up);
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 v[8 * q + 2 * e] *= dact<EPI>(up[e].x);

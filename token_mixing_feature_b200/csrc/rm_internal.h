@@ -189,7 +189,8 @@ cudaError_t launch_moe_bwd_combine(const void* dZ, const void* dSg, const MoeWor
 // Router weight-gradient partials over blocks of RB samples (see rm_moe.cu).
 cudaError_t launch_router_grad(const void* S, const float* dR, float* part, float* part_b, int B, int T, int D, int Ne,
                                int RB, cudaStream_t s);
-// loss[0] += lambda * sum of x[0 .. n), in a fixed order.
-cudaError_t launch_add_scaled_sum(const float* x, long long n, float lambda, float* loss, cudaStream_t s);
+// loss[0] += lambda * sum of x[0 .. n), in a fixed order; part: 256 floats of scratch.
+cudaError_t launch_add_scaled_sum(const float* x, long long n, float lambda, float* loss, float* part,
+                                  cudaStream_t s);
 
 }  // namespace rm

@@ -14,6 +14,8 @@
 // in ascending sample order.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "rm_device.cuh"
 
 namespace rm {
@@ -583,25 +585,35 @@ __global__ void __launch_bounds__(kThreads) router_grad_kernel(const __nv_bfloat
         for (int jj = 0; jj < 8; ++jj)
 #pragma unroll
             for (int e = 0; e < 8; ++e) a[jj][e] = 0.f;
-        for (int b = b0; b < b1; ++b) {
-            const long long row = (long long)b * T + t;
-            float dr[8];
-            bool any = false;
+        for (int bq = b0; bq < b1; bq += 4) {   // four rows' loads in flight, summed in row order
+            float dr[4][8];
+            uint4 sv[4];
+            bool any[4];
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                dr[jj] = j0 + jj < Ne ? __ldg(dR + row * Ne + j0 + jj) : 0.f;
-                any |= dr[jj] != 0.f;
+            for (int q = 0; q < 4; ++q) {
+                const int b = bq + q;
+                const long long row = (long long)b * T + t;
+                any[q] = false;
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    dr[q][jj] = (b < b1 && j0 + jj < Ne) ? __ldg(dR + row * Ne + j0 + jj) : 0.f;
+                    any[q] |= dr[q][jj] != 0.f;
+                }
+                if (any[q] && col) sv[q] = __ldcg(reinterpret_cast<const uint4*>(S + row * D) + v);
             }
-            if (!any || !col) continue;
-            float2 sp[4];
-            unpack_pairs(__ldcg(reinterpret_cast<const uint4*>(S + row * D) + v), sp);
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                if (dr[jj] != 0.f) {
+            for (int q = 0; q < 4; ++q) {
+                if (!any[q] || !col) continue;
+                float2 sp[4];
+                unpack_pairs(sv[q], sp);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        a[jj][2 * q] = fmaf(dr[jj], sp[q].x, a[jj][2 * q]);
-                        a[jj][2 * q + 1] = fmaf(dr[jj], sp[q].y, a[jj][2 * q + 1]);
+                for (int jj = 0; jj < 8; ++jj) {
+                    if (dr[q][jj] != 0.f) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            a[jj][2 * e] = fmaf(dr[q][jj], sp[e].x, a[jj][2 * e]);
+                            a[jj][2 * e + 1] = fmaf(dr[q][jj], sp[e].y, a[jj][2 * e + 1]);
+                        }
                     }
                 }
             }
@@ -624,22 +636,37 @@ __global__ void __launch_bounds__(kThreads) router_grad_kernel(const __nv_bfloat
     }
 }
 
-// loss[0] += lambda * sum of x[0 .. n) (one CTA, a fixed order: thread i sums
-// x[i], x[i + 1024], ...; then a fixed tree).
-__global__ void __launch_bounds__(1024) add_scaled_sum_kernel(const float* __restrict__ x, long long n, float lambda,
-                                                              float* __restrict__ loss) {
+// loss[0] += lambda * sum of x[0 .. n), in a fixed order: CTA p sums chunk
+// p of kSumChunks equal chunks (thread i over elements i, i + 256, ..., then
+// a fixed tree) into part[p]; one warp adds the chunk sums (lane l over
+// chunks l, l + 32, ..., then a fixed butterfly).
+constexpr int kSumChunks = 256;
+
+__global__ void __launch_bounds__(256) sum_chunks_kernel(const float* __restrict__ x, long long n,
+                                                         float* __restrict__ part) {
     pdl_enter();
-    __shared__ float red[32];
+    __shared__ float red[8];
+    const long long chunk = (n + gridDim.x - 1) / gridDim.x;
+    const long long i0 = blockIdx.x * chunk, i1 = min(n, i0 + chunk);
     float a = 0.f;
-    for (long long i = threadIdx.x; i < n; i += blockDim.x) a += __ldcg(x + i);
+    for (long long i = i0 + threadIdx.x; i < i1; i += blockDim.x) a += __ldcg(x + i);
     a = warp_sum(a);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
     __syncthreads();
-    if (threadIdx.x < 32) {
-        float v = red[threadIdx.x];
-        v = warp_sum(v);
-        if (threadIdx.x == 0) loss[0] += lambda * v;
+    if (threadIdx.x == 0) {
+        float t = 0.f;
+        for (int w = 0; w < 8; ++w) t += red[w];
+        part[blockIdx.x] = t;
     }
+}
+
+__global__ void __launch_bounds__(32) add_scaled_parts_kernel(const float* __restrict__ part, int np, float lambda,
+                                                               float* __restrict__ loss) {
+    pdl_enter();
+    float a = 0.f;
+    for (int i = threadIdx.x; i < np; i += 32) a += __ldcg(part + i);
+    a = warp_sum(a);
+    if (threadIdx.x == 0) loss[0] += lambda * a;
 }
 
 }  // namespace
@@ -697,13 +724,18 @@ cudaError_t launch_moe_bwd_combine(const void* dZ, const void* dSg, const MoeWor
 cudaError_t launch_router_grad(const void* S, const float* dR, float* part, float* part_b, int B, int T, int D, int Ne,
                                int RB, cudaStream_t s) {
     const int nrb = (B + RB - 1) / RB;
-    const dim3 grid((unsigned)((D / 8 + kThreads - 1) / kThreads), (unsigned)nrb, (unsigned)T);
-    return launch_pdl(router_grad_kernel, grid, kThreads, 0, s, static_cast<const __nv_bfloat16*>(S), dR, part, part_b,
+    const int nv = D / 8;
+    const int threads = nv < kThreads ? std::max(32, (nv + 31) / 32 * 32) : kThreads;
+    const dim3 grid((unsigned)((nv + threads - 1) / threads), (unsigned)nrb, (unsigned)T);
+    return launch_pdl(router_grad_kernel, grid, threads, 0, s, static_cast<const __nv_bfloat16*>(S), dR, part, part_b,
                       B, T, D, Ne, RB);
 }
 
-cudaError_t launch_add_scaled_sum(const float* x, long long n, float lambda, float* loss, cudaStream_t s) {
-    return launch_pdl(add_scaled_sum_kernel, 1, 1024, 0, s, x, n, lambda, loss);
+cudaError_t launch_add_scaled_sum(const float* x, long long n, float lambda, float* loss, float* part,
+                                  cudaStream_t s) {
+    cudaError_t e = launch_pdl(sum_chunks_kernel, kSumChunks, 256, 0, s, x, n, part);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(add_scaled_parts_kernel, 1, 32, 0, s, (const float*)part, kSumChunks, lambda, loss);
 }
 
 }  // namespace rm

@@ -101,8 +101,8 @@ __global__ void __launch_bounds__(kThreads) head_logit_kernel(const float* poole
 // dw[n] = sum_b dlogit_b pooled[b, n] and gpool[b, n] = dlogit_b w[n] / T,
 // the gradient of every token row of the last block's output.  CTA = 32
 // columns; warp w takes samples b = w, w + kRedWarps, ... in ascending order
-// and the warp sums are added in warp order.  One thread adds up the loss and
-// dc in ascending b.
+// and the warp sums are added in warp order.  Warp 0 of CTA 0 adds up the
+// loss and dc: lane l over b = l, l + 32, ..., then a fixed butterfly.
 __global__ void __launch_bounds__(32 * kRedWarps) head_grad_kernel(const float* pooled,
                                                                   const __nv_bfloat16* __restrict__ w,
                                                                   const float* dlogit, const float* lterm, float* dw,
@@ -129,14 +129,18 @@ __global__ void __launch_bounds__(32 * kRedWarps) head_grad_kernel(const float* 
         for (int q = 0; q < kRedWarps; ++q) t += red[q][lane];
         dw[n] = t;
     }
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (blockIdx.x == 0 && warp == 0) {
         float l = 0.f, c = 0.f;
-        for (int b = 0; b < B; ++b) {
+        for (int b = lane; b < B; b += 32) {
             l += __ldcg(lterm + b);
             c += __ldcg(dlogit + b);
         }
-        *loss = l / (float)B;
-        *dc = c;
+        l = warp_sum(l);
+        c = warp_sum(c);
+        if (lane == 0) {
+            *loss = l / (float)B;
+            *dc = c;
+        }
     }
 }
 
@@ -371,8 +375,48 @@ __global__ void __launch_bounds__(32 * kRedWarps) reduce_parts_kernel(const floa
     }
 }
 
+// scratch[(g * gridDim.z + c) * N + n] = sum of slices [c*CH, min(J, c*CH + CH))
+// of column n of group g, in the same warp-split order as reduce_parts_kernel.
+__global__ void __launch_bounds__(32 * kRedWarps) reduce_chunks_kernel(const float* part, float* scratch, int G, int J,
+                                                                       int N, int CH) {
+    pdl_enter();
+    __shared__ float red[kRedWarps][33];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, W = blockDim.x >> 5;
+    const int n = blockIdx.x * 32 + lane, g = blockIdx.y, c = blockIdx.z;
+    const int j0 = c * CH, j1 = min(J, j0 + CH);
+    float a = 0.f;
+    if (n < N) {
+        const float* p = part + (long long)g * J * N + n;
+        for (int j = j0 + warp; j < j1; j += W) a += __ldcg(p + (long long)j * N);
+    }
+    red[warp][lane] = a;
+    __syncthreads();
+    if (warp == 0 && n < N) {
+        float t = 0.f;
+        for (int w = 0; w < W; ++w) t += red[w][lane];
+        scratch[((long long)g * gridDim.z + c) * N + n] = t;
+    }
+}
+
 // Ordered reduction of J slices per column: about eight slices per warp.
-inline cudaError_t launch_reduce_parts(const float* part, float* out, int G, int J, int N, cudaStream_t s) {
+// When the (column block, group) grid is too small to fill the GPU and J is
+// large, the slices are first reduced in fixed chunks of kRedChunk into
+// `scratch` (ceil(J / kRedChunk) x G x N floats), then those chunk sums in
+// order: a fixed order for a given shape (deterministic).
+constexpr int kRedChunk = 64;
+inline cudaError_t launch_reduce_parts(const float* part, float* out, int G, int J, int N, cudaStream_t s,
+                                       float* scratch = nullptr) {
+    const long long ctas = (long long)((N + 31) / 32) * G;
+    if (scratch && ctas < 2 * 148 && J > 2 * kRedChunk) {
+        const int JS = (J + kRedChunk - 1) / kRedChunk;
+        // chunk c of group g: slices [c*kRedChunk, ...) of g -> scratch[(g*JS + c)*N + n]
+        const int W = std::min(kRedWarps, kRedChunk / 8);
+        cudaError_t e = launch_pdl(reduce_chunks_kernel, dim3((N + 31) / 32, G, JS), dim3(32 * W), 0, s, part,
+                                   scratch, G, J, N, kRedChunk);
+        if (e != cudaSuccess) return e;
+        part = scratch;
+        J = JS;
+    }
     const int W = std::min(kRedWarps, std::max(1, (J + 7) / 8));
     return launch_pdl(reduce_parts_kernel, dim3((N + 31) / 32, G), dim3(32 * W), 0, s, part, out, G, J, N);
 }
@@ -515,6 +559,8 @@ struct rm_trainer {
     float *pooled, *dlogit, *lterm, *gpool;
     unsigned char *dY, *dU, *dS, *dX;
     float *pg, *pb, *pdb, *pcol, *pcol2;
+    float* rscratch;         // chunk sums of the two-stage ordered reductions
+    float* lreg_part;        // chunk sums of L_reg
     float* sk_ws;
     int* sk_cnt;
     // shared, sparse MoE backward
@@ -620,7 +666,8 @@ cudaError_t moe_backward(rm_trainer* t, const rm_block_weights& w, const rm_bloc
         if ((e = rm::launch_reduce_parts((const float*)t->prt, pass ? gr.Wr_infer : gr.Wr, T, nrb_b, Ne * D, s)) !=
             cudaSuccess)
             return e;
-        if ((e = rm::launch_reduce_parts((const float*)t->prt_b, pass ? gr.br_infer : gr.br, T, nrb_b, Ne, s)) !=
+        if ((e = rm::launch_reduce_parts((const float*)t->prt_b, pass ? gr.br_infer : gr.br, T, nrb_b, Ne, s,
+                                         t->rscratch)) !=
             cudaSuccess)
             return e;
     }
@@ -742,6 +789,13 @@ rm_status rm_train_create(const rm_config* cfg, rm_trainer** out) {
         t->pdb = carve<float>(base, off, (size_t)c.T * t->nsb * c.D * 4);
         t->pcol = carve<float>(base, off, col_parts * 4);
         t->pcol2 = carve<float>(base, off, col_parts * 4);
+        {
+            const size_t ch = (size_t)rm::kRedChunk;
+            const size_t r1 = (nrb_rows + ch - 1) / ch * c.D, r2 = ((size_t)c.T * t->nsb + ch - 1) / ch * c.D;
+            const size_t r3 = (nrb_b + ch - 1) / ch * (size_t)c.T * std::max(Ne, 1);
+            t->rscratch = carve<float>(base, off, std::max(std::max(r1, r2), r3) * 4);
+        }
+        t->lreg_part = carve<float>(base, off, 256 * 4);
         t->sk_cnt = carve<int>(base, off, rm::gemm_tc_split_cnt_ints(t->num_sms) * sizeof(int));
         t->sk_ws = carve<float>(base, off, rm::gemm_tc_split_ws_bytes(t->num_sms));
         if (Ne) {
@@ -910,7 +964,7 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
     if (Ne && t->lambda > 0.f)   // + lambda L_reg: the regularised gates of every MoE block, in block order
         for (int l = 0; l < L; ++l)
             RM_TRY(rm::launch_add_scaled_sum(blocks[l].Wr_infer ? t->gates_inf[l] : t->moe[l].gates,
-                                             (long long)B * T * Ne, t->lambda, loss, s));
+                                             (long long)B * T * Ne, t->lambda, loss, t->lreg_part, s));
 
     // ------------------------------------------------------------ backward
     const int nsb = (B + t->SB - 1) / t->SB;
@@ -932,8 +986,8 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
             RM_TRY(rm::launch_pdl(rm::ln2_bwd_kernel<false>, dim3(nsb, T), dim3(lnb_threads), 0, s,
                                   (const __nv_bfloat16*)t->dX, (const float*)nullptr, Yl, (const float2*)t->ystats[l],
                                   P, w.ln2_g, c.ln_eps, dY, t->pg, t->pb, t->pdb, B, T, D, t->SB));
-        RM_TRY(rm::launch_reduce_parts((const float*)t->pg, gr.ln2_g, 1, T * nsb, D, s));
-        RM_TRY(rm::launch_reduce_parts((const float*)t->pb, gr.ln2_b, 1, T * nsb, D, s));
+        RM_TRY(rm::launch_reduce_parts((const float*)t->pg, gr.ln2_g, 1, T * nsb, D, s, t->rscratch));
+        RM_TRY(rm::launch_reduce_parts((const float*)t->pb, gr.ln2_b, 1, T * nsb, D, s, t->rscratch));
         if (Ne) {
             RM_TRY(moe_backward(t, w, gr, l, B, s));
         } else {
@@ -989,8 +1043,8 @@ rm_status rm_train_step(rm_trainer* t, const rm_block_weights* blocks, const voi
                               dim3(rm::kThreads), 0, s, (const __nv_bfloat16*)t->dS,
                               (const __nv_bfloat16*)t->XH1[l], t->pcol, t->pcol2, B * T, D, 0LL, (long long)D,
                               rm::kColRows));
-        RM_TRY(rm::launch_reduce_parts((const float*)t->pcol2, gr.ln1_g, 1, nrb, D, s));
-        RM_TRY(rm::launch_reduce_parts((const float*)t->pcol, gr.ln1_b, 1, nrb, D, s));
+        RM_TRY(rm::launch_reduce_parts((const float*)t->pcol2, gr.ln1_g, 1, nrb, D, s, t->rscratch));
+        RM_TRY(rm::launch_reduce_parts((const float*)t->pcol, gr.ln1_b, 1, nrb, D, s, t->rscratch));
         // LN1 backward and the mixing's transpose: dX (the stack input's gradient for l = 0)
         __nv_bfloat16* dXo = (l == 0 && dX0) ? static_cast<__nv_bfloat16*>(dX0)
                                              : reinterpret_cast<__nv_bfloat16*>(t->dX);
