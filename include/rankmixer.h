@@ -232,6 +232,34 @@ rm_status rm_pffn_forward_static(const rm_block_weights *w, const void *S, void 
                                  int D, int hidden, rm_dtype dtype, int act, int *device_status,
                                  rm_stream_t stream);
 
+/* ---- token-sharded forward (one rank's share) ------------------------------
+ * G ranks each own Tl = T / G consecutive tokens: their rows of every sample
+ * [B, Tl, D] and their per-token FFN weights.  The token mixing with H = T
+ * then needs chunk h of every token's row on the rank owning token h: an
+ * all-to-all between the ranks ("特征交叉 —— RankMixer 精读笔记": the mixing
+ * works like an all-to-all; "重新理解 RankMixer" section 3.3, model sharding).
+ * The handle is created with cfg->T = Tl (the rank's tokens).  Per block:
+ *   rm_tokshard_pack: Xh = LN(Za + Zb) with (ln_g, ln_b) (the previous
+ *     block's LN2 of V + S), or Za alone (ln_g = ln_b = Zb = NULL: the stack
+ *     input); Xh [B, Tl, D] is written (kept for the residual) and its
+ *     column range [r D/G, (r+1) D/G) of each row to send + r * B*Tl*D/G,
+ *     laid out [r][b][tq][D/G], for an equal-split all-to-all of send into
+ *     recv (B*Tl*D elements each, bf16);
+ *   rm_tokshard_mix_ln: S = LN1(TokenMixing(Xh) + Xh) for the rank's tokens,
+ *     the mixed pieces read from recv ([q][b][tq][D/G]);
+ *   rm_pffn_forward on S with the rank's token weights (W1 + rank*Tl*kD*D, ...);
+ *   after the last block rm_tokshard_pool: pooled_part [B, D] float = ln2_g *
+ *     mean over the rank's tokens of xhat(V + S) + ln2_b; the pooled output
+ *     is the mean of the G ranks' parts.
+ * Supported: bf16, dense FFN, Add & Norm after mixing, D % G == 0,
+ * (D / G) % 8 == 0, (D / T) % 8 == 0, D <= 2048; else RM_ERR_UNSUPPORTED. */
+rm_status rm_tokshard_pack(rm_handle *h, const void *Za, const void *Zb, const float *ln_g, const float *ln_b,
+                           void *Xh, void *send, int B, int world, rm_stream_t stream);
+rm_status rm_tokshard_mix_ln(rm_handle *h, const void *recv, const void *Xh, const float *ln1_g, const float *ln1_b,
+                             void *S, int B, int world, rm_stream_t stream);
+rm_status rm_tokshard_pool(rm_handle *h, const void *V, const void *S, const float *ln2_g, const float *ln2_b,
+                           float *pooled_part, int B, rm_stream_t stream);
+
 /* ---- training step (dense and sparse-MoE bf16 stacks) ---------------------
  * One training step of a stack of L dense RankMixer blocks with the sigmoid
  * head: the forward pass (keeping what the backward pass needs), the task loss

@@ -552,6 +552,53 @@ rm_status rm_host_wait(rm_handle* h) {
     return cuda_status(cudaStreamSynchronize(h->d2h));
 }
 
+// ---- token-sharded forward (one rank's share; the caller runs the all-to-all)
+namespace {
+rm_status check_shard(const rm_handle* h, int B, int world) {
+    if (!h) return RM_ERR_INVALID_ARG;
+    const rm_config& c = h->cfg;
+    if (B < 1 || B > c.B_max || world < 1) return RM_ERR_INVALID_ARG;
+    if (c.dtype != RM_BF16 || c.n_experts != 0 || c.D % 8 || c.D > 2048) return RM_ERR_UNSUPPORTED;
+    const long long T = (long long)c.T * world;
+    if (c.D % world || (c.D / world) % 8 || c.D % T || (c.D / T) % 8) return RM_ERR_UNSUPPORTED;
+    return RM_OK;
+}
+}  // namespace
+
+rm_status rm_tokshard_pack(rm_handle* h, const void* Za, const void* Zb, const float* ln_g, const float* ln_b,
+                           void* Xh, void* send, int B, int world, rm_stream_t stream) {
+    rm_status st = check_shard(h, B, world);
+    if (st != RM_OK) return st;
+    if (!aligned16(Za) || !aligned16_or_null(Zb) || !aligned16(Xh) || !aligned16(send)) return RM_ERR_INVALID_ARG;
+    if ((ln_g == nullptr) != (ln_b == nullptr) || !aligned16_or_null(ln_g) || !aligned16_or_null(ln_b))
+        return RM_ERR_INVALID_ARG;
+    return cuda_status(rm::launch_shard_pack(Za, Zb, ln_g, ln_b, h->cfg.ln_eps, Xh, send, B, h->cfg.T, h->cfg.D,
+                                             world, stream));
+}
+
+rm_status rm_tokshard_mix_ln(rm_handle* h, const void* recv, const void* Xh, const float* ln1_g, const float* ln1_b,
+                             void* S, int B, int world, rm_stream_t stream) {
+    rm_status st = check_shard(h, B, world);
+    if (st != RM_OK) return st;
+    if (!h->cfg.mix_addnorm) return RM_ERR_UNSUPPORTED;
+    if (!aligned16(recv) || !aligned16(Xh) || !aligned16(S) || !aligned16(ln1_g) || !aligned16(ln1_b))
+        return RM_ERR_INVALID_ARG;
+    ProfScope ps(h, RM_K_MIX_LN, stream);
+    return cuda_status(rm::launch_shard_mix_ln(recv, Xh, ln1_g, ln1_b, h->cfg.ln_eps, S, B, h->cfg.T, h->cfg.D, world,
+                                               stream));
+}
+
+rm_status rm_tokshard_pool(rm_handle* h, const void* V, const void* S, const float* ln2_g, const float* ln2_b,
+                           float* pooled_part, int B, rm_stream_t stream) {
+    rm_status st = check_shard(h, B, 1);
+    if (st != RM_OK) return st;
+    if (!aligned16(V) || !aligned16(S) || !aligned16(ln2_g) || !aligned16(ln2_b) || !aligned16(pooled_part))
+        return RM_ERR_INVALID_ARG;
+    ProfScope ps(h, RM_K_LN_POOL, stream);
+    return cuda_status(
+        rm::launch_shard_pool(V, S, ln2_g, ln2_b, h->cfg.ln_eps, pooled_part, B, h->cfg.T, h->cfg.D, stream));
+}
+
 rm_status rm_padsplit_tokenize(rm_handle* h, const void* const* groups, const int* widths, int n_groups, void* X0,
                                int B, rm_stream_t stream) {
     rm_status st = check_batch(h, B);

@@ -193,4 +193,12 @@ cudaError_t launch_router_grad(const void* S, const float* dR, float* part, floa
 cudaError_t launch_add_scaled_sum(const float* x, long long n, float lambda, float* loss, float* part,
                                   cudaStream_t s);
 
+// Token-sharded forward (rm_shard.cu): G ranks of Tl = T / G tokens each.
+cudaError_t launch_shard_pack(const void* Za, const void* Zb, const float* g, const float* bt, float eps, void* Xh,
+                              void* send, int B, int Tl, int D, int G, cudaStream_t s);
+cudaError_t launch_shard_mix_ln(const void* recv, const void* Xh, const float* g, const float* bt, float eps, void* S,
+                                int B, int Tl, int D, int G, cudaStream_t s);
+cudaError_t launch_shard_pool(const void* V, const void* Sres, const float* g, const float* bt, float eps,
+                              float* pooled_part, int B, int Tl, int D, cudaStream_t s);
+
 }  // namespace rm

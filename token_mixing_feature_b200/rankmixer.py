@@ -28,7 +28,7 @@ EXPORTED = (
     "rm_profile_begin", "rm_profile_end", "rm_kernel_name", "rm_pffn_forward_static",
     "rm_stack_forward_host_async", "rm_host_wait",
     "rm_train_create", "rm_train_destroy", "rm_train_workspace_bytes", "rm_train_step", "rm_train_sync_status",
-    "rm_train_set_reg",
+    "rm_train_set_reg", "rm_tokshard_pack", "rm_tokshard_mix_ln", "rm_tokshard_pool",
 )
 RM_STATIC_SCRATCH_BYTES = 16 << 20
 RM_K_COUNT = 11
@@ -94,6 +94,9 @@ def _load() -> ctypes.CDLL:
                                vp, vp, vp, vp, vp, ci, vp]),
         "rm_train_sync_status": (st, [vp, vp]),
         "rm_train_set_reg": (st, [vp, ctypes.c_float]),
+        "rm_tokshard_pack": (st, [vp, vp, vp, vp, vp, vp, vp, ci, ci, vp]),
+        "rm_tokshard_mix_ln": (st, [vp, vp, vp, vp, vp, vp, ci, ci, vp]),
+        "rm_tokshard_pool": (st, [vp, vp, vp, vp, vp, vp, ci, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -365,3 +368,19 @@ def rm_train_step(t: Trainer, blocks: Sequence[Dict], X0, head_w, head_b, labels
 
 def rm_train_sync_status(t: Trainer, stream=None) -> int:
     return _lib.rm_train_sync_status(t.ptr, _stream(stream))
+
+
+# ------------------------------------------------------- token-sharded forward
+def rm_tokshard_pack(h: Handle, Za, Zb, ln_g, ln_b, Xh, send, B: int, world: int, stream=None) -> None:
+    _check(_lib.rm_tokshard_pack(h.ptr, _ptr(Za), _ptr(Zb), _ptr(ln_g), _ptr(ln_b), _ptr(Xh), _ptr(send), B, world,
+                                 _stream(stream)), "rm_tokshard_pack")
+
+
+def rm_tokshard_mix_ln(h: Handle, recv, Xh, ln1_g, ln1_b, S, B: int, world: int, stream=None) -> None:
+    _check(_lib.rm_tokshard_mix_ln(h.ptr, _ptr(recv), _ptr(Xh), _ptr(ln1_g), _ptr(ln1_b), _ptr(S), B, world,
+                                   _stream(stream)), "rm_tokshard_mix_ln")
+
+
+def rm_tokshard_pool(h: Handle, V, S, ln2_g, ln2_b, pooled_part, B: int, stream=None) -> None:
+    _check(_lib.rm_tokshard_pool(h.ptr, _ptr(V), _ptr(S), _ptr(ln2_g), _ptr(ln2_b), _ptr(pooled_part), B,
+                                 _stream(stream)), "rm_tokshard_pool")
