@@ -472,14 +472,13 @@ __global__ void __launch_bounds__(kMixMaxThreads, 2) mix_ln_kernel(
 // merged from the producer's partials (one warp per row) into shared memory;
 // then thread u takes (sample u / nv, 16-byte column vector u % nv) and sums
 // that column over the sample's T rows in ascending t (deterministic), with
-// twelve rows' loads in flight at a time straight from global memory (no
+// eight rows' loads in flight at a time straight from global memory (no
 // staging: each element is read once, and many small CTAs keep enough loads
 // in flight to cover the memory latency).
 constexpr int kPoolThreads = 256;
+constexpr int kPoolRowsInFlight = 8;
 
-// XOUT: also write LN(x) (gamma/beta held across the row loop, eight rows in
-// flight); else twelve rows' loads in flight.
-template <typename E, bool XOUT>
+template <typename E>
 __global__ void __launch_bounds__(kPoolThreads, 3) ln_pool_kernel(const E* X, const float2* pstats, int P,
                                                               const float* __restrict__ g,
                                                               const float* __restrict__ bta, float* __restrict__ pooled,
@@ -520,15 +519,12 @@ __global__ void __launch_bounds__(kPoolThreads, 3) ln_pool_kernel(const E* X, co
     __syncthreads();
     const int nv = D / V;
     const float invT = 1.0f / T;
-    constexpr int kPoolRowsInFlight = XOUT ? 8 : 12;
     for (int u = tid; u < ns * nv; u += blockDim.x) {
         const int sm = u / nv, c0 = (u - sm * nv) * V;
         const E* col = X + (size_t)(b0 + sm) * T * D + c0;
         float2 gp[NP], bp[NP];
-        if (XOUT) {
-            load_pairs(g + c0, gp);
-            load_pairs(bta + c0, bp);
-        }
+        load_pairs(g + c0, gp);
+        load_pairs(bta + c0, bp);
         float2 acc[NP];
 #pragma unroll
         for (int j = 0; j < NP; ++j) acc[j] = f2(0.f);
@@ -550,17 +546,13 @@ __global__ void __launch_bounds__(kPoolThreads, 3) ln_pool_kernel(const E* X, co
                         x[j] = f2_fma(x[j], r2, mr2);   // (x - m_t) r_t
                         acc[j] = f2_add(acc[j], x[j]);
                     }
-                    if (XOUT) {
+                    if (Xout) {
 #pragma unroll
                         for (int j = 0; j < NP; ++j) x[j] = f2_fma(x[j], gp[j], bp[j]);
                         *reinterpret_cast<uint4*>(Xout + ((size_t)(b0 + sm) * T + t) * D + c0) = pack_pairs(x);
                     }
                 }
             }
-        }
-        if (!XOUT) {
-            load_pairs(g + c0, gp);
-            load_pairs(bta + c0, bp);
         }
         float4* dst = reinterpret_cast<float4*>(pooled + (size_t)(b0 + sm) * D + c0);
 #pragma unroll
@@ -744,11 +736,8 @@ cudaError_t ln_pool_go(const void* X, RowStats stats, const float* g, const floa
     const int threads = std::max(64, (spc * nv + 31) / 32 * 32);
     const size_t smem = sizeof(float) * 2 * (size_t)spc * T;
     const int grid = (B + spc - 1) / spc;
-    if (Xout)
-        return launch_pdl(ln_pool_kernel<E, true>, grid, threads, smem, s, static_cast<const E*>(X), stats.part,
-                          stats.P, g, b, pooled, static_cast<E*>(Xout), B, T, D, eps, spc);
-    return launch_pdl(ln_pool_kernel<E, false>, grid, threads, smem, s, static_cast<const E*>(X), stats.part, stats.P,
-                      g, b, pooled, static_cast<E*>(nullptr), B, T, D, eps, spc);
+    return launch_pdl(ln_pool_kernel<E>, grid, threads, smem, s, static_cast<const E*>(X), stats.part, stats.P, g,
+                      b, pooled, static_cast<E*>(Xout), B, T, D, eps, spc);
 }
 
 }  // namespace
