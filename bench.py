@@ -380,6 +380,8 @@ def main():
                     help="time direct launches instead of replaying the step captured in a CUDA graph")
     ap.add_argument("--train", action="store_true",
                     help="time one training step (forward, loss, every gradient) of the dense workload instead")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the stack with e4m3 FFN operands (rm_stack_forward_fp8) instead, one GPU")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -398,6 +400,8 @@ def main():
         return run_reference(a, wl, cfg, rank, world)
     if a.train:
         return run_train(a, wl, cfg, rank, world, local)
+    if a.fp8:
+        return run_fp8(a, wl, cfg, local)
 
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
@@ -553,6 +557,72 @@ def main():
     if pg:
         pg.barrier(device_ids=[local])
         pg.destroy_process_group()
+
+
+def run_fp8(a, wl, cfg, local):
+    """K steps of the stack with e4m3 FFN operands (weights quantised once per
+    output channel, S and H per token row inside the step), replayed from a
+    CUDA graph; FLOPs as the bf16 stack, against the e4m3 dense peak taken as
+    twice the measured bf16 burst peak (the datasheet's fp8 : bf16 ratio)."""
+    if wl.n_experts or wl.dtype != "bf16" or wl.group_widths:
+        raise SystemExit("the e4m3 stack covers the dense bf16 workloads")
+    from token_mixing_feature_b200 import rankmixer as rm
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    runner = Runner(wl, device)
+    st = runner.st
+    B, T, D, Hd, L = wl.B, wl.T, wl.D, wl.hidden, wl.L
+    qblocks = []
+    for blk in st.blocks:
+        q = {}
+        for k, rows, K in (("W1", T * Hd, D), ("W2", T * D, Hd)):
+            q[k + "q"] = torch.empty(rows * K, dtype=torch.uint8, device=device)
+            q[k + "s"] = torch.empty(rows, device=device)
+            rm.rm_quantize_fp8(blk[k], q[k + "q"], q[k + "s"], rows, K)
+        qblocks.append(q)
+    stream = torch.cuda.Stream(device)
+
+    def step():
+        rm.rm_stack_forward_fp8(st.h, st.blocks, qblocks, runner.X0, runner.pooled, B, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(a.warmup):
+            step()
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    torch.cuda.synchronize(device)
+    if rm.rm_sync_status(st.h) != rm.RM_OK:
+        raise SystemExit("device error during warm-up")
+    sampler = ClockSampler(local)
+    wall0 = time.time()
+    ms = time_steps(graph.replay, a.steps, stream)
+    wall1 = time.time()
+    sampler.stop()
+    clocks = sampler.summary(wall0 - 0.05, wall1 + 0.05)
+    peaks, peak_src = load_peaks()
+    flops = 4.0 * B * T * D * Hd * L
+    nbytes = L * 2 * T * D * Hd + B * T * D * 2
+    sec = ms / 1e3 / a.steps
+    f8_peak = 2.0 * peaks["bf16_tflops"]
+    t_roof = roofline.roofline_seconds(flops, nbytes, f8_peak * 1e12, peaks["hbm_gbs"] * 1e9)
+    line = {
+        "metric": "RankMixer stack fwd samples/s with e4m3 FFN operands on 1\u00d7B200",
+        "value": B * a.steps / (ms / 1e3), "unit": "samples/s", "n_gpus": 1, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": ms / a.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 x e4m3 -> f32 FFN products, bf16 elsewhere",
+        "data": "synthetic (seeded N(0,1) inputs, Xavier-normal weights)",
+        "config": dict(cfg, mode="fp8", launch="cuda_graph"),
+        "tflops": flops / sec / 1e12,
+        "stack_roofline": {"flops": flops, "bytes": nbytes, "t_roof_ms": t_roof * 1e3, "frac": t_roof / sec,
+                           "peaks": f"e4m3 {f8_peak:.1f} TFLOP/s (2 x the measured bf16 burst, the datasheet "
+                                    f"ratio), HBM {peaks['hbm_gbs']} GB/s, of {peak_src}"},
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    del graph
+    st.close()
 
 
 def run_train(a, wl, cfg, rank, world, local):

@@ -232,6 +232,35 @@ rm_status rm_pffn_forward_static(const rm_block_weights *w, const void *S, void 
                                  int D, int hidden, rm_dtype dtype, int act, int *device_status,
                                  rm_stream_t stream);
 
+/* ---- stack with e4m3 (fp8) FFN weights ------------------------------------
+ * Lower-precision serving of the dense bf16 stack (8-bit serving is only
+ * mentioned, in section 4.1 of the least reliable of the pages; the scheme
+ * here is this library's own): the FFN
+ * weights are quantised once to e4m3 with one fp32 scale per output channel,
+ * and in every block S and the FFN hidden H are quantised per token row, so
+ * both FFN projections run on the tensor cores' kind::f8f6f4 path and
+ * dequantise in their epilogues (acc * scale_row * scale_channel, then the
+ * bias, GELU / residual and LayerNorm partials as in the bf16 stack).
+ * e4m3 keeps 3 mantissa bits: results differ from the bf16 stack by a few
+ * percent relative L2 (the tests derive their bound from that rounding).
+ *
+ * rm_quantize_fp8: dst[r][k] = e4m3(src[r][k] / scale[r]) with scale[r] =
+ *   max_k |src[r][k]| / 448 (1 for an all-zero row), src bf16 [rows][K],
+ *   dst one byte per element, K % 16 == 0.  For W1 [T][kD][D] call it with
+ *   rows = T*kD, K = D; for W2 [T][D][kD] with rows = T*D, K = kD.
+ * rm_stack_forward_fp8: as rm_stack_forward (pooled output only) with the
+ *   quantised weights of every block in q[l] (the biases, LayerNorm
+ *   parameters come from blocks[l]); dense bf16 handles with D % 64 == 0 and
+ *   hidden % 16 == 0, else RM_ERR_UNSUPPORTED.  The first call allocates the
+ *   quantised activations (B_max*T*(D + kD) bytes + scales). */
+typedef struct {
+    const void *W1q, *W2q;          /* e4m3 [T][kD][D], [T][D][kD]     */
+    const float *W1s, *W2s;         /* scales [T][kD], [T][D]          */
+} rm_fp8_weights;
+rm_status rm_quantize_fp8(const void *src, void *dst, float *scale, long long rows, int K, rm_stream_t stream);
+rm_status rm_stack_forward_fp8(rm_handle *h, const rm_block_weights *blocks, const rm_fp8_weights *q, const void *X0,
+                               float *pooled, int B, rm_stream_t stream);
+
 /* ---- token-sharded forward (one rank's share) ------------------------------
  * G ranks each own Tl = T / G consecutive tokens: their rows of every sample
  * [B, Tl, D] and their per-token FFN weights.  The token mixing with H = T

@@ -14,7 +14,7 @@ HEADER = os.path.join(ROOT, "include", "rankmixer.h")
 def _declared():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(rm_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(rm_[a-z0-9_]+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")

@@ -46,6 +46,13 @@ struct rm_handle {
     float* sk_ws;     // split-K partial tiles of the dense tcgen05 GEMMs (null for fp32 / MoE)
     int* sk_cnt;      // their arrival counters (zero between launches)
     rm::MoeWork moe;
+    // e4m3 stack (allocated on its first call): the quantised S and H and their
+    // per-row scales
+    void* f8ws;
+    void* S8;
+    void* H8;
+    float* sS;
+    float* sH;
     int* err;       // [0] error word, [1] site
     unsigned long long budget_ns;
     int last_site;
@@ -410,6 +417,7 @@ rm_status rm_destroy(rm_handle* h) {
         }
     }
     cudaError_t e = cudaFree(h->ws);
+    if (h->f8ws) cudaFree(h->f8ws);
     cudaSetDevice(cur);
     delete h;
     return cuda_status(e);
@@ -483,6 +491,92 @@ rm_status rm_stack_forward(rm_handle* h, const rm_block_weights* blocks, const v
     for (int l = 0; l < h->cfg.L; ++l)
         if ((st = check_block_weights(h, &blocks[l], true)) != RM_OK) return st;
     return run_stack(h, blocks, X0, pooled, Xlast, B, stream);
+}
+
+rm_status rm_quantize_fp8(const void* src, void* dst, float* scale, long long rows, int K, rm_stream_t stream) {
+    if (!aligned16(src) || !aligned16(dst) || !scale || rows < 0 || K < 16 || K % 16) return RM_ERR_INVALID_ARG;
+    if (rows == 0) return RM_OK;
+    return cuda_status(rm::launch_quant_rows(src, dst, scale, rows, K, stream));
+}
+
+rm_status rm_stack_forward_fp8(rm_handle* h, const rm_block_weights* blocks, const rm_fp8_weights* q, const void* X0,
+                               float* pooled, int B, rm_stream_t stream) {
+    rm_status st = check_batch(h, B);
+    if (st != RM_OK) return st;
+    const rm_config& c = h->cfg;
+    if (c.dtype != RM_BF16 || c.n_experts != 0 || c.D % 64 || c.hidden % 16) return RM_ERR_UNSUPPORTED;
+    if (!blocks || !q || !aligned16(X0) || !aligned16(pooled)) return RM_ERR_INVALID_ARG;
+    for (int l = 0; l < c.L; ++l) {
+        if ((st = check_block_weights(h, &blocks[l], true)) != RM_OK) return st;
+        if (!aligned16(q[l].W1q) || !aligned16(q[l].W2q) || !aligned16(q[l].W1s) || !aligned16(q[l].W2s))
+            return RM_ERR_INVALID_ARG;
+    }
+    const size_t rows = (size_t)c.B_max * c.T;
+    if (!h->f8ws) {   // first call: the quantised activations and their scales
+        const size_t s8 = round_up(rows * c.D, 256), h8 = round_up(rows * c.hidden, 256),
+                     sc = round_up(rows * sizeof(float), 256);
+        if (cudaMalloc(&h->f8ws, s8 + h8 + 2 * sc) != cudaSuccess) {
+            cudaGetLastError();
+            h->f8ws = nullptr;
+            return RM_ERR_OOM;
+        }
+        unsigned char* b = static_cast<unsigned char*>(h->f8ws);
+        h->S8 = b;
+        h->H8 = b + s8;
+        h->sS = reinterpret_cast<float*>(b + s8 + h8);
+        h->sH = reinterpret_cast<float*>(b + s8 + h8 + sc);
+    }
+    cudaStream_t s = stream;
+    for (int l = 0; l < c.L; ++l) {
+        const rm_block_weights* w = &blocks[l];
+        const rm_block_weights* prev = l ? &blocks[l - 1] : nullptr;
+        cudaError_t e;
+        {
+            ProfScope ps(h, RM_K_MIX_LN, s);
+            e = rm::launch_mix_ln(c.dtype, l ? h->Y : X0, prev ? prev->ln2_g : nullptr, prev ? prev->ln2_b : nullptr,
+                                  rm::RowStats{h->ystats, h->stat_P}, w->ln1_g, w->ln1_b, h->S, B, c.T, c.D,
+                                  c.ln_eps, c.mix_addnorm, h->num_sms, derr(h), h->budget_ns, s);
+        }
+        // S rows (b, t) and H rows (t, b), each with its own scale
+        if (e == cudaSuccess) e = rm::launch_quant_rows(h->S, h->S8, h->sS, (long long)B * c.T, c.D, s);
+        rm::GroupedGemm g1{};
+        g1.G = c.T; g1.M = B; g1.N = c.hidden; g1.K = c.D;
+        g1.A = h->S8; g1.a_gstride = c.D; g1.a_ld = (long long)c.T * c.D;
+        g1.W = q[l].W1q;
+        g1.out = h->H; g1.o_gstride = (long long)B * c.hidden; g1.o_ld = c.hidden;
+        g1.bias = static_cast<const float*>(w->b1);
+        g1.epi = rm::f8_epi_for_act(c.act);
+        g1.ascale = h->sS; g1.as_gstride = 1; g1.as_ld = c.T;
+        g1.wscale = q[l].W1s;
+        g1.sk_ws = h->sk_ws; g1.sk_cnt = h->sk_cnt;
+        if (e == cudaSuccess) {
+            ProfScope ps(h, RM_K_GEMM1, s);
+            e = rm::launch_gemm_tc(g1, derr(h), h->budget_ns, h->num_sms, s);
+        }
+        if (e == cudaSuccess) e = rm::launch_quant_rows(h->H, h->H8, h->sH, (long long)c.T * B, c.hidden, s);
+        rm::GroupedGemm g2{};
+        g2.G = c.T; g2.M = B; g2.N = c.D; g2.K = c.hidden;
+        g2.A = h->H8; g2.a_gstride = (long long)B * c.hidden; g2.a_ld = c.hidden;
+        g2.W = q[l].W2q;
+        g2.out = h->Y; g2.o_gstride = c.D; g2.o_ld = (long long)c.T * c.D;
+        g2.bias = static_cast<const float*>(w->b2);
+        g2.resid = h->S; g2.r_gstride = c.D; g2.r_ld = (long long)c.T * c.D;
+        g2.epi = rm::EPI_F8_BIAS_RESID;
+        g2.stats = h->ystats; g2.s_gstride = h->stat_P; g2.s_ld = (long long)c.T * h->stat_P;
+        g2.ascale = h->sH; g2.as_gstride = B; g2.as_ld = 1;
+        g2.wscale = q[l].W2s;
+        g2.sk_ws = h->sk_ws; g2.sk_cnt = h->sk_cnt;
+        if (e == cudaSuccess) {
+            ProfScope ps(h, RM_K_GEMM2, s);
+            e = rm::launch_gemm_tc(g2, derr(h), h->budget_ns, h->num_sms, s);
+        }
+        if (e != cudaSuccess) return RM_ERR_CUDA;
+    }
+    const rm_block_weights* last = &blocks[c.L - 1];
+    ProfScope ps(h, RM_K_LN_POOL, s);
+    return cuda_status(rm::launch_ln_pool(c.dtype, h->Y, rm::RowStats{h->ystats, h->stat_P}, last->ln2_g,
+                                          last->ln2_b, pooled, nullptr, B, c.T, c.D, c.ln_eps, h->num_sms, derr(h),
+                                          h->budget_ns, s));
 }
 
 rm_status rm_stack_forward_host(rm_handle* h, const rm_block_weights* blocks, const void* X0_host,

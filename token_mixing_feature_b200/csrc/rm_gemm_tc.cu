@@ -78,6 +78,10 @@ struct KParams {
     // of the compacted A and W operands (grp_cnt a multiple of 64, the padding
     // rows zero); group coordinate 0 in both maps.
     int vark;
+    // e4m3 operands (EPI_F8_*): dequantisation scales of A's rows and W's rows
+    const float* ascale;
+    long long as_gstride, as_ld;
+    const float* wscale;
     DeviceErr err;
     unsigned long long budget_ns;
 };
@@ -260,6 +264,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     static_assert(!BMN || C::BN_LOCAL % 64 == 0, "N-major W tiles are whole 64-row boxes");
     constexpr bool DACT = EPI == EPI_DACT_TANH || EPI == EPI_DACT_ERF || EPI == EPI_DACT_RELU;
     constexpr bool F32OUT = EPI == EPI_F32;
+    // e4m3 operands: the bf16 epilogue EB after dequantisation; a ring stage
+    // holds KE = 128 one-byte K elements per row instead of 64 bf16
+    constexpr bool F8 = EPI >= EPI_F8_GELU_TANH;
+    constexpr int EB = EPI == EPI_F8_GELU_TANH ? EPI_GELU_TANH
+                       : EPI == EPI_F8_GELU_ERF ? EPI_GELU_ERF
+                       : EPI == EPI_F8_RELU ? EPI_RELU
+                       : EPI == EPI_F8_BIAS_RESID ? EPI_BIAS_RESID : EPI;
+    constexpr int KE = F8 ? 128 : BK;
+    static_assert(!(F8 && (VAR || AMN || BMN || CG == 0)), "e4m3 operands: dense, K-major");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     unsigned char* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -324,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const WaitCtx wc{abort_flag, p.budget_ns, p.err};
     const int nblk = (p.N + BN - 1) / BN;
     const int mblk = (p.M + C::TM - 1) / C::TM;
-    const int num_kb = (p.K + BK - 1) / BK;
+    const int num_kb = (p.K + KE - 1) / KE;
     const long long total = p.var_rows ? (long long)mt_table[p.G] * nblk
                                        : p.full_tiles + ((long long)p.G * nblk * mblk - p.full_tiles) * p.nsplit;
     const long long unit = blockIdx.x / CG, nunits = gridDim.x / CG;
@@ -347,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t fb = full0 + 8 * k;
                     if (leader) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
                     const uint32_t sb = sbase + k * C::STAGE_BYTES + C::A_BYTES;
-                    const int kc = (it0.kb_lo + k) * BK;
+                    const int kc = (it0.kb_lo + k) * KE;
                     load_operand<BMN, C::BN_LOCAL, CG == 2>(sb, &tmB, CG == 2 ? mapa_shared(fb, 0) : fb, kc, nb0,
                                                             t0.g, p.w_g_inner);
                 }
@@ -368,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t fb = full0 + 8 * stage;
                     if (leader && !pre) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
                     const uint32_t sa = sbase + stage * C::STAGE_BYTES;
-                    const int kc = kb * BK + item.koff;
+                    const int kc = kb * KE + item.koff;
                     // the pair counts bytes on the even CTA's barrier
                     const uint32_t fbl = CG == 2 ? mapa_shared(fb, 0) : fb;
                     load_operand<AMN, BM, CG == 2>(sa, &tmA, fbl, kc, t.arow, t.ag, p.a_g_inner);
@@ -391,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         pdl_wait();   // (reads no global memory; keeps every thread ordered after the previous kernel)
         if (lane == 0 && leader) {
             // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = idesc_bf16_f32(C::TM, BN, AMN, BMN);
+            constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(C::TM, BN) : idesc_bf16_f32(C::TM, BN, AMN, BMN);
             // per K = 16 step: 32 bytes along a K-major row, or 16 K rows (2 KB)
             // of an M/N-major tile; descriptors count 16-byte units
             constexpr uint64_t a_step = AMN ? 128 : 2, b_step = BMN ? 128 : 2;
@@ -419,10 +432,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         const uint32_t accum = (kb != item.kb_lo || k != 0) ? 1u : 0u;
-                        if (CG == 2)
-                            tc_mma_f16_pair(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, accum);
-                        else
-                            tc_mma_f16(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, accum);
+                        if constexpr (F8) {   // (a K step of 32 bytes, as for bf16)
+                            if (CG == 2)
+                                tc_mma_f8_pair(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, accum);
+                            else
+                                tc_mma_f8(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, accum);
+                        } else {
+                            if (CG == 2)
+                                tc_mma_f16_pair(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, accum);
+                            else
+                                tc_mma_f16(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, accum);
+                        }
                     }
                     if (CG == 2) tc_commit_pair_mc(empty0 + 8 * stage, 0x3);
                     else tc_commit(empty0 + 8 * stage);
@@ -461,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t stg = staging0 + (uint32_t)ew * 4096u;
         const uint32_t rbar = rbar0 + 8u * (uint32_t)ew;
         uint32_t rphase = 0;
-        const bool has_resid = (EPI == EPI_BIAS_RESID || DACT) && p.resid != nullptr;
+        const bool has_resid = (EB == EPI_BIAS_RESID || DACT) && p.resid != nullptr;
         const uint32_t my_row = stg + (uint32_t)lane * 128u;
         const uint32_t swz = (uint32_t)(lane & 7);
         int it = 0;
@@ -567,6 +587,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     else mbar_arrive(tempty0 + 8 * acc);
                 }
                 if (!live) continue;
+                if constexpr (F8) {   // dequantise: acc * ascale[row] * wscale[g][n + e]
+                    const int mrow = wrow0 + lane;
+                    const float sa =
+                        mrow < p.M ? __ldg(p.ascale + (long long)t.g * p.as_gstride + (long long)mrow * p.as_ld) : 0.f;
+                    const float4* ws4 = reinterpret_cast<const float4*>(p.wscale + (long long)t.g * p.N + n);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        if (n + 4 * q < p.N) {
+                            const float4 w = __ldg(ws4 + q);
+                            v[4 * q] *= sa * w.x;
+                            v[4 * q + 1] *= sa * w.y;
+                            v[4 * q + 2] *= sa * w.z;
+                            v[4 * q + 3] *= sa * w.w;
+                        }
+                    }
+                }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     if (bias_g && n + 16 * q < p.N) {
@@ -584,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                if ((EPI == EPI_RELU || EPI == EPI_GELU_TANH || EPI == EPI_GELU_ERF) && p.save_pre) {
+                if ((EB == EPI_RELU || EB == EPI_GELU_TANH || EB == EPI_GELU_ERF) && p.save_pre) {
                     // the activation's input, kept for the backward pass: its own
                     // store through the staging buffer, before the activation
 #pragma unroll
@@ -603,20 +639,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     __syncwarp();
                 }
-                if (EPI == EPI_RELU) {
+                if (EB == EPI_RELU) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e) v[e] = fmaxf(v[e], 0.0f);
-                } else if (EPI == EPI_GELU_TANH) {
+                } else if (EB == EPI_GELU_TANH) {
 #pragma unroll
                     for (int e = 0; e < 64; e += 2) {
                         const float2 y = gelu_tanh_pair(make_float2(v[e], v[e + 1]));
                         v[e] = y.x;
                         v[e + 1] = y.y;
                     }
-                } else if (EPI == EPI_GELU_ERF) {
+                } else if (EB == EPI_GELU_ERF) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e) v[e] = 0.5f * v[e] * (1.0f + erff(v[e] * 0.7071067811865476f));
-                } else if (EPI == EPI_BIAS_RESID || DACT) {
+                } else if (EB == EPI_BIAS_RESID || DACT) {
                     if (has_resid) {
                         if (!mbar_wait(rbar, rphase, wc, SITE_TC_EPILOGUE)) {
                             ok = false;
@@ -670,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t w[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) w[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-                if (EPI == EPI_BIAS_RESID && p.stats != nullptr && wrow0 + lane < p.M) {
+                if (EB == EPI_BIAS_RESID && p.stats != nullptr && wrow0 + lane < p.M) {
                     // LayerNorm partials of the stored (rounded) 64 values: (mean, M2)
                     float2 a1 = f2(0.f);
 #pragma unroll
@@ -913,6 +949,18 @@ cudaError_t launch_bn(int epi, const Maps& m, const KParams& kp, int grid, cudaS
         case EPI_BIAS_GATE:
             if constexpr (VAR) return launch_typed<BN, EPI_BIAS_GATE, CG, VAR>(m, kp, grid, s);
             break;
+        case EPI_F8_GELU_TANH:
+            if constexpr (!VAR) return launch_typed<BN, EPI_F8_GELU_TANH, CG, VAR>(m, kp, grid, s);
+            break;
+        case EPI_F8_GELU_ERF:
+            if constexpr (!VAR) return launch_typed<BN, EPI_F8_GELU_ERF, CG, VAR>(m, kp, grid, s);
+            break;
+        case EPI_F8_RELU:
+            if constexpr (!VAR) return launch_typed<BN, EPI_F8_RELU, CG, VAR>(m, kp, grid, s);
+            break;
+        case EPI_F8_BIAS_RESID:
+            if constexpr (!VAR) return launch_typed<BN, EPI_F8_BIAS_RESID, CG, VAR>(m, kp, grid, s);
+            break;
     }
     return cudaErrorInvalidValue;
 }
@@ -989,6 +1037,9 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     if (!var && mn && (!g.w_mn || (g.a_mn != f32out) || (!g.a_mn && !dact && g.epi != EPI_BIAS_RESID)))
         return cudaErrorInvalidValue;
     if (vark && (!g.a_mn || !g.w_mn || !f32out || !g.grp_off || !g.vark_cnt)) return cudaErrorInvalidValue;
+    const bool f8 = g.epi >= EPI_F8_GELU_TANH;
+    if (f8 && (var || vark || mn || !g.ascale || !g.wscale || g.K % 16)) return cudaErrorInvalidValue;
+    const uint64_t ae = f8 ? 1 : 2;   // bytes per A / W element
     if (f32out && !mn) return cudaErrorInvalidValue;
     if (dact && !mn) return cudaErrorInvalidValue;
     if (dact && !g.resid) return cudaErrorInvalidValue;
@@ -1015,7 +1066,8 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     kp.stats = g.stats;
     kp.s_gstride = g.s_gstride;
     kp.s_ld = g.s_ld;
-    if (g.stats && (var || g.epi != EPI_BIAS_RESID || g.N % 64)) return cudaErrorInvalidValue;
+    if (g.stats && (var || (g.epi != EPI_BIAS_RESID && g.epi != EPI_F8_BIAS_RESID) || g.N % 64))
+        return cudaErrorInvalidValue;
     kp.full_tiles = 0;
     kp.nsplit = 1;
     kp.sk_ws = g.sk_ws;
@@ -1024,6 +1076,10 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     // activation epilogues with resid set: resid receives the pre-activation values
     kp.save_pre = (g.resid && (g.epi == EPI_GELU_TANH || g.epi == EPI_GELU_ERF || g.epi == EPI_RELU)) ? 1 : 0;
     kp.w_g_inner = 0;
+    kp.ascale = g.ascale;
+    kp.as_gstride = g.as_gstride;
+    kp.as_ld = g.as_ld;
+    kp.wscale = g.wscale;
     kp.err = err;
     kp.budget_ns = budget_ns;
 
@@ -1063,11 +1119,11 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
         }
     } else if (g.a_gstride <= g.a_ld) {
         // group stride inside the row stride, e.g. S [B, T, D]: dims (K, G, M)
-        ok = make_map(&m.a, g.A, g.K, g.G, g.M, g.a_gstride * 2, g.a_ld * 2, 1, BM);
+        ok = make_map_e(&m.a, g.A, g.K, g.G, g.M, g.a_gstride * ae, g.a_ld * ae, 1, BM, (int)ae);
         kp.a_g_inner = 1;
     } else {
         // groups outermost, e.g. H [T, B, kD]: dims (K, M, G)
-        ok = make_map(&m.a, g.A, g.K, g.M, g.G, g.a_ld * 2, g.a_gstride * 2, BM, 1);
+        ok = make_map_e(&m.a, g.A, g.K, g.M, g.G, g.a_ld * ae, g.a_gstride * ae, BM, 1, (int)ae);
         kp.a_g_inner = 0;
     }
     const long long w_ld = g.w_ld ? g.w_ld : g.K, w_gs = g.w_ld ? g.w_gstride : (long long)g.N * g.K;
@@ -1083,7 +1139,7 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
             ok = ok && make_map(&m.b, g.W, g.N, g.K, g.G, w_ld * 2, w_gs * 2, BK, 1);
         }
     } else {
-        ok = ok && make_map(&m.b, g.W, g.K, g.N, g.G, w_ld * 2, w_gs * 2, (uint32_t)(bn / cg), 1);
+        ok = ok && make_map_e(&m.b, g.W, g.K, g.N, g.G, w_ld * ae, w_gs * ae, (uint32_t)(bn / cg), 1, (int)ae);
     }
     if (!var) {
         // output (and residual) tiles of 32 rows x 64 columns (32 for float
@@ -1108,7 +1164,8 @@ cudaError_t launch_gemm_tc(const GroupedGemm& g, DeviceErr err, uint64_t budget_
     if (!var) {
         const long long tiles = (long long)g.G * ((g.M + BM * cg - 1) / (BM * cg)) * ((g.N + bn - 1) / bn);
         if (tiles == 0) return cudaSuccess;
-        const int num_kb = (g.K + BK - 1) / BK;
+        const int ke = f8 ? 128 : BK;   // K elements per ring stage
+        const int num_kb = (g.K + ke - 1) / ke;
         const int S = (g.sk_ws && g.sk_cnt && !vark) ? split_slices(tiles, units, num_kb) : 1;
         if (const char* e = getenv("RM_GEMM_SPLIT"))   // tuning override: 0 disables the split tail
             if (atoi(e) == 0 && S > 1) return launch_gemm_tc_nosplit(g, err, budget_ns, num_sms, s);

@@ -78,7 +78,16 @@ enum Epilogue : int {
     EPI_DACT_ERF = 6,    // bf16( acc * GELU_erf'(U) )
     EPI_DACT_RELU = 7,   // bf16( acc * [U > 0] )
     EPI_F32 = 8,         // float( acc )   (out is float)
+    // e4m3 operands (kind::f8f6f4; dense, K-major): acc is first dequantised,
+    // acc * ascale[row] * wscale[g][n], then as the bf16 epilogue named
+    EPI_F8_GELU_TANH = 9,
+    EPI_F8_GELU_ERF = 10,
+    EPI_F8_RELU = 11,
+    EPI_F8_BIAS_RESID = 12,
 };
+inline int f8_epi_for_act(int act) {
+    return act == RM_ACT_GELU_ERF ? EPI_F8_GELU_ERF : act == RM_ACT_RELU ? EPI_F8_RELU : EPI_F8_GELU_TANH;
+}
 inline int epi_for_act(int act) { return act == RM_ACT_GELU_ERF ? EPI_GELU_ERF : act == RM_ACT_RELU ? EPI_RELU : EPI_GELU_TANH; }
 inline int dact_epi_for_act(int act) {
     return act == RM_ACT_GELU_ERF ? EPI_DACT_ERF : act == RM_ACT_RELU ? EPI_DACT_RELU : EPI_DACT_TANH;
@@ -133,6 +142,11 @@ struct GroupedGemm {
     // at least 64, the padding rows zero).  grp_cnt must be null.
     bool vark;
     const int* vark_cnt;
+    // e4m3 operands (EPI_F8_*): A and W hold one byte per element; row (g, m)
+    // of A has scale ascale[g*as_gstride + m*as_ld], row (g, n) of W wscale[g*N + n].
+    const float* ascale;
+    long long as_gstride, as_ld;
+    const float* wscale;
     // Optional split-K workspace for the dense tcgen05 path (both null: no
     // split).  sk_ws holds gemm_tc_split_ws_bytes(num_sms) bytes; sk_cnt holds
     // gemm_tc_split_cnt_ints(num_sms) ints, zero before the first use (the
@@ -192,6 +206,10 @@ cudaError_t launch_router_grad(const void* S, const float* dR, float* part, floa
 // loss[0] += lambda * sum of x[0 .. n), in a fixed order; part: 256 floats of scratch.
 cudaError_t launch_add_scaled_sum(const float* x, long long n, float lambda, float* loss, float* part,
                                   cudaStream_t s);
+
+// e4m3 rows (rm_fp8.cu): dst[r][k] = e4m3(src[r][k] / scale[r]), scale[r] =
+// absmax of row r / 448 (1 for a zero row); src bf16 [rows][K], K % 16 == 0.
+cudaError_t launch_quant_rows(const void* src, void* dst, float* scale, long long rows, int K, cudaStream_t s);
 
 // Token-sharded forward (rm_shard.cu): G ranks of Tl = T / G tokens each.
 cudaError_t launch_shard_pack(const void* Za, const void* Zb, const float* g, const float* bt, float eps, void* Xh,

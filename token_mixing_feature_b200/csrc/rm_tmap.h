@@ -28,21 +28,28 @@ inline EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// 3-D tensor map: dims d0 (contiguous), d1, d2 with byte strides s1, s2;
-// box (one 128-byte swizzle row of d0: 64 bf16 or 32 float, b1, b2),
-// 128-byte swizzle, zero fill out of bounds.
-inline bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
-                     uint64_t s2, uint32_t b1, uint32_t b2, bool f32 = false) {
+// 3-D tensor map of esz-byte elements (1: e4m3 bytes, 2: bf16, 4: float):
+// dims d0 (contiguous), d1, d2 with byte strides s1, s2; box (one 128-byte
+// swizzle row of d0: 128 / esz elements, b1, b2), 128-byte swizzle, zero fill
+// out of bounds.
+inline bool make_map_e(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                       uint64_t s2, uint32_t b1, uint32_t b2, int esz) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {d0, d1, d2};
     cuuint64_t strides[2] = {s1, s2};
-    cuuint32_t box[3] = {f32 ? 32u : 64u, b1, b2};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / esz), b1, b2};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    const CUtensorMapDataType dt = esz == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : esz == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                              : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+inline bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                     uint64_t s2, uint32_t b1, uint32_t b2, bool f32 = false) {
+    return make_map_e(m, base, d0, d1, d2, s1, s2, b1, b2, f32 ? 4 : 2);
 }
 
 }  // namespace rm

@@ -29,6 +29,7 @@ EXPORTED = (
     "rm_stack_forward_host_async", "rm_host_wait",
     "rm_train_create", "rm_train_destroy", "rm_train_workspace_bytes", "rm_train_step", "rm_train_sync_status",
     "rm_train_set_reg", "rm_tokshard_pack", "rm_tokshard_mix_ln", "rm_tokshard_pool",
+    "rm_quantize_fp8", "rm_stack_forward_fp8",
 )
 RM_STATIC_SCRATCH_BYTES = 16 << 20
 RM_K_COUNT = 11
@@ -44,6 +45,10 @@ class rm_config(ctypes.Structure):
 class rm_block_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("W1", "b1", "W2", "b2", "ln1_g", "ln1_b", "ln2_g", "ln2_b", "Wr", "br", "Wr_infer", "br_infer")]
+
+
+class rm_fp8_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W1q", "W2q", "W1s", "W2s")]
 
 
 class rm_block_grads(ctypes.Structure):
@@ -97,6 +102,9 @@ def _load() -> ctypes.CDLL:
         "rm_tokshard_pack": (st, [vp, vp, vp, vp, vp, vp, vp, ci, ci, vp]),
         "rm_tokshard_mix_ln": (st, [vp, vp, vp, vp, vp, vp, ci, ci, vp]),
         "rm_tokshard_pool": (st, [vp, vp, vp, vp, vp, vp, ci, vp]),
+        "rm_quantize_fp8": (st, [vp, vp, vp, ctypes.c_longlong, ci, vp]),
+        "rm_stack_forward_fp8": (st, [vp, ctypes.POINTER(rm_block_weights), ctypes.POINTER(rm_fp8_weights), vp, vp,
+                                      ci, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -384,3 +392,19 @@ def rm_tokshard_mix_ln(h: Handle, recv, Xh, ln1_g, ln1_b, S, B: int, world: int,
 def rm_tokshard_pool(h: Handle, V, S, ln2_g, ln2_b, pooled_part, B: int, stream=None) -> None:
     _check(_lib.rm_tokshard_pool(h.ptr, _ptr(V), _ptr(S), _ptr(ln2_g), _ptr(ln2_b), _ptr(pooled_part), B,
                                  _stream(stream)), "rm_tokshard_pool")
+
+
+# ------------------------------------------------- stack with e4m3 FFN weights
+def rm_quantize_fp8(src, dst, scale, rows: int, K: int, stream=None) -> None:
+    _check(_lib.rm_quantize_fp8(_ptr(src), _ptr(dst), _ptr(scale), rows, K, _stream(stream)), "rm_quantize_fp8")
+
+
+def rm_stack_forward_fp8(h: Handle, blocks: Sequence[Dict], qblocks: Sequence[Dict], X0, pooled, B: int,
+                         stream=None) -> None:
+    """qblocks: per block {"W1q", "W2q", "W1s", "W2s"} device tensors."""
+    arr = _block_array(blocks)
+    qarr = (rm_fp8_weights * len(qblocks))()
+    for i, q in enumerate(qblocks):
+        qarr[i] = rm_fp8_weights(**{n: _ptr(q[n]) for n, _ in rm_fp8_weights._fields_})
+    _check(_lib.rm_stack_forward_fp8(h.ptr, arr, qarr, _ptr(X0), _ptr(pooled), B, _stream(stream)),
+           "rm_stack_forward_fp8")
