@@ -246,7 +246,8 @@ rm_status rm_pffn_forward_static(const rm_block_weights *w, const void *S, void 
  *
  * rm_quantize_fp8: dst[r][k] = e4m3(src[r][k] / scale[r]) with scale[r] =
  *   max_k |src[r][k]| / 448 (1 for an all-zero row), src bf16 [rows][K],
- *   dst one byte per element, K % 16 == 0.  For W1 [T][kD][D] call it with
+ *   dst one byte per element, K % 16 == 0 (else RM_ERR_INVALID_ARG), K <=
+ *   16384 and rows < 2^31 (else RM_ERR_UNSUPPORTED).  For W1 [T][kD][D] call it with
  *   rows = T*kD, K = D; for W2 [T][D][kD] with rows = T*D, K = kD.
  * rm_stack_forward_fp8: as rm_stack_forward (pooled output only) with the
  *   quantised weights of every block in q[l] (the biases, LayerNorm

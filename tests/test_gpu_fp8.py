@@ -17,7 +17,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_common import dev, host64, rel_l2
+from gpu_common import dev, host64, rel_l2, sample_rows
 from token_mixing_feature_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -43,11 +43,18 @@ def _e4m3_round(x: np.ndarray) -> np.ndarray:
     return np.sign(x) * r * ulp
 
 
-def test_quantize_rows_matches_definition(rm):
+@pytest.mark.parametrize("rows,K", [
+    (40, 96),        # 12 vectors a row: one partial warp
+    (24, 1536),      # S rows at D = 1536: 192 threads, one vector each
+    (9, 2064),       # 258 vectors: two a thread, the second ragged
+    (12, 6144),      # H rows at kD = 6144: three vectors a thread
+    (5, 12304),      # 1538 vectors: the eight-vector form with seven in use
+    (3, 16384),      # the largest row
+])
+def test_quantize_rows_matches_definition(rm, rows, K):
     g = torch.Generator().manual_seed(3)
-    rows, K = 40, 96
     x = (torch.randn(rows, K, generator=g) * torch.logspace(-3, 2, rows).unsqueeze(1)).to(torch.bfloat16)
-    x[7] = 0                                                    # an all-zero row gets scale 1
+    x[rows // 2] = 0                                            # an all-zero row gets scale 1
     q = torch.empty(rows, K, dtype=torch.uint8, device="cuda")
     sc = torch.empty(rows, device="cuda")
     rm.rm_quantize_fp8(dev(x), q, sc, rows, K)
@@ -97,3 +104,56 @@ def test_fp8_stack(rm, O, B, T, D, hidden, L, act):
     assert r_bf <= FP8_REL_L2, f"fp8 vs bf16 stack: rel L2 {r_bf:.3e}"
     assert r_or > 1e-3   # the quantisation is really in the path
     st.close()
+
+
+def test_fp8_stack_rm1b_graph_sampled(rm, O):
+    """The rm1b stack with e4m3 FFN operands as the benchmark runs it: weights
+    quantised once, the step captured in a CUDA graph on a side stream and
+    replayed there; the replay equals a direct launch bit for bit, and sampled
+    rows of the pooled output stay within the e4m3 bound of the oracle."""
+    from token_mixing_feature_b200.stack import RankMixerStack
+    wl = synth.WORKLOADS["rm1b"]
+    B, T, D, Hd = wl.B, wl.T, wl.D, wl.hidden
+    d = synth.make_inputs(wl)
+    st = RankMixerStack(wl, d["blocks"])
+    qblocks = [_quantize_block(rm, blk, T, D, Hd) for blk in d["blocks"]]
+    X0 = dev(d["X0"])
+    pooled = torch.empty(B, D, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        rm.rm_stack_forward_fp8(st.h, st.blocks, qblocks, X0, pooled, B, side)
+        side.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            rm.rm_stack_forward_fp8(st.h, st.blocks, qblocks, X0, pooled, B, side)
+    torch.cuda.synchronize()
+    pooled.zero_()
+    with torch.cuda.stream(side):
+        g.replay()
+    torch.cuda.synchronize()
+    got = pooled.clone()
+    direct = torch.empty_like(pooled)
+    rm.rm_stack_forward_fp8(st.h, st.blocks, qblocks, X0, direct, B)
+    torch.cuda.synchronize()
+    assert rm.rm_sync_status(st.h) == rm.RM_OK
+    assert torch.equal(got, direct)
+    idx = sample_rows(B, 8)
+    ref = O.stack(synth.make_x0(wl, samples=idx), d["blocks"], want_all=False, want_last=False)
+    r = rel_l2(host64(got[idx.to("cuda")]), ref["pooled"])
+    assert 1e-3 < r <= FP8_REL_L2, f"fp8 rm1b vs oracle: rel L2 {r:.3e}"
+    del g
+    st.close()
+
+
+def test_quantize_rejects_unsupported(rm):
+    x = torch.zeros(2, 16400, dtype=torch.bfloat16, device="cuda")
+    q = torch.empty(2, 16400, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(2, device="cuda")
+    with pytest.raises(rm.RankMixerError) as e:
+        rm.rm_quantize_fp8(x, q, sc, 2, 16400)          # rows longer than 16384
+    assert e.value.status == rm.RM_ERR_UNSUPPORTED
+    with pytest.raises(rm.RankMixerError) as e:
+        rm.rm_quantize_fp8(x, q, sc, 2, 24)             # K not a multiple of 16
+    assert e.value.status == rm.RM_ERR_INVALID_ARG
+    rm.rm_quantize_fp8(x, q, sc, 0, 16)                 # no rows: nothing to do

@@ -495,6 +495,7 @@ rm_status rm_stack_forward(rm_handle* h, const rm_block_weights* blocks, const v
 
 rm_status rm_quantize_fp8(const void* src, void* dst, float* scale, long long rows, int K, rm_stream_t stream) {
     if (!aligned16(src) || !aligned16(dst) || !scale || rows < 0 || K < 16 || K % 16) return RM_ERR_INVALID_ARG;
+    if (K > 16384 || rows > 0x7fffffffLL) return RM_ERR_UNSUPPORTED;   // one CTA per row, <= 8 vectors a thread
     if (rows == 0) return RM_OK;
     return cuda_status(rm::launch_quant_rows(src, dst, scale, rows, K, stream));
 }
