@@ -539,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 64 * half; c < BN; c += 128) {
                 const int n = t.n0 + c;
                 const bool live = n < p.N;   // warp-uniform
-                if (!F32OUT) {   // (float output alternates two buffers below)
+                if (!F32OUT) {   // (float output: transposed line stores below)
                     if (lane == 0) bulk_wait_read_all();   // the previous store has read the buffer
                     __syncwarp();
                 }
@@ -679,11 +679,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if constexpr (F32OUT) {
-                    // two 32-column float halves through the staging buffer
+                    // Two 32-column float halves, transposed through the
+                    // staging buffer: the lanes write their rows, then read
+                    // back four whole rows per instruction (8 lanes x 16 bytes
+                    // a row) and store them as full 128-byte lines.  No bulk
+                    // store to wait for, so a warp's stores are not limited
+                    // to one 4 KB buffer in flight.
+                    float* obase = reinterpret_cast<float*>(p.out) + (long long)t.g * p.o_gstride;
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
-                        if (lane == 0) bulk_wait_read_all();   // the previous store has read the buffer
-                        __syncwarp();
+                        const int n2 = n + 32 * hh;
+                        if (n2 >= p.N) break;   // warp-uniform; N is a multiple of 32
+                        __syncwarp();          // every lane has read the previous half
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             const float* q = v + 32 * hh + 4 * j;
@@ -693,12 +700,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          "r"(__float_as_uint(q[2])), "r"(__float_as_uint(q[3]))
                                          : "memory");
                         }
-                        fence_proxy_async_shared();
                         __syncwarp();
-                        if (lane == 0) {
-                            if (p.o_g_inner) tma_store_3d(&tmO, stg, n + 32 * hh, t.g, wrow0);
-                            else tma_store_3d(&tmO, stg, n + 32 * hh, wrow0, t.g);
-                            bulk_commit_group();
+                        const uint32_t ju = (uint32_t)(lane & 7);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int r = 4 * i + (lane >> 3);
+                            uint32_t x0, x1, x2, x3;
+                            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+                                         : "r"(stg + (uint32_t)r * 128u + ((ju ^ (uint32_t)(r & 7)) << 4))
+                                         : "memory");
+                            if (wrow0 + r < p.M)
+                                __stcs(reinterpret_cast<float4*>(obase + (long long)(wrow0 + r) * p.o_ld + n2 +
+                                                                 4 * (int)ju),
+                                       make_float4(__uint_as_float(x0), __uint_as_float(x1), __uint_as_float(x2),
+                                                   __uint_as_float(x3)));
                         }
                     }
                     continue;
