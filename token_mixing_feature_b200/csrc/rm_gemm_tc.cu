@@ -467,9 +467,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Each warp owns 32 accumulator rows (its TMEM lane quarter) and half
         // of the BN columns, in 64-column chunks: tcgen05.ld -> registers ->
         // bias / GELU / residual -> bf16 into a 128-byte-swizzled 32 x 64
-        // staging buffer -> one TMA bulk store.  The residual tile arrives in
-        // the same buffer by TMA first.  The accumulator is released right
-        // after the tile's last tcgen05.ld.
+        // staging buffer -> one TMA bulk store (float output instead goes
+        // through the buffer as a transpose and leaves as whole 128-byte
+        // lines from the registers).  The residual tile arrives in the same
+        // buffer by TMA first.  The accumulator is released right after the
+        // tile's last tcgen05.ld.
         const int ew = warp - 2;
         const int quarter = warp & 3;
         const int half = ew >> 2;
