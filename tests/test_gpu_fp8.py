@@ -44,8 +44,9 @@ def _e4m3_round(x: np.ndarray) -> np.ndarray:
 
 
 @pytest.mark.parametrize("rows,K", [
-    (40, 96),        # 12 vectors a row: one partial warp
-    (24, 1536),      # S rows at D = 1536: 192 threads, one vector each
+    (40, 96),        # 12 vectors a row: one partial warp, four rows a CTA
+    (24, 1536),      # S rows at D = 1536: 192 threads, one vector each, four rows a CTA
+    (25, 1536),      # the last CTA's four rows ragged
     (9, 2064),       # 258 vectors: two a thread, the second ragged
     (12, 6144),      # H rows at kD = 6144: three vectors a thread
     (5, 12304),      # 1538 vectors: the eight-vector form with seven in use
