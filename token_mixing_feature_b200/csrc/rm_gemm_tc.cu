@@ -254,6 +254,26 @@ __device__ __forceinline__ float dact(float u) {
     }
 }
 
+// The derivative at a pair of points: the tanh form in paired fp32
+// instructions (two elements an instruction, tanh from the SFU), the other
+// activations element by element.
+template <int EPI>
+__device__ __forceinline__ float2 dact_pair(float2 u) {
+    if constexpr (EPI == EPI_DACT_TANH) {
+        const float c = 0.7978845608028654f;
+        const float2 u2 = f2_mul(u, u);
+        const float2 a = f2_mul(u, f2_fma(u2, f2(c * 0.044715f), f2(c)));      // c (u + 0.044715 u^3)
+        float2 th;
+        asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(a.x));
+        asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(a.y));
+        const float2 hd = f2_mul(f2_mul(u, f2(0.5f)), f2_fma(u2, f2(3.0f * 0.044715f * c), f2(c)));
+        const float2 sech2 = f2_fma(th, make_float2(-th.x, -th.y), f2(1.0f));   // 1 - tanh^2
+        return f2_fma(hd, sech2, f2_fma(th, f2(0.5f), f2(0.5f)));
+    } else {
+        return make_float2(dact<EPI>(u.x), dact<EPI>(u.y));
+    }
+}
+
 template <int BN, int EPI, int CG, bool VAR, bool AMN = false, bool BMN = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -672,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const float2 a = make_float2(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
-                                const float2 y = DACT ? f2_mul(a, make_float2(dact<EPI>(rp[e].x), dact<EPI>(rp[e].y)))
+                                const float2 y = DACT ? f2_mul(a, dact_pair<EPI>(rp[e]))
                                                       : f2_add(a, rp[e]);
                                 v[8 * j + 2 * e] = y.x;
                                 v[8 * j + 2 * e + 1] = y.y;
@@ -847,8 +867,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             unpack_pairs(uc[q], up);
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                v[8 * q + 2 * e] *= dact<EPI>(up[e].x);
-                                v[8 * q + 2 * e + 1] *= dact<EPI>(up[e].y);
+                                const float2 y = f2_mul(make_float2(v[8 * q + 2 * e], v[8 * q + 2 * e + 1]),
+                                                        dact_pair<EPI>(up[e]));
+                                v[8 * q + 2 * e] = y.x;
+                                v[8 * q + 2 * e + 1] = y.y;
                             }
                         }
                     } else if (EPI == EPI_BIAS_GATE) {
